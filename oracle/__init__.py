@@ -1,0 +1,207 @@
+"""CPU oracle of the NVFP4 FlashAttention forward (ctypes binding).
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by __graft_entry__.smoke() and by
+the CPU-baseline leg of bench.py, never by the product path. The arithmetic is
+in fp4attn_oracle.cpp, which shares nothing with the CUDA sources.
+
+Every function has CPU pins in tests/test_oracle_*.py; none is "parity
+unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fp4attn_oracle.cpp")
+_LIB = os.path.join(_HERE, "libfp4attn_oracle.so")
+_lib = None
+
+FLAG_QP_DENOMINATOR = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle (g++, no fused multiply-add contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["g++", "-O2", "-std=c++17", "-ffp-contract=off", "-fno-fast-math",
+                               "-fPIC", "-shared", "-pthread", "-o", tmp, _SRC])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        f32, u8, i32, i64, u32 = (ctypes.c_float, ctypes.c_uint8, ctypes.c_int, ctypes.c_int64,
+                                  ctypes.c_uint32)
+        vp = ctypes.c_void_p
+        lib.ora_e2m1_encode.argtypes = [f32]
+        lib.ora_e2m1_encode.restype = u8
+        lib.ora_e2m1_decode.argtypes = [u8]
+        lib.ora_e2m1_decode.restype = f32
+        lib.ora_e4m3_encode.argtypes = [f32]
+        lib.ora_e4m3_encode.restype = u8
+        lib.ora_e4m3_decode.argtypes = [u8]
+        lib.ora_e4m3_decode.restype = f32
+        lib.ora_e2m1_encode_range.argtypes = [u32, i64, vp, i32]
+        lib.ora_e2m1_encode_range.restype = None
+        lib.ora_e4m3_encode_range.argtypes = [u32, i64, vp, i32]
+        lib.ora_e4m3_encode_range.restype = None
+        lib.ora_amax_bf16.argtypes = [vp, i64]
+        lib.ora_amax_bf16.restype = f32
+        lib.ora_tensor_scale.argtypes = [f32, vp, vp]
+        lib.ora_tensor_scale.restype = None
+        lib.ora_quantize_block.argtypes = [vp, i32, f32, vp, vp]
+        lib.ora_quantize_block.restype = None
+        lib.ora_quantize_rows.argtypes = [vp, i64, i32, f32, vp, vp, i32]
+        lib.ora_quantize_rows.restype = None
+        lib.ora_quantize_tokens_T.argtypes = [vp, i32, i32, f32, vp, vp, i32]
+        lib.ora_quantize_tokens_T.restype = None
+        lib.ora_scores_head.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32]
+        lib.ora_scores_head.restype = i32
+        lib.ora_attn_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, i32,
+                                     vp, i64, vp, vp, vp, i32]
+        lib.ora_attn_fwd.restype = i32
+        _lib = lib
+    return _lib
+
+
+def _threads(n: int | None) -> int:
+    return int(n) if n else max(1, os.cpu_count() or 1)
+
+
+def _c(a: np.ndarray, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# ------------------------------------------------------------- formats ----
+def e2m1_encode(y: float) -> int:
+    return int(_load().ora_e2m1_encode(float(y)))
+
+
+def e2m1_decode(c: int) -> float:
+    return float(_load().ora_e2m1_decode(int(c)))
+
+
+def e4m3_encode(y: float) -> int:
+    return int(_load().ora_e4m3_encode(float(y)))
+
+
+def e4m3_decode(c: int) -> float:
+    return float(_load().ora_e4m3_decode(int(c)))
+
+
+def e2m1_encode_range(start: int, count: int, threads: int | None = None) -> np.ndarray:
+    """Codes of fp32 bit patterns start..start+count-1 (0xFF marks NaN inputs)."""
+    out = np.empty(count, dtype=np.uint8)
+    _load().ora_e2m1_encode_range(start, count, out.ctypes.data, _threads(threads))
+    return out
+
+
+def e4m3_encode_range(start: int, count: int, threads: int | None = None) -> np.ndarray:
+    out = np.empty(count, dtype=np.uint8)
+    _load().ora_e4m3_encode_range(start, count, out.ctypes.data, _threads(threads))
+    return out
+
+
+# ----------------------------------------------------------- quantizer ----
+def amax_bf16(x: np.ndarray) -> float:
+    x = _c(x, np.uint16)
+    return float(_load().ora_amax_bf16(x.ctypes.data, x.size))
+
+
+def tensor_scale(amax: float) -> tuple[float, float]:
+    """(s_enc, d) of a tensor whose absolute maximum is amax."""
+    s, d = ctypes.c_float(), ctypes.c_float()
+    _load().ora_tensor_scale(float(amax), ctypes.byref(s), ctypes.byref(d))
+    return s.value, d.value
+
+
+def quantize_block(x, s_enc: float) -> tuple[np.ndarray, int]:
+    """One block (<= 16 fp32 values): (codes, one per byte; scale byte)."""
+    x = _c(x, np.float32)
+    assert x.size <= 16
+    codes = np.zeros(x.size, dtype=np.uint8)
+    e = ctypes.c_uint8()
+    _load().ora_quantize_block(x.ctypes.data, x.size, float(s_enc), codes.ctypes.data,
+                               ctypes.byref(e))
+    return codes, int(e.value)
+
+
+def quantize_rows(x_bf16: np.ndarray, s_enc: float, threads: int | None = None):
+    """Blocks of 16 along the last axis. Returns (codes [..., D/2], scales [..., D/16])."""
+    x = _c(x_bf16, np.uint16)
+    D = x.shape[-1]
+    rows = x.size // D
+    codes = np.empty(x.shape[:-1] + (D // 2,), dtype=np.uint8)
+    scales = np.empty(x.shape[:-1] + (D // 16,), dtype=np.uint8)
+    _load().ora_quantize_rows(x.ctypes.data, rows, D, float(s_enc), codes.ctypes.data,
+                              scales.ctypes.data, _threads(threads))
+    return codes, scales
+
+
+def quantize_tokens_T(x_bf16: np.ndarray, s_enc: float, npad: int | None = None):
+    """x [N, D]: blocks of 16 tokens per channel, transposed.
+    Returns (codes [D, npad/2], scales [D, npad/16])."""
+    x = _c(x_bf16, np.uint16)
+    N, D = x.shape
+    npad = npad or (N + 15) // 16 * 16
+    codes = np.empty((D, npad // 2), dtype=np.uint8)
+    scales = np.empty((D, npad // 16), dtype=np.uint8)
+    _load().ora_quantize_tokens_T(x.ctypes.data, N, D, float(s_enc), codes.ctypes.data,
+                                  scales.ctypes.data, npad)
+    return codes, scales
+
+
+# ----------------------------------------------------------- attention ----
+def scores_head(q, k, b: int, h: int, threads: int | None = None) -> np.ndarray:
+    q = _c(q, np.uint16)
+    k = _c(k, np.uint16)
+    B, H, N, D = q.shape
+    Hkv = k.shape[1]
+    S = np.empty((N, N), dtype=np.float32)
+    rc = _load().ora_scores_head(q.ctypes.data, k.ctypes.data, B, H, Hkv, N, D, b, h,
+                                 S.ctypes.data, _threads(threads))
+    if rc:
+        raise ValueError("ora_scores_head: bad arguments")
+    return S
+
+
+def attn_fwd(q, k, v, causal: bool, softmax_scale: float = 0.0, rows=None, Bc: int = 128,
+             flags: int = 0, threads: int | None = None, want_f64: bool = False,
+             want_ml: bool = False):
+    """The tiled NVFP4 attention forward on the CPU.
+
+    q [B,H,N,D], k/v [B,Hkv,N,D] as uint16 bf16 bit patterns. rows: None (every
+    row; the outputs have q's shape) or int64 [n, 3] triples (b, h, i) (outputs
+    [n, D]). Returns a dict with "bf16" (uint16) and optionally "f64" and "ml"."""
+    q = _c(q, np.uint16)
+    k = _c(k, np.uint16)
+    v = _c(v, np.uint16)
+    B, H, N, D = q.shape
+    Hkv = k.shape[1]
+    if rows is None:
+        shape, rp, nrows = (B, H, N, D), None, 0
+    else:
+        rows = _c(rows, np.int64).reshape(-1, 3)
+        shape, rp, nrows = (rows.shape[0], D), rows.ctypes.data, rows.shape[0]
+    out = np.empty(shape, dtype=np.uint16)
+    f64 = np.empty(shape, dtype=np.float64) if want_f64 else None
+    ml = np.empty(shape[:-1] + (2,), dtype=np.float64) if want_ml else None
+    rc = _load().ora_attn_fwd(q.ctypes.data, k.ctypes.data, v.ctypes.data, B, H, Hkv, N, D,
+                              int(bool(causal)), float(softmax_scale), Bc, flags, rp, nrows,
+                              out.ctypes.data, f64.ctypes.data if f64 is not None else None,
+                              ml.ctypes.data if ml is not None else None, _threads(threads))
+    if rc:
+        raise ValueError("ora_attn_fwd: bad arguments")
+    res = {"bf16": out}
+    if want_f64:
+        res["f64"] = f64
+    if want_ml:
+        res["ml"] = ml
+    return res

@@ -1,0 +1,497 @@
+// CPU oracle for the NVFP4 FlashAttention forward.
+//
+// TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the CPU-baseline
+// leg of the benchmark load this file's library. The CUDA path shares no code,
+// header, table or constant generator with it.
+//
+// Plain, slow and written to be checked by eye against the method:
+//  * "4-bit attention" runs both QK^T and PV as 4-bit block-scaled
+//    contractions while the online-softmax state stays in higher precision
+//    [HiFA4 summary, theflow.svmpsp.dev related-papers feed; EFQ-Softmax
+//    abstract, scholarbro.com page "AVQ Attention: Adaptive Vector-Quantized
+//    Attention"].
+//  * The operand format is block-scaled E2M1, named NVFP4 [TetraJet-v2
+//    abstract, searcharxiv.com author page "Pengle Zhang"; Minima summary,
+//    theflow feed; EFQ-Softmax abstract].
+//  * The probability path is exp-then-quantize: shifted-score exponentials in
+//    higher precision form a temporary probability block that is quantized
+//    before the low-bit PV product; the FlashAttention row-maximum update,
+//    historical rescaling, high-precision accumulation and final normalisation
+//    are kept [EFQ-Softmax abstract].
+// The pages give no formula for any of these steps. Where this file fixes one
+// (format constants, scale recipe, rounding, masking, GQA mapping, the
+// denominator) it states the reading it takes.
+//
+// Precision: quantisation runs in IEEE fp32, one correctly rounded operation
+// per step and never a fused multiply-add (build with -ffp-contract=off).
+// Dot products of dequantised operands are exact in double: every product has
+// at most 12 significant bits and a sum over <= 128 terms spans at most 50
+// bits of binary exponent, below double's 53.
+//
+// Parity pins: every function here is pinned by the CPU tests (tests/
+// test_oracle_*.py): format tables written from the format definitions, brute
+// force nearest-value search, exactly representable round trips, hand-worked
+// attention examples (tests/golden/), closed forms (uniform scores, one key),
+// and brute-force fp64 attention within an a-posteriori FP4 error bound.
+#include <algorithm>
+#include <atomic>
+#include <cfloat>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+namespace {
+
+// ---------------------------------------------------------------- bf16 ----
+float bf16_to_f32(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+uint16_t f32_to_bf16_rne(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  if ((u & 0x7FFFFFFFu) > 0x7F800000u) return (uint16_t)((u >> 16) | 0x40);
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+// ---------------------------------------------------------------- E2M1 ----
+// E2M1: 1 sign bit (bit 3), 2 exponent bits, 1 mantissa bit. Magnitudes of
+// codes 0..7 are {0, 0.5, 1, 1.5, 2, 3, 4, 6}.
+const float kE2M1Mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+
+// Round to nearest, ties to the even code (mantissa bit 0); magnitudes above
+// 6 saturate to 6 (the "satfinite" behaviour). The sign bit is copied from the
+// input, so -0 and small negatives that round to zero give code 8.
+uint8_t e2m1_encode(float y) {
+  uint8_t s = std::signbit(y) ? 8 : 0;
+  float a = std::fabs(y);
+  uint8_t c;
+  if (a <= 0.25f) c = 0;        // tie 0.25 -> code 0
+  else if (a < 0.75f) c = 1;
+  else if (a <= 1.25f) c = 2;   // ties 0.75 and 1.25 -> code 2
+  else if (a < 1.75f) c = 3;
+  else if (a <= 2.5f) c = 4;    // ties 1.75 and 2.5 -> code 4
+  else if (a < 3.5f) c = 5;
+  else if (a <= 5.0f) c = 6;    // ties 3.5 and 5 -> code 6
+  else c = 7;                   // (5, inf] -> 6
+  return s | c;
+}
+
+float e2m1_decode(uint8_t c) {
+  float m = kE2M1Mag[c & 7];
+  return (c & 8) ? -m : m;
+}
+
+// ---------------------------------------------------------------- E4M3 ----
+// E4M3 (OCP FP8 E4M3): bias 7, no infinities, 0x7F/0xFF are NaN, largest
+// finite magnitude 0x7E = 448, subnormals m * 2^-9.
+float e4m3_decode(uint8_t c) {
+  int e = (c >> 3) & 15, m = c & 7;
+  float mag;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0) mag = std::ldexp((float)m, -9);
+  else mag = std::ldexp(1.0f + m / 8.0f, e - 7);
+  return (c & 0x80) ? -mag : mag;
+}
+
+// Round to nearest, ties to the even code; magnitudes above 448 saturate to
+// 448 (satfinite). Nearest-value search over the 127 finite magnitudes.
+uint8_t e4m3_encode(float y) {
+  if (std::isnan(y)) return 0x7F;
+  uint8_t s = std::signbit(y) ? 0x80 : 0;
+  float a = std::fabs(y);
+  static float mags[127];
+  static bool init = false;
+  if (!init) {  // benign race: every thread writes the same values
+    for (int c = 0; c < 127; ++c) mags[c] = e4m3_decode((uint8_t)c);
+    init = true;
+  }
+  if (a >= 448.0f) return s | 0x7E;
+  // first code whose magnitude is >= a
+  int hi = (int)(std::lower_bound(mags, mags + 127, a) - mags);
+  if (hi == 0) return s;  // a == 0
+  int lo = hi - 1;
+  double dlo = (double)a - mags[lo], dhi = (double)mags[hi] - a;
+  int c;
+  if (dlo < dhi) c = lo;
+  else if (dhi < dlo) c = hi;
+  else c = (lo % 2 == 0) ? lo : hi;
+  return s | (uint8_t)c;
+}
+
+// ------------------------------------------------------- NVFP4 recipe ----
+// Reading (the pages name NVFP4 and "block-scaled E2M1" but give no recipe):
+// the standard two-level NVFP4 scaling. One fp32 scale per tensor maps the
+// tensor's absolute maximum onto 6 * 448 = 2688, the product of the largest
+// E2M1 and E4M3 magnitudes; each block of 16 elements carries an E4M3 scale.
+const float kTensorRange = 2688.0f;  // 6 * 448
+
+// s_enc = 2688 / amax; amax == 0 gives s_enc = 1; a non-finite quotient
+// saturates to FLT_MAX. The decode scale is d = 1 / s_enc.
+void tensor_scale(float amax, float* s_enc, float* d) {
+  float s = (amax > 0.0f) ? kTensorRange / amax : 1.0f;
+  if (!std::isfinite(s)) s = FLT_MAX;
+  *s_enc = s;
+  *d = 1.0f / s;
+}
+
+// One block (n <= 16 values; absent values of a tail block count as zero):
+//   a = max |x_i|
+//   e = E4M3(fl(fl(a / 6) * s_enc))
+//   r = fl(s_enc / dec(e)), or 0 when dec(e) == 0
+//   code_i = E2M1(fl(x_i * r))
+// Each operation is one correctly rounded fp32 operation.
+void quantize_block(const float* x, int n, float s_enc, uint8_t* codes, uint8_t* scale) {
+  float a = 0.0f;
+  for (int i = 0; i < n; ++i) a = std::max(a, std::fabs(x[i]));
+  float t = a / 6.0f;
+  t = t * s_enc;
+  uint8_t e = e4m3_encode(t);
+  float de = e4m3_decode(e);
+  float r = (de == 0.0f) ? 0.0f : s_enc / de;
+  for (int i = 0; i < n; ++i) {
+    float y = x[i] * r;
+    codes[i] = e2m1_encode(y);
+  }
+  *scale = e;
+}
+
+float amax_bf16(const uint16_t* x, int64_t n) {
+  float a = 0.0f;
+  for (int64_t i = 0; i < n; ++i) a = std::max(a, std::fabs(bf16_to_f32(x[i])));
+  return a;
+}
+
+template <class F>
+void parallel_for(int64_t n, int nthreads, F&& f) {
+  if (nthreads <= 0) nthreads = (int)std::max(1u, std::thread::hardware_concurrency());
+  if (nthreads == 1 || n < 2) {
+    for (int64_t i = 0; i < n; ++i) f(i);
+    return;
+  }
+  std::atomic<int64_t> next(0);
+  std::vector<std::thread> ts;
+  for (int t = 0; t < nthreads; ++t)
+    ts.emplace_back([&] {
+      for (int64_t i; (i = next.fetch_add(1)) < n;) f(i);
+    });
+  for (auto& t : ts) t.join();
+}
+
+// Rows of `cols` values, blocks of 16 along the row (Q and K: along D).
+// codes [rows][cols/2]: element 2i in the low nibble of byte i.
+// scales [rows][cols/16].
+void quantize_rows(const uint16_t* x, int64_t rows, int cols, float s_enc, uint8_t* codes,
+                   uint8_t* scales, int nthreads) {
+  const int nb = cols / 16;
+  parallel_for(rows, nthreads, [&](int64_t r) {
+    float blk[16];
+    uint8_t c[16];
+    for (int b = 0; b < nb; ++b) {
+      for (int i = 0; i < 16; ++i) blk[i] = bf16_to_f32(x[r * cols + b * 16 + i]);
+      quantize_block(blk, 16, s_enc, c, &scales[r * nb + b]);
+      for (int i = 0; i < 8; ++i)
+        codes[r * (cols / 2) + b * 8 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+    }
+  });
+}
+
+// V: blocks of 16 consecutive tokens for each channel d, stored transposed.
+// x [N][D]; codes [D][npad/2], scales [D][npad/16]; tokens >= N count as 0.
+void quantize_tokens_T(const uint16_t* x, int N, int D, float s_enc, uint8_t* codes,
+                       uint8_t* scales, int npad) {
+  const int nb = npad / 16;
+  for (int d = 0; d < D; ++d)
+    for (int b = 0; b < nb; ++b) {
+      float blk[16];
+      uint8_t c[16];
+      for (int i = 0; i < 16; ++i) {
+        int n = b * 16 + i;
+        blk[i] = (n < N) ? bf16_to_f32(x[(int64_t)n * D + d]) : 0.0f;
+      }
+      quantize_block(blk, 16, s_enc, c, &scales[(int64_t)d * nb + b]);
+      for (int i = 0; i < 8; ++i)
+        codes[(int64_t)d * (npad / 2) + b * 8 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+    }
+}
+
+// Dequantised value in the contraction's own units: E2M1 value times the E4M3
+// block scale. The tensor scale d is applied after the contraction.
+inline double deq(uint8_t code, uint8_t scale) {
+  return (double)e2m1_decode(code) * (double)e4m3_decode(scale);
+}
+
+const float kLog2e = 1.44269504088896340736f;  // fl32(1 / ln 2)
+
+struct Tensors {
+  const uint16_t *q, *k, *v;
+  int B, H, Hkv, N, D;
+  float sq, dq, sk, dk, sv, dv;
+};
+
+// K and V of one (b, kv-head), dequantised to contraction units, [N][D].
+struct KVGroup {
+  std::vector<double> K, V;
+};
+
+KVGroup make_group(const Tensors& T, int b, int hk) {
+  const int N = T.N, D = T.D;
+  const int64_t off = ((int64_t)b * T.Hkv + hk) * N * D;
+  KVGroup g;
+  g.K.resize((size_t)N * D);
+  g.V.resize((size_t)N * D);
+  std::vector<uint8_t> kc((size_t)N * D / 2), ks((size_t)N * D / 16);
+  quantize_rows(T.k + off, N, D, T.sk, kc.data(), ks.data(), 1);
+  for (int64_t n = 0; n < N; ++n)
+    for (int d = 0; d < D; ++d) {
+      uint8_t byte = kc[n * (D / 2) + d / 2];
+      uint8_t c = (d & 1) ? (byte >> 4) : (byte & 15);
+      g.K[n * D + d] = deq(c, ks[n * (D / 16) + d / 16]);
+    }
+  const int npad = (N + 15) / 16 * 16;
+  std::vector<uint8_t> vc((size_t)D * npad / 2), vs((size_t)D * npad / 16);
+  quantize_tokens_T(T.v + off, N, D, T.sv, vc.data(), vs.data(), npad);
+  for (int d = 0; d < D; ++d)
+    for (int64_t n = 0; n < N; ++n) {
+      uint8_t byte = vc[d * (npad / 2) + n / 2];
+      uint8_t c = (n & 1) ? (byte >> 4) : (byte & 15);
+      g.V[n * D + d] = deq(c, vs[d * (npad / 16) + n / 16]);
+    }
+  return g;
+}
+
+enum { FLAG_QP_DENOMINATOR = 1 };
+
+// One query row: the tiled forward over key tiles of Bc keys.
+//   S_ij = fl32(exact dot product of dequantised q_i, k_j)
+//   x_ij = fl32(S_ij * c), c = fl32(fl32(fl32(d_Q d_K) * softmax_scale) * log2 e)
+//   masked (causal j > i, top-left aligned) -> -inf
+// per tile: m_new = max(m, max_j x_ij); alpha = exp2(m - m_new) (0 while m is -inf)
+//   p_ij = fl32(exp2(x_ij - m_new)) (double exp2, rounded once)
+//   l = alpha l + sum_j p_ij         (reading: the denominator sums the fp32 p
+//                                     before quantisation; flag: sum of p~)
+//   p~ = NVFP4(p) per 16 keys with the fixed tensor scale 2688 (p <= 1)
+//   O = alpha O + sum_j p~_ij v~_j   (exact tile product, accumulated in double)
+// out = bf16(fl32(O * fl32(d_P d_V) / l)), d_P = fl32(1 / 2688).
+void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float c, int Bc,
+                 int causal, int flags, double* o_out, double* ml_out, uint16_t* bf_out) {
+  const int N = T.N, D = T.D;
+  // quantise the query row
+  const uint16_t* qrow = T.q + (((int64_t)b * T.H + h) * N + i) * D;
+  std::vector<uint8_t> qc(D / 2), qs(D / 16);
+  quantize_rows(qrow, 1, D, T.sq, qc.data(), qs.data(), 1);
+  std::vector<double> qd(D);
+  for (int d = 0; d < D; ++d) {
+    uint8_t byte = qc[d / 2];
+    qd[d] = deq((d & 1) ? (byte >> 4) : (byte & 15), qs[d / 16]);
+  }
+  float sP, dP;
+  tensor_scale(1.0f, &sP, &dP);  // P: a-priori amax 1, so s_enc = 2688
+  std::vector<double> O(D, 0.0);
+  std::vector<float> x(Bc), p(Bc);
+  std::vector<double> pq(Bc);
+  double m = -INFINITY, l = 0.0;
+  const int ntiles = (N + Bc - 1) / Bc;
+  for (int t = 0; t < ntiles; ++t) {
+    const int j0 = t * Bc, j1 = std::min(j0 + Bc, N);
+    if (causal && j0 > i) break;  // fully masked tiles contribute nothing
+    float mt = -INFINITY;
+    for (int j = j0; j < j1; ++j) {
+      float xv = -INFINITY;
+      if (!(causal && j > i)) {
+        double s = 0.0;
+        const double* kr = &g.K[(int64_t)j * D];
+        for (int d = 0; d < D; ++d) s += qd[d] * kr[d];
+        float sf = (float)s;
+        xv = sf * c;
+      }
+      x[j - j0] = xv;
+      mt = std::max(mt, xv);
+    }
+    double m_new = std::max(m, (double)mt);
+    double alpha = (m == -INFINITY) ? 0.0 : std::exp2(m - m_new);
+    for (int jj = 0; jj < Bc; ++jj) {
+      int j = j0 + jj;
+      p[jj] = (j < j1 && x[jj] != -INFINITY) ? (float)std::exp2((double)x[jj] - m_new) : 0.0f;
+    }
+    // P quantisation, blocks of 16 keys from the tile start
+    for (int b0 = 0; b0 < Bc; b0 += 16) {
+      int n = std::min(16, Bc - b0);
+      uint8_t codes[16], e;
+      quantize_block(&p[b0], n, sP, codes, &e);
+      for (int u = 0; u < n; ++u) pq[b0 + u] = deq(codes[u], e);
+    }
+    double lt = 0.0;
+    if (flags & FLAG_QP_DENOMINATOR)
+      for (int jj = 0; jj < Bc; ++jj) lt += pq[jj] * (double)dP;
+    else
+      for (int jj = 0; jj < Bc; ++jj) lt += (double)p[jj];
+    l = alpha * l + lt;
+    for (int d = 0; d < D; ++d) {
+      double acc = 0.0;
+      for (int j = j0; j < j1; ++j) acc += pq[j - j0] * g.V[(int64_t)j * D + d];
+      O[d] = alpha * O[d] + acc;
+    }
+    m = m_new;
+  }
+  const float fpv = dP * T.dv;
+  for (int d = 0; d < D; ++d) {
+    double y = O[d] * (double)fpv / l;
+    if (o_out) o_out[d] = y;
+    if (bf_out) bf_out[d] = f32_to_bf16_rne((float)y);
+  }
+  if (ml_out) {
+    ml_out[0] = m;
+    ml_out[1] = l;
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+uint8_t ora_e2m1_encode(float y) { return e2m1_encode(y); }
+float ora_e2m1_decode(uint8_t c) { return e2m1_decode(c); }
+uint8_t ora_e4m3_encode(float y) { return e4m3_encode(y); }
+float ora_e4m3_decode(uint8_t c) { return e4m3_decode(c); }
+
+// Codes of the fp32 bit patterns start .. start+count-1, one byte each; NaN
+// inputs (outside the contract) give the marker 0xFF.
+void ora_e2m1_encode_range(uint32_t start, int64_t count, uint8_t* out, int nthreads) {
+  const int64_t chunk = 1 << 16;
+  parallel_for((count + chunk - 1) / chunk, nthreads, [&](int64_t c) {
+    int64_t hi = std::min(count, (c + 1) * chunk);
+    for (int64_t i = c * chunk; i < hi; ++i) {
+      uint32_t u = start + (uint32_t)i;
+      float f;
+      std::memcpy(&f, &u, 4);
+      out[i] = std::isnan(f) ? 0xFF : e2m1_encode(f);
+    }
+  });
+}
+
+void ora_e4m3_encode_range(uint32_t start, int64_t count, uint8_t* out, int nthreads) {
+  e4m3_encode(0.0f);  // build the magnitude table before the threads start
+  const int64_t chunk = 1 << 16;
+  parallel_for((count + chunk - 1) / chunk, nthreads, [&](int64_t c) {
+    int64_t hi = std::min(count, (c + 1) * chunk);
+    for (int64_t i = c * chunk; i < hi; ++i) {
+      uint32_t u = start + (uint32_t)i;
+      float f;
+      std::memcpy(&f, &u, 4);
+      out[i] = std::isnan(f) ? 0xFF : e4m3_encode(f);
+    }
+  });
+}
+
+float ora_amax_bf16(const uint16_t* x, int64_t n) { return amax_bf16(x, n); }
+
+void ora_tensor_scale(float amax, float* s_enc, float* d) { tensor_scale(amax, s_enc, d); }
+
+// One block of n <= 16 fp32 values: n codes (one per byte) and the scale byte.
+void ora_quantize_block(const float* x, int n, float s_enc, uint8_t* codes, uint8_t* scale) {
+  quantize_block(x, n, s_enc, codes, scale);
+}
+
+void ora_quantize_rows(const uint16_t* x, int64_t rows, int cols, float s_enc, uint8_t* codes,
+                       uint8_t* scales, int nthreads) {
+  e4m3_encode(0.0f);
+  quantize_rows(x, rows, cols, s_enc, codes, scales, nthreads);
+}
+
+void ora_quantize_tokens_T(const uint16_t* x, int N, int D, float s_enc, uint8_t* codes,
+                           uint8_t* scales, int npad) {
+  quantize_tokens_T(x, N, D, s_enc, codes, scales, npad);
+}
+
+// Unscaled scores of one head: S[i][j] = fl32(exact q~_i . k~_j), contraction
+// units (before d_Q d_K), no mask. S is [N][N].
+int ora_scores_head(const uint16_t* q, const uint16_t* k, int B, int H, int Hkv, int N, int D,
+                    int b, int h, float* S, int nthreads) {
+  if (B <= 0 || H <= 0 || Hkv <= 0 || H % Hkv || N <= 0 || D % 16 || b >= B || h >= H) return -1;
+  e4m3_encode(0.0f);
+  Tensors T{q, k, k, B, H, Hkv, N, D, 0, 0, 0, 0, 0, 0};
+  tensor_scale(amax_bf16(q, (int64_t)B * H * N * D), &T.sq, &T.dq);
+  tensor_scale(amax_bf16(k, (int64_t)B * Hkv * N * D), &T.sk, &T.dk);
+  const int hk = h / (H / Hkv);
+  std::vector<uint8_t> qc((size_t)N * D / 2), qs((size_t)N * D / 16), kc(qc.size()), ks(qs.size());
+  quantize_rows(q + ((int64_t)b * H + h) * N * D, N, D, T.sq, qc.data(), qs.data(), nthreads);
+  quantize_rows(k + ((int64_t)b * Hkv + hk) * N * D, N, D, T.sk, kc.data(), ks.data(), nthreads);
+  auto val = [&](const std::vector<uint8_t>& c, const std::vector<uint8_t>& s, int64_t n, int d) {
+    uint8_t byte = c[n * (D / 2) + d / 2];
+    return deq((d & 1) ? (byte >> 4) : (byte & 15), s[n * (D / 16) + d / 16]);
+  };
+  parallel_for(N, nthreads, [&](int64_t i) {
+    for (int j = 0; j < N; ++j) {
+      double s = 0.0;
+      for (int d = 0; d < D; ++d) s += val(qc, qs, i, d) * val(kc, ks, j, d);
+      S[i * N + j] = (float)s;
+    }
+  });
+  return 0;
+}
+
+// The tiled NVFP4 attention forward.
+//   q [B][H][N][D], k and v [B][Hkv][N][D], bf16 bit patterns.
+//   rows: nrows (b, h, i) triples to compute, or NULL for every row.
+//   out_bf16 / out_f64: [nrows][D] (or [B][H][N][D] when rows is NULL); either
+//   may be NULL. out_ml: [nrows][2] final (m, l), may be NULL.
+//   Bc: key tile (128 on the path); flags: 1 = denominator from p~.
+// Returns 0, or -1 on bad arguments.
+int ora_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H, int Hkv,
+                 int N, int D, int causal, float softmax_scale, int Bc, int flags,
+                 const int64_t* rows, int64_t nrows, uint16_t* out_bf16, double* out_f64,
+                 double* out_ml, int nthreads) {
+  if (B <= 0 || H <= 0 || Hkv <= 0 || H % Hkv || N <= 0 || D <= 0 || D % 16 || Bc <= 0 ||
+      Bc % 16)
+    return -1;
+  e4m3_encode(0.0f);
+  Tensors T{q, k, v, B, H, Hkv, N, D, 0, 0, 0, 0, 0, 0};
+  tensor_scale(amax_bf16(q, (int64_t)B * H * N * D), &T.sq, &T.dq);
+  tensor_scale(amax_bf16(k, (int64_t)B * Hkv * N * D), &T.sk, &T.dk);
+  tensor_scale(amax_bf16(v, (int64_t)B * Hkv * N * D), &T.sv, &T.dv);
+  if (!(softmax_scale > 0.0f)) softmax_scale = 1.0f / std::sqrt((float)D);
+  float c = T.dq * T.dk;
+  c = c * softmax_scale;
+  c = c * kLog2e;
+
+  std::vector<int64_t> all;
+  if (!rows) {
+    nrows = (int64_t)B * H * N;
+    all.resize((size_t)nrows * 3);
+    for (int64_t r = 0; r < nrows; ++r) {
+      all[r * 3 + 0] = r / ((int64_t)H * N);
+      all[r * 3 + 1] = (r / N) % H;
+      all[r * 3 + 2] = r % N;
+    }
+    rows = all.data();
+  }
+  for (int64_t r = 0; r < nrows; ++r)
+    if (rows[r * 3] < 0 || rows[r * 3] >= B || rows[r * 3 + 1] < 0 || rows[r * 3 + 1] >= H ||
+        rows[r * 3 + 2] < 0 || rows[r * 3 + 2] >= N)
+      return -1;
+  const int G = H / Hkv;
+  for (int b = 0; b < B; ++b)
+    for (int hk = 0; hk < Hkv; ++hk) {
+      std::vector<int64_t> mine;
+      for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r * 3] == b && rows[r * 3 + 1] / G == hk) mine.push_back(r);
+      if (mine.empty()) continue;
+      KVGroup g = make_group(T, b, hk);
+      parallel_for((int64_t)mine.size(), nthreads, [&](int64_t u) {
+        int64_t r = mine[u];
+        row_forward(T, g, b, (int)rows[r * 3 + 1], (int)rows[r * 3 + 2], c, Bc, causal, flags,
+                    out_f64 ? out_f64 + r * D : nullptr, out_ml ? out_ml + r * 2 : nullptr,
+                    out_bf16 ? out_bf16 + r * D : nullptr);
+      });
+    }
+  return 0;
+}
+
+}  // extern "C"
