@@ -1,0 +1,306 @@
+"""Benchmark of the NVFP4 FlashAttention forward on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step is one pass of the whole path over one batch of the workload: amax
+and NVFP4 quantisation of Q, K and V, then the fused attention forward (one
+fp4_attn_fwd call). value = algorithmic FLOPs (4*B*H*N^2*D, halved when causal)
+of all ranks / the slowest rank's device time. Under torchrun every rank runs
+its own replica of the workload (the path needs no exchange between ranks).
+Inputs are seeded synthetic tensors; the default workload is the video-DiT
+latent grid (B1 H24 N32760 D128).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FP4 attention fwd TFLOPS at 1 B200 and % of dense FP4 tensor peak"
+FP4_DATASHEET_TFLOPS = 9000.0  # NVIDIA B200 dense FP4, no sparsity
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="video_dit")
+    ap.add_argument("--impl", default="fp4attn", choices=["fp4attn", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=0,
+                    help="query rows in the oracle's timed sample (0: one per head)")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            m = json.load(f)
+        return m, "MEASURED_PEAKS.json"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, \
+            "fallback"
+
+
+class Clocks:
+    """nvidia-smi samples (every 200 ms) while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.proc = index, None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        mhz, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                maxes.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(maxes),
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+def flush_l2(buf):
+    buf.add_(1)
+
+
+def cpu_baseline(wl, q, k, v, rows_total: int):
+    """The oracle, as it stands, on a bounded sample: `rows_total` seeded query
+    rows spread over the heads (plus the quantisation of K and V it needs)."""
+    import numpy as np
+    import oracle
+    import synth
+    oracle.build()
+    per_head = max(1, rows_total // (wl.B * wl.H))
+    rows = synth.sample_rows(wl, per_head)
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    oracle.attn_fwd(q, k, v, causal=wl.causal, rows=rows, threads=threads)
+    dt = time.perf_counter() - t0
+    keys = (rows[:, 2] + 1).astype(np.float64) if wl.causal else np.full(len(rows), wl.N, np.float64)
+    flops = float((4.0 * wl.D * keys).sum())
+    return {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+            "sample": f"{len(rows)} seeded query rows ({per_head} per head) of {wl.name}, "
+                      f"plus quantising all of K and V; {dt:.1f} s",
+            "seconds": dt}
+
+
+def run_reference(args, wl):
+    """The reference arm: the CPU oracle on a bounded sample per step."""
+    import numpy as np
+    import synth
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    synth.build()
+    q, k, v = synth.workload_inputs(wl)
+    rows_total = args.cpu_rows or wl.B * wl.H
+    times, res = [], None
+    for i in range(args.warmup + args.steps):
+        res = cpu_baseline(wl, q, k, v, rows_total)
+        if i >= args.warmup:
+            times.append(res["seconds"])
+    flops = res["value"] * res["seconds"] * 1e12
+    val = flops / statistics.mean(times) / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOPS",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": statistics.mean(times) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64/f32 (CPU oracle)",
+            "data": "synthetic", "config": {**wl.describe(), "sample": res["sample"]},
+            "cpu_baseline": {k2: res[k2] for k2 in ("kind", "cores", "sample")} | {"value": val},
+            "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    import synth
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+        return
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import bit_attention_transformers_b200 as fa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    fa.lib()
+
+    synth.build()
+    shape_q = (wl.B, wl.H, wl.N, wl.D)
+    shape_kv = (wl.B, wl.Hkv, wl.N, wl.D)
+    hq = torch.empty(shape_q, dtype=torch.bfloat16, pin_memory=True)
+    hk = torch.empty(shape_kv, dtype=torch.bfloat16, pin_memory=True)
+    hv = torch.empty(shape_kv, dtype=torch.bfloat16, pin_memory=True)
+    synth.workload_inputs(wl, outs=[t.view(torch.int16).numpy().view(np.uint16) for t in (hq, hk, hv)])
+    q, k, v = hq.to(dev), hk.to(dev), hv.to(dev)
+    out = torch.empty_like(q)
+    ws = fa.workspace(wl.B, wl.H, wl.Hkv, wl.N, wl.D, dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    flops = wl.flops
+
+    def step():
+        fa.fp4_attn_fwd(q, k, v, causal=wl.causal, out=out, ws=ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def timed(fn, n):
+        """Device time (ms) of each of n calls of fn, L2 flushed before each."""
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
+        for s, e in evs:
+            flush_l2(flush)
+            s.record(stream)
+            fn()
+            e.record(stream)
+        torch.cuda.synchronize()
+        return [s.elapsed_time(e) for s, e in evs]
+
+    for _ in range(args.warmup):
+        step()
+    fa.fp4_status()
+    barrier()
+    with Clocks(local) as clk:
+        step_ms = timed(step, args.steps)
+    barrier()
+    fa.fp4_status()
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+
+    # the fused attention kernel alone (same inputs, already quantised)
+    qq = fa.fp4_quantize(q, fa.FP4_BLOCK_ALONG_D)
+    kq = fa.fp4_quantize(k, fa.FP4_BLOCK_ALONG_D)
+    vq = fa.fp4_quantize(v, fa.FP4_BLOCK_ALONG_N_T)
+
+    def kernel():
+        fa.fp4_attn_fwd_quantized(qq, kq, vq, wl.B, wl.H, wl.Hkv, causal=wl.causal, out=out)
+
+    for _ in range(args.warmup):
+        kernel()
+    k_ms = statistics.mean(timed(kernel, args.steps))
+    fa.fp4_status()
+
+    # end to end: pinned host inputs -> device -> fp4_attn_fwd -> host output
+    hout = torch.empty(shape_q, dtype=torch.bfloat16, pin_memory=True)
+
+    def e2e():
+        fa.fp4_attn_fwd_host(hq, hk, hv, causal=wl.causal, out=hout, device=dev)
+
+    for _ in range(max(1, args.warmup // 2)):
+        e2e()
+    barrier()
+    e_ms = timed(e2e, max(1, args.steps // 2))
+    barrier()
+    e_total = sum(e_ms)
+    if world > 1:
+        t = torch.tensor([e_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_total = float(t.item())
+    e2e_value = world * flops / (e_total / len(e_ms) * 1e-3) / 1e12
+    fa.fp4_status()
+
+    peaks, src = measured_peaks()
+    fp4_peak = 4.0 * peaks["bf16_tflops"]  # dense FP4 = 4x dense bf16 (nominal 9 vs 2.25 PF)
+    achieved = flops / (k_ms * 1e-3) / 1e12
+    traffic = None
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
+        "data": "synthetic",
+        "config": {**wl.describe(), "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (bf16 Q/K/V of "
+                         f"{(hq.numel() + 2 * hk.numel()) * 2 / 1e6:.0f} MB); "
+                         "L2 also flushed (252 MB write) before every timed step"},
+        "pct_of_fp4_peak": {"value": 100.0 * value / world / FP4_DATASHEET_TFLOPS,
+                            "peak_tflops": FP4_DATASHEET_TFLOPS,
+                            "peak": "9 PFLOP/s dense FP4, NVIDIA B200 datasheet"},
+        "attn_kernel_ms": k_ms,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak,
+                     "unit": "TFLOP/s", "frac": achieved / fp4_peak, "traffic": traffic,
+                     "peak_source": f"4 x measured dense bf16 ({peaks['bf16_tflops']} TFLOP/s, "
+                                    f"{src}); fraction of measured"},
+        "e2e": {"value": e2e_value, "unit": "TFLOPS",
+                "h2d_bytes_per_step": (hq.numel() + hk.numel() + hv.numel()) * 2,
+                "d2h_bytes_per_step": hout.numel() * 2},
+        "gpu_launches": 5 * args.steps,
+    }
+    c = clk.summary()
+    if c:
+        line["clocks"] = c
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = {k2: v2 for k2, v2 in
+                                cpu_baseline(wl, hq.view(torch.int16).numpy().view(np.uint16),
+                                             hk.view(torch.int16).numpy().view(np.uint16),
+                                             hv.view(torch.int16).numpy().view(np.uint16),
+                                             args.cpu_rows or wl.B * wl.H).items()
+                                if k2 != "seconds"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,239 @@
+"""NVFP4 (4-bit) FlashAttention forward for B200: Python binding of libfp4attn.
+
+A thin ctypes layer over the C ABI in include/fp4attn.h: it marshals torch
+tensors (device memory and streams only) into the library's calls and raises
+on error. Every step of the computation runs in the library's CUDA kernels;
+there is no fallback path. The names are the C ABI's.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_ROOT = os.path.dirname(_HERE)
+_SRC_DIR = os.path.join(_HERE, "csrc")
+_LIB_PATH = os.path.join(_HERE, "libfp4attn.so")
+_HEADER = os.path.join(_ROOT, "include", "fp4attn.h")
+
+FP4_OK = 0
+FP4_ERR_INVALID_ARG = 1
+FP4_ERR_UNSUPPORTED = 2
+FP4_ERR_WORKSPACE = 3
+FP4_ERR_CUDA = 4
+FP4_ERR_TIMEOUT = 5
+FP4_BLOCK_ALONG_D = 0
+FP4_BLOCK_ALONG_N_T = 1
+
+# Every symbol include/fp4attn.h declares.
+EXPORTS = ("fp4_codes_bytes", "fp4_scales_bytes", "fp4_attn_workspace_bytes", "fp4_quantize",
+           "fp4_attn_fwd", "fp4_attn_fwd_quantized", "fp4_status", "fp4_last_error",
+           "fp4_probe_cvt")
+
+NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
+              "-Xcompiler", "-fPIC", "-shared"]
+
+
+class Fp4Error(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"fp4attn error {code}: {msg}")
+        self.code = code
+
+
+def _sources():
+    return [os.path.join(_SRC_DIR, f) for f in sorted(os.listdir(_SRC_DIR))
+            if f.endswith((".cu", ".cuh"))] + [_HEADER]
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile libfp4attn.so in-tree for sm_100a (nvcc; no GPU needed)."""
+    newest = max(os.path.getmtime(s) for s in _sources())
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < newest:
+        nvcc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "bin", "nvcc")
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = [nvcc, *NVCC_FLAGS, "-o", tmp, os.path.join(_SRC_DIR, "fp4attn.cu")]
+        if verbose:
+            cmd.insert(1, "-Xptxas=-v")
+        subprocess.check_call(cmd)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+_lib = None
+
+
+def lib():
+    """The loaded library. Raises if it has not been built: there is no fallback."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"{_LIB_PATH} is missing: run bit_attention_transformers_b200.build()")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, i32, i64, u32, f32, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                      ctypes.c_uint32, ctypes.c_float, ctypes.c_size_t)
+        L.fp4_codes_bytes.argtypes = [i32, i32, i32, i32]
+        L.fp4_codes_bytes.restype = sz
+        L.fp4_scales_bytes.argtypes = [i32, i32, i32, i32]
+        L.fp4_scales_bytes.restype = sz
+        L.fp4_attn_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+        L.fp4_attn_workspace_bytes.restype = sz
+        L.fp4_quantize.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp]
+        L.fp4_quantize.restype = i32
+        L.fp4_attn_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, sz]
+        L.fp4_attn_fwd.restype = i32
+        L.fp4_attn_fwd_quantized.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
+        L.fp4_attn_fwd_quantized.restype = i32
+        L.fp4_status.argtypes = [vp]
+        L.fp4_status.restype = i32
+        L.fp4_last_error.argtypes = []
+        L.fp4_last_error.restype = ctypes.c_char_p
+        L.fp4_probe_cvt.argtypes = [u32, i64, i32, vp, vp]
+        L.fp4_probe_cvt.restype = i32
+        _lib = L
+    return _lib
+
+
+class _Tensor(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("amax", ctypes.c_void_p)]
+
+
+def _check(rc: int):
+    if rc != FP4_OK:
+        raise Fp4Error(rc, lib().fp4_last_error().decode())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr())
+
+
+# ------------------------------------------------------------------ sizes ----
+def fp4_codes_bytes(G: int, N: int, D: int, axis: int) -> int:
+    return lib().fp4_codes_bytes(G, N, D, axis)
+
+
+def fp4_scales_bytes(G: int, N: int, D: int, axis: int) -> int:
+    return lib().fp4_scales_bytes(G, N, D, axis)
+
+
+def fp4_attn_workspace_bytes(B: int, H: int, Hkv: int, N: int, D: int) -> int:
+    return lib().fp4_attn_workspace_bytes(B, H, Hkv, N, D)
+
+
+# --------------------------------------------------------------- quantise ----
+@dataclass
+class Fp4Tensor:
+    """A quantised tensor on the device (layouts in include/fp4attn.h)."""
+    codes: "object"
+    scales: "object"
+    amax: "object"
+    G: int
+    N: int
+    D: int
+    axis: int
+
+
+def fp4_quantize(x, axis: int = FP4_BLOCK_ALONG_D, stream=None) -> Fp4Tensor:
+    """x: bf16 CUDA tensor [..., N, D] (the leading dims form the groups G)."""
+    import torch
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous()
+    N, D = x.shape[-2], x.shape[-1]
+    G = x.numel() // (N * D)
+    codes = torch.empty(fp4_codes_bytes(G, N, D, axis), dtype=torch.uint8, device=x.device)
+    scales = torch.empty(fp4_scales_bytes(G, N, D, axis), dtype=torch.uint8, device=x.device)
+    amax = torch.empty(4, dtype=torch.float32, device=x.device)
+    _check(lib().fp4_quantize(_ptr(x), G, N, D, axis, _ptr(codes), _ptr(scales), _ptr(amax),
+                              _stream(stream)))
+    return Fp4Tensor(codes, scales, amax, G, N, D, axis)
+
+
+# -------------------------------------------------------------- attention ----
+_ws_cache: dict = {}
+
+
+def workspace(B, H, Hkv, N, D, device):
+    """A cached device workspace large enough for fp4_attn_fwd on this shape."""
+    import torch
+    need = fp4_attn_workspace_bytes(B, H, Hkv, N, D)
+    key = (str(device),)
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(need, dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def fp4_attn_fwd(q, k, v, causal: bool = False, softmax_scale: float | None = None, out=None,
+                 stream=None, ws=None):
+    """NVFP4 attention forward. q [B,H,N,D], k/v [B,Hkv,N,D]: contiguous bf16
+    CUDA tensors. Returns out [B,H,N,D] bf16."""
+    import torch
+    B, H, N, D = q.shape
+    Hkv = k.shape[1]
+    for t in (q, k, v):
+        assert t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()
+    assert k.shape == (B, Hkv, N, D) and v.shape == (B, Hkv, N, D)
+    if out is None:
+        out = torch.empty_like(q)
+    if ws is None:
+        ws = workspace(B, H, Hkv, N, D, q.device)
+    _check(lib().fp4_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, Hkv, N, D,
+                              int(bool(causal)), float(softmax_scale or 0.0), _stream(stream),
+                              _ptr(ws), ws.numel()))
+    return out
+
+
+def fp4_attn_fwd_quantized(qq: Fp4Tensor, kq: Fp4Tensor, vq: Fp4Tensor, B: int, H: int,
+                           Hkv: int, causal: bool = False, softmax_scale: float | None = None,
+                           out=None, stream=None):
+    """The fused forward alone on tensors fp4_quantize() produced."""
+    import torch
+    N, D = qq.N, qq.D
+    if out is None:
+        out = torch.empty((B, H, N, D), dtype=torch.bfloat16, device=qq.codes.device)
+    ts = [_Tensor(t.codes.data_ptr(), t.scales.data_ptr(), t.amax.data_ptr()) for t in (qq, kq, vq)]
+    _check(lib().fp4_attn_fwd_quantized(ctypes.byref(ts[0]), ctypes.byref(ts[1]),
+                                        ctypes.byref(ts[2]), _ptr(out), B, H, Hkv, N, D,
+                                        int(bool(causal)), float(softmax_scale or 0.0),
+                                        _stream(stream)))
+    return out
+
+
+def fp4_attn_fwd_host(q, k, v, causal: bool = False, softmax_scale: float | None = None,
+                      out=None, device="cuda", stream=None):
+    """End-to-end call on host buffers: copies q, k, v (pinned CPU bf16
+    tensors) to the device, runs fp4_attn_fwd, copies the output back into
+    `out` (a pinned CPU tensor) and returns it once the stream has finished."""
+    import torch
+    dq = q.to(device, non_blocking=True)
+    dk = k.to(device, non_blocking=True)
+    dv = v.to(device, non_blocking=True)
+    o = fp4_attn_fwd(dq, dk, dv, causal, softmax_scale, stream=stream)
+    if out is None:
+        out = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    out.copy_(o, non_blocking=True)
+    torch.cuda.current_stream().synchronize()
+    return out
+
+
+def fp4_status(stream=None):
+    """Synchronise and raise if a kernel reported an expired wait."""
+    _check(lib().fp4_status(_stream(stream)))
+
+
+def fp4_probe_cvt(start: int, count: int, kind: int, out=None, stream=None):
+    import torch
+    if out is None:
+        out = torch.empty(count, dtype=torch.uint8, device="cuda")
+    _check(lib().fp4_probe_cvt(start, count, kind, _ptr(out), _stream(stream)))
+    return out

@@ -1,0 +1,364 @@
+// Host side of the fp4attn C ABI (include/fp4attn.h): argument validation,
+// workspace layout, TMA descriptors and kernel launches. No device memory is
+// allocated here; every buffer belongs to the caller.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/fp4attn.h"
+#include "attn_fwd.cuh"
+#include "quantize.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+fp4_status_t fail(fp4_status_t s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+#define FP4_CUDA(call)                                                                  \
+  do {                                                                                  \
+    cudaError_t e_ = (call);                                                            \
+    if (e_ != cudaSuccess)                                                              \
+      return fail(FP4_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_));        \
+  } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+bool g_attr_done[kMaxDevices];
+int g_num_sms[kMaxDevices];
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// sm_100 check, per-device one-time kernel attributes, SM count.
+fp4_status_t device_setup(int* dev_out, int* sms_out) {
+  int dev;
+  FP4_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(FP4_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_attr_done[dev]) {
+    int major = 0, minor = 0, sms = 0;
+    FP4_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+    FP4_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+    FP4_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    if (major != 10 || minor != 0)
+      return fail(FP4_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
+                  dev, major, minor);
+    FP4_CUDA(cudaFuncSetAttribute(fp4::attn_fwd_kernel<128, false>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  fp4::AttnSmem<128>::kBytes));
+    FP4_CUDA(cudaFuncSetAttribute(fp4::attn_fwd_kernel<128, true>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  fp4::AttnSmem<128>::kBytes));
+    FP4_CUDA(cudaFuncSetAttribute(fp4::attn_fwd_kernel<64, false>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  fp4::AttnSmem<64>::kBytes));
+    FP4_CUDA(cudaFuncSetAttribute(fp4::attn_fwd_kernel<64, true>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  fp4::AttnSmem<64>::kBytes));
+    if (!g_encode) {
+      cudaDriverEntryPointQueryResult q;
+      void* fn = nullptr;
+      FP4_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+      if (q != cudaDriverEntryPointSuccess || !fn)
+        return fail(FP4_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    g_num_sms[dev] = sms;
+    g_attr_done[dev] = true;
+  }
+  *dev_out = dev;
+  *sms_out = g_num_sms[dev];
+  return FP4_OK;
+}
+
+// 2D uint8 tensor map: rows x inner bytes, box rows x box_inner bytes.
+fp4_status_t tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                     uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FP4_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return FP4_OK;
+}
+
+struct WsLayout {
+  size_t amax, qc, qs, kc, ks, vc, vs, total;
+};
+
+size_t codes_bytes(int64_t G, int64_t N, int64_t D) { return (size_t)(G * round_up(N, 128) * D / 2); }
+size_t scales_bytes(int64_t G, int64_t N, int64_t D, fp4_axis_t axis) {
+  const int64_t Npad = round_up(N, 128);
+  return axis == FP4_BLOCK_ALONG_D ? (size_t)(G * Npad * D / 16) : (size_t)(G * (Npad / 64) * 512);
+}
+
+WsLayout ws_layout(int B, int H, int Hkv, int N, int D) {
+  WsLayout w;
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    size_t o = off;
+    off += (size_t)round_up((int64_t)n, 1024);
+    return o;
+  };
+  const int64_t Gq = (int64_t)B * H, Gk = (int64_t)B * Hkv;
+  w.amax = take(256);
+  w.qc = take(codes_bytes(Gq, N, D));
+  w.qs = take(scales_bytes(Gq, N, D, FP4_BLOCK_ALONG_D));
+  w.kc = take(codes_bytes(Gk, N, D));
+  w.ks = take(scales_bytes(Gk, N, D, FP4_BLOCK_ALONG_D));
+  w.vc = take(codes_bytes(Gk, N, D));
+  w.vs = take(scales_bytes(Gk, N, D, FP4_BLOCK_ALONG_N_T));
+  w.total = off;
+  return w;
+}
+
+fp4_status_t check_shape(int B, int H, int Hkv, int N, int D) {
+  if (B < 1 || H < 1 || Hkv < 1 || N < 1)
+    return fail(FP4_ERR_INVALID_ARG, "B, H, Hkv and N must be >= 1 (got %d, %d, %d, %d)", B, H,
+                Hkv, N);
+  if (H % Hkv) return fail(FP4_ERR_INVALID_ARG, "H (%d) must be a multiple of Hkv (%d)", H, Hkv);
+  if (D != 64 && D != 128) return fail(FP4_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", D);
+  if (B > 65535 || H > 65535) return fail(FP4_ERR_INVALID_ARG, "B and H must be <= 65535");
+  const int64_t Npad = round_up(N, 128);
+  if ((int64_t)B * H * Npad > INT32_MAX || (int64_t)B * Hkv * D > INT32_MAX ||
+      Npad / 128 > INT32_MAX)
+    return fail(FP4_ERR_INVALID_ARG, "problem too large");
+  return FP4_OK;
+}
+
+fp4_status_t launch_amax(const void* x0, int64_t n0, const void* x1, int64_t n1, const void* x2,
+                         int64_t n2, float* a0, float* a1, float* a2, int sms,
+                         cudaStream_t stream) {
+  const int tensors = x2 ? 3 : (x1 ? 2 : 1);
+  FP4_CUDA(cudaMemsetAsync(a0, 0, sizeof(float), stream));
+  if (x1) FP4_CUDA(cudaMemsetAsync(a1, 0, sizeof(float), stream));
+  if (x2) FP4_CUDA(cudaMemsetAsync(a2, 0, sizeof(float), stream));
+  dim3 grid(sms * 4, tensors);
+  fp4::amax3_kernel<<<grid, 256, 0, stream>>>(
+      static_cast<const uint4*>(x0), n0 / 8, static_cast<const uint4*>(x1), n1 / 8,
+      static_cast<const uint4*>(x2), n2 / 8, reinterpret_cast<unsigned*>(a0),
+      reinterpret_cast<unsigned*>(a1), reinterpret_cast<unsigned*>(a2));
+  FP4_CUDA(cudaGetLastError());
+  return FP4_OK;
+}
+
+fp4_status_t launch_quant(const void* x, int64_t G, int N, int D, fp4_axis_t axis, uint8_t* codes,
+                          uint8_t* scales, const float* amax, int sms, cudaStream_t stream) {
+  const int64_t Npad = round_up(N, 128);
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  if (axis == FP4_BLOCK_ALONG_D) {
+    const int64_t total = G * Npad * (D / 16);
+    const int64_t blocks = std::min<int64_t>((total + 255) / 256, (int64_t)sms * 16);
+    if (D == 128)
+      fp4::quant_rows_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(xb, (int)G, N, (int)Npad,
+                                                                       amax, codes, scales);
+    else
+      fp4::quant_rows_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(xb, (int)G, N, (int)Npad,
+                                                                      amax, codes, scales);
+  } else {
+    const int64_t blocks = G * (Npad / 128);
+    if (blocks > INT32_MAX) return fail(FP4_ERR_INVALID_ARG, "problem too large");
+    if (D == 128)
+      fp4::quant_tokens_T_kernel<128><<<(unsigned)blocks, 128, 0, stream>>>(
+          xb, (int)G, N, (int)Npad, amax, codes, scales);
+    else
+      fp4::quant_tokens_T_kernel<64><<<(unsigned)blocks, 128, 0, stream>>>(
+          xb, (int)G, N, (int)Npad, amax, codes, scales);
+  }
+  FP4_CUDA(cudaGetLastError());
+  return FP4_OK;
+}
+
+fp4_status_t launch_attn(const uint8_t* qc, const uint8_t* qs, const float* qa, const uint8_t* kc,
+                         const uint8_t* ks, const float* ka, const uint8_t* vc, const uint8_t* vs,
+                         const float* va, void* out, int B, int H, int Hkv, int N, int D,
+                         int causal, float softmax_scale, cudaStream_t stream) {
+  const int64_t Npad = round_up(N, 128);
+  const int64_t Gq = (int64_t)B * H, Gk = (int64_t)B * Hkv;
+  const CUtensorMapSwizzle swQK =
+      D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUtensorMap tq, tk, tv;
+  fp4_status_t s;
+  if ((s = tmap_2d(&tq, qc, D / 2, Gq * Npad, D / 2, 128, swQK)) != FP4_OK) return s;
+  if ((s = tmap_2d(&tk, kc, D / 2, Gk * Npad, D / 2, 128, swQK)) != FP4_OK) return s;
+  if ((s = tmap_2d(&tv, vc, Npad / 2, Gk * D, 64, D, CU_TENSOR_MAP_SWIZZLE_64B)) != FP4_OK)
+    return s;
+  fp4::AttnParams p;
+  p.q_sf = qs;
+  p.k_sf = ks;
+  p.v_sf = vs;
+  p.amax_q = qa;
+  p.amax_k = ka;
+  p.amax_v = va;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.H = H;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.Npad = (int)Npad;
+  p.ntq = (int)(Npad / 128);
+  p.softmax_scale = (softmax_scale > 0.0f && std::isfinite(softmax_scale))
+                        ? softmax_scale
+                        : 1.0f / std::sqrt((float)D);
+  dim3 grid(p.ntq, H, B);
+  const int smem = D == 128 ? fp4::AttnSmem<128>::kBytes : fp4::AttnSmem<64>::kBytes;
+  if (D == 128) {
+    if (causal)
+      fp4::attn_fwd_kernel<128, true><<<grid, fp4::kAttnThreads, smem, stream>>>(tq, tk, tv, p);
+    else
+      fp4::attn_fwd_kernel<128, false><<<grid, fp4::kAttnThreads, smem, stream>>>(tq, tk, tv, p);
+  } else {
+    if (causal)
+      fp4::attn_fwd_kernel<64, true><<<grid, fp4::kAttnThreads, smem, stream>>>(tq, tk, tv, p);
+    else
+      fp4::attn_fwd_kernel<64, false><<<grid, fp4::kAttnThreads, smem, stream>>>(tq, tk, tv, p);
+  }
+  FP4_CUDA(cudaGetLastError());
+  return FP4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fp4_codes_bytes(int G, int N, int D, fp4_axis_t) {
+  if (G < 1 || N < 1 || D < 16) return 0;
+  return codes_bytes(G, N, D);
+}
+
+size_t fp4_scales_bytes(int G, int N, int D, fp4_axis_t axis) {
+  if (G < 1 || N < 1 || D < 16) return 0;
+  return scales_bytes(G, N, D, axis);
+}
+
+size_t fp4_attn_workspace_bytes(int B, int H, int Hkv, int N, int D) {
+  if (check_shape(B, H, Hkv, N, D) != FP4_OK) return 0;
+  return ws_layout(B, H, Hkv, N, D).total;
+}
+
+fp4_status_t fp4_quantize(const void* x, int G, int N, int D, fp4_axis_t axis, uint8_t* codes,
+                          uint8_t* scales, float* amax, void* stream) {
+  g_last_error.clear();
+  fp4_status_t s;
+  if ((s = check_shape(1, G, G, N, D)) != FP4_OK) return s;
+  if (axis != FP4_BLOCK_ALONG_D && axis != FP4_BLOCK_ALONG_N_T)
+    return fail(FP4_ERR_INVALID_ARG, "axis %d", (int)axis);
+  if (!x || !codes || !scales || !amax) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(amax))
+    return fail(FP4_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  int dev, sms;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t n = (int64_t)G * N * D;
+  if ((s = launch_amax(x, n, nullptr, 0, nullptr, 0, amax, nullptr, nullptr, sms, st)) != FP4_OK)
+    return s;
+  return launch_quant(x, G, N, D, axis, codes, scales, amax, sms, st);
+}
+
+fp4_status_t fp4_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int H,
+                          int Hkv, int N, int D, int causal, float softmax_scale, void* stream,
+                          void* workspace, size_t workspace_bytes) {
+  g_last_error.clear();
+  fp4_status_t s;
+  if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
+  if (!q || !k || !v || !out || !workspace) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace))
+    return fail(FP4_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const WsLayout w = ws_layout(B, H, Hkv, N, D);
+  if (workspace_bytes < w.total)
+    return fail(FP4_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, w.total);
+  int dev, sms;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* amax = reinterpret_cast<float*>(ws + w.amax);
+  const int64_t nq = (int64_t)B * H * N * D, nkv = (int64_t)B * Hkv * N * D;
+  if ((s = launch_amax(q, nq, k, nkv, v, nkv, amax, amax + 1, amax + 2, sms, st)) != FP4_OK)
+    return s;
+  if ((s = launch_quant(q, (int64_t)B * H, N, D, FP4_BLOCK_ALONG_D, ws + w.qc, ws + w.qs, amax,
+                        sms, st)) != FP4_OK)
+    return s;
+  if ((s = launch_quant(k, (int64_t)B * Hkv, N, D, FP4_BLOCK_ALONG_D, ws + w.kc, ws + w.ks,
+                        amax + 1, sms, st)) != FP4_OK)
+    return s;
+  if ((s = launch_quant(v, (int64_t)B * Hkv, N, D, FP4_BLOCK_ALONG_N_T, ws + w.vc, ws + w.vs,
+                        amax + 2, sms, st)) != FP4_OK)
+    return s;
+  return launch_attn(ws + w.qc, ws + w.qs, amax, ws + w.kc, ws + w.ks, amax + 1, ws + w.vc,
+                     ws + w.vs, amax + 2, out, B, H, Hkv, N, D, causal, softmax_scale, st);
+}
+
+fp4_status_t fp4_attn_fwd_quantized(const fp4_tensor_t* q, const fp4_tensor_t* k,
+                                    const fp4_tensor_t* v, void* out, int B, int H, int Hkv,
+                                    int N, int D, int causal, float softmax_scale, void* stream) {
+  g_last_error.clear();
+  fp4_status_t s;
+  if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
+  if (!q || !k || !v || !out) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  const fp4_tensor_t* t[3] = {q, k, v};
+  for (auto* x : t) {
+    if (!x->codes || !x->scales || !x->amax) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(x->codes) || !aligned16(x->scales) ||
+        (reinterpret_cast<uintptr_t>(x->amax) & 3u))
+      return fail(FP4_ERR_INVALID_ARG, "codes/scales must be 16-byte aligned");
+  }
+  if (!aligned16(out)) return fail(FP4_ERR_INVALID_ARG, "out must be 16-byte aligned");
+  int dev, sms;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  return launch_attn(q->codes, q->scales, q->amax, k->codes, k->scales, k->amax, v->codes,
+                     v->scales, v->amax, out, B, H, Hkv, N, D, causal, softmax_scale,
+                     static_cast<cudaStream_t>(stream));
+}
+
+fp4_status_t fp4_status(void* stream) {
+  FP4_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  FP4_CUDA(cudaGetLastError());
+  unsigned err = 0;
+  FP4_CUDA(cudaMemcpyFromSymbol(&err, fp4::g_fp4_err, sizeof(err)));
+  if (err) {
+    const unsigned zero = 0;
+    FP4_CUDA(cudaMemcpyToSymbol(fp4::g_fp4_err, &zero, sizeof(zero)));
+    return fail(FP4_ERR_TIMEOUT, "a kernel's bounded wait expired (device error word %u)", err);
+  }
+  return FP4_OK;
+}
+
+const char* fp4_last_error(void) { return g_last_error.c_str(); }
+
+fp4_status_t fp4_probe_cvt(uint32_t start, int64_t count, int kind, uint8_t* out, void* stream) {
+  g_last_error.clear();
+  if (count < 0 || (kind != 0 && kind != 1) || (count > 0 && !out))
+    return fail(FP4_ERR_INVALID_ARG, "bad probe arguments");
+  if ((int64_t)start + count > (int64_t)1 << 32)
+    return fail(FP4_ERR_INVALID_ARG, "range beyond 2^32");
+  int dev, sms;
+  fp4_status_t s;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  if (count == 0) return FP4_OK;
+  fp4::probe_cvt_kernel<<<sms * 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(start, count,
+                                                                                 kind, out);
+  FP4_CUDA(cudaGetLastError());
+  return FP4_OK;
+}
+
+}  // extern "C"

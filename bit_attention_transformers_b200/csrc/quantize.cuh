@@ -1,0 +1,220 @@
+// NVFP4 quantisation of Q, K and V on sm_100a (HBM-bound).
+//
+// Format and recipe: block-scaled E2M1 operands (NVFP4) [TetraJet-v2 abstract,
+// searcharxiv.com author page "Pengle Zhang"; EFQ-Softmax abstract, scholarbro.com
+// page "AVQ Attention: Adaptive Vector-Quantized Attention"]. The pages give no
+// recipe; this file implements the standard two-level NVFP4 reading:
+//   s_enc = 2688 / amax (1 when amax == 0, FLT_MAX when the quotient overflows)
+//   per 16-element block: e = E4M3(fl(fl(a_b / 6) * s_enc)),
+//                         r = fl(s_enc / dec(e)) (0 when dec(e) == 0),
+//                         code_i = E2M1(fl(x_i * r))
+// with one correctly rounded fp32 operation per step (no FMA contraction) and
+// the hardware round-to-nearest-even, saturating conversions.
+//
+// Layouts written (all per group g = one (batch, head)):
+//   codes along D  (Q, K): [g][Npad][D/2] bytes, rows >= N zero.
+//   codes along tokens (V): [g][D][Npad/2] bytes (V transposed), tokens >= N zero.
+//   scales: the tensor-core block-scale layout, 512-byte atoms. An atom holds
+//     the scales of 128 rows x 4 consecutive 16-blocks; row r (0..127) and
+//     block k (0..3) sit at byte (r % 32) * 16 + (r / 32) * 4 + k.
+//     Along D: atom (tile = n / 128, chunk = block / 4) at
+//       ((g * Npad/128 + tile) * D/64 + chunk) * 512.
+//     Along tokens: rows are the D channels (padded to 128 with zeros), atom
+//       chunk = token_block / 4 at (g * Npad/64 + chunk) * 512.
+#pragma once
+#include <cfloat>
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace fp4 {
+
+constexpr float kTensorRange = 2688.0f;  // 6 * 448: largest E2M1 times largest E4M3
+
+__device__ __forceinline__ float tensor_senc(float amax) {
+  float s = (amax > 0.0f) ? __fdiv_rn(kTensorRange, amax) : 1.0f;
+  if (!isfinite(s)) s = FLT_MAX;
+  return s;
+}
+
+// One 16-element block: codes into lo (elements 0..7) and hi (8..15), returns
+// the E4M3 scale byte.
+__device__ __forceinline__ uint32_t quant_block16(const float* x, float s_enc, uint32_t& lo,
+                                                  uint32_t& hi) {
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(x[i]));
+  const float t = __fmul_rn(__fdiv_rn(a, 6.0f), s_enc);
+  const uint32_t e = cvt_e4m3(t);
+  const float de = e4m3_to_f32(e);
+  const float r = (de == 0.0f) ? 0.0f : __fdiv_rn(s_enc, de);
+  float y[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(x[i], r);
+  lo = cvt_e2m1x8(y);
+  hi = cvt_e2m1x8(y + 8);
+  return e;
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& w, float* f) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(u[i] << 16);
+    f[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// amax of up to three bf16 tensors (blockIdx.y selects the tensor). The result
+// is max |x| as fp32 bits, reduced with an integer atomicMax: for non-negative
+// floats the bit patterns order like the values, and a bf16 magnitude shifted
+// left by 16 is exactly its fp32 pattern. The outputs must be zeroed first.
+__global__ void __launch_bounds__(256) amax3_kernel(const uint4* __restrict__ x0, int64_t n0,
+                                                    const uint4* __restrict__ x1, int64_t n1,
+                                                    const uint4* __restrict__ x2, int64_t n2,
+                                                    unsigned* __restrict__ out0,
+                                                    unsigned* __restrict__ out1,
+                                                    unsigned* __restrict__ out2) {
+  const uint4* x = blockIdx.y == 0 ? x0 : (blockIdx.y == 1 ? x1 : x2);
+  const int64_t n = blockIdx.y == 0 ? n0 : (blockIdx.y == 1 ? n1 : n2);
+  unsigned* out = blockIdx.y == 0 ? out0 : (blockIdx.y == 1 ? out1 : out2);
+  if (x == nullptr) return;
+  uint32_t m = 0;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const uint4 w = ld_nc_v4(x + i);
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      m = max(m, u[k] & 0x7FFFu);
+      m = max(m, (u[k] >> 16) & 0x7FFFu);
+    }
+  }
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  __shared__ uint32_t wm[8];
+  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t r = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r = max(r, wm[w]);
+    if (r) atomicMax(out, r << 16);
+  }
+}
+
+// Blocks of 16 along D (Q and K). One thread per block; the four scales of a
+// row's consecutive blocks are gathered with shuffles into one 32-bit store.
+template <int D>
+__global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16* __restrict__ x, int G,
+                                                         int N, int Npad,
+                                                         const float* __restrict__ amax,
+                                                         uint8_t* __restrict__ codes,
+                                                         uint8_t* __restrict__ sf) {
+  constexpr int NB = D / 16;
+  const float s_enc = tensor_senc(*amax);
+  const int64_t total = (int64_t)G * Npad * NB;  // a multiple of 32
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int lane = threadIdx.x & 31;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i - lane < total;
+       i += stride) {
+    const bool valid = i < total;  // warp-uniform: total and the warp base are multiples of 32
+    const int64_t r = i / NB;
+    const int kb = (int)(i % NB);
+    const int64_t g = r / Npad;
+    const int n = (int)(r % Npad);
+    float xv[16];
+    if (valid && n < N) {
+      const __nv_bfloat16* src = x + ((g * N + n) * D + kb * 16);
+      bf16x8_to_f32(ld_nc_v4(src), xv);
+      bf16x8_to_f32(ld_nc_v4(src + 8), xv + 8);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 16; ++k) xv[k] = 0.0f;
+    }
+    uint32_t lo, hi;
+    const uint32_t e = quant_block16(xv, s_enc, lo, hi);
+    if (valid) *reinterpret_cast<uint2*>(codes + r * (D / 2) + kb * 8) = make_uint2(lo, hi);
+    // gather the scales of blocks kb..kb+3 (lanes l..l+3) into lane l (kb % 4 == 0)
+    const uint32_t e1 = __shfl_down_sync(0xFFFFFFFFu, e, 1);
+    const uint32_t e2 = __shfl_down_sync(0xFFFFFFFFu, e, 2);
+    const uint32_t e3 = __shfl_down_sync(0xFFFFFFFFu, e, 3);
+    if (valid && (kb & 3) == 0) {
+      const int tile = n >> 7, rr = n & 127;
+      const int64_t atom = (g * (Npad >> 7) + tile) * (D / 64) + (kb >> 2);
+      *reinterpret_cast<uint32_t*>(sf + atom * 512 + (rr & 31) * 16 + (rr >> 5) * 4) =
+          e | (e1 << 8) | (e2 << 16) | (e3 << 24);
+    }
+  }
+}
+
+// Blocks of 16 tokens per channel (V), written transposed. One CTA per
+// (group, 128-token tile): the tile is staged in shared memory, then thread d
+// quantises channel d's eight token blocks.
+template <int D>
+__global__ void __launch_bounds__(128) quant_tokens_T_kernel(const __nv_bfloat16* __restrict__ v,
+                                                             int G, int N, int Npad,
+                                                             const float* __restrict__ amax,
+                                                             uint8_t* __restrict__ codes,
+                                                             uint8_t* __restrict__ sf) {
+  __shared__ __align__(16) uint16_t tile[128 * D];
+  const int ntile = Npad >> 7;
+  const int64_t g = blockIdx.x / ntile;
+  const int t = blockIdx.x % ntile;
+  const float s_enc = tensor_senc(*amax);
+  // stage: 128 tokens x D channels, zero beyond N
+  constexpr int VEC = D / 8;  // uint4 per token row
+  for (int idx = threadIdx.x; idx < 128 * VEC; idx += blockDim.x) {
+    const int tok = idx / VEC, c = idx % VEC;
+    const int n = t * 128 + tok;
+    uint4 w = make_uint4(0, 0, 0, 0);
+    if (n < N) w = ld_nc_v4(v + ((g * N + n) * D + c * 8));
+    *reinterpret_cast<uint4*>(&tile[tok * D + c * 8]) = w;
+  }
+  __syncthreads();
+  const int d = threadIdx.x;
+  uint32_t e4[2] = {0, 0};
+  if (d < D) {
+    uint32_t out[16];
+#pragma unroll
+    for (int tb = 0; tb < 8; ++tb) {
+      float xv[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) xv[i] = __uint_as_float((uint32_t)tile[(tb * 16 + i) * D + d] << 16);
+      uint32_t lo, hi;
+      const uint32_t e = quant_block16(xv, s_enc, lo, hi);
+      out[2 * tb] = lo;
+      out[2 * tb + 1] = hi;
+      e4[tb >> 2] |= e << (8 * (tb & 3));
+    }
+    uint4* dst = reinterpret_cast<uint4*>(codes + (g * D + d) * (int64_t)(Npad / 2) + t * 64);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      dst[k] = make_uint4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
+  }
+  // scales: rows are channels (padded to 128 with zeros), two atoms per tile
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    const int64_t atom = g * (Npad >> 6) + t * 2 + c;
+    *reinterpret_cast<uint32_t*>(sf + atom * 512 + (d & 31) * 16 + (d >> 5) * 4) = e4[c];
+  }
+}
+
+// Hardware conversion probe over fp32 bit patterns start + i: kind 0 gives
+// the E2M1 code (one per byte), kind 1 the E4M3 byte.
+__global__ void probe_cvt_kernel(uint32_t start, int64_t count, int kind, uint8_t* __restrict__ out) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += stride) {
+    const float x = __uint_as_float(start + (uint32_t)i);
+    out[i] = (uint8_t)(kind == 0 ? (cvt_e2m1x2(x, 0.0f) & 15u) : cvt_e4m3(x));
+  }
+}
+
+}  // namespace fp4

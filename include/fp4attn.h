@@ -1,0 +1,150 @@
+/*
+ * fp4attn: NVFP4 (4-bit) FlashAttention forward on NVIDIA B200 (sm_100a).
+ *
+ * C ABI. Every pointer argument is a device pointer owned by the caller unless
+ * stated otherwise; the library allocates no device memory on any call path,
+ * keeps no state between calls beyond a per-device error word, and launches
+ * its work asynchronously on the caller's stream (a cudaStream_t passed as
+ * void*; NULL is the legacy default stream). Arguments are validated before
+ * anything is launched: a call that returns an error has launched nothing.
+ * Kernel-side failures (a bounded wait that expired) are reported later by
+ * fp4_status(). Functions are thread-safe; fp4_last_error() is per thread.
+ *
+ * Method. The pages this library restates describe 4-bit attention in which
+ * both QK^T and PV run as 4-bit block-scaled contractions while the online-
+ * softmax state stays in higher precision (HiFA4 summary, theflow.svmpsp.dev
+ * related-papers feed), the probability tile is formed from exponentials in
+ * higher precision and quantised before the low-bit PV product, and the
+ * FlashAttention row-maximum update, historical rescaling, high-precision
+ * accumulation and final normalisation are kept (EFQ-Softmax abstract,
+ * scholarbro.com page "AVQ Attention: Adaptive Vector-Quantized Attention").
+ * The operand format is block-scaled E2M1, NVFP4 (TetraJet-v2 abstract,
+ * searcharxiv.com author page "Pengle Zhang"), run on the FP4 tensor cores of
+ * Blackwell GPUs (SageAttention3 abstract, same page).
+ *
+ * NVFP4 as implemented (the pages name the format but give no recipe; this is
+ * the standard two-level reading):
+ *   element   E2M1 code, 4 bits: magnitudes {0,.5,1,1.5,2,3,4,6}, sign bit 3;
+ *             two codes per byte, element 2i in the low nibble of byte i
+ *   block     16 consecutive elements share one E4M3 scale byte (UE4M3)
+ *   tensor    one fp32 scale s_enc = 2688 / amax (1 if amax == 0, FLT_MAX on
+ *             overflow), amax = max |x| over the whole tensor
+ *   block scale  e = E4M3(fl(fl(a_b / 6) * s_enc)), a_b = block max |x|
+ *   codes        E2M1(fl(x * r)), r = fl(s_enc / dec(e)) or 0 if dec(e) == 0
+ *   conversions  round to nearest even, saturating (E2M1 to +-6, E4M3 to 448)
+ *   value        x ~= val(code) * dec(e) / s_enc
+ *
+ * Attention forward (fp4_attn_fwd), per query row i of head h:
+ *   S_ij = (q~_i . k~_j) as a block-scaled FP4 contraction, fp32 accumulation
+ *   x_ij = S_ij * d_Q * d_K * softmax_scale * log2(e), masked keys -> -inf
+ *   keys in tiles of 128 (the tile is part of the method: the running maximum
+ *   is updated once per tile): m_new = max(m, max_j x_ij), alpha = 2^(m-m_new)
+ *   p_ij = 2^(x_ij - m_new) in fp32; l = alpha l + sum_j p_ij (fp32, before
+ *   quantisation); O = alpha O + NVFP4(p) . v~ with P quantised per 16 keys
+ *   with the fixed tensor scale 2688 (p <= 1); out = O d_P d_V / l, bf16.
+ *   Causal masking keeps keys j <= i (query and key positions aligned at 0).
+ *   Grouped heads: query head h reads key/value head h / (H / Hkv).
+ *
+ * Tensor layouts (row-major, contiguous, 16-byte aligned base pointers):
+ *   q, out  bf16 [B][H][N][D]      k, v  bf16 [B][Hkv][N][D]
+ *   D in {64, 128}; H % Hkv == 0; N >= 1; B, H <= 65535.
+ */
+#ifndef FP4ATTN_H_
+#define FP4ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FP4_OK = 0,
+  FP4_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or shape */
+  FP4_ERR_UNSUPPORTED = 2, /* head dim not in {64,128}, or the device is not sm_100 */
+  FP4_ERR_WORKSPACE = 3,   /* workspace smaller than fp4_attn_workspace_bytes() */
+  FP4_ERR_CUDA = 4,        /* a CUDA runtime call failed (message in fp4_last_error) */
+  FP4_ERR_TIMEOUT = 5      /* a kernel's bounded wait expired (from fp4_status) */
+} fp4_status_t;
+
+typedef enum {
+  FP4_BLOCK_ALONG_D = 0,  /* Q, K: blocks of 16 along the head dimension */
+  FP4_BLOCK_ALONG_N_T = 1 /* V: blocks of 16 along tokens, stored transposed */
+} fp4_axis_t;
+
+/*
+ * A quantised tensor as fp4_quantize() writes it (device pointers).
+ * Npad = N rounded up to a multiple of 128; G = B*H (Q) or B*Hkv (K, V).
+ *   FP4_BLOCK_ALONG_D:   codes [G][Npad][D/2] (rows >= N are zero)
+ *   FP4_BLOCK_ALONG_N_T: codes [G][D][Npad/2] (tokens >= N are zero)
+ *   scales: the tensor-core block-scale layout in 512-byte atoms; an atom holds
+ *   128 rows x 4 consecutive blocks, row r and block k at byte
+ *   (r % 32) * 16 + (r / 32) * 4 + k.
+ *     ALONG_D:   atom ((g * Npad/128 + n/128) * D/64 + block/4) for row n
+ *     ALONG_N_T: rows are the D channels (padded to 128 with zero scales);
+ *                atom (g * Npad/64 + token_block/4)
+ *   amax: one fp32, max |x| of the whole source tensor.
+ */
+typedef struct {
+  const uint8_t* codes;
+  const uint8_t* scales;
+  const float* amax;
+} fp4_tensor_t;
+
+/* Bytes of codes / scales fp4_quantize() writes for a [G][N][D] tensor. */
+size_t fp4_codes_bytes(int G, int N, int D, fp4_axis_t axis);
+size_t fp4_scales_bytes(int G, int N, int D, fp4_axis_t axis);
+
+/* Workspace fp4_attn_fwd() needs (holds quantised Q, K, V and their maxima). */
+size_t fp4_attn_workspace_bytes(int B, int H, int Hkv, int N, int D);
+
+/*
+ * NVFP4 quantisation of one bf16 tensor x [G][N][D] (steps: amax over the whole
+ * tensor, then codes and block scales as described above).
+ * Outputs codes (fp4_codes_bytes), scales (fp4_scales_bytes) and *amax (one
+ * fp32) in device memory; all three must be 16-byte aligned.
+ */
+fp4_status_t fp4_quantize(const void* x, int G, int N, int D, fp4_axis_t axis, uint8_t* codes,
+                          uint8_t* scales, float* amax, void* stream);
+
+/*
+ * The NVFP4 attention forward: quantises q and k along D and v along tokens
+ * into the workspace, then runs the fused forward. softmax_scale <= 0 (or NaN)
+ * selects 1/sqrt(D). out may not alias q, k, v or the workspace.
+ */
+fp4_status_t fp4_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int H,
+                          int Hkv, int N, int D, int causal, float softmax_scale, void* stream,
+                          void* workspace, size_t workspace_bytes);
+
+/*
+ * The fused forward alone, on tensors fp4_quantize() produced (q with
+ * FP4_BLOCK_ALONG_D and G = B*H; k with FP4_BLOCK_ALONG_D and v with
+ * FP4_BLOCK_ALONG_N_T, G = B*Hkv), all for the same N and D.
+ */
+fp4_status_t fp4_attn_fwd_quantized(const fp4_tensor_t* q, const fp4_tensor_t* k,
+                                    const fp4_tensor_t* v, void* out, int B, int H, int Hkv,
+                                    int N, int D, int causal, float softmax_scale, void* stream);
+
+/*
+ * Synchronises the stream, then returns FP4_ERR_TIMEOUT if a kernel of this
+ * library reported an expired wait on the current device since the last call
+ * (and clears the report), FP4_ERR_CUDA on a CUDA error, else FP4_OK.
+ */
+fp4_status_t fp4_status(void* stream);
+
+/* Message of the last failing call on this thread ("" if none). */
+const char* fp4_last_error(void);
+
+/*
+ * Test support: the hardware conversion applied to the fp32 bit patterns
+ * start .. start+count-1, one output byte each: kind 0 = E2M1 code (as the
+ * quantiser's cvt produces it), kind 1 = E4M3 byte. out: device, count bytes.
+ */
+fp4_status_t fp4_probe_cvt(uint32_t start, int64_t count, int kind, uint8_t* out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4ATTN_H_ */

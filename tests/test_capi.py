@@ -1,0 +1,79 @@
+"""The C-ABI library: builds for sm_100a, loads, exports every symbol the header
+declares, and rejects bad arguments on the host before launching anything.
+No test here needs a GPU or launches a kernel."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import bit_attention_transformers_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    fa.build()
+    return fa.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "fp4attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return set(re.findall(r"\b(fp4_\w+)\s*\(", src))
+
+
+def test_header_and_binding_agree():
+    assert _declared() == set(fa.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_sizes(L):
+    # Npad = 384 for N = 300; codes 4 bits per element, scales 1 byte per 16
+    assert fa.fp4_codes_bytes(3, 300, 128, fa.FP4_BLOCK_ALONG_D) == 3 * 384 * 64
+    assert fa.fp4_scales_bytes(3, 300, 128, fa.FP4_BLOCK_ALONG_D) == 3 * 384 * 8
+    assert fa.fp4_scales_bytes(3, 300, 64, fa.FP4_BLOCK_ALONG_N_T) == 3 * 6 * 512
+    ws = fa.fp4_attn_workspace_bytes(2, 8, 2, 1000, 128)
+    assert ws >= 2 * 8 * 1024 * 64 + 2 * 2 * 1024 * 64 * 2
+    assert fa.fp4_attn_workspace_bytes(1, 3, 2, 10, 128) == 0  # H % Hkv != 0
+    assert fa.fp4_attn_workspace_bytes(1, 1, 1, 10, 96) == 0   # unsupported D
+
+
+def _call_fwd(L, q=16, k=16, v=16, out=16, B=1, H=1, Hkv=1, N=8, D=128, ws=1 << 20,
+              wsz=1 << 30):
+    vp = ctypes.c_void_p
+    return L.fp4_attn_fwd(vp(q), vp(k), vp(v), vp(out), B, H, Hkv, N, D, 0, 0.0, vp(0), vp(ws),
+                          wsz)
+
+
+def test_argument_errors_launch_nothing(L):
+    # fake, never dereferenced addresses: validation fails before any CUDA call
+    assert _call_fwd(L, D=96) == fa.FP4_ERR_UNSUPPORTED
+    assert _call_fwd(L, H=3, Hkv=2) == fa.FP4_ERR_INVALID_ARG
+    assert _call_fwd(L, N=0) == fa.FP4_ERR_INVALID_ARG
+    assert _call_fwd(L, q=0) == fa.FP4_ERR_INVALID_ARG
+    assert _call_fwd(L, k=24) == fa.FP4_ERR_INVALID_ARG  # misaligned
+    assert _call_fwd(L, wsz=100) == fa.FP4_ERR_WORKSPACE
+    assert b"workspace" in L.fp4_last_error()
+    vp = ctypes.c_void_p
+    assert L.fp4_quantize(vp(16), 1, 8, 128, 7, vp(16), vp(16), vp(16), vp(0)) == \
+        fa.FP4_ERR_INVALID_ARG
+    assert L.fp4_quantize(vp(16), 1, 8, 128, 0, vp(0), vp(16), vp(16), vp(0)) == \
+        fa.FP4_ERR_INVALID_ARG
+    assert L.fp4_probe_cvt(0xFFFFFFF0, 64, 0, vp(16), vp(0)) == fa.FP4_ERR_INVALID_ARG
+    assert L.fp4_probe_cvt(0, 16, 3, vp(16), vp(0)) == fa.FP4_ERR_INVALID_ARG
+
+
+def test_product_path_does_not_touch_the_oracle():
+    """The package, its sources and bench's GPU leg never import the oracle."""
+    pkg = os.path.join(ROOT, "bit_attention_transformers_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".c", ".cpp")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in txt.lower(), f

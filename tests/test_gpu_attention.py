@@ -1,0 +1,119 @@
+"""Attention parity: the CUDA forward (through the C ABI) against the oracle.
+
+Bar: per element |O_gpu - O_oracle| <= 2e-3 * max|V| and, per head, cosine
+similarity >= 0.9999 between the two outputs. Sizes the oracle finishes in
+seconds (several key tiles, ragged tails, causal, grouped heads, D = 64 and
+128) are checked on every row; the five workloads at full size are checked
+on every row (tiny, heavy-tailed) or on seeded sampled rows (the others).
+"""
+import os
+
+import numpy as np
+import pytest
+
+import bit_attention_transformers_b200 as fa
+from _util import bf16_bits_to_f32, bits_to_float, golden_tensors, load_golden
+from gpu_util import run_attn
+
+ATOL_REL = 2e-3
+COS_MIN = 0.9999
+
+
+def compare(gpu_rows, ora_rows, heads, vmax, label):
+    """gpu_rows/ora_rows: uint16 [n, D]; heads: [n] head id of each row."""
+    g = bf16_bits_to_f32(gpu_rows).astype(np.float64)
+    o = bf16_bits_to_f32(ora_rows).astype(np.float64)
+    assert np.isfinite(g).all(), label
+    err = np.abs(g - o).max()
+    worst_cos = 1.0
+    for h in np.unique(heads):
+        a, b = g[heads == h].ravel(), o[heads == h].ravel()
+        na, nb = np.linalg.norm(a), np.linalg.norm(b)
+        cos = 1.0 if na == 0 and nb == 0 else float(a @ b / (na * nb))
+        worst_cos = min(worst_cos, cos)
+    print(f"{label}: max|err| = {err:.3g} ({err / vmax:.3g} max|V|), min head cosine = "
+          f"{worst_cos:.7f}")
+    assert err <= ATOL_REL * vmax, (label, err, vmax)
+    assert worst_cos >= COS_MIN, (label, worst_cos)
+
+
+def run_full(ora, q, k, v, causal, label, softmax_scale=0.0):
+    B, H, N, D = q.shape
+    got = run_attn(q, k, v, causal, softmax_scale)
+    want = ora.attn_fwd(q, k, v, causal=causal, softmax_scale=softmax_scale)["bf16"]
+    heads = np.repeat(np.arange(B * H), N)
+    vmax = float(np.abs(bf16_bits_to_f32(v)).max())
+    compare(got.reshape(-1, D), want.reshape(-1, D), heads, vmax, label)
+
+
+SMALL = [  # B, H, Hkv, N, D, causal
+    (1, 2, 2, 256, 64, False),
+    (1, 2, 1, 300, 128, False),
+    (1, 2, 1, 300, 128, True),
+    (2, 4, 2, 130, 64, True),
+    (1, 1, 1, 1, 128, False),
+    (1, 1, 1, 1, 64, True),
+    (1, 3, 1, 513, 128, False),
+    (1, 2, 2, 1000, 64, True),
+    (1, 1, 1, 127, 128, True),
+    (1, 2, 2, 129, 128, False),
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("B,H,Hkv,N,D,causal", SMALL)
+def test_attention_small(ora, syn, B, H, Hkv, N, D, causal):
+    s = 1000 + N * 7 + D + 3 * H + int(causal)
+    q = syn.normal_bf16(B * H * N * D, seed=s, stream=1, scale=1.5).reshape(B, H, N, D)
+    k = syn.normal_bf16(B * Hkv * N * D, seed=s, stream=2, scale=1.5).reshape(B, Hkv, N, D)
+    v = syn.normal_bf16(B * Hkv * N * D, seed=s, stream=3).reshape(B, Hkv, N, D)
+    run_full(ora, q, k, v, causal, f"B{B} H{H} Hkv{Hkv} N{N} D{D} causal={causal}")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", ["attn_4x4.json", "attn_2x2_gqa.json"])
+@pytest.mark.parametrize("causal", [False, True])
+def test_attention_golden(ora, name, causal):
+    g = load_golden(name)
+    q, k, v = golden_tensors(g)
+    run_full(ora, q, k, v, causal, f"{name} causal={causal}",
+             softmax_scale=bits_to_float(g["softmax_scale_bits"]))
+
+
+@pytest.mark.gpu
+def test_attention_uniform_and_peaked(ora, syn):
+    """Q = 0 (every weight equal) and large-magnitude Q/K (peaked rows)."""
+    B, H, N, D = 1, 2, 400, 128
+    v = syn.normal_bf16(B * H * N * D, seed=77).reshape(B, H, N, D)
+    k = syn.normal_bf16(B * H * N * D, seed=78, scale=4.0).reshape(B, H, N, D)
+    run_full(ora, np.zeros_like(v), k, v, False, "Q=0")
+    q = syn.normal_bf16(B * H * N * D, seed=79, scale=4.0).reshape(B, H, N, D)
+    run_full(ora, q, k, v, True, "peaked causal")
+
+
+def _rows_per_head(wl):
+    env = os.environ.get("FP4_ORACLE_ROWS_PER_HEAD")
+    if env and wl.oracle_rows_per_head:
+        return int(env)
+    return wl.oracle_rows_per_head
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name", ["tiny", "heavy_tailed", "llm_prefill", "video_dit",
+                                  "long_context"])
+def test_attention_workloads(ora, syn, name):
+    wl = syn.WORKLOADS[name]
+    q, k, v = syn.workload_inputs(wl)
+    got = run_attn(q, k, v, wl.causal)
+    vmax = float(np.abs(bf16_bits_to_f32(v)).max())
+    per_head = _rows_per_head(wl)
+    if per_head == 0:
+        want = ora.attn_fwd(q, k, v, causal=wl.causal)["bf16"]
+        heads = np.repeat(np.arange(wl.B * wl.H), wl.N)
+        compare(got.reshape(-1, wl.D), want.reshape(-1, wl.D), heads, vmax, name)
+        return
+    rows = syn.sample_rows(wl, per_head)
+    want = ora.attn_fwd(q, k, v, causal=wl.causal, rows=rows)["bf16"]
+    got_rows = got[rows[:, 0], rows[:, 1], rows[:, 2]]
+    compare(got_rows, want, rows[:, 0] * wl.H + rows[:, 1], vmax,
+            f"{name} ({per_head} rows/head)")
