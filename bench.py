@@ -36,6 +36,8 @@ def parse():
     ap.add_argument("--workload", default="video_dit")
     ap.add_argument("--impl", default="fp4attn", choices=["fp4attn", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override H and Hkv (keeping their ratio) for a smaller profiling case")
     ap.add_argument("--cpu-rows", type=int, default=0,
                     help="query rows in the oracle's timed sample (0: one per head)")
     return ap.parse_args()
@@ -159,6 +161,10 @@ def main():
     args = parse()
     import synth
     wl = synth.WORKLOADS[args.workload]
+    if args.heads:
+        import dataclasses
+        g = wl.H // wl.Hkv
+        wl = dataclasses.replace(wl, H=args.heads, Hkv=max(1, args.heads // g))
     if args.impl == "reference":
         run_reference(args, wl)
         return

@@ -21,6 +21,8 @@ _LIB = os.path.join(_HERE, "libfp4attn_oracle.so")
 _lib = None
 
 FLAG_QP_DENOMINATOR = 1
+FLAG_FLIP_BOUND = 2
+FLAG_PERTURB_P = 4
 
 
 def build(force: bool = False) -> str:
@@ -65,7 +67,7 @@ def _load():
         lib.ora_scores_head.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32]
         lib.ora_scores_head.restype = i32
         lib.ora_attn_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, i32,
-                                     vp, i64, vp, vp, vp, i32]
+                                     vp, i64, vp, vp, vp, vp, i32]
         lib.ora_attn_fwd.restype = i32
         _lib = lib
     return _lib
@@ -174,12 +176,17 @@ def scores_head(q, k, b: int, h: int, threads: int | None = None) -> np.ndarray:
 
 def attn_fwd(q, k, v, causal: bool, softmax_scale: float = 0.0, rows=None, Bc: int = 128,
              flags: int = 0, threads: int | None = None, want_f64: bool = False,
-             want_ml: bool = False):
+             want_ml: bool = False, want_flip: bool = False):
     """The tiled NVFP4 attention forward on the CPU.
 
     q [B,H,N,D], k/v [B,Hkv,N,D] as uint16 bf16 bit patterns. rows: None (every
     row; the outputs have q's shape) or int64 [n, 3] triples (b, h, i) (outputs
-    [n, D]). Returns a dict with "bf16" (uint16) and optionally "f64" and "ml"."""
+    [n, D]). Returns a dict with "bf16" (uint16) and optionally "f64" (unrounded
+    output), "ml" (final m, l and the flip bound's eps per row) and "flip" (the
+    flip bound, output units:
+    how far another correct fp32 evaluation of the row can move each output
+    through P codes or block scales that lie within its rounding uncertainty of
+    a boundary)."""
     q = _c(q, np.uint16)
     k = _c(k, np.uint16)
     v = _c(v, np.uint16)
@@ -192,11 +199,15 @@ def attn_fwd(q, k, v, causal: bool, softmax_scale: float = 0.0, rows=None, Bc: i
         shape, rp, nrows = (rows.shape[0], D), rows.ctypes.data, rows.shape[0]
     out = np.empty(shape, dtype=np.uint16)
     f64 = np.empty(shape, dtype=np.float64) if want_f64 else None
-    ml = np.empty(shape[:-1] + (2,), dtype=np.float64) if want_ml else None
+    ml = np.empty(shape[:-1] + (3,), dtype=np.float64) if want_ml else None
+    flip = np.empty(shape, dtype=np.float64) if want_flip else None
+    if want_flip:
+        flags |= FLAG_FLIP_BOUND
     rc = _load().ora_attn_fwd(q.ctypes.data, k.ctypes.data, v.ctypes.data, B, H, Hkv, N, D,
                               int(bool(causal)), float(softmax_scale), Bc, flags, rp, nrows,
                               out.ctypes.data, f64.ctypes.data if f64 is not None else None,
-                              ml.ctypes.data if ml is not None else None, _threads(threads))
+                              ml.ctypes.data if ml is not None else None,
+                              flip.ctypes.data if flip is not None else None, _threads(threads))
     if rc:
         raise ValueError("ora_attn_fwd: bad arguments")
     res = {"bf16": out}
@@ -204,4 +215,6 @@ def attn_fwd(q, k, v, causal: bool, softmax_scale: float = 0.0, rows=None, Bc: i
         res["f64"] = f64
     if want_ml:
         res["ml"] = ml
+    if want_flip:
+        res["flip"] = flip
     return res

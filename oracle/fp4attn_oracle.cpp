@@ -266,7 +266,25 @@ KVGroup make_group(const Tensors& T, int b, int hk) {
   return g;
 }
 
-enum { FLAG_QP_DENOMINATOR = 1 };
+enum { FLAG_QP_DENOMINATOR = 1, FLAG_FLIP_BOUND = 2, FLAG_PERTURB_P = 4 };
+
+// E2M1 rounding boundaries of |y| between codes c and c+1 (c = 0..6).
+const float kE2M1Mid[7] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.0f};
+
+// Codes of a block with a given scale byte e (the second half of the block
+// recipe), used to evaluate the other rounding of a block scale.
+void quantize_block_with_scale(const float* x, int n, float s_enc, uint8_t e, uint8_t* codes) {
+  float de = e4m3_decode(e);
+  float r = (de == 0.0f) ? 0.0f : s_enc / de;
+  for (int i = 0; i < n; ++i) codes[i] = e2m1_encode(x[i] * r);
+}
+
+uint64_t mix64(uint64_t z) {
+  z += 0x9E3779B97F4A7C15ULL;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBULL;
+  return z ^ (z >> 31);
+}
 
 // One query row: the tiled forward over key tiles of Bc keys.
 //   S_ij = fl32(exact dot product of dequantised q_i, k_j)
@@ -279,9 +297,23 @@ enum { FLAG_QP_DENOMINATOR = 1 };
 //   p~ = NVFP4(p) per 16 keys with the fixed tensor scale 2688 (p <= 1)
 //   O = alpha O + sum_j p~_ij v~_j   (exact tile product, accumulated in double)
 // out = bf16(fl32(O * fl32(d_P d_V) / l)), d_P = fl32(1 / 2688).
+//
+// Flip bound (diagnostic, FLAG_FLIP_BOUND): a P code or block scale is a
+// rounding decision; another correct fp32 evaluation of the same row (a
+// different accumulation order of S, another exp2 within a few ulp) may land
+// on the other side of a rounding boundary. For every decision whose input lies
+// within eps of a boundary, the bound adds |p~ change| * |v~_jd| (propagated
+// like O) to flip[d] (output units), plus eps |out_d| for the continuous
+// change of the denominator. eps is four times the relative
+// uncertainty of p from: S rounding (2^-22 of sum_d |q~_d k~_d|, for the key
+// and for the row maximum), two fp32 roundings of the exponent argument and
+// 2^-21 for the exponential. FLAG_PERTURB_P multiplies each p by
+// (1 + u eps/4), u uniform in [-1, 1] (seeded by the row), to test the bound.
 void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float c, int Bc,
-                 int causal, int flags, double* o_out, double* ml_out, uint16_t* bf_out) {
+                 int causal, int flags, double* o_out, double* ml_out, uint16_t* bf_out,
+                 double* flip_out) {
   const int N = T.N, D = T.D;
+  const bool want_flip = (flags & (FLAG_FLIP_BOUND | FLAG_PERTURB_P)) != 0;
   // quantise the query row
   const uint16_t* qrow = T.q + (((int64_t)b * T.H + h) * N + i) * D;
   std::vector<uint8_t> qc(D / 2), qs(D / 16);
@@ -293,32 +325,55 @@ void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float 
   }
   float sP, dP;
   tensor_scale(1.0f, &sP, &dP);  // P: a-priori amax 1, so s_enc = 2688
-  std::vector<double> O(D, 0.0);
+  std::vector<double> O(D, 0.0), F(D, 0.0);
   std::vector<float> x(Bc), p(Bc);
-  std::vector<double> pq(Bc);
-  double m = -INFINITY, l = 0.0;
+  std::vector<double> pq(Bc), A(Bc, 0.0), eps(Bc, 0.0), dlt(Bc, 0.0);
+  double m = -INFINITY, l = 0.0, epsmax = 0.0;
   const int ntiles = (N + Bc - 1) / Bc;
+  const uint64_t rowkey = mix64(((uint64_t)b * 65536 + h) * 4294967296ULL + (uint64_t)i);
   for (int t = 0; t < ntiles; ++t) {
     const int j0 = t * Bc, j1 = std::min(j0 + Bc, N);
     if (causal && j0 > i) break;  // fully masked tiles contribute nothing
     float mt = -INFINITY;
+    double amx = 0.0;
     for (int j = j0; j < j1; ++j) {
       float xv = -INFINITY;
+      double aj = 0.0;
       if (!(causal && j > i)) {
         double s = 0.0;
         const double* kr = &g.K[(int64_t)j * D];
         for (int d = 0; d < D; ++d) s += qd[d] * kr[d];
+        if (want_flip)
+          for (int d = 0; d < D; ++d) aj += std::fabs(qd[d] * kr[d]);
         float sf = (float)s;
         xv = sf * c;
       }
       x[j - j0] = xv;
-      mt = std::max(mt, xv);
+      A[j - j0] = aj;
+      if (xv > mt) {
+        mt = xv;
+        amx = aj;
+      }
     }
     double m_new = std::max(m, (double)mt);
     double alpha = (m == -INFINITY) ? 0.0 : std::exp2(m - m_new);
     for (int jj = 0; jj < Bc; ++jj) {
       int j = j0 + jj;
-      p[jj] = (j < j1 && x[jj] != -INFINITY) ? (float)std::exp2((double)x[jj] - m_new) : 0.0f;
+      bool live = j < j1 && x[jj] != -INFINITY;
+      p[jj] = live ? (float)std::exp2((double)x[jj] - m_new) : 0.0f;
+      eps[jj] = 0.0;
+      if (live && want_flip) {
+        const double u = std::ldexp(1.0, -22);
+        eps[jj] = std::log(2.0) * ((double)c * u * (A[jj] + amx) +
+                                   u * (std::fabs((double)x[jj]) + std::fabs(m_new))) +
+                  std::ldexp(1.0, -21);
+        if (flags & FLAG_PERTURB_P) {
+          double uu = (double)(mix64(rowkey ^ mix64((uint64_t)j)) >> 11) * std::ldexp(1.0, -53);
+          p[jj] = (float)((double)p[jj] * (1.0 + (2.0 * uu - 1.0) * eps[jj]));
+        }
+        eps[jj] *= 4.0;
+        epsmax = std::max(epsmax, eps[jj]);
+      }
     }
     // P quantisation, blocks of 16 keys from the tile start
     for (int b0 = 0; b0 < Bc; b0 += 16) {
@@ -326,6 +381,34 @@ void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float 
       uint8_t codes[16], e;
       quantize_block(&p[b0], n, sP, codes, &e);
       for (int u = 0; u < n; ++u) pq[b0 + u] = deq(codes[u], e);
+      if (!(flags & FLAG_FLIP_BOUND)) continue;
+      const float de = e4m3_decode(e);
+      const float r = (de == 0.0f) ? 0.0f : sP / de;
+      double epsb = 0.0;
+      for (int u = 0; u < n; ++u) {
+        dlt[b0 + u] = 0.0;
+        epsb = std::max(epsb, eps[b0 + u]);
+        float y = std::fabs(p[b0 + u] * r);
+        for (int k2 = 0; k2 < 7; ++k2)
+          if (std::fabs((double)y - kE2M1Mid[k2]) <= eps[b0 + u] * (double)y + 1e-30)
+            dlt[b0 + u] = std::max(dlt[b0 + u],
+                                   (double)(kE2M1Mag[k2 + 1] - kE2M1Mag[k2]) * (double)de);
+      }
+      // the block scale's own rounding
+      float a = 0.0f;
+      for (int u = 0; u < n; ++u) a = std::max(a, std::fabs(p[b0 + u]));
+      float tt = (a / 6.0f) * sP;
+      int other = (tt >= de) ? e + 1 : e - 1;
+      if (a > 0.0f && other >= 0 && other <= 126) {
+        double mid = 0.5 * ((double)de + (double)e4m3_decode((uint8_t)other));
+        if (std::fabs((double)tt - mid) <= epsb * (double)tt + 1e-30) {
+          uint8_t alt[16];
+          quantize_block_with_scale(&p[b0], n, sP, (uint8_t)other, alt);
+          for (int u = 0; u < n; ++u)
+            dlt[b0 + u] = std::max(dlt[b0 + u],
+                                   std::fabs(deq(alt[u], (uint8_t)other) - pq[b0 + u]));
+        }
+      }
     }
     double lt = 0.0;
     if (flags & FLAG_QP_DENOMINATOR)
@@ -334,9 +417,12 @@ void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float 
       for (int jj = 0; jj < Bc; ++jj) lt += (double)p[jj];
     l = alpha * l + lt;
     for (int d = 0; d < D; ++d) {
-      double acc = 0.0;
+      double acc = 0.0, fl = 0.0;
       for (int j = j0; j < j1; ++j) acc += pq[j - j0] * g.V[(int64_t)j * D + d];
+      if (flags & FLAG_FLIP_BOUND)
+        for (int j = j0; j < j1; ++j) fl += dlt[j - j0] * std::fabs(g.V[(int64_t)j * D + d]);
       O[d] = alpha * O[d] + acc;
+      F[d] = alpha * F[d] + fl;
     }
     m = m_new;
   }
@@ -345,10 +431,13 @@ void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float 
     double y = O[d] * (double)fpv / l;
     if (o_out) o_out[d] = y;
     if (bf_out) bf_out[d] = f32_to_bf16_rne((float)y);
+    // decisions near a boundary, plus the continuous change of l (|dl| <= eps l)
+    if (flip_out) flip_out[d] = F[d] * (double)fpv / l + epsmax * std::fabs(y);
   }
   if (ml_out) {
     ml_out[0] = m;
     ml_out[1] = l;
+    ml_out[2] = epsmax;
   }
 }
 
@@ -441,13 +530,16 @@ int ora_scores_head(const uint16_t* q, const uint16_t* k, int B, int H, int Hkv,
 //   q [B][H][N][D], k and v [B][Hkv][N][D], bf16 bit patterns.
 //   rows: nrows (b, h, i) triples to compute, or NULL for every row.
 //   out_bf16 / out_f64: [nrows][D] (or [B][H][N][D] when rows is NULL); either
-//   may be NULL. out_ml: [nrows][2] final (m, l), may be NULL.
-//   Bc: key tile (128 on the path); flags: 1 = denominator from p~.
+//   may be NULL. out_ml: [nrows][3] final (m, l) and the largest relative
+//   uncertainty eps of the row's p (nonzero with flags 2 or 4), may be NULL.
+//   Bc: key tile (128 on the path); flags: 1 = denominator from p~,
+//   2 = flip bound into out_flip ([nrows][D], may be NULL otherwise),
+//   4 = perturb p within the flip bound's uncertainty (tests the bound).
 // Returns 0, or -1 on bad arguments.
 int ora_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H, int Hkv,
                  int N, int D, int causal, float softmax_scale, int Bc, int flags,
                  const int64_t* rows, int64_t nrows, uint16_t* out_bf16, double* out_f64,
-                 double* out_ml, int nthreads) {
+                 double* out_ml, double* out_flip, int nthreads) {
   if (B <= 0 || H <= 0 || Hkv <= 0 || H % Hkv || N <= 0 || D <= 0 || D % 16 || Bc <= 0 ||
       Bc % 16)
     return -1;
@@ -487,8 +579,8 @@ int ora_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B,
       parallel_for((int64_t)mine.size(), nthreads, [&](int64_t u) {
         int64_t r = mine[u];
         row_forward(T, g, b, (int)rows[r * 3 + 1], (int)rows[r * 3 + 2], c, Bc, causal, flags,
-                    out_f64 ? out_f64 + r * D : nullptr, out_ml ? out_ml + r * 2 : nullptr,
-                    out_bf16 ? out_bf16 + r * D : nullptr);
+                    out_f64 ? out_f64 + r * D : nullptr, out_ml ? out_ml + r * 3 : nullptr,
+                    out_bf16 ? out_bf16 + r * D : nullptr, out_flip ? out_flip + r * D : nullptr);
       });
     }
   return 0;

