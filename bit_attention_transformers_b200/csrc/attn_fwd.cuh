@@ -12,7 +12,13 @@
 //   warp 0      TMA producer: Q once, K/V tiles (+ their scales) into a ring
 //   warp 1      TMEM owner and MMA issuer (one thread): S = Q K^T into a
 //               double-buffered TMEM tile, O += P V into a TMEM accumulator
-//   warps 2..9  softmax: two threads per query row, 64 keys each
+//   warps 2-3   idle (they complete the first warpgroup)
+//   warps 4..11 softmax: one thread per query row and two streams per
+//               32-row quadrant: stream s takes the key tiles t = s mod 2
+//               (S buffer s, P buffer s), so two tiles are in flight on every
+//               SM sub-partition; the running maximum, the only value a tile
+//               needs from the one before, passes between the two streams
+//               through shared memory
 // TMEM columns: S0 [0,128) S1 [128,256) O [256,256+D) scales from 384.
 // Every wait is bounded (2 s of %globaltimer); on expiry the kernel sets the
 // device error word, stops issuing, drains its tensor-core work and returns.
@@ -29,7 +35,10 @@ namespace fp4 {
 constexpr int kBM = 128;                    // query rows per CTA
 constexpr int kBN = 128;                    // keys per tile (the method's Bc)
 constexpr int kStages = 3;                  // K/V ring depth
-constexpr int kAttnThreads = 320;           // 10 warps
+constexpr int kAttnThreads = 384;  // 12 warps = 3 warpgroups
+// Register budgets after the warpgroups re-balance: 128 x 56 + 256 x 224 equals
+// the 384 x 168 registers the block is launched with.
+constexpr uint32_t kRegsCtl = 56, kRegsSoftmax = 224;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kLog2e = 1.44269504088896340736f;
 
@@ -56,20 +65,6 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity))
     if (globaltimer_ns() - t0 > kTimeoutNs / 20) return;
-}
-
-// bar.sync over the softmax warps that also ORs a per-thread flag.
-__device__ __forceinline__ bool softmax_bar_or(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred pi, po;\n\t"
-      "setp.ne.u32 pi, %1, 0;\n\t"
-      "bar.red.or.pred po, 1, 256, pi;\n\t"
-      "selp.u32 %0, 1, 0, po;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)v)
-      : "memory");
-  return r != 0;
 }
 
 struct AttnParams {
@@ -99,7 +94,7 @@ struct AttnSmem {
   static constexpr int oKsf = oQsf + 1024;
   static constexpr int oVsf = oKsf + kStages * 1024;
   static constexpr int oPsf = oVsf + kStages * 1024;
-  static constexpr int oRed = oPsf + 2 * 1024;  // float [2][2][128]
+  static constexpr int oRed = oPsf + 2 * 1024;  // float [2][128] running max per stream, [2][128] l
   static constexpr int oPtab = oRed + 2048;     // float [128]
   static constexpr int oBar = oPtab + 512;      // mbarriers
   static constexpr int oTmem = oBar + 256;
@@ -116,8 +111,9 @@ enum : int {
   kBarSFull = kBarVEmpty + kStages,
   kBarSEmpty = kBarSFull + 2,
   kBarPFull = kBarSEmpty + 2,
-  kBarO = kBarPFull + 2,
-  kBarDrain = kBarO + 1,
+  kBarO = kBarPFull + 2,            // [2]: PV of tile t completes O[t & 1]
+  kBarMax = kBarO + 2,              // [4 quadrants][2]: running max of tile t published
+  kBarDrain = kBarMax + 8,
   kNumBars = kBarDrain + 1
 };
 
@@ -153,10 +149,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(kBarSFull + s), 1);
-      mbar_init(bar(kBarSEmpty + s), 8);
-      mbar_init(bar(kBarPFull + s), 8);
+      mbar_init(bar(kBarSEmpty + s), 4);
+      mbar_init(bar(kBarPFull + s), 4);
+      mbar_init(bar(kBarO + s), 1);
     }
-    mbar_init(bar(kBarO), 1);
+    for (int s = 0; s < 8; ++s) mbar_init(bar(kBarMax + s), 1);
     mbar_init(bar(kBarDrain), 1);
     fence_mbar_init();
   }
@@ -181,6 +178,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + L::oTmem);
 
+  if (warp < 4) {
+  regs_dec<kRegsCtl>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -208,61 +207,62 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Order per tile t: S_{t+2} as soon as the softmax has read S_t out of
+    // TMEM (early in tile t), then PV_t once P_t is written (end of tile t).
     if (lane == 0) {
       constexpr uint32_t kSw = (D == 128) ? 4u : 6u;     // 64- or 32-byte swizzle
       constexpr uint32_t kSboQK = (D == 128) ? 512u : 256u;
       constexpr uint32_t kIdS = idesc_mxf4nvf4(kBM, kBN);
       constexpr uint32_t kIdO = idesc_mxf4nvf4(kBM, D);
-      const uint32_t tS[2] = {tmem + kColS, tmem + kColS + kBN};
       const uint32_t tO = tmem + kColO, tQsf = tmem + kColQsf;
+      auto issue_s = [&](int t) -> bool {
+        const int st = t % kStages;
+        const uint32_t tKsf = tmem + kColKsf + 8 * (t & 1);
+        if (!wait_bar(bar(kBarKFull + st), (t / kStages) & 1)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kc = 0; kc < D / 64; ++kc)
+          tc_cp_32x128b_x4(tKsf + 4 * kc, smem_desc(sb + L::oKsf + st * 1024 + 512 * kc, 0, 128, 0));
+#pragma unroll
+        for (int kc = 0; kc < D / 64; ++kc)
+          mma_mxf4nvf4(tmem + kColS + (t & 1) * kBN, smem_desc(sb + L::oQ + 32 * kc, 16, kSboQK, kSw),
+                       smem_desc(sb + L::oK + st * L::kK + 32 * kc, 16, kSboQK, kSw), kIdS,
+                       tQsf + 4 * kc, tKsf + 4 * kc, kc > 0 ? 1u : 0u);
+        tc_commit(bar(kBarSFull + (t & 1)));
+        tc_commit(bar(kBarKEmpty + st));
+        return true;
+      };
       bool ok = wait_bar(bar(kBarQ), 0);
       if (ok) {
         tc_fence_after();
 #pragma unroll
         for (int kc = 0; kc < D / 64; ++kc)
           tc_cp_32x128b_x4(tQsf + 4 * kc, smem_desc(sb + L::oQsf + 512 * kc, 0, 128, 0));
+        ok = issue_s(0) && (nt < 2 || issue_s(1));
       }
-      for (int j = 0; ok && j <= nt; ++j) {
-        if (j < nt) {
-          const int st = j % kStages;
-          const uint32_t tKsf = tmem + kColKsf + 8 * (j & 1);
-          if (!(ok = wait_bar(bar(kBarKFull + st), (j / kStages) & 1))) break;
-          if (j >= 2 && !(ok = wait_bar(bar(kBarSEmpty + (j & 1)), ((j >> 1) - 1) & 1))) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kc = 0; kc < D / 64; ++kc)
-            tc_cp_32x128b_x4(tKsf + 4 * kc,
-                             smem_desc(sb + L::oKsf + st * 1024 + 512 * kc, 0, 128, 0));
-#pragma unroll
-          for (int kc = 0; kc < D / 64; ++kc)
-            mma_mxf4nvf4(tS[j & 1], smem_desc(sb + L::oQ + 32 * kc, 16, kSboQK, kSw),
-                         smem_desc(sb + L::oK + st * L::kK + 32 * kc, 16, kSboQK, kSw), kIdS,
-                         tQsf + 4 * kc, tKsf + 4 * kc, kc > 0 ? 1u : 0u);
-          tc_commit(bar(kBarSFull + (j & 1)));
-          tc_commit(bar(kBarKEmpty + st));
+      for (int t = 0; ok && t < nt; ++t) {
+        if (t + 2 < nt) {
+          if (!(ok = wait_bar(bar(kBarSEmpty + (t & 1)), (t >> 1) & 1))) break;
+          if (!(ok = issue_s(t + 2))) break;
         }
-        if (j >= 1) {
-          const int t = j - 1, st = t % kStages;
-          const uint32_t tPsf = tmem + kColPsf + 8 * (t & 1);
-          const uint32_t tVsf = tmem + kColVsf + 8 * (t & 1);
-          if (!(ok = wait_bar(bar(kBarVFull + st), (t / kStages) & 1))) break;
-          if (!(ok = wait_bar(bar(kBarPFull + (t & 1)), (t >> 1) & 1))) break;
-          tc_fence_after();
+        const int st = t % kStages;
+        const uint32_t tPsf = tmem + kColPsf + 8 * (t & 1);
+        const uint32_t tVsf = tmem + kColVsf + 8 * (t & 1);
+        if (!(ok = wait_bar(bar(kBarVFull + st), (t / kStages) & 1))) break;
+        if (!(ok = wait_bar(bar(kBarPFull + (t & 1)), (t >> 1) & 1))) break;
+        tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            tc_cp_32x128b_x4(tPsf + 4 * c,
-                             smem_desc(sb + L::oPsf + (t & 1) * 1024 + 512 * c, 0, 128, 0));
-            tc_cp_32x128b_x4(tVsf + 4 * c,
-                             smem_desc(sb + L::oVsf + st * 1024 + 512 * c, 0, 128, 0));
-          }
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-            mma_mxf4nvf4(tO, smem_desc(sb + L::oP + (t & 1) * L::kP + 32 * c, 16, 512, 4),
-                         smem_desc(sb + L::oV + st * L::kV + 32 * c, 16, 512, 4), kIdO,
-                         tPsf + 4 * c, tVsf + 4 * c, (t > 0 || c > 0) ? 1u : 0u);
-          tc_commit(bar(kBarO));
-          tc_commit(bar(kBarVEmpty + st));
+        for (int c = 0; c < 2; ++c) {
+          tc_cp_32x128b_x4(tPsf + 4 * c, smem_desc(sb + L::oPsf + (t & 1) * 1024 + 512 * c, 0, 128, 0));
+          tc_cp_32x128b_x4(tVsf + 4 * c, smem_desc(sb + L::oVsf + st * 1024 + 512 * c, 0, 128, 0));
         }
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+          mma_mxf4nvf4(tO, smem_desc(sb + L::oP + (t & 1) * L::kP + 32 * c, 16, 512, 4),
+                       smem_desc(sb + L::oV + st * L::kV + 32 * c, 16, 512, 4), kIdO,
+                       tPsf + 4 * c, tVsf + 4 * c, (t > 0 || c > 0) ? 1u : 0u);
+        tc_commit(bar(kBarO + (t & 1)));
+        tc_commit(bar(kBarVEmpty + st));
       }
       if (!ok) {  // drain whatever was issued before giving up
         tc_commit(bar(kBarDrain));
@@ -270,129 +270,165 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
     }
     __syncwarp();
+  }
   } else {
+    regs_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax
-    const int sw = warp - 2;
-    const int half = sw >> 2;             // keys [64*half, 64*half+64) of each tile
+    const int stream = (warp - 4) >> 2;   // key tiles t with t % 2 == stream
     const int quad = warp & 3;            // TMEM lanes 32*quad .. 32*quad+31
     const int row = quad * 32 + lane;     // query row within the tile
     const int qrow = qt * kBM + row;
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
-    float* red = reinterpret_cast<float*>(sm + L::oRed);
+    float* mval = reinterpret_cast<float*>(sm + L::oRed);  // [2][128]: running max after tile t, slot t & 1
+    float* lval = mval + 2 * kBM;                          // [2][128]: each stream's row sum
     const float sq = tensor_senc(*p.amax_q), sk = tensor_senc(*p.amax_k),
                 sv = tensor_senc(*p.amax_v);
     const float dq = __fdiv_rn(1.0f, sq), dk = __fdiv_rn(1.0f, sk), dv = __fdiv_rn(1.0f, sv);
     const float c = __fmul_rn(__fmul_rn(__fmul_rn(dq, dk), p.softmax_scale), kLog2e);
     const float fpv = __fmul_rn(__fdiv_rn(1.0f, kTensorRange), dv);  // d_P * d_V
-    float m_old = -INFINITY, l = 0.0f;
+    const uint64_t c2 = pk(c, c);
+    float m_own = -INFINITY;   // running max after this stream's previous tile
+    float m_last = -INFINITY;  // running max after the last tile processed
+    float l = 0.0f;            // this stream's row sum, relative to m_own
     bool fail = false;
-    int j = 0;
-    for (; j < nt; ++j) {
-      float s[64];
-      bool ok = __all_sync(0xFFFFFFFFu, wait_bar(bar(kBarSFull + (j & 1)), (j >> 1) & 1));
+    for (int t = stream; t < nt; t += 2) {
+      float s[kBN];
+      bool ok = __all_sync(0xFFFFFFFFu, wait_bar(bar(kBarSFull + stream), (t >> 1) & 1));
       if (ok) {
         tc_fence_after();
-        tmem_ld32(tl + kColS + (j & 1) * kBN + half * 64, s);
-        tmem_ld32(tl + kColS + (j & 1) * kBN + half * 64 + 32, s + 32);
+#pragma unroll
+        for (int cc = 0; cc < kBN; cc += 32) tmem_ld32(tl + kColS + stream * kBN + cc, s + cc);
         tmem_wait_ld();
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBarSEmpty + (j & 1)));
+      if (lane == 0) mbar_arrive(bar(kBarSEmpty + stream));
       // mask: keys beyond N, and (causal) keys after the query
-      const int key0 = j * kBN + half * 64;
-      if (key0 + 64 > p.N || (CAUSAL && key0 + 63 > qrow)) {
+      const int key0 = t * kBN;
+      if (key0 + kBN > p.N || (CAUSAL && key0 + kBN - 1 > qrow)) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
+        for (int i = 0; i < kBN; ++i)
           if (key0 + i >= p.N || (CAUSAL && key0 + i > qrow)) s[i] = -INFINITY;
       }
-      float bm[4];
+      float bm[8];
 #pragma unroll
-      for (int bk = 0; bk < 4; ++bk) {
-        float m0 = fmax3(s[16 * bk + 0], s[16 * bk + 1], s[16 * bk + 2]);
-        float m1 = fmax3(s[16 * bk + 3], s[16 * bk + 4], s[16 * bk + 5]);
-        float m2 = fmax3(s[16 * bk + 6], s[16 * bk + 7], s[16 * bk + 8]);
-        float m3 = fmax3(s[16 * bk + 9], s[16 * bk + 10], s[16 * bk + 11]);
-        float m4 = fmax3(s[16 * bk + 12], s[16 * bk + 13], s[16 * bk + 14]);
-        bm[bk] = fmax3(fmax3(m0, m1, m2), fmax3(m3, m4, s[16 * bk + 15]), -INFINITY);
+      for (int bk = 0; bk < 8; ++bk) {
+        const float* x = s + 16 * bk;
+        const float a0 = fmax3(x[0], x[1], x[2]), a1 = fmax3(x[3], x[4], x[5]),
+                    a2 = fmax3(x[6], x[7], x[8]), a3 = fmax3(x[9], x[10], x[11]),
+                    a4 = fmax3(x[12], x[13], x[14]);
+        bm[bk] = fmaxf(fmax3(a0, a1, a2), fmax3(a3, a4, x[15]));
       }
-      const float tmax = fmax3(fmaxf(bm[0], bm[1]), bm[2], bm[3]);
-      red[((j & 1) * 2 + half) * kBM + row] = tmax;
-      fail = softmax_bar_or(!ok || fail);
-      if (fail) break;
-      const float mx = fmaxf(tmax, red[((j & 1) * 2 + (half ^ 1)) * kBM + row]);
-      const float m_new = fmaxf(m_old, __fmul_rn(mx, c));
-      const float alpha = (m_old == -INFINITY) ? 0.0f : ex2_approx(m_old - m_new);
+      const float mx = fmaxf(fmax3(bm[0], bm[1], bm[2]),
+                             fmaxf(fmax3(bm[3], bm[4], bm[5]), fmax3(bm[6], bm[7], -INFINITY)));
+      // running max: the previous tile's (the other stream) and this tile's
+      float m_prev = -INFINITY;
+      if (t > 0) {
+        ok = __all_sync(0xFFFFFFFFu,
+                        wait_bar(bar(kBarMax + quad * 2 + (stream ^ 1)), ((t - 1) >> 1) & 1));
+        m_prev = mval[(stream ^ 1) * kBM + row];
+      }
+      if (!ok) {
+        fail = true;
+        break;
+      }
+      const float m_new = fmaxf(m_prev, __fmul_rn(mx, c));
+      mval[stream * kBM + row] = m_new;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBarMax + quad * 2 + stream));
+      const float alpha = (m_prev == -INFINITY) ? 0.0f : ex2_approx(m_prev - m_new);
       const float neg_m = (m_new == -INFINITY) ? 0.0f : -m_new;
-      float ls = 0.0f;
+      const uint64_t nm2 = pk(neg_m, neg_m);
+      // P -> NVFP4 per 16 keys with the fixed tensor scale 2688 (p <= 1):
+      // p = 2^(x - m) in fp32, block scale e = E4M3(448 a_b) with
+      // a_b = 2^(max_b - m), codes E2M1(p r) with r = 2688 / dec(e)
+      uint32_t pc[16];
+      uint32_t sfw[2] = {0u, 0u};
+      float lsum = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        s[i] = ex2_approx(fmaf(s[i], c, neg_m));
-        ls += s[i];
-      }
-      l = fmaf(l, alpha, ls);
-      // P -> NVFP4 per 16 keys (fixed tensor scale 2688: p <= 1)
-      uint32_t pc[8];
-      uint32_t sfw = 0;
-#pragma unroll
-      for (int bk = 0; bk < 4; ++bk) {
+      for (int bk = 0; bk < 8; ++bk) {
         const float a = ex2_approx(fmaf(bm[bk], c, neg_m));
         const uint32_t e = cvt_e4m3(__fmul_rn(a, 448.0f));
         const float r = ptab[e];
+        const uint64_t r2 = pk(r, r);
         float y[16];
+        uint64_t acc = 0;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) y[i] = __fmul_rn(s[16 * bk + i], r);
+        for (int i = 0; i < 8; ++i) {
+          float u0, u1;
+          upk(fma2(pk(s[16 * bk + 2 * i], s[16 * bk + 2 * i + 1]), c2, nm2), u0, u1);
+          const uint64_t pp = pk(ex2_approx(u0), ex2_approx(u1));
+          acc = (i == 0) ? pp : add2(acc, pp);
+          upk(mul2(pp, r2), y[2 * i], y[2 * i + 1]);
+        }
+        float a0, a1;
+        upk(acc, a0, a1);
+        lsum += a0 + a1;
         pc[2 * bk] = cvt_e2m1x8(y);
         pc[2 * bk + 1] = cvt_e2m1x8(y + 8);
-        sfw |= e << (8 * bk);
+        sfw[bk >> 2] |= e << (8 * (bk & 3));
       }
-      // PV of the previous tile must be complete before O is rescaled and
-      // before this tile's P buffer (last read two tiles ago) is overwritten
-      if (j >= 1) ok = __all_sync(0xFFFFFFFFu, wait_bar(bar(kBarO), (j - 1) & 1));
+      // this stream's sum, carried to the new running max
+      l = (m_own == -INFINITY) ? lsum : fmaf(l, ex2_approx(m_own - m_new), lsum);
+      m_own = m_new;
+      m_last = m_new;
+      // PV of the previous tile (the other stream's) must be complete before O
+      // is rescaled and before P buffer `stream` (read by PV two tiles ago) is
+      // overwritten
+      if (t >= 1) ok = __all_sync(0xFFFFFFFFu, wait_bar(bar(kBarO + (stream ^ 1)), ((t - 1) >> 1) & 1));
       if (!ok) {
         fail = true;
-      } else if (j >= 1 && __any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
+        break;
+      }
+      if (t >= 1 && __any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
         tc_fence_after();
+        const uint64_t al2 = pk(alpha, alpha);
 #pragma unroll
-        for (int cc = 0; cc < D / 2; cc += 16) {
+        for (int cc = 0; cc < D; cc += 16) {
           float o[16];
-          const uint32_t ta = tl + kColO + half * (D / 2) + cc;
+          const uint32_t ta = tl + kColO + cc;
           tmem_ld16(ta, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) o[i] *= alpha;
+          for (int i = 0; i < 8; ++i) upk(mul2(pk(o[2 * i], o[2 * i + 1]), al2), o[2 * i], o[2 * i + 1]);
           tmem_st16(ta, o);
         }
         tmem_wait_st();
       }
-      uint8_t* pbuf = sm + L::oP + (j & 1) * L::kP;
+      // codes: the row's 64 bytes (64-byte swizzle); scales: two 4-block atoms
+      uint8_t* pbuf = sm + L::oP + stream * L::kP + row * 64;
 #pragma unroll
-      for (int k2 = 0; k2 < 2; ++k2) {
-        const int chunk = (half * 2 + k2) ^ ((row >> 1) & 3);  // 64-byte swizzle
-        *reinterpret_cast<uint4*>(pbuf + row * 64 + chunk * 16) =
+      for (int k2 = 0; k2 < 4; ++k2)
+        *reinterpret_cast<uint4*>(pbuf + ((k2 ^ ((row >> 1) & 3)) * 16)) =
             make_uint4(pc[4 * k2], pc[4 * k2 + 1], pc[4 * k2 + 2], pc[4 * k2 + 3]);
-      }
-      *reinterpret_cast<uint32_t*>(sm + L::oPsf + (j & 1) * 1024 + half * 512 + (row & 31) * 16 +
-                                   (row >> 5) * 4) = sfw;
+      uint8_t* psf = sm + L::oPsf + stream * 1024 + (row & 31) * 16 + (row >> 5) * 4;
+      *reinterpret_cast<uint32_t*>(psf) = sfw[0];
+      *reinterpret_cast<uint32_t*>(psf + 512) = sfw[1];
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kBarPFull + (j & 1)));
-      m_old = m_new;
+      if (lane == 0) mbar_arrive(bar(kBarPFull + stream));
     }
     // ------------------------------------------------------------ epilogue
-    bool ok = !fail && __all_sync(0xFFFFFFFFu, wait_bar(bar(kBarO), (nt - 1) & 1));
-    red[((nt & 1) * 2 + half) * kBM + row] = l;
-    fail = softmax_bar_or(!ok);
+    // both streams carry their sums to the final running max (the last tile's)
+    const int tlast = nt - 1;
+    bool ok = !fail && __all_sync(0xFFFFFFFFu, wait_bar(bar(kBarO + (tlast & 1)), (tlast >> 1) & 1));
+    if (stream != (tlast & 1) && ok)
+      ok = __all_sync(0xFFFFFFFFu, wait_bar(bar(kBarMax + quad * 2 + (tlast & 1)), (tlast >> 1) & 1));
+    const float m_fin = ok ? mval[(tlast & 1) * kBM + row] : 0.0f;
+    const float l_own = (nt > stream && m_last != -INFINITY) ? l * ex2_approx(m_last - m_fin) : 0.0f;
+    lval[stream * kBM + row] = l_own;
+    fail = bar_red_or(1 + quad, 64, !ok);
     if (!fail) {
       tc_fence_after();
-      const float ltot = l + red[((nt & 1) * 2 + (half ^ 1)) * kBM + row];
+      const float ltot = lval[row] + lval[kBM + row];
       const float inv = __fdiv_rn(fpv, ltot);
-      __nv_bfloat16* dst = p.out + ((int64_t)gq * p.N + qrow) * D + half * (D / 2);
+      constexpr int DH = D / 2;             // each stream writes half the channels
+      __nv_bfloat16* dst = p.out + ((int64_t)gq * p.N + qrow) * D + stream * DH;
 #pragma unroll
-      for (int cc = 0; cc < D / 2; cc += 32) {
+      for (int cc = 0; cc < DH; cc += 32) {
         float o[32];
-        tmem_ld32(tl + kColO + half * (D / 2) + cc, o);
+        tmem_ld32(tl + kColO + stream * DH + cc, o);
         tmem_wait_ld();
         if (qrow < p.N) {
           uint32_t w[16];

@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -47,6 +48,15 @@ int g_num_sms[kMaxDevices];
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
+using AttnKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                            const fp4::AttnParams);
+
+// The fused kernel for head dim D and causal masking.
+AttnKernel attn_kernel(int D, int causal) {
+  if (D == 128) return causal ? fp4::attn_fwd_kernel<128, true> : fp4::attn_fwd_kernel<128, false>;
+  return causal ? fp4::attn_fwd_kernel<64, true> : fp4::attn_fwd_kernel<64, false>;
+}
+
 // sm_100 check, per-device one-time kernel attributes, SM count.
 fp4_status_t device_setup(int* dev_out, int* sms_out) {
   int dev;
@@ -61,18 +71,11 @@ fp4_status_t device_setup(int* dev_out, int* sms_out) {
     if (major != 10 || minor != 0)
       return fail(FP4_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
                   dev, major, minor);
-    FP4_CUDA(cudaFuncSetAttribute(fp4::attn_fwd_kernel<128, false>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  fp4::AttnSmem<128>::kBytes));
-    FP4_CUDA(cudaFuncSetAttribute(fp4::attn_fwd_kernel<128, true>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  fp4::AttnSmem<128>::kBytes));
-    FP4_CUDA(cudaFuncSetAttribute(fp4::attn_fwd_kernel<64, false>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  fp4::AttnSmem<64>::kBytes));
-    FP4_CUDA(cudaFuncSetAttribute(fp4::attn_fwd_kernel<64, true>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  fp4::AttnSmem<64>::kBytes));
+    for (int d = 0; d < 2; ++d)
+      for (int causal = 0; causal < 2; ++causal)
+        FP4_CUDA(cudaFuncSetAttribute(attn_kernel(d ? 128 : 64, causal),
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      d ? fp4::AttnSmem<128>::kBytes : fp4::AttnSmem<64>::kBytes));
     if (!g_encode) {
       cudaDriverEntryPointQueryResult q;
       void* fn = nullptr;
@@ -222,17 +225,7 @@ fp4_status_t launch_attn(const uint8_t* qc, const uint8_t* qs, const float* qa, 
                         : 1.0f / std::sqrt((float)D);
   dim3 grid(p.ntq, H, B);
   const int smem = D == 128 ? fp4::AttnSmem<128>::kBytes : fp4::AttnSmem<64>::kBytes;
-  if (D == 128) {
-    if (causal)
-      fp4::attn_fwd_kernel<128, true><<<grid, fp4::kAttnThreads, smem, stream>>>(tq, tk, tv, p);
-    else
-      fp4::attn_fwd_kernel<128, false><<<grid, fp4::kAttnThreads, smem, stream>>>(tq, tk, tv, p);
-  } else {
-    if (causal)
-      fp4::attn_fwd_kernel<64, true><<<grid, fp4::kAttnThreads, smem, stream>>>(tq, tk, tv, p);
-    else
-      fp4::attn_fwd_kernel<64, false><<<grid, fp4::kAttnThreads, smem, stream>>>(tq, tk, tv, p);
-  }
+  attn_kernel(D, causal)<<<grid, fp4::kAttnThreads, smem, stream>>>(tq, tk, tv, p);
   FP4_CUDA(cudaGetLastError());
   return FP4_OK;
 }
