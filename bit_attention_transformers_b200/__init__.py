@@ -29,8 +29,9 @@ FP4_BLOCK_ALONG_N_T = 1
 
 # Every symbol include/fp4attn.h declares.
 EXPORTS = ("fp4_codes_bytes", "fp4_scales_bytes", "fp4_attn_workspace_bytes", "fp4_quantize",
-           "fp4_attn_fwd", "fp4_attn_fwd_quantized", "fp4_status", "fp4_last_error",
-           "fp4_probe_cvt")
+           "fp4_attn_fwd", "fp4_attn_fwd_quantized", "fp4_attn_fwd_noalloc", "fp4_status",
+           "fp4_last_error", "fp4_probe_cvt")
+FP4_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-shared"]
@@ -85,6 +86,8 @@ def lib():
         L.fp4_attn_fwd.restype = i32
         L.fp4_attn_fwd_quantized.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
         L.fp4_attn_fwd_quantized.restype = i32
+        L.fp4_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
+        L.fp4_attn_fwd_noalloc.restype = i32
         L.fp4_status.argtypes = [vp]
         L.fp4_status.restype = i32
         L.fp4_last_error.argtypes = []
@@ -190,6 +193,26 @@ def fp4_attn_fwd(q, k, v, causal: bool = False, softmax_scale: float | None = No
     _check(lib().fp4_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, Hkv, N, D,
                               int(bool(causal)), float(softmax_scale or 0.0), _stream(stream),
                               _ptr(ws), ws.numel()))
+    return out
+
+
+def fp4_attn_fwd_noalloc(q, k, v, causal: bool = False, softmax_scale: float | None = None,
+                         out=None, stream=None):
+    """fp4_attn_fwd for callers that cannot allocate device memory: the
+    scratch is the library's built-in FP4_NOALLOC_SCRATCH_BYTES array, shared
+    by every call on a device (calls that overlap on the GPU race on it), and
+    larger problems are rejected. `out` must be given to avoid any allocation
+    here (it is created only as a convenience when omitted)."""
+    import torch
+    B, H, N, D = q.shape
+    Hkv = k.shape[1]
+    for t in (q, k, v):
+        assert t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().fp4_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, Hkv, N, D,
+                                      int(bool(causal)), float(softmax_scale or 0.0),
+                                      _stream(stream)))
     return out
 
 

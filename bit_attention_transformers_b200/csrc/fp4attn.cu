@@ -323,6 +323,42 @@ fp4_status_t fp4_attn_fwd_quantized(const fp4_tensor_t* q, const fp4_tensor_t* k
                      static_cast<cudaStream_t>(stream));
 }
 
+// Scratch for fp4_attn_fwd_noalloc: reserved in every GPU's copy of this
+// module; its device address is looked up once per device.
+static __device__ __align__(256) uint8_t g_fp4_noalloc_scratch[FP4_NOALLOC_SCRATCH_BYTES];
+static void* g_noalloc_ptr[kMaxDevices];
+
+fp4_status_t fp4_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, int B,
+                                  int H, int Hkv, int N, int D, int causal, float softmax_scale,
+                                  void* stream) {
+  g_last_error.clear();
+  fp4_status_t s;
+  if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
+  const size_t need = ws_layout(B, H, Hkv, N, D).total;
+  if (need > FP4_NOALLOC_SCRATCH_BYTES)
+    return fail(FP4_ERR_WORKSPACE,
+                "this problem needs %zu bytes of scratch; the built-in scratch of "
+                "fp4_attn_fwd_noalloc holds %zu (use fp4_attn_fwd with a workspace)",
+                need, (size_t)FP4_NOALLOC_SCRATCH_BYTES);
+  int dev, sms;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  void* scratch;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_noalloc_ptr[dev]) {
+      void* ptr = nullptr;
+      cudaError_t e = cudaGetSymbolAddress(&ptr, g_fp4_noalloc_scratch);
+      if (e != cudaSuccess || !ptr)
+        return fail(FP4_ERR_CUDA, "cudaGetSymbolAddress of the scratch failed: %s",
+                    cudaGetErrorString(e));
+      g_noalloc_ptr[dev] = ptr;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  return fp4_attn_fwd(q, k, v, out, B, H, Hkv, N, D, causal, softmax_scale, stream, scratch,
+                      FP4_NOALLOC_SCRATCH_BYTES);
+}
+
 fp4_status_t fp4_status(void* stream) {
   FP4_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
   FP4_CUDA(cudaGetLastError());

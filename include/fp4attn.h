@@ -127,6 +127,28 @@ fp4_status_t fp4_attn_fwd_quantized(const fp4_tensor_t* q, const fp4_tensor_t* k
                                     int N, int D, int causal, float softmax_scale, void* stream);
 
 /*
+ * fp4_attn_fwd without a caller-supplied workspace, for callers that cannot
+ * allocate device memory: code whose device memory is owned by a host
+ * framework that hands it no allocator, or code that must not call
+ * cudaMalloc because it may synchronise the device. This entry point has no
+ * counterpart on the source pages; it only changes where the scratch lives.
+ *
+ * The scratch is one array of FP4_NOALLOC_SCRATCH_BYTES in this library's
+ * device memory, reserved on every GPU that loads the library until the
+ * process exits. Problems whose workspace (fp4_attn_workspace_bytes) exceeds
+ * it are rejected with FP4_ERR_WORKSPACE and launch nothing. Every call uses
+ * the same array: calls whose work overlaps on the GPU (other streams, other
+ * host threads, other devices' calls are fine) race on it and must be
+ * ordered by the caller. The first call on a device looks up the array's
+ * device address and caches it; make that first call before any stream
+ * capture. No call allocates or frees memory. Arguments as fp4_attn_fwd.
+ */
+#define FP4_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+fp4_status_t fp4_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, int B,
+                                  int H, int Hkv, int N, int D, int causal, float softmax_scale,
+                                  void* stream);
+
+/*
  * Synchronises the stream, then returns FP4_ERR_TIMEOUT if a kernel of this
  * library reported an expired wait on the current device since the last call
  * (and clears the report), FP4_ERR_CUDA on a CUDA error, else FP4_OK.
