@@ -5,8 +5,12 @@ python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl re
 One step is one pass of the whole path over one batch of the workload: amax
 and NVFP4 quantisation of Q, K and V, then the fused attention forward (one
 fp4_attn_fwd call). value = algorithmic FLOPs (4*B*H*N^2*D, halved when causal)
-of all ranks / the slowest rank's device time. Under torchrun every rank runs
-its own replica of the workload (the path needs no exchange between ranks).
+of all ranks / the slowest rank's device time. Under torchrun (N > 1 ranks) the
+heads are sharded: the job is N times the workload's (batch, key/value head)
+units, each rank owns one workload-sized slab of them (weak scaling), and a step
+is fp4_attn_fwd_sharded: the three tensor maxima of the rank's shard, one NCCL
+all-reduce (MAX) of those three floats, quantisation with the global maxima and
+the fused forward, so codes match a single-GPU run over the whole job.
 Inputs are seeded synthetic tensors; the default workload is the video-DiT
 latent grid (B1 H24 N32760 D128).
 """
@@ -190,16 +194,22 @@ def main():
     hq = torch.empty(shape_q, dtype=torch.bfloat16, pin_memory=True)
     hk = torch.empty(shape_kv, dtype=torch.bfloat16, pin_memory=True)
     hv = torch.empty(shape_kv, dtype=torch.bfloat16, pin_memory=True)
-    synth.workload_inputs(wl, outs=[t.view(torch.int16).numpy().view(np.uint16) for t in (hq, hk, hv)])
+    # rank r holds units r*B*Hkv .. (r+1)*B*Hkv - 1 of the job: its own heads, its own data
+    synth.workload_inputs(wl, seed=wl.seed + 7919 * rank,
+                          outs=[t.view(torch.int16).numpy().view(np.uint16) for t in (hq, hk, hv)])
     q, k, v = hq.to(dev), hk.to(dev), hv.to(dev)
     out = torch.empty_like(q)
+    qf, kf, vf, outf = (t.view(-1, wl.N, wl.D) for t in (q, k, v, out))
     ws = fa.workspace(wl.B, wl.H, wl.Hkv, wl.N, wl.D, dev)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
     flops = wl.flops
 
     def step():
-        fa.fp4_attn_fwd(q, k, v, causal=wl.causal, out=out, ws=ws)
+        if world > 1:
+            fa.fp4_attn_fwd_sharded(qf, kf, vf, causal=wl.causal, out=outf)
+        else:
+            fa.fp4_attn_fwd(q, k, v, causal=wl.causal, out=out, ws=ws)
 
     def barrier():
         if world > 1:
@@ -251,7 +261,14 @@ def main():
     hout = torch.empty(shape_q, dtype=torch.bfloat16, pin_memory=True)
 
     def e2e():
-        fa.fp4_attn_fwd_host(hq, hk, hv, causal=wl.causal, out=hout, device=dev)
+        if world > 1:
+            for d, h in ((q, hq), (k, hk), (v, hv)):
+                d.copy_(h, non_blocking=True)
+            fa.fp4_attn_fwd_sharded(qf, kf, vf, causal=wl.causal, out=outf)
+            hout.copy_(out, non_blocking=True)
+            stream.synchronize()
+        else:
+            fa.fp4_attn_fwd_host(hq, hk, hv, causal=wl.causal, out=hout, device=dev)
 
     for _ in range(max(1, args.warmup // 2)):
         e2e()
@@ -275,7 +292,10 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
         "data": "synthetic",
-        "config": {**wl.describe(), "parallelism": f"replicas x{world}",
+        "config": {**wl.describe(),
+                   "parallelism": (f"heads sharded over {world} ranks ({world} x B*Hkv units, "
+                                   "one all-reduce MAX of 3 floats per step)") if world > 1
+                   else "1 GPU",
                    "l2": "inputs larger than L2 (bf16 Q/K/V of "
                          f"{(hq.numel() + 2 * hk.numel()) * 2 / 1e6:.0f} MB); "
                          "L2 also flushed (252 MB write) before every timed step"},
@@ -290,7 +310,8 @@ def main():
         "e2e": {"value": e2e_value, "unit": "TFLOPS",
                 "h2d_bytes_per_step": (hq.numel() + hk.numel() + hv.numel()) * 2,
                 "d2h_bytes_per_step": hout.numel() * 2},
-        "gpu_launches": 5 * args.steps,
+        # per step: amax (1, or 3 when sharded), 3 quantisations, the fused forward
+        "gpu_launches": (7 if world > 1 else 5) * args.steps,
     }
     c = clk.summary()
     if c:

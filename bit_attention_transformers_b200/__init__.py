@@ -29,8 +29,8 @@ FP4_BLOCK_ALONG_N_T = 1
 
 # Every symbol include/fp4attn.h declares.
 EXPORTS = ("fp4_codes_bytes", "fp4_scales_bytes", "fp4_attn_workspace_bytes", "fp4_quantize",
-           "fp4_attn_fwd", "fp4_attn_fwd_quantized", "fp4_attn_fwd_noalloc", "fp4_status",
-           "fp4_last_error", "fp4_probe_cvt")
+           "fp4_amax", "fp4_quantize_scaled", "fp4_attn_fwd", "fp4_attn_fwd_quantized",
+           "fp4_attn_fwd_noalloc", "fp4_status", "fp4_last_error", "fp4_probe_cvt")
 FP4_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
@@ -82,6 +82,10 @@ def lib():
         L.fp4_attn_workspace_bytes.restype = sz
         L.fp4_quantize.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp]
         L.fp4_quantize.restype = i32
+        L.fp4_amax.argtypes = [vp, i32, i32, i32, vp, vp]
+        L.fp4_amax.restype = i32
+        L.fp4_quantize_scaled.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp]
+        L.fp4_quantize_scaled.restype = i32
         L.fp4_attn_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, sz]
         L.fp4_attn_fwd.restype = i32
         L.fp4_attn_fwd_quantized.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
@@ -146,18 +150,41 @@ class Fp4Tensor:
     axis: int
 
 
-def fp4_quantize(x, axis: int = FP4_BLOCK_ALONG_D, stream=None) -> Fp4Tensor:
-    """x: bf16 CUDA tensor [..., N, D] (the leading dims form the groups G)."""
+def _gnd(x):
     import torch
     assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous()
     N, D = x.shape[-2], x.shape[-1]
-    G = x.numel() // (N * D)
+    return x.numel() // (N * D), N, D
+
+
+def fp4_quantize(x, axis: int = FP4_BLOCK_ALONG_D, stream=None, amax=None) -> Fp4Tensor:
+    """x: bf16 CUDA tensor [..., N, D] (the leading dims form the groups G).
+    With `amax` (a float32 CUDA tensor whose first element is the tensor
+    maximum, e.g. combined over shards) the tensor scale comes from it
+    (fp4_quantize_scaled); otherwise max |x| is computed first."""
+    import torch
+    G, N, D = _gnd(x)
     codes = torch.empty(fp4_codes_bytes(G, N, D, axis), dtype=torch.uint8, device=x.device)
     scales = torch.empty(fp4_scales_bytes(G, N, D, axis), dtype=torch.uint8, device=x.device)
-    amax = torch.empty(4, dtype=torch.float32, device=x.device)
-    _check(lib().fp4_quantize(_ptr(x), G, N, D, axis, _ptr(codes), _ptr(scales), _ptr(amax),
-                              _stream(stream)))
+    if amax is None:
+        amax = torch.empty(4, dtype=torch.float32, device=x.device)
+        _check(lib().fp4_quantize(_ptr(x), G, N, D, axis, _ptr(codes), _ptr(scales), _ptr(amax),
+                                  _stream(stream)))
+    else:
+        assert amax.is_cuda and amax.dtype == torch.float32
+        _check(lib().fp4_quantize_scaled(_ptr(x), G, N, D, axis, _ptr(amax), _ptr(codes),
+                                         _ptr(scales), _stream(stream)))
     return Fp4Tensor(codes, scales, amax, G, N, D, axis)
+
+
+def fp4_amax(x, out=None, stream=None):
+    """max |x| of a bf16 CUDA tensor [..., N, D] into out[0] (float32 CUDA)."""
+    import torch
+    G, N, D = _gnd(x)
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=x.device)
+    _check(lib().fp4_amax(_ptr(x), G, N, D, _ptr(out), _stream(stream)))
+    return out
 
 
 # -------------------------------------------------------------- attention ----
@@ -260,3 +287,6 @@ def fp4_probe_cvt(start: int, count: int, kind: int, out=None, stream=None):
         out = torch.empty(count, dtype=torch.uint8, device="cuda")
     _check(lib().fp4_probe_cvt(start, count, kind, _ptr(out), _stream(stream)))
     return out
+
+
+from .sharded import allreduce_max_, fp4_attn_fwd_sharded, shard_rows, shard_units  # noqa: E402

@@ -268,6 +268,38 @@ fp4_status_t fp4_quantize(const void* x, int G, int N, int D, fp4_axis_t axis, u
   return launch_quant(x, G, N, D, axis, codes, scales, amax, sms, st);
 }
 
+fp4_status_t fp4_amax(const void* x, int G, int N, int D, float* amax, void* stream) {
+  g_last_error.clear();
+  fp4_status_t s;
+  if ((s = check_shape(1, G, G, N, D)) != FP4_OK) return s;
+  if (!x || !amax) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(amax) & 3u))
+    return fail(FP4_ERR_INVALID_ARG, "x must be 16-byte and amax 4-byte aligned");
+  int dev, sms;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  return launch_amax(x, (int64_t)G * N * D, nullptr, 0, nullptr, 0, amax, nullptr, nullptr, sms,
+                     static_cast<cudaStream_t>(stream));
+}
+
+fp4_status_t fp4_quantize_scaled(const void* x, int G, int N, int D, fp4_axis_t axis,
+                                 const float* amax, uint8_t* codes, uint8_t* scales,
+                                 void* stream) {
+  g_last_error.clear();
+  fp4_status_t s;
+  if ((s = check_shape(1, G, G, N, D)) != FP4_OK) return s;
+  if (axis != FP4_BLOCK_ALONG_D && axis != FP4_BLOCK_ALONG_N_T)
+    return fail(FP4_ERR_INVALID_ARG, "axis %d", (int)axis);
+  if (!x || !codes || !scales || !amax) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) ||
+      (reinterpret_cast<uintptr_t>(amax) & 3u))
+    return fail(FP4_ERR_INVALID_ARG,
+                "x, codes and scales must be 16-byte aligned, amax 4-byte aligned");
+  int dev, sms;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  return launch_quant(x, G, N, D, axis, codes, scales, amax, sms,
+                      static_cast<cudaStream_t>(stream));
+}
+
 fp4_status_t fp4_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int H,
                           int Hkv, int N, int D, int causal, float softmax_scale, void* stream,
                           void* workspace, size_t workspace_bytes) {

@@ -1,0 +1,90 @@
+"""Head-sharded NVFP4 attention forward across ranks (one process per GPU).
+
+Every (batch, key/value head) unit of attention, with its G = H / Hkv query
+heads, is independent of every other unit. The one quantity that couples them
+is the NVFP4 tensor scale, which the recipe forms from max |x| over the whole
+tensor (one fp32 scale per tensor: TetraJet-v2 abstract, NVFP4). So a tensor
+held in shards is quantised exactly as the whole tensor would be: every rank
+takes its shard's maxima of Q, K and V, one all-reduce (MAX) of those three
+floats makes them global, and every rank then quantises its own shard with
+them and runs the fused forward on it. Codes, scales and outputs are then the
+same, bit for bit, as one GPU's run over the whole tensors; the outputs stay
+sharded by head and nothing else crosses between ranks.
+
+The units are the B * Hkv (batch, key/value head) pairs in memory order,
+split into contiguous ranges, so that a rank's share of q viewed as
+[B * H, N, D] and of k, v viewed as [B * Hkv, N, D] is one contiguous slab.
+"""
+from __future__ import annotations
+
+
+def shard_units(B: int, Hkv: int, world: int, rank: int) -> tuple[int, int]:
+    """[u0, u1): the (batch, key/value head) units of `rank`, unit u = b * Hkv + kv_head.
+
+    Ranges are contiguous and in rank order, their sizes differ by at most one,
+    and ranks beyond the number of units get an empty range."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} of world {world}")
+    if B < 0 or Hkv < 1:
+        raise ValueError(f"B={B}, Hkv={Hkv}")
+    base, extra = divmod(B * Hkv, world)
+    u0 = rank * base + min(rank, extra)
+    return u0, u0 + base + (1 if rank < extra else 0)
+
+
+def shard_rows(B: int, H: int, Hkv: int, world: int, rank: int) -> tuple[slice, slice]:
+    """Slices of the leading dim of q viewed as [B * H, N, D] and of k, v viewed
+    as [B * Hkv, N, D] that `rank` owns (query head h of a batch reads key/value
+    head h / G, so the query rows of unit u are u * G .. u * G + G - 1)."""
+    if H % Hkv:
+        raise ValueError(f"H ({H}) must be a multiple of Hkv ({Hkv})")
+    g = H // Hkv
+    u0, u1 = shard_units(B, Hkv, world, rank)
+    return slice(u0 * g, u1 * g), slice(u0, u1)
+
+
+def allreduce_max_(t, group=None):
+    """In place: t = elementwise max of t over the ranks of `group`.
+
+    A no-op unless torch.distributed has a process group with more than one
+    rank (NCCL for CUDA tensors; any backend that supports MAX for others)."""
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return t
+
+
+def fp4_attn_fwd_sharded(q, k, v, causal: bool = False, softmax_scale: float | None = None,
+                         group=None, out=None, stream=None):
+    """This rank's part of a head-sharded NVFP4 attention forward.
+
+    q: this rank's query heads, a contiguous bf16 CUDA tensor [..., N, D] whose
+    leading dims hold Gq = U * G heads in unit order; k, v: its U key/value
+    heads, [..., N, D]. Every rank of `group` calls this with the same N, D,
+    G, causal and softmax_scale, an empty shard (U = 0) included: it still
+    takes part in the all-reduce. Returns `out` (like q) with this rank's
+    output heads."""
+    import torch
+    from . import (FP4_BLOCK_ALONG_D, FP4_BLOCK_ALONG_N_T, fp4_amax, fp4_attn_fwd_quantized,
+                   fp4_quantize)
+    N, D = q.shape[-2], q.shape[-1]
+    if k.shape[-2:] != (N, D) or v.shape != k.shape:
+        raise ValueError("q, k, v must share N and D, and k and v their shape")
+    gq, gkv = q.numel() // (N * D), k.numel() // (N * D)
+    if (gkv == 0) != (gq == 0) or (gkv and gq % gkv):
+        raise ValueError(f"{gq} query heads for {gkv} key/value heads")
+    amax = torch.zeros(3, dtype=torch.float32, device=q.device)
+    if gkv:
+        fp4_amax(q, amax[0:1], stream)
+        fp4_amax(k, amax[1:2], stream)
+        fp4_amax(v, amax[2:3], stream)
+    allreduce_max_(amax, group)
+    if out is None:
+        out = torch.empty_like(q)
+    if gkv == 0:
+        return out
+    qq = fp4_quantize(q, FP4_BLOCK_ALONG_D, stream, amax=amax[0:1])
+    kq = fp4_quantize(k, FP4_BLOCK_ALONG_D, stream, amax=amax[1:2])
+    vq = fp4_quantize(v, FP4_BLOCK_ALONG_N_T, stream, amax=amax[2:3])
+    fp4_attn_fwd_quantized(qq, kq, vq, 1, gq, gkv, causal, softmax_scale, out=out, stream=stream)
+    return out

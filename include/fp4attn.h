@@ -109,6 +109,31 @@ fp4_status_t fp4_quantize(const void* x, int G, int N, int D, fp4_axis_t axis, u
                           uint8_t* scales, float* amax, void* stream);
 
 /*
+ * The tensor maximum alone (the first step of fp4_quantize): *amax = max |x|
+ * over a bf16 tensor x [G][N][D] (shape rules as fp4_quantize; x 16-byte
+ * aligned, amax one fp32 in device memory, 4-byte aligned). With
+ * fp4_quantize_scaled this splits fp4_quantize in two, so that a tensor held
+ * in shards (by head, one shard per GPU) can be quantised exactly as the whole
+ * tensor would be: each shard's maximum is computed here, the maxima are
+ * combined by max across the shards (the head-sharded forward all-reduces
+ * them), and every shard is then quantised with the combined value. The
+ * pages' recipe has one fp32 scale per tensor (TetraJet-v2 abstract); this
+ * entry point only lets that scale be formed from shards.
+ */
+fp4_status_t fp4_amax(const void* x, int G, int N, int D, float* amax, void* stream);
+
+/*
+ * fp4_quantize with the tensor maximum given instead of computed: the tensor
+ * scale is s_enc = 2688 / *amax, read on the device when the kernel runs
+ * (amax: one fp32 in device memory, 4-byte aligned; it must be >= max |x|,
+ * else the largest blocks saturate to the E4M3 maximum 448). Writes codes
+ * and scales as fp4_quantize (16-byte aligned); *amax is not modified.
+ */
+fp4_status_t fp4_quantize_scaled(const void* x, int G, int N, int D, fp4_axis_t axis,
+                                 const float* amax, uint8_t* codes, uint8_t* scales,
+                                 void* stream);
+
+/*
  * The NVFP4 attention forward: quantises q and k along D and v along tokens
  * into the workspace, then runs the fused forward. softmax_scale <= 0 (or NaN)
  * selects 1/sqrt(D). out may not alias q, k, v or the workspace.

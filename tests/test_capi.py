@@ -65,6 +65,16 @@ def test_argument_errors_launch_nothing(L):
         fa.FP4_ERR_INVALID_ARG
     assert L.fp4_quantize(vp(16), 1, 8, 128, 0, vp(0), vp(16), vp(16), vp(0)) == \
         fa.FP4_ERR_INVALID_ARG
+    assert L.fp4_amax(vp(16), 1, 8, 96, vp(16), vp(0)) == fa.FP4_ERR_UNSUPPORTED
+    assert L.fp4_amax(vp(16), 1, 8, 128, vp(0), vp(0)) == fa.FP4_ERR_INVALID_ARG
+    assert L.fp4_amax(vp(24), 1, 8, 128, vp(16), vp(0)) == fa.FP4_ERR_INVALID_ARG  # misaligned x
+    assert L.fp4_amax(vp(16), 1, 8, 128, vp(18), vp(0)) == fa.FP4_ERR_INVALID_ARG  # misaligned amax
+    assert L.fp4_quantize_scaled(vp(16), 1, 8, 128, 2, vp(16), vp(16), vp(16), vp(0)) == \
+        fa.FP4_ERR_INVALID_ARG
+    assert L.fp4_quantize_scaled(vp(16), 1, 8, 128, 1, vp(0), vp(16), vp(16), vp(0)) == \
+        fa.FP4_ERR_INVALID_ARG
+    assert L.fp4_quantize_scaled(vp(16), 0, 8, 128, 1, vp(4), vp(16), vp(16), vp(0)) == \
+        fa.FP4_ERR_INVALID_ARG
     assert L.fp4_probe_cvt(0xFFFFFFF0, 64, 0, vp(16), vp(0)) == fa.FP4_ERR_INVALID_ARG
     assert L.fp4_probe_cvt(0, 16, 3, vp(16), vp(0)) == fa.FP4_ERR_INVALID_ARG
 
