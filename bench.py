@@ -17,6 +17,7 @@ latent grid (B1 H24 N32760 D128).
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -30,6 +31,12 @@ sys.path.insert(0, ROOT)
 METRIC = "FP4 attention fwd TFLOPS at 1 B200 and % of dense FP4 tensor peak"
 FP4_DATASHEET_TFLOPS = 9000.0  # NVIDIA B200 dense FP4, no sparsity
 L2_BYTES = 126 * 1024 * 1024
+# DRAM bytes (read + write) of one attention-kernel launch on the full video-DiT
+# workload, from ncu (dram__bytes_read.sum + dram__bytes_write.sum, one pass;
+# profiles/attn_fwd_traffic_video_dit.md). They hold only for the kernel source
+# they were taken on, identified by its hash; otherwise traffic is reported null.
+ATTN_TRAFFIC = {"workload": "video_dit", "bytes": 171.07e6 + 156.07e6,
+                "attn_fwd_sha256": "d118fd94ac8b00d407f1fc48af0930efaea761c8d965698189cf2efe43f09bfd"}
 
 
 def parse():
@@ -287,6 +294,11 @@ def main():
     fp4_peak = 4.0 * peaks["bf16_tflops"]  # dense FP4 = 4x dense bf16 (nominal 9 vs 2.25 PF)
     achieved = flops / (k_ms * 1e-3) / 1e12
     traffic = None
+    src = os.path.join(ROOT, "bit_attention_transformers_b200", "csrc", "attn_fwd.cuh")
+    with open(src, "rb") as f:
+        if (wl.name == ATTN_TRAFFIC["workload"] and not args.heads and
+                hashlib.sha256(f.read()).hexdigest() == ATTN_TRAFFIC["attn_fwd_sha256"]):
+            traffic = ATTN_TRAFFIC["bytes"]
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,

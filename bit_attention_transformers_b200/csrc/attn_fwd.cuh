@@ -10,9 +10,11 @@
 //
 // Per CTA: one tile of 128 query rows of one (batch, head); key tiles of 128.
 //   warp 0      TMA producer: Q once, K/V tiles (+ their scales) into a ring
-//   warp 1      TMEM owner and MMA issuer (one thread): S = Q K^T into a
-//               double-buffered TMEM tile, O += P V into a TMEM accumulator
-//   warps 2-3   idle (they complete the first warpgroup)
+//   warp 1      TMEM owner and S issuer (one thread): S = Q K^T into a
+//               double-buffered TMEM tile, S_{t+2} as soon as S_t has been read
+//   warp 2      PV issuer (one thread): O += P V into a TMEM accumulator once
+//               P_t is written; each issuer commits only its own operations
+//   warp 3      idle (it completes the first warpgroup)
 //   warps 4..11 softmax: one thread per query row and two streams per
 //               32-row quadrant: stream s takes the key tiles t = s mod 2
 //               (S buffer s, P buffer s), so two tiles are in flight on every
@@ -113,8 +115,8 @@ enum : int {
   kBarPFull = kBarSEmpty + 2,
   kBarO = kBarPFull + 2,            // [2]: PV of tile t completes O[t & 1]
   kBarMax = kBarO + 2,              // [4 quadrants][2]: running max of tile t published
-  kBarDrain = kBarMax + 8,
-  kNumBars = kBarDrain + 1
+  kBarDrain = kBarMax + 8,  // [2]: S issuer, PV issuer
+  kNumBars = kBarDrain + 2
 };
 
 constexpr uint32_t kTmemCols = 512;
@@ -155,6 +157,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int s = 0; s < 8; ++s) mbar_init(bar(kBarMax + s), 1);
     mbar_init(bar(kBarDrain), 1);
+    mbar_init(bar(kBarDrain + 1), 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -205,68 +208,72 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                   1024, bar(kBarVFull + st));
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    // Order per tile t: S_{t+2} as soon as the softmax has read S_t out of
-    // TMEM (early in tile t), then PV_t once P_t is written (end of tile t).
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
+    // warp 1 issues S_{t+2} as soon as the softmax has read S_t; warp 2 issues
+    // PV_t once P_t is written. Each commits only its own operations.
     if (lane == 0) {
       constexpr uint32_t kSw = (D == 128) ? 4u : 6u;     // 64- or 32-byte swizzle
       constexpr uint32_t kSboQK = (D == 128) ? 512u : 256u;
       constexpr uint32_t kIdS = idesc_mxf4nvf4(kBM, kBN);
       constexpr uint32_t kIdO = idesc_mxf4nvf4(kBM, D);
       const uint32_t tO = tmem + kColO, tQsf = tmem + kColQsf;
-      auto issue_s = [&](int t) -> bool {
-        const int st = t % kStages;
-        const uint32_t tKsf = tmem + kColKsf + 8 * (t & 1);
-        if (!wait_bar(bar(kBarKFull + st), (t / kStages) & 1)) return false;
-        tc_fence_after();
+      bool ok = true;
+      if (warp == 1) {
+        auto issue_s = [&](int t) -> bool {
+          const int st = t % kStages;
+          const uint32_t tKsf = tmem + kColKsf + 8 * (t & 1);
+          if (!wait_bar(bar(kBarKFull + st), (t / kStages) & 1)) return false;
+          tc_fence_after();
 #pragma unroll
-        for (int kc = 0; kc < D / 64; ++kc)
-          tc_cp_32x128b_x4(tKsf + 4 * kc, smem_desc(sb + L::oKsf + st * 1024 + 512 * kc, 0, 128, 0));
+          for (int kc = 0; kc < D / 64; ++kc)
+            tc_cp_32x128b_x4(tKsf + 4 * kc, smem_desc(sb + L::oKsf + st * 1024 + 512 * kc, 0, 128, 0));
 #pragma unroll
-        for (int kc = 0; kc < D / 64; ++kc)
-          mma_mxf4nvf4(tmem + kColS + (t & 1) * kBN, smem_desc(sb + L::oQ + 32 * kc, 16, kSboQK, kSw),
-                       smem_desc(sb + L::oK + st * L::kK + 32 * kc, 16, kSboQK, kSw), kIdS,
-                       tQsf + 4 * kc, tKsf + 4 * kc, kc > 0 ? 1u : 0u);
-        tc_commit(bar(kBarSFull + (t & 1)));
-        tc_commit(bar(kBarKEmpty + st));
-        return true;
-      };
-      bool ok = wait_bar(bar(kBarQ), 0);
-      if (ok) {
-        tc_fence_after();
+          for (int kc = 0; kc < D / 64; ++kc)
+            mma_mxf4nvf4(tmem + kColS + (t & 1) * kBN, smem_desc(sb + L::oQ + 32 * kc, 16, kSboQK, kSw),
+                         smem_desc(sb + L::oK + st * L::kK + 32 * kc, 16, kSboQK, kSw), kIdS,
+                         tQsf + 4 * kc, tKsf + 4 * kc, kc > 0 ? 1u : 0u);
+          tc_commit(bar(kBarSFull + (t & 1)));
+          tc_commit(bar(kBarKEmpty + st));
+          return true;
+        };
+        ok = wait_bar(bar(kBarQ), 0);
+        if (ok) {
+          tc_fence_after();
 #pragma unroll
-        for (int kc = 0; kc < D / 64; ++kc)
-          tc_cp_32x128b_x4(tQsf + 4 * kc, smem_desc(sb + L::oQsf + 512 * kc, 0, 128, 0));
-        ok = issue_s(0) && (nt < 2 || issue_s(1));
-      }
-      for (int t = 0; ok && t < nt; ++t) {
-        if (t + 2 < nt) {
+          for (int kc = 0; kc < D / 64; ++kc)
+            tc_cp_32x128b_x4(tQsf + 4 * kc, smem_desc(sb + L::oQsf + 512 * kc, 0, 128, 0));
+          ok = issue_s(0) && (nt < 2 || issue_s(1));
+        }
+        for (int t = 0; ok && t + 2 < nt; ++t) {
           if (!(ok = wait_bar(bar(kBarSEmpty + (t & 1)), (t >> 1) & 1))) break;
-          if (!(ok = issue_s(t + 2))) break;
+          ok = issue_s(t + 2);
         }
-        const int st = t % kStages;
-        const uint32_t tPsf = tmem + kColPsf + 8 * (t & 1);
-        const uint32_t tVsf = tmem + kColVsf + 8 * (t & 1);
-        if (!(ok = wait_bar(bar(kBarVFull + st), (t / kStages) & 1))) break;
-        if (!(ok = wait_bar(bar(kBarPFull + (t & 1)), (t >> 1) & 1))) break;
-        tc_fence_after();
+      } else {
+        for (int t = 0; ok && t < nt; ++t) {
+          const int st = t % kStages;
+          const uint32_t tPsf = tmem + kColPsf + 8 * (t & 1);
+          const uint32_t tVsf = tmem + kColVsf + 8 * (t & 1);
+          if (!(ok = wait_bar(bar(kBarVFull + st), (t / kStages) & 1))) break;
+          if (!(ok = wait_bar(bar(kBarPFull + (t & 1)), (t >> 1) & 1))) break;
+          tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          tc_cp_32x128b_x4(tPsf + 4 * c, smem_desc(sb + L::oPsf + (t & 1) * 1024 + 512 * c, 0, 128, 0));
-          tc_cp_32x128b_x4(tVsf + 4 * c, smem_desc(sb + L::oVsf + st * 1024 + 512 * c, 0, 128, 0));
+          for (int c = 0; c < 2; ++c) {
+            tc_cp_32x128b_x4(tPsf + 4 * c, smem_desc(sb + L::oPsf + (t & 1) * 1024 + 512 * c, 0, 128, 0));
+            tc_cp_32x128b_x4(tVsf + 4 * c, smem_desc(sb + L::oVsf + st * 1024 + 512 * c, 0, 128, 0));
+          }
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+            mma_mxf4nvf4(tO, smem_desc(sb + L::oP + (t & 1) * L::kP + 32 * c, 16, 512, 4),
+                         smem_desc(sb + L::oV + st * L::kV + 32 * c, 16, 512, 4), kIdO,
+                         tPsf + 4 * c, tVsf + 4 * c, (t > 0 || c > 0) ? 1u : 0u);
+          tc_commit(bar(kBarO + (t & 1)));
+          tc_commit(bar(kBarVEmpty + st));
         }
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-          mma_mxf4nvf4(tO, smem_desc(sb + L::oP + (t & 1) * L::kP + 32 * c, 16, 512, 4),
-                       smem_desc(sb + L::oV + st * L::kV + 32 * c, 16, 512, 4), kIdO,
-                       tPsf + 4 * c, tVsf + 4 * c, (t > 0 || c > 0) ? 1u : 0u);
-        tc_commit(bar(kBarO + (t & 1)));
-        tc_commit(bar(kBarVEmpty + st));
       }
-      if (!ok) {  // drain whatever was issued before giving up
-        tc_commit(bar(kBarDrain));
-        drain_wait(bar(kBarDrain), 0);
+      if (!ok) {  // drain whatever this issuer issued before giving up
+        tc_commit(bar(kBarDrain + (warp - 1)));
+        drain_wait(bar(kBarDrain + (warp - 1)), 0);
       }
     }
     __syncwarp();
