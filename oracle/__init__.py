@@ -23,6 +23,7 @@ _lib = None
 FLAG_QP_DENOMINATOR = 1
 FLAG_FLIP_BOUND = 2
 FLAG_PERTURB_P = 4
+FLAG_EFQ = 8  # EFQ-Softmax P generation (exp-free), denominator from its p~
 
 
 def build(force: bool = False) -> str:
@@ -64,6 +65,8 @@ def _load():
         lib.ora_quantize_rows.restype = None
         lib.ora_quantize_tokens_T.argtypes = [vp, i32, i32, f32, vp, vp, i32]
         lib.ora_quantize_tokens_T.restype = None
+        lib.ora_efq_block.argtypes = [vp, i32, vp, vp]
+        lib.ora_efq_block.restype = i32
         lib.ora_scores_head.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32]
         lib.ora_scores_head.restype = i32
         lib.ora_attn_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, i32,
@@ -158,6 +161,18 @@ def quantize_tokens_T(x_bf16: np.ndarray, s_enc: float, npad: int | None = None)
     _load().ora_quantize_tokens_T(x.ctypes.data, N, D, float(s_enc), codes.ctypes.data,
                                   scales.ctypes.data, npad)
     return codes, scales
+
+
+def efq_block(z) -> tuple[np.ndarray, int, int | None]:
+    """EFQ-Softmax P of one block: z = n <= 16 shifted scores x - m (float64,
+    -inf for masked keys). Returns (codes, scale byte, E or None when every key
+    is masked); p~ = val(code) * 2^E, stored with P's tensor scale 2^-10."""
+    z = _c(z, np.float64)
+    assert z.size <= 16
+    codes = np.zeros(z.size, dtype=np.uint8)
+    e = ctypes.c_uint8()
+    E = _load().ora_efq_block(z.ctypes.data, z.size, codes.ctypes.data, ctypes.byref(e))
+    return codes, int(e.value), (None if E == -(1 << 31) else int(E))
 
 
 # ----------------------------------------------------------- attention ----

@@ -18,6 +18,10 @@
 //    before the low-bit PV product; the FlashAttention row-maximum update,
 //    historical rescaling, high-precision accumulation and final normalisation
 //    are kept [EFQ-Softmax abstract].
+//  * Flag 8 replaces that path with EFQ-Softmax: E2M1 codes generated straight
+//    from the shifted scores by an exponent-only block scale and one affine
+//    rule, the same operand in numerator and denominator [EFQ-Softmax
+//    abstract]; the reading is at efq_block.
 // The pages give no formula for any of these steps. Where this file fixes one
 // (format constants, scale recipe, rounding, masking, GQA mapping, the
 // denominator) it states the reading it takes.
@@ -266,7 +270,59 @@ KVGroup make_group(const Tensors& T, int b, int hk) {
   return g;
 }
 
-enum { FLAG_QP_DENOMINATOR = 1, FLAG_FLIP_BOUND = 2, FLAG_PERTURB_P = 4 };
+enum { FLAG_QP_DENOMINATOR = 1, FLAG_FLIP_BOUND = 2, FLAG_PERTURB_P = 4, FLAG_EFQ = 8 };
+
+// EFQ-Softmax P generation for one block of n <= 16 keys of one row
+// [EFQ-Softmax abstract, scholarbro.com page "AVQ Attention: Adaptive
+// Vector-Quantized Attention": for each microscaling block, an exponent-only
+// scale chosen from the local maximum, the shifted scores mapped to a
+// normalised residual domain, nonnegative E2M1 codes from a single affine rule;
+// the same operand feeds the numerator and the denominator]. The abstract gives
+// no formula; the reading taken here:
+//   z_u = x_u - m          shifted scores (log2 units, <= 0; -inf when masked)
+//   E = floor(max_u z_u) - 2   exponent-only scale 2^E: the microscaling shared
+//                          exponent, 2 being E2M1's largest exponent
+//   r_u = z_u - E          residual; the block maximum has r in [2, 3)
+//   c_u = min(7, max(0, rne(2 r_u + 2)))   the affine rule: two E2M1 codes per
+//                          binade, code 2 = 1.0, code 4 = 2.0, code 6 = 4.0;
+//                          rne = round half to even
+//   p~_u = val(c_u) 2^E
+// Stored as NVFP4 with P's tensor scale 2^-10 (kEfqScaleExp): the block's scale
+// byte is the E4M3 value 2^(E + 10), exact for E + 10 in [-9, 8]; E <= -2 since
+// z <= 0, and a block with E + 10 < -9 has no such byte and is zero.
+// z is exact in double (fp32 x minus fp32 m). Returns E (INT32_MIN when every
+// key is masked).
+const int kEfqScaleExp = 10;
+
+int efq_block(const double* z, int n, uint8_t* codes, uint8_t* scale) {
+  double b = -INFINITY;
+  for (int u = 0; u < n; ++u) b = std::max(b, z[u]);
+  for (int u = 0; u < n; ++u) codes[u] = 0;
+  *scale = 0;
+  if (b == -INFINITY) return INT32_MIN;
+  const int E = (int)std::floor(b) - 2;
+  if (E + kEfqScaleExp < -9) return E;
+  *scale = e4m3_encode(std::ldexp(1.0f, E + kEfqScaleExp));
+  for (int u = 0; u < n; ++u) {
+    if (z[u] == -INFINITY) continue;
+    double t = std::nearbyint(2.0 * (z[u] - E) + 2.0);  // default rounding: ties to even
+    codes[u] = (uint8_t)std::min(7.0, std::max(0.0, t));
+  }
+  return E;
+}
+
+// The codes of a block for a given E (to evaluate the other rounding of floor).
+void efq_block_with_exp(const double* z, int n, int E, uint8_t* codes, uint8_t* scale) {
+  for (int u = 0; u < n; ++u) codes[u] = 0;
+  *scale = 0;
+  if (E + kEfqScaleExp < -9 || E + kEfqScaleExp > 8) return;
+  *scale = e4m3_encode(std::ldexp(1.0f, E + kEfqScaleExp));
+  for (int u = 0; u < n; ++u) {
+    if (z[u] == -INFINITY) continue;
+    double t = std::nearbyint(2.0 * (z[u] - E) + 2.0);
+    codes[u] = (uint8_t)std::min(7.0, std::max(0.0, t));
+  }
+}
 
 // E2M1 rounding boundaries of |y| between codes c and c+1 (c = 0..6).
 const float kE2M1Mid[7] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.0f};
@@ -286,6 +342,73 @@ uint64_t mix64(uint64_t z) {
   return z ^ (z >> 31);
 }
 
+// EFQ P of one key tile: pq[jj] = val(c) dec(e) per key (units of d_P = 2^-10).
+// Flip bound: t = 2 (x - m - E) + 2 decides the codes, floor(max z) decides E.
+// Another correct fp32 evaluation (S accumulated in another order, t formed as
+// fma(s, 2c, 2 - 2 (m + E)) with one rounding per operation) moves t by at most
+//   2 c u (A_j + A_max) + 2 u |x| + 8 u |m| + 4 u |E| + 10 u,  u = 2^-22
+// (A_j = sum_d |q~_d k~_d| of the key, A_max that of the row maximum); eps_t is
+// four times this. A code whose t lies within eps_t of a rounding point k + 1/2
+// (k = 0..6) may take the neighbouring code; a block whose max z lies within
+// eps_t of an integer may take the other E, except max z = 0 exactly: that block
+// holds the running maximum, and max z = fl(x_max) - m is then exactly 0 in
+// every evaluation that forms it that way. FLAG_PERTURB_P moves each z < 0 by
+// up to eps_t / 8 (seeded by the row) to test the bound.
+void efq_tile(const std::vector<float>& x, const std::vector<double>& A, double amx, float c,
+              double m_new, int Bc, int j0, int j1, int flags, uint64_t rowkey,
+              std::vector<double>& pq, std::vector<double>& dlt, double& epsmax) {
+  const double u = std::ldexp(1.0, -22);
+  std::vector<double> z(Bc), eb(Bc, 0.0);
+  for (int jj = 0; jj < Bc; ++jj) {
+    const bool live = j0 + jj < j1 && x[jj] != -INFINITY;
+    z[jj] = live ? (double)x[jj] - m_new : -INFINITY;
+    dlt[jj] = 0.0;
+    if (live) {
+      eb[jj] = 4.0 * (2.0 * (double)c * u * (A[jj] + amx) + 2.0 * u * std::fabs((double)x[jj]) +
+                      8.0 * u * std::fabs(m_new) + 10.0 * u);
+      if ((flags & FLAG_PERTURB_P) && z[jj] < 0.0) {
+        double uu = (double)(mix64(rowkey ^ mix64((uint64_t)(j0 + jj))) >> 11) *
+                    std::ldexp(1.0, -53);
+        z[jj] = std::min(0.0, z[jj] + (2.0 * uu - 1.0) * eb[jj] / 8.0);
+      }
+    }
+  }
+  for (int b0 = 0; b0 < Bc; b0 += 16) {
+    const int n = std::min(16, Bc - b0);
+    uint8_t codes[16], e;
+    const int E = efq_block(&z[b0], n, codes, &e);
+    for (int k = 0; k < n; ++k) pq[b0 + k] = deq(codes[k], e);
+    if (E == INT32_MIN) continue;
+    const double de = (double)e4m3_decode(e);
+    double ebk = 0.0, b = -INFINITY;
+    for (int k = 0; k < n; ++k) {
+      if (z[b0 + k] == -INFINITY) continue;
+      const double et = eb[b0 + k] + 16.0 * u * std::fabs((double)E);
+      epsmax = std::max(epsmax, et);
+      ebk = std::max(ebk, et);
+      b = std::max(b, z[b0 + k]);
+      if (!(flags & FLAG_FLIP_BOUND)) continue;
+      const double t = 2.0 * (z[b0 + k] - E) + 2.0;
+      for (int k2 = 0; k2 < 7; ++k2)
+        if (std::fabs(t - (k2 + 0.5)) <= et)
+          dlt[b0 + k] = std::max(dlt[b0 + k], (double)(kE2M1Mag[k2 + 1] - kE2M1Mag[k2]) * de);
+    }
+    if (!(flags & FLAG_FLIP_BOUND)) continue;
+    // the other rounding of floor(max z)
+    const double fb = std::floor(b);
+    int other = INT32_MIN;
+    if (b == 0.0) other = INT32_MIN;  // the running maximum's block: exact
+    else if (b - fb <= ebk) other = E - 1;
+    else if (fb + 1.0 - b <= ebk) other = E + 1;
+    if (other != INT32_MIN) {
+      uint8_t alt[16], ealt;
+      efq_block_with_exp(&z[b0], n, other, alt, &ealt);
+      for (int k = 0; k < n; ++k)
+        dlt[b0 + k] = std::max(dlt[b0 + k], std::fabs(deq(alt[k], ealt) - pq[b0 + k]));
+    }
+  }
+}
+
 // One query row: the tiled forward over key tiles of Bc keys.
 //   S_ij = fl32(exact dot product of dequantised q_i, k_j)
 //   x_ij = fl32(S_ij * c), c = fl32(fl32(fl32(d_Q d_K) * softmax_scale) * log2 e)
@@ -297,6 +420,9 @@ uint64_t mix64(uint64_t z) {
 //   p~ = NVFP4(p) per 16 keys with the fixed tensor scale 2688 (p <= 1)
 //   O = alpha O + sum_j p~_ij v~_j   (exact tile product, accumulated in double)
 // out = bf16(fl32(O * fl32(d_P d_V) / l)), d_P = fl32(1 / 2688).
+// With FLAG_EFQ the P block comes from efq_block instead (no exponential of
+// the scores), l sums those p~ (the same operand in numerator and
+// denominator) and d_P = 2^-10.
 //
 // Flip bound (diagnostic, FLAG_FLIP_BOUND): a P code or block scale is a
 // rounding decision; another correct fp32 evaluation of the same row (a
@@ -323,11 +449,14 @@ void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float 
     uint8_t byte = qc[d / 2];
     qd[d] = deq((d & 1) ? (byte >> 4) : (byte & 15), qs[d / 16]);
   }
+  const bool efq = (flags & FLAG_EFQ) != 0;
   float sP, dP;
   tensor_scale(1.0f, &sP, &dP);  // P: a-priori amax 1, so s_enc = 2688
+  if (efq) dP = std::ldexp(1.0f, -kEfqScaleExp);
   std::vector<double> O(D, 0.0), F(D, 0.0);
   std::vector<float> x(Bc), p(Bc);
-  std::vector<double> pq(Bc), A(Bc, 0.0), eps(Bc, 0.0), dlt(Bc, 0.0);
+  std::vector<double> pq(Bc), A(Bc, 0.0), eps(Bc, 0.0), dlt(Bc, 0.0), z(Bc);
+  double Fl = 0.0;  // flip bound of the p~ denominator (EFQ), in units of pq
   double m = -INFINITY, l = 0.0, epsmax = 0.0;
   const int ntiles = (N + Bc - 1) / Bc;
   const uint64_t rowkey = mix64(((uint64_t)b * 65536 + h) * 4294967296ULL + (uint64_t)i);
@@ -357,65 +486,74 @@ void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float 
     }
     double m_new = std::max(m, (double)mt);
     double alpha = (m == -INFINITY) ? 0.0 : std::exp2(m - m_new);
-    for (int jj = 0; jj < Bc; ++jj) {
-      int j = j0 + jj;
-      bool live = j < j1 && x[jj] != -INFINITY;
-      p[jj] = live ? (float)std::exp2((double)x[jj] - m_new) : 0.0f;
-      eps[jj] = 0.0;
-      if (live && want_flip) {
-        const double u = std::ldexp(1.0, -22);
-        eps[jj] = std::log(2.0) * ((double)c * u * (A[jj] + amx) +
-                                   u * (std::fabs((double)x[jj]) + std::fabs(m_new))) +
-                  std::ldexp(1.0, -21);
-        if (flags & FLAG_PERTURB_P) {
-          double uu = (double)(mix64(rowkey ^ mix64((uint64_t)j)) >> 11) * std::ldexp(1.0, -53);
-          p[jj] = (float)((double)p[jj] * (1.0 + (2.0 * uu - 1.0) * eps[jj]));
-        }
-        eps[jj] *= 4.0;
-        epsmax = std::max(epsmax, eps[jj]);
-      }
-    }
-    // P quantisation, blocks of 16 keys from the tile start
-    for (int b0 = 0; b0 < Bc; b0 += 16) {
-      int n = std::min(16, Bc - b0);
-      uint8_t codes[16], e;
-      quantize_block(&p[b0], n, sP, codes, &e);
-      for (int u = 0; u < n; ++u) pq[b0 + u] = deq(codes[u], e);
-      if (!(flags & FLAG_FLIP_BOUND)) continue;
-      const float de = e4m3_decode(e);
-      const float r = (de == 0.0f) ? 0.0f : sP / de;
-      double epsb = 0.0;
-      for (int u = 0; u < n; ++u) {
-        dlt[b0 + u] = 0.0;
-        epsb = std::max(epsb, eps[b0 + u]);
-        float y = std::fabs(p[b0 + u] * r);
-        for (int k2 = 0; k2 < 7; ++k2)
-          if (std::fabs((double)y - kE2M1Mid[k2]) <= eps[b0 + u] * (double)y + 1e-30)
-            dlt[b0 + u] = std::max(dlt[b0 + u],
-                                   (double)(kE2M1Mag[k2 + 1] - kE2M1Mag[k2]) * (double)de);
-      }
-      // the block scale's own rounding
-      float a = 0.0f;
-      for (int u = 0; u < n; ++u) a = std::max(a, std::fabs(p[b0 + u]));
-      float tt = (a / 6.0f) * sP;
-      int other = (tt >= de) ? e + 1 : e - 1;
-      if (a > 0.0f && other >= 0 && other <= 126) {
-        double mid = 0.5 * ((double)de + (double)e4m3_decode((uint8_t)other));
-        if (std::fabs((double)tt - mid) <= epsb * (double)tt + 1e-30) {
-          uint8_t alt[16];
-          quantize_block_with_scale(&p[b0], n, sP, (uint8_t)other, alt);
-          for (int u = 0; u < n; ++u)
-            dlt[b0 + u] = std::max(dlt[b0 + u],
-                                   std::fabs(deq(alt[u], (uint8_t)other) - pq[b0 + u]));
+    if (efq) {
+      efq_tile(x, A, amx, c, m_new, Bc, j0, j1, flags, rowkey, pq, dlt, epsmax);
+    } else {
+      for (int jj = 0; jj < Bc; ++jj) {
+        int j = j0 + jj;
+        bool live = j < j1 && x[jj] != -INFINITY;
+        p[jj] = live ? (float)std::exp2((double)x[jj] - m_new) : 0.0f;
+        eps[jj] = 0.0;
+        if (live && want_flip) {
+          const double u = std::ldexp(1.0, -22);
+          eps[jj] = std::log(2.0) * ((double)c * u * (A[jj] + amx) +
+                                     u * (std::fabs((double)x[jj]) + std::fabs(m_new))) +
+                    std::ldexp(1.0, -21);
+          if (flags & FLAG_PERTURB_P) {
+            double uu = (double)(mix64(rowkey ^ mix64((uint64_t)j)) >> 11) * std::ldexp(1.0, -53);
+            p[jj] = (float)((double)p[jj] * (1.0 + (2.0 * uu - 1.0) * eps[jj]));
+          }
+          eps[jj] *= 4.0;
+          epsmax = std::max(epsmax, eps[jj]);
         }
       }
-    }
-    double lt = 0.0;
-    if (flags & FLAG_QP_DENOMINATOR)
+      // P quantisation, blocks of 16 keys from the tile start
+      for (int b0 = 0; b0 < Bc; b0 += 16) {
+        int n = std::min(16, Bc - b0);
+        uint8_t codes[16], e;
+        quantize_block(&p[b0], n, sP, codes, &e);
+        for (int u = 0; u < n; ++u) pq[b0 + u] = deq(codes[u], e);
+        if (!(flags & FLAG_FLIP_BOUND)) continue;
+        const float de = e4m3_decode(e);
+        const float r = (de == 0.0f) ? 0.0f : sP / de;
+        double epsb = 0.0;
+        for (int u = 0; u < n; ++u) {
+          dlt[b0 + u] = 0.0;
+          epsb = std::max(epsb, eps[b0 + u]);
+          float y = std::fabs(p[b0 + u] * r);
+          for (int k2 = 0; k2 < 7; ++k2)
+            if (std::fabs((double)y - kE2M1Mid[k2]) <= eps[b0 + u] * (double)y + 1e-30)
+              dlt[b0 + u] = std::max(dlt[b0 + u],
+                                     (double)(kE2M1Mag[k2 + 1] - kE2M1Mag[k2]) * (double)de);
+        }
+        // the block scale's own rounding
+        float a = 0.0f;
+        for (int u = 0; u < n; ++u) a = std::max(a, std::fabs(p[b0 + u]));
+        float tt = (a / 6.0f) * sP;
+        int other = (tt >= de) ? e + 1 : e - 1;
+        if (a > 0.0f && other >= 0 && other <= 126) {
+          double mid = 0.5 * ((double)de + (double)e4m3_decode((uint8_t)other));
+          if (std::fabs((double)tt - mid) <= epsb * (double)tt + 1e-30) {
+            uint8_t alt[16];
+            quantize_block_with_scale(&p[b0], n, sP, (uint8_t)other, alt);
+            for (int u = 0; u < n; ++u)
+              dlt[b0 + u] = std::max(dlt[b0 + u],
+                                     std::fabs(deq(alt[u], (uint8_t)other) - pq[b0 + u]));
+          }
+        }
+      }
+    }  // exp-then-quantize
+    double lt = 0.0, flt = 0.0;
+    if (efq) {
+      for (int jj = 0; jj < Bc; ++jj) lt += pq[jj] * (double)dP;
+      if (flags & FLAG_FLIP_BOUND)
+        for (int jj = 0; jj < Bc; ++jj) flt += dlt[jj];
+    } else if (flags & FLAG_QP_DENOMINATOR)
       for (int jj = 0; jj < Bc; ++jj) lt += pq[jj] * (double)dP;
     else
       for (int jj = 0; jj < Bc; ++jj) lt += (double)p[jj];
     l = alpha * l + lt;
+    Fl = alpha * Fl + flt;
     for (int d = 0; d < D; ++d) {
       double acc = 0.0, fl = 0.0;
       for (int j = j0; j < j1; ++j) acc += pq[j - j0] * g.V[(int64_t)j * D + d];
@@ -431,8 +569,14 @@ void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float 
     double y = O[d] * (double)fpv / l;
     if (o_out) o_out[d] = y;
     if (bf_out) bf_out[d] = f32_to_bf16_rne((float)y);
-    // decisions near a boundary, plus the continuous change of l (|dl| <= eps l)
-    if (flip_out) flip_out[d] = F[d] * (double)fpv / l + epsmax * std::fabs(y);
+    // decisions near a boundary, plus the change of l: continuous (|dl| <= eps l)
+    // for the fp32-p denominator; for EFQ's p~ denominator the same flips move
+    // l by up to Fl d_P, so y moves by at most (|dO| + |y| |dl|) / (l - |dl|)
+    if (flip_out) {
+      const double dl = Fl * (double)dP;
+      flip_out[d] = !efq ? F[d] * (double)fpv / l + epsmax * std::fabs(y)
+                    : (l > dl ? (F[d] * (double)fpv + std::fabs(y) * dl) / (l - dl) : INFINITY);
+    }
   }
   if (ml_out) {
     ml_out[0] = m;
@@ -499,6 +643,14 @@ void ora_quantize_tokens_T(const uint16_t* x, int N, int D, float s_enc, uint8_t
   quantize_tokens_T(x, N, D, s_enc, codes, scales, npad);
 }
 
+// EFQ P generation of one block (n <= 16 shifted scores z, -inf when masked):
+// n codes and the scale byte (P tensor scale 2^-10); returns E (INT32_MIN when
+// every key is masked).
+int ora_efq_block(const double* z, int n, uint8_t* codes, uint8_t* scale) {
+  e4m3_encode(0.0f);
+  return efq_block(z, n, codes, scale);
+}
+
 // Unscaled scores of one head: S[i][j] = fl32(exact q~_i . k~_j), contraction
 // units (before d_Q d_K), no mask. S is [N][N].
 int ora_scores_head(const uint16_t* q, const uint16_t* k, int B, int H, int Hkv, int N, int D,
@@ -534,7 +686,8 @@ int ora_scores_head(const uint16_t* q, const uint16_t* k, int B, int H, int Hkv,
 //   uncertainty eps of the row's p (nonzero with flags 2 or 4), may be NULL.
 //   Bc: key tile (128 on the path); flags: 1 = denominator from p~,
 //   2 = flip bound into out_flip ([nrows][D], may be NULL otherwise),
-//   4 = perturb p within the flip bound's uncertainty (tests the bound).
+//   4 = perturb p within the flip bound's uncertainty (tests the bound),
+//   8 = EFQ-Softmax P generation (efq_block), denominator from its p~.
 // Returns 0, or -1 on bad arguments.
 int ora_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H, int Hkv,
                  int N, int D, int causal, float softmax_scale, int Bc, int flags,
