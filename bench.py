@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="video_dit")
     ap.add_argument("--impl", default="fp4attn", choices=["fp4attn", "reference"])
+    ap.add_argument("--variant", default="exp", choices=["exp", "efq"],
+                    help="P generation: exp-then-quantize (the default path) or EFQ-Softmax")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0,
                     help="override H and Hkv (keeping their ratio) for a smaller profiling case")
@@ -212,11 +214,13 @@ def main():
     stream = torch.cuda.current_stream()
     flops = wl.flops
 
+    efq = args.variant == "efq"
+
     def step():
         if world > 1:
-            fa.fp4_attn_fwd_sharded(qf, kf, vf, causal=wl.causal, out=outf)
+            fa.fp4_attn_fwd_sharded(qf, kf, vf, causal=wl.causal, out=outf, efq=efq)
         else:
-            fa.fp4_attn_fwd(q, k, v, causal=wl.causal, out=out, ws=ws)
+            fa.fp4_attn_fwd(q, k, v, causal=wl.causal, out=out, ws=ws, efq=efq)
 
     def barrier():
         if world > 1:
@@ -257,7 +261,8 @@ def main():
     vq = fa.fp4_quantize(v, fa.FP4_BLOCK_ALONG_N_T)
 
     def kernel():
-        fa.fp4_attn_fwd_quantized(qq, kq, vq, wl.B, wl.H, wl.Hkv, causal=wl.causal, out=out)
+        fa.fp4_attn_fwd_quantized(qq, kq, vq, wl.B, wl.H, wl.Hkv, causal=wl.causal, out=out,
+                                  efq=efq)
 
     for _ in range(args.warmup):
         kernel()
@@ -271,11 +276,11 @@ def main():
         if world > 1:
             for d, h in ((q, hq), (k, hk), (v, hv)):
                 d.copy_(h, non_blocking=True)
-            fa.fp4_attn_fwd_sharded(qf, kf, vf, causal=wl.causal, out=outf)
+            fa.fp4_attn_fwd_sharded(qf, kf, vf, causal=wl.causal, out=outf, efq=efq)
             hout.copy_(out, non_blocking=True)
             stream.synchronize()
         else:
-            fa.fp4_attn_fwd_host(hq, hk, hv, causal=wl.causal, out=hout, device=dev)
+            fa.fp4_attn_fwd_host(hq, hk, hv, causal=wl.causal, out=hout, device=dev, efq=efq)
 
     for _ in range(max(1, args.warmup // 2)):
         e2e()
@@ -294,9 +299,9 @@ def main():
     fp4_peak = 4.0 * peaks["bf16_tflops"]  # dense FP4 = 4x dense bf16 (nominal 9 vs 2.25 PF)
     achieved = flops / (k_ms * 1e-3) / 1e12
     traffic = None
-    src = os.path.join(ROOT, "bit_attention_transformers_b200", "csrc", "attn_fwd.cuh")
-    with open(src, "rb") as f:
-        if (wl.name == ATTN_TRAFFIC["workload"] and not args.heads and
+    kernel_src = os.path.join(ROOT, "bit_attention_transformers_b200", "csrc", "attn_fwd.cuh")
+    with open(kernel_src, "rb") as f:
+        if (wl.name == ATTN_TRAFFIC["workload"] and not args.heads and not efq and
                 hashlib.sha256(f.read()).hexdigest() == ATTN_TRAFFIC["attn_fwd_sha256"]):
             traffic = ATTN_TRAFFIC["bytes"]
     line = {
@@ -305,6 +310,7 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
         "data": "synthetic",
         "config": {**wl.describe(),
+                   "p_generation": "EFQ-Softmax" if efq else "exp-then-quantize",
                    "parallelism": (f"heads sharded over {world} ranks ({world} x B*Hkv units, "
                                    "one all-reduce MAX of 3 floats per step)") if world > 1
                    else "1 GPU",

@@ -30,7 +30,8 @@ FP4_BLOCK_ALONG_N_T = 1
 # Every symbol include/fp4attn.h declares.
 EXPORTS = ("fp4_codes_bytes", "fp4_scales_bytes", "fp4_attn_workspace_bytes", "fp4_quantize",
            "fp4_amax", "fp4_quantize_scaled", "fp4_attn_fwd", "fp4_attn_fwd_quantized",
-           "fp4_attn_fwd_noalloc", "fp4_status", "fp4_last_error", "fp4_probe_cvt")
+           "fp4_attn_fwd_efq", "fp4_attn_fwd_quantized_efq", "fp4_attn_fwd_noalloc",
+           "fp4_status", "fp4_last_error", "fp4_probe_cvt")
 FP4_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
@@ -90,6 +91,10 @@ def lib():
         L.fp4_attn_fwd.restype = i32
         L.fp4_attn_fwd_quantized.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
         L.fp4_attn_fwd_quantized.restype = i32
+        L.fp4_attn_fwd_efq.argtypes = L.fp4_attn_fwd.argtypes
+        L.fp4_attn_fwd_efq.restype = i32
+        L.fp4_attn_fwd_quantized_efq.argtypes = L.fp4_attn_fwd_quantized.argtypes
+        L.fp4_attn_fwd_quantized_efq.restype = i32
         L.fp4_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
         L.fp4_attn_fwd_noalloc.restype = i32
         L.fp4_status.argtypes = [vp]
@@ -204,9 +209,10 @@ def workspace(B, H, Hkv, N, D, device):
 
 
 def fp4_attn_fwd(q, k, v, causal: bool = False, softmax_scale: float | None = None, out=None,
-                 stream=None, ws=None):
+                 stream=None, ws=None, efq: bool = False):
     """NVFP4 attention forward. q [B,H,N,D], k/v [B,Hkv,N,D]: contiguous bf16
-    CUDA tensors. Returns out [B,H,N,D] bf16."""
+    CUDA tensors. Returns out [B,H,N,D] bf16. efq=True calls fp4_attn_fwd_efq
+    (P from EFQ-Softmax instead of exp-then-quantize)."""
     import torch
     B, H, N, D = q.shape
     Hkv = k.shape[1]
@@ -217,9 +223,9 @@ def fp4_attn_fwd(q, k, v, causal: bool = False, softmax_scale: float | None = No
         out = torch.empty_like(q)
     if ws is None:
         ws = workspace(B, H, Hkv, N, D, q.device)
-    _check(lib().fp4_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, Hkv, N, D,
-                              int(bool(causal)), float(softmax_scale or 0.0), _stream(stream),
-                              _ptr(ws), ws.numel()))
+    fn = lib().fp4_attn_fwd_efq if efq else lib().fp4_attn_fwd
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, Hkv, N, D, int(bool(causal)),
+              float(softmax_scale or 0.0), _stream(stream), _ptr(ws), ws.numel()))
     return out
 
 
@@ -245,22 +251,22 @@ def fp4_attn_fwd_noalloc(q, k, v, causal: bool = False, softmax_scale: float | N
 
 def fp4_attn_fwd_quantized(qq: Fp4Tensor, kq: Fp4Tensor, vq: Fp4Tensor, B: int, H: int,
                            Hkv: int, causal: bool = False, softmax_scale: float | None = None,
-                           out=None, stream=None):
-    """The fused forward alone on tensors fp4_quantize() produced."""
+                           out=None, stream=None, efq: bool = False):
+    """The fused forward alone on tensors fp4_quantize() produced
+    (fp4_attn_fwd_quantized_efq with efq=True)."""
     import torch
     N, D = qq.N, qq.D
     if out is None:
         out = torch.empty((B, H, N, D), dtype=torch.bfloat16, device=qq.codes.device)
     ts = [_Tensor(t.codes.data_ptr(), t.scales.data_ptr(), t.amax.data_ptr()) for t in (qq, kq, vq)]
-    _check(lib().fp4_attn_fwd_quantized(ctypes.byref(ts[0]), ctypes.byref(ts[1]),
-                                        ctypes.byref(ts[2]), _ptr(out), B, H, Hkv, N, D,
-                                        int(bool(causal)), float(softmax_scale or 0.0),
-                                        _stream(stream)))
+    fn = lib().fp4_attn_fwd_quantized_efq if efq else lib().fp4_attn_fwd_quantized
+    _check(fn(ctypes.byref(ts[0]), ctypes.byref(ts[1]), ctypes.byref(ts[2]), _ptr(out), B, H,
+              Hkv, N, D, int(bool(causal)), float(softmax_scale or 0.0), _stream(stream)))
     return out
 
 
 def fp4_attn_fwd_host(q, k, v, causal: bool = False, softmax_scale: float | None = None,
-                      out=None, device="cuda", stream=None):
+                      out=None, device="cuda", stream=None, efq: bool = False):
     """End-to-end call on host buffers: copies q, k, v (pinned CPU bf16
     tensors) to the device, runs fp4_attn_fwd, copies the output back into
     `out` (a pinned CPU tensor) and returns it once the stream has finished."""
@@ -268,7 +274,7 @@ def fp4_attn_fwd_host(q, k, v, causal: bool = False, softmax_scale: float | None
     dq = q.to(device, non_blocking=True)
     dk = k.to(device, non_blocking=True)
     dv = v.to(device, non_blocking=True)
-    o = fp4_attn_fwd(dq, dk, dv, causal, softmax_scale, stream=stream)
+    o = fp4_attn_fwd(dq, dk, dv, causal, softmax_scale, stream=stream, efq=efq)
     if out is None:
         out = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
     out.copy_(o, non_blocking=True)

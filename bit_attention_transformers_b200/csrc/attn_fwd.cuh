@@ -22,6 +22,18 @@
 //               needs from the one before, passes between the two streams
 //               through shared memory
 // TMEM columns: S0 [0,128) S1 [128,256) O [256,256+D) scales from 384.
+//
+// EFQ variant (template flag EFQ) [EFQ-Softmax abstract]: P is generated
+// without exponentials. Per 16-key block, E = floor(max z) - 2 with z = x - m
+// (max z formed as fl(x_max) - m, exactly 0 in the block of the running
+// maximum); codes clamp(rne(2 (z - E) + 2), 0, 7), computed as
+// rne(7 * sat(s c' + o)) with c' = 2c/7 and o = (2 - 2 (m + E)) / 7: one
+// saturating FMA (the clamp) and one FMA that adds 2^23 (the rounding) per
+// score, the low mantissa bits being the code; scale byte 2^(E + 10) (P's
+// tensor scale 2^-10). The denominator P~1 comes from the tensor cores: two
+// more MMAs per tile multiply P~ by a constant all-ones FP4 tile into 16 TMEM
+// columns beside O (L [256+D, 256+D+16)), so the same rescaling applies to
+// it; the scale columns then start at 400.
 // Every wait is bounded (2 s of %globaltimer); on expiry the kernel sets the
 // device error word, stops issuing, drains its tensor-core work and returns.
 #pragma once
@@ -92,7 +104,9 @@ struct AttnSmem {
   static constexpr int oK = oQ + kQ;
   static constexpr int oV = oK + kStages * kK;
   static constexpr int oP = oV + kStages * kV;
-  static constexpr int oQsf = oP + 2 * kP;
+  static constexpr int oOnes = oP + 2 * kP;     // EFQ: 16 x 128 FP4 ones (code 2), 1 KB
+  static constexpr int oOnesSf = oOnes + 1024;  // EFQ: one scale atom of 1.0 (E4M3 0x38)
+  static constexpr int oQsf = oOnesSf + 512;
   static constexpr int oKsf = oQsf + 1024;
   static constexpr int oVsf = oKsf + kStages * 1024;
   static constexpr int oPsf = oVsf + kStages * 1024;
@@ -120,14 +134,26 @@ enum : int {
 };
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColO = 256, kColQsf = 384, kColKsf = 392, kColPsf = 408,
-                   kColVsf = 424;
+constexpr uint32_t kColS = 0, kColO = 256;
+// Scale-factor columns: after O (at most 128 columns) and, for EFQ, the 16
+// denominator columns beside it.
+template <bool EFQ>
+struct TmemCols {
+  static constexpr uint32_t kSf = EFQ ? 400 : 384;
+  static constexpr uint32_t kQsf = kSf, kKsf = kSf + 8, kPsf = kSf + 24, kVsf = kSf + 40,
+                            kOnesSf = kSf + 56;
+};
+constexpr float kInv7 = 1.0f / 7.0f;
+constexpr float kRound = 8388608.0f;  // 2^23: x + 2^23 rounds x (0 <= x < 2^22) to an integer
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool EFQ>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using L = AttnSmem<D>;
+  using TC = TmemCols<EFQ>;
+  constexpr uint32_t kColQsf = TC::kQsf, kColKsf = TC::kKsf, kColPsf = TC::kPsf,
+                     kColVsf = TC::kVsf, kColL = kColO + D;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -175,6 +201,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t e = threadIdx.x - 64;
     const float de = e4m3_to_f32(e);
     ptab[e] = (e >= 127u || de == 0.0f) ? 0.0f : __fdiv_rn(kTensorRange, de);
+  }
+  if (EFQ && threadIdx.x >= 192 && threadIdx.x < 288) {
+    // the all-ones B operand of P~1 (every code 2 = 1.0) and its scales (1.0)
+    const int i = threadIdx.x - 192;  // 96 threads x 16 bytes = 1536 bytes
+    *reinterpret_cast<uint4*>(sm + L::oOnes + 16 * i) =
+        i < 64 ? make_uint4(0x22222222u, 0x22222222u, 0x22222222u, 0x22222222u)
+               : make_uint4(0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -250,6 +284,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           ok = issue_s(t + 2);
         }
       } else {
+        if (EFQ) tc_cp_32x128b_x4(tmem + TC::kOnesSf, smem_desc(sb + L::oOnesSf, 0, 128, 0));
         for (int t = 0; ok && t < nt; ++t) {
           const int st = t % kStages;
           const uint32_t tPsf = tmem + kColPsf + 8 * (t & 1);
@@ -267,6 +302,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mma_mxf4nvf4(tO, smem_desc(sb + L::oP + (t & 1) * L::kP + 32 * c, 16, 512, 4),
                          smem_desc(sb + L::oV + st * L::kV + 32 * c, 16, 512, 4), kIdO,
                          tPsf + 4 * c, tVsf + 4 * c, (t > 0 || c > 0) ? 1u : 0u);
+          if (EFQ) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              mma_mxf4nvf4(tmem + kColL, smem_desc(sb + L::oP + (t & 1) * L::kP + 32 * c, 16, 512, 4),
+                           smem_desc(sb + L::oOnes + 32 * c, 16, 512, 4), idesc_mxf4nvf4(kBM, 16),
+                           tPsf + 4 * c, tmem + TC::kOnesSf, (t > 0 || c > 0) ? 1u : 0u);
+          }
           tc_commit(bar(kBarO + (t & 1)));
           tc_commit(bar(kBarVEmpty + st));
         }
@@ -294,6 +336,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const float c = __fmul_rn(__fmul_rn(__fmul_rn(dq, dk), p.softmax_scale), kLog2e);
     const float fpv = __fmul_rn(__fdiv_rn(1.0f, kTensorRange), dv);  // d_P * d_V
     const uint64_t c2 = pk(c, c);
+    const float c27 = __fdiv_rn(__fmul_rn(2.0f, c), 7.0f);  // EFQ: slope of the affine rule / 7
     float m_own = -INFINITY;   // running max after this stream's previous tile
     float m_last = -INFINITY;  // running max after the last tile processed
     float l = 0.0f;            // this stream's row sum, relative to m_own
@@ -346,34 +389,73 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float alpha = (m_prev == -INFINITY) ? 0.0f : ex2_approx(m_prev - m_new);
       const float neg_m = (m_new == -INFINITY) ? 0.0f : -m_new;
       const uint64_t nm2 = pk(neg_m, neg_m);
-      // P -> NVFP4 per 16 keys with the fixed tensor scale 2688 (p <= 1):
-      // p = 2^(x - m) in fp32, block scale e = E4M3(448 a_b) with
-      // a_b = 2^(max_b - m), codes E2M1(p r) with r = 2688 / dec(e)
       uint32_t pc[16];
       uint32_t sfw[2] = {0u, 0u};
       float lsum = 0.0f;
+      if constexpr (EFQ) {
+        // EFQ-Softmax: per block, E = floor(max z) - 2 and scale byte 2^(E + 10);
+        // per score, code = rne(7 sat((2 (z - E) + 2) / 7)) from the bits of
+        // fma(sat(s c' + o), 7, 2^23); eight codes per word by shift-and-add
+        // (the eight 2^23 exponents leave the constant 0xFB000000 behind)
 #pragma unroll
-      for (int bk = 0; bk < 8; ++bk) {
-        const float a = ex2_approx(fmaf(bm[bk], c, neg_m));
-        const uint32_t e = cvt_e4m3(__fmul_rn(a, 448.0f));
-        const float r = ptab[e];
-        const uint64_t r2 = pk(r, r);
-        float y[16];
-        uint64_t acc = 0;
+        for (int bk = 0; bk < 8; ++bk) {
+          const float bz = __fsub_rn(__fmul_rn(bm[bk], c), m_new);  // max z of the block
+          uint32_t e = 0u;
+          float o7 = 0.0f;
+          if (bz > -INFINITY) {
+            const float Ef = floorf(bz) - 2.0f;
+            const int k = __float2int_rz(Ef) + 10;
+            e = k >= -6 ? (uint32_t)(k + 7) << 3 : (k >= -9 ? 1u << (k + 9) : 0u);
+            o7 = __fmul_rn(fmaf(-2.0f, __fadd_rn(m_new, Ef), 2.0f), kInv7);
+          }
+          const uint64_t r2 = pk(kRound, kRound);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float u0, u1;
-          upk(fma2(pk(s[16 * bk + 2 * i], s[16 * bk + 2 * i + 1]), c2, nm2), u0, u1);
-          const uint64_t pp = pk(ex2_approx(u0), ex2_approx(u1));
-          acc = (i == 0) ? pp : add2(acc, pp);
-          upk(mul2(pp, r2), y[2 * i], y[2 * i + 1]);
+          for (int h8 = 0; h8 < 2; ++h8) {
+            uint32_t f[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int j = 16 * bk + 8 * h8 + 2 * i;
+              const float t0 = fma_sat(s[j], c27, o7), t1 = fma_sat(s[j + 1], c27, o7);
+              float f0, f1;
+              upk(fma2(pk(t0, t1), pk(7.0f, 7.0f), r2), f0, f1);
+              f[2 * i] = __float_as_uint(f0);
+              f[2 * i + 1] = __float_as_uint(f1);
+            }
+            uint32_t w = f[7];
+#pragma unroll
+            for (int i = 6; i >= 0; --i) w = (w << 4) + f[i];
+            pc[2 * bk + h8] = w - 0xFB000000u;
+          }
+          sfw[bk >> 2] |= e << (8 * (bk & 3));
         }
-        float a0, a1;
-        upk(acc, a0, a1);
-        lsum += a0 + a1;
-        pc[2 * bk] = cvt_e2m1x8(y);
-        pc[2 * bk + 1] = cvt_e2m1x8(y + 8);
-        sfw[bk >> 2] |= e << (8 * (bk & 3));
+      } else {
+        // P -> NVFP4 per 16 keys with the fixed tensor scale 2688 (p <= 1):
+        // p = 2^(x - m) in fp32, block scale e = E4M3(448 a_b) with
+        // a_b = 2^(max_b - m), codes E2M1(p r) with r = 2688 / dec(e)
+#pragma unroll
+        for (int bk = 0; bk < 8; ++bk) {
+          const float a = ex2_approx(fmaf(bm[bk], c, neg_m));
+          const uint32_t e = cvt_e4m3(__fmul_rn(a, 448.0f));
+          const float r = ptab[e];
+          const uint64_t r2 = pk(r, r);
+          float y[16];
+          uint64_t acc = 0;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float u0, u1;
+            upk(fma2(pk(s[16 * bk + 2 * i], s[16 * bk + 2 * i + 1]), c2, nm2), u0, u1);
+            const uint64_t pp = pk(ex2_approx(u0), ex2_approx(u1));
+            acc = (i == 0) ? pp : add2(acc, pp);
+            upk(mul2(pp, r2), y[2 * i], y[2 * i + 1]);
+          }
+          float a0, a1;
+          upk(acc, a0, a1);
+          lsum += a0 + a1;
+          pc[2 * bk] = cvt_e2m1x8(y);
+          pc[2 * bk + 1] = cvt_e2m1x8(y + 8);
+          sfw[bk >> 2] |= e << (8 * (bk & 3));
+        }
+
       }
       // this stream's sum, carried to the new running max
       l = (m_own == -INFINITY) ? lsum : fmaf(l, ex2_approx(m_own - m_new), lsum);
@@ -391,7 +473,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_after();
         const uint64_t al2 = pk(alpha, alpha);
 #pragma unroll
-        for (int cc = 0; cc < D; cc += 16) {
+        for (int cc = 0; cc < D + (EFQ ? 16 : 0); cc += 16) {
           float o[16];
           const uint32_t ta = tl + kColO + cc;
           tmem_ld16(ta, o);
@@ -428,8 +510,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     fail = bar_red_or(1 + quad, 64, !ok);
     if (!fail) {
       tc_fence_after();
-      const float ltot = lval[row] + lval[kBM + row];
-      const float inv = __fdiv_rn(fpv, ltot);
+      float inv;
+      if constexpr (EFQ) {
+        // P~1 accumulated beside O in the same units: out = O d_V / (P~1)
+        float lq[16];
+        tmem_ld16(tl + kColL, lq);
+        tmem_wait_ld();
+        inv = __fdiv_rn(dv, lq[0]);
+      } else {
+        inv = __fdiv_rn(fpv, lval[row] + lval[kBM + row]);
+      }
       constexpr int DH = D / 2;             // each stream writes half the channels
       __nv_bfloat16* dst = p.out + ((int64_t)gq * p.N + qrow) * D + stream * DH;
 #pragma unroll

@@ -52,9 +52,15 @@ using AttnKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensor
                             const fp4::AttnParams);
 
 // The fused kernel for head dim D and causal masking.
-AttnKernel attn_kernel(int D, int causal) {
-  if (D == 128) return causal ? fp4::attn_fwd_kernel<128, true> : fp4::attn_fwd_kernel<128, false>;
-  return causal ? fp4::attn_fwd_kernel<64, true> : fp4::attn_fwd_kernel<64, false>;
+AttnKernel attn_kernel(int D, int causal, int efq) {
+  if (efq) {
+    if (D == 128)
+      return causal ? fp4::attn_fwd_kernel<128, true, true> : fp4::attn_fwd_kernel<128, false, true>;
+    return causal ? fp4::attn_fwd_kernel<64, true, true> : fp4::attn_fwd_kernel<64, false, true>;
+  }
+  if (D == 128)
+    return causal ? fp4::attn_fwd_kernel<128, true, false> : fp4::attn_fwd_kernel<128, false, false>;
+  return causal ? fp4::attn_fwd_kernel<64, true, false> : fp4::attn_fwd_kernel<64, false, false>;
 }
 
 // sm_100 check, per-device one-time kernel attributes, SM count.
@@ -73,9 +79,10 @@ fp4_status_t device_setup(int* dev_out, int* sms_out) {
                   dev, major, minor);
     for (int d = 0; d < 2; ++d)
       for (int causal = 0; causal < 2; ++causal)
-        FP4_CUDA(cudaFuncSetAttribute(attn_kernel(d ? 128 : 64, causal),
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      d ? fp4::AttnSmem<128>::kBytes : fp4::AttnSmem<64>::kBytes));
+        for (int efq = 0; efq < 2; ++efq)
+          FP4_CUDA(cudaFuncSetAttribute(attn_kernel(d ? 128 : 64, causal, efq),
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        d ? fp4::AttnSmem<128>::kBytes : fp4::AttnSmem<64>::kBytes));
     if (!g_encode) {
       cudaDriverEntryPointQueryResult q;
       void* fn = nullptr;
@@ -196,7 +203,7 @@ fp4_status_t launch_quant(const void* x, int64_t G, int N, int D, fp4_axis_t axi
 fp4_status_t launch_attn(const uint8_t* qc, const uint8_t* qs, const float* qa, const uint8_t* kc,
                          const uint8_t* ks, const float* ka, const uint8_t* vc, const uint8_t* vs,
                          const float* va, void* out, int B, int H, int Hkv, int N, int D,
-                         int causal, float softmax_scale, cudaStream_t stream) {
+                         int causal, float softmax_scale, int efq, cudaStream_t stream) {
   const int64_t Npad = round_up(N, 128);
   const int64_t Gq = (int64_t)B * H, Gk = (int64_t)B * Hkv;
   const CUtensorMapSwizzle swQK =
@@ -225,9 +232,65 @@ fp4_status_t launch_attn(const uint8_t* qc, const uint8_t* qs, const float* qa, 
                         : 1.0f / std::sqrt((float)D);
   dim3 grid(p.ntq, H, B);
   const int smem = D == 128 ? fp4::AttnSmem<128>::kBytes : fp4::AttnSmem<64>::kBytes;
-  attn_kernel(D, causal)<<<grid, fp4::kAttnThreads, smem, stream>>>(tq, tk, tv, p);
+  attn_kernel(D, causal, efq)<<<grid, fp4::kAttnThreads, smem, stream>>>(tq, tk, tv, p);
   FP4_CUDA(cudaGetLastError());
   return FP4_OK;
+}
+
+fp4_status_t attn_fwd_any(const void* q, const void* k, const void* v, void* out, int B, int H,
+                          int Hkv, int N, int D, int causal, float softmax_scale, void* stream,
+                          void* workspace, size_t workspace_bytes, int efq) {
+  g_last_error.clear();
+  fp4_status_t s;
+  if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
+  if (!q || !k || !v || !out || !workspace) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace))
+    return fail(FP4_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const WsLayout w = ws_layout(B, H, Hkv, N, D);
+  if (workspace_bytes < w.total)
+    return fail(FP4_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, w.total);
+  int dev, sms;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* amax = reinterpret_cast<float*>(ws + w.amax);
+  const int64_t nq = (int64_t)B * H * N * D, nkv = (int64_t)B * Hkv * N * D;
+  if ((s = launch_amax(q, nq, k, nkv, v, nkv, amax, amax + 1, amax + 2, sms, st)) != FP4_OK)
+    return s;
+  if ((s = launch_quant(q, (int64_t)B * H, N, D, FP4_BLOCK_ALONG_D, ws + w.qc, ws + w.qs, amax,
+                        sms, st)) != FP4_OK)
+    return s;
+  if ((s = launch_quant(k, (int64_t)B * Hkv, N, D, FP4_BLOCK_ALONG_D, ws + w.kc, ws + w.ks,
+                        amax + 1, sms, st)) != FP4_OK)
+    return s;
+  if ((s = launch_quant(v, (int64_t)B * Hkv, N, D, FP4_BLOCK_ALONG_N_T, ws + w.vc, ws + w.vs,
+                        amax + 2, sms, st)) != FP4_OK)
+    return s;
+  return launch_attn(ws + w.qc, ws + w.qs, amax, ws + w.kc, ws + w.ks, amax + 1, ws + w.vc,
+                     ws + w.vs, amax + 2, out, B, H, Hkv, N, D, causal, softmax_scale, efq, st);
+}
+
+fp4_status_t attn_fwd_quantized_any(const fp4_tensor_t* q, const fp4_tensor_t* k,
+                                    const fp4_tensor_t* v, void* out, int B, int H, int Hkv,
+                                    int N, int D, int causal, float softmax_scale, void* stream,
+                                    int efq) {
+  g_last_error.clear();
+  fp4_status_t s;
+  if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
+  if (!q || !k || !v || !out) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  const fp4_tensor_t* t[3] = {q, k, v};
+  for (auto* x : t) {
+    if (!x->codes || !x->scales || !x->amax) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(x->codes) || !aligned16(x->scales) ||
+        (reinterpret_cast<uintptr_t>(x->amax) & 3u))
+      return fail(FP4_ERR_INVALID_ARG, "codes/scales must be 16-byte aligned");
+  }
+  if (!aligned16(out)) return fail(FP4_ERR_INVALID_ARG, "out must be 16-byte aligned");
+  int dev, sms;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  return launch_attn(q->codes, q->scales, q->amax, k->codes, k->scales, k->amax, v->codes,
+                     v->scales, v->amax, out, B, H, Hkv, N, D, causal, softmax_scale, efq,
+                     static_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -303,57 +366,31 @@ fp4_status_t fp4_quantize_scaled(const void* x, int G, int N, int D, fp4_axis_t 
 fp4_status_t fp4_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int H,
                           int Hkv, int N, int D, int causal, float softmax_scale, void* stream,
                           void* workspace, size_t workspace_bytes) {
-  g_last_error.clear();
-  fp4_status_t s;
-  if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
-  if (!q || !k || !v || !out || !workspace) return fail(FP4_ERR_INVALID_ARG, "null pointer");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace))
-    return fail(FP4_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
-  const WsLayout w = ws_layout(B, H, Hkv, N, D);
-  if (workspace_bytes < w.total)
-    return fail(FP4_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, w.total);
-  int dev, sms;
-  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* amax = reinterpret_cast<float*>(ws + w.amax);
-  const int64_t nq = (int64_t)B * H * N * D, nkv = (int64_t)B * Hkv * N * D;
-  if ((s = launch_amax(q, nq, k, nkv, v, nkv, amax, amax + 1, amax + 2, sms, st)) != FP4_OK)
-    return s;
-  if ((s = launch_quant(q, (int64_t)B * H, N, D, FP4_BLOCK_ALONG_D, ws + w.qc, ws + w.qs, amax,
-                        sms, st)) != FP4_OK)
-    return s;
-  if ((s = launch_quant(k, (int64_t)B * Hkv, N, D, FP4_BLOCK_ALONG_D, ws + w.kc, ws + w.ks,
-                        amax + 1, sms, st)) != FP4_OK)
-    return s;
-  if ((s = launch_quant(v, (int64_t)B * Hkv, N, D, FP4_BLOCK_ALONG_N_T, ws + w.vc, ws + w.vs,
-                        amax + 2, sms, st)) != FP4_OK)
-    return s;
-  return launch_attn(ws + w.qc, ws + w.qs, amax, ws + w.kc, ws + w.ks, amax + 1, ws + w.vc,
-                     ws + w.vs, amax + 2, out, B, H, Hkv, N, D, causal, softmax_scale, st);
+  return attn_fwd_any(q, k, v, out, B, H, Hkv, N, D, causal, softmax_scale, stream, workspace,
+                      workspace_bytes, 0);
+}
+
+fp4_status_t fp4_attn_fwd_efq(const void* q, const void* k, const void* v, void* out, int B,
+                              int H, int Hkv, int N, int D, int causal, float softmax_scale,
+                              void* stream, void* workspace, size_t workspace_bytes) {
+  return attn_fwd_any(q, k, v, out, B, H, Hkv, N, D, causal, softmax_scale, stream, workspace,
+                      workspace_bytes, 1);
 }
 
 fp4_status_t fp4_attn_fwd_quantized(const fp4_tensor_t* q, const fp4_tensor_t* k,
                                     const fp4_tensor_t* v, void* out, int B, int H, int Hkv,
                                     int N, int D, int causal, float softmax_scale, void* stream) {
-  g_last_error.clear();
-  fp4_status_t s;
-  if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
-  if (!q || !k || !v || !out) return fail(FP4_ERR_INVALID_ARG, "null pointer");
-  const fp4_tensor_t* t[3] = {q, k, v};
-  for (auto* x : t) {
-    if (!x->codes || !x->scales || !x->amax) return fail(FP4_ERR_INVALID_ARG, "null pointer");
-    if (!aligned16(x->codes) || !aligned16(x->scales) ||
-        (reinterpret_cast<uintptr_t>(x->amax) & 3u))
-      return fail(FP4_ERR_INVALID_ARG, "codes/scales must be 16-byte aligned");
-  }
-  if (!aligned16(out)) return fail(FP4_ERR_INVALID_ARG, "out must be 16-byte aligned");
-  int dev, sms;
-  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
-  return launch_attn(q->codes, q->scales, q->amax, k->codes, k->scales, k->amax, v->codes,
-                     v->scales, v->amax, out, B, H, Hkv, N, D, causal, softmax_scale,
-                     static_cast<cudaStream_t>(stream));
+  return attn_fwd_quantized_any(q, k, v, out, B, H, Hkv, N, D, causal, softmax_scale, stream, 0);
 }
+
+fp4_status_t fp4_attn_fwd_quantized_efq(const fp4_tensor_t* q, const fp4_tensor_t* k,
+                                        const fp4_tensor_t* v, void* out, int B, int H, int Hkv,
+                                        int N, int D, int causal, float softmax_scale,
+                                        void* stream) {
+  return attn_fwd_quantized_any(q, k, v, out, B, H, Hkv, N, D, causal, softmax_scale, stream, 1);
+}
+
+
 
 // Scratch for fp4_attn_fwd_noalloc: reserved in every GPU's copy of this
 // module; its device address is looked up once per device.

@@ -55,7 +55,7 @@ def allreduce_max_(t, group=None):
 
 
 def fp4_attn_fwd_sharded(q, k, v, causal: bool = False, softmax_scale: float | None = None,
-                         group=None, out=None, stream=None):
+                         group=None, out=None, stream=None, efq: bool = False):
     """This rank's part of a head-sharded NVFP4 attention forward.
 
     q: this rank's query heads, a contiguous bf16 CUDA tensor [..., N, D] whose
@@ -63,7 +63,7 @@ def fp4_attn_fwd_sharded(q, k, v, causal: bool = False, softmax_scale: float | N
     heads, [..., N, D]. Every rank of `group` calls this with the same N, D,
     G, causal and softmax_scale, an empty shard (U = 0) included: it still
     takes part in the all-reduce. Returns `out` (like q) with this rank's
-    output heads."""
+    output heads. efq selects the EFQ-Softmax P generation."""
     import torch
     from . import (FP4_BLOCK_ALONG_D, FP4_BLOCK_ALONG_N_T, fp4_amax, fp4_attn_fwd_quantized,
                    fp4_quantize)
@@ -86,5 +86,6 @@ def fp4_attn_fwd_sharded(q, k, v, causal: bool = False, softmax_scale: float | N
     qq = fp4_quantize(q, FP4_BLOCK_ALONG_D, stream, amax=amax[0:1])
     kq = fp4_quantize(k, FP4_BLOCK_ALONG_D, stream, amax=amax[1:2])
     vq = fp4_quantize(v, FP4_BLOCK_ALONG_N_T, stream, amax=amax[2:3])
-    fp4_attn_fwd_quantized(qq, kq, vq, 1, gq, gkv, causal, softmax_scale, out=out, stream=stream)
+    fp4_attn_fwd_quantized(qq, kq, vq, 1, gq, gkv, causal, softmax_scale, out=out, stream=stream,
+                           efq=efq)
     return out

@@ -152,6 +152,30 @@ fp4_status_t fp4_attn_fwd_quantized(const fp4_tensor_t* q, const fp4_tensor_t* k
                                     int N, int D, int causal, float softmax_scale, void* stream);
 
 /*
+ * The EFQ-Softmax variant of fp4_attn_fwd / fp4_attn_fwd_quantized (same
+ * arguments, layouts and errors). P is generated without exponentials
+ * (EFQ-Softmax abstract, scholarbro.com page "AVQ Attention: Adaptive
+ * Vector-Quantized Attention": an exponent-only scale per microscaling block
+ * chosen from the local maximum, the shifted scores mapped to a residual
+ * domain, nonnegative E2M1 codes from a single affine rule, and the same
+ * operand in the numerator P~V and the denominator P~1). The abstract gives no
+ * formula; the reading implemented, per 16-key block of a row with
+ * z = x - m (log2 units) and the running maximum m updated as above:
+ *   E = floor(max z) - 2            (shared exponent; 2 = E2M1's largest)
+ *   code = clamp(rne(2 (z - E) + 2), 0, 7)   (rne: round half to even)
+ *   p~ = val(code) * 2^E            (block scale byte 2^(E + 10), P's tensor
+ *                                     scale 2^-10; a block with E < -19 is zero)
+ *   l = alpha l + sum_j p~_j,  out = O / l  (O and l both from p~).
+ */
+fp4_status_t fp4_attn_fwd_efq(const void* q, const void* k, const void* v, void* out, int B,
+                              int H, int Hkv, int N, int D, int causal, float softmax_scale,
+                              void* stream, void* workspace, size_t workspace_bytes);
+fp4_status_t fp4_attn_fwd_quantized_efq(const fp4_tensor_t* q, const fp4_tensor_t* k,
+                                        const fp4_tensor_t* v, void* out, int B, int H, int Hkv,
+                                        int N, int D, int causal, float softmax_scale,
+                                        void* stream);
+
+/*
  * fp4_attn_fwd without a caller-supplied workspace, for callers that cannot
  * allocate device memory: code whose device memory is owned by a host
  * framework that hands it no allocator, or code that must not call

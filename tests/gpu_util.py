@@ -36,10 +36,10 @@ def scales_tokens_logical(native: np.ndarray, G: int, N: int, D: int):
     return full[:, :D, :], full[:, D:, :]
 
 
-def run_attn(q, k, v, causal: bool, softmax_scale: float = 0.0) -> np.ndarray:
+def run_attn(q, k, v, causal: bool, softmax_scale: float = 0.0, efq: bool = False) -> np.ndarray:
     import torch
     out = fa.fp4_attn_fwd(to_dev(q), to_dev(k), to_dev(v), causal=causal,
-                          softmax_scale=softmax_scale or None)
+                          softmax_scale=softmax_scale or None, efq=efq)
     torch.cuda.synchronize()
     fa.fp4_status()
     return from_dev(out)
