@@ -35,8 +35,8 @@ L2_BYTES = 126 * 1024 * 1024
 # workload, from ncu (dram__bytes_read.sum + dram__bytes_write.sum, one pass;
 # profiles/attn_fwd_traffic_video_dit.md). They hold only for the kernel source
 # they were taken on, identified by its hash; otherwise traffic is reported null.
-ATTN_TRAFFIC = {"workload": "video_dit", "bytes": 171.07e6 + 156.07e6,
-                "attn_fwd_sha256": "d118fd94ac8b00d407f1fc48af0930efaea761c8d965698189cf2efe43f09bfd"}
+ATTN_TRAFFIC = {"workload": "video_dit", "bytes": 170.08e6 + 155.86e6,
+                "attn_fwd_sha256": "d1f520670fe34a2b5a5f613a5ed9f996b304785a670cef48f4dabe1994c93bd4"}
 
 
 def parse():

@@ -31,7 +31,7 @@ FP4_BLOCK_ALONG_N_T = 1
 EXPORTS = ("fp4_codes_bytes", "fp4_scales_bytes", "fp4_attn_workspace_bytes", "fp4_quantize",
            "fp4_amax", "fp4_quantize_scaled", "fp4_attn_fwd", "fp4_attn_fwd_quantized",
            "fp4_attn_fwd_efq", "fp4_attn_fwd_quantized_efq", "fp4_attn_fwd_noalloc",
-           "fp4_status", "fp4_last_error", "fp4_probe_cvt")
+           "fp4_status", "fp4_last_error", "fp4_probe_cvt", "fp4_test_wait_timeout")
 FP4_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
@@ -103,6 +103,8 @@ def lib():
         L.fp4_last_error.restype = ctypes.c_char_p
         L.fp4_probe_cvt.argtypes = [u32, i64, i32, vp, vp]
         L.fp4_probe_cvt.restype = i32
+        L.fp4_test_wait_timeout.argtypes = [ctypes.c_uint64, vp, vp]
+        L.fp4_test_wait_timeout.restype = i32
         _lib = L
     return _lib
 
@@ -285,6 +287,16 @@ def fp4_attn_fwd_host(q, k, v, causal: bool = False, softmax_scale: float | None
 def fp4_status(stream=None):
     """Synchronise and raise if a kernel reported an expired wait."""
     _check(lib().fp4_status(_stream(stream)))
+
+
+def fp4_test_wait_timeout(limit_ns: int, stream=None):
+    """Test support: a bounded wait that nothing ends; returns the device int
+    that receives 0 once the wait has expired (the next fp4_status raises
+    FP4_ERR_TIMEOUT)."""
+    import torch
+    ok = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    _check(lib().fp4_test_wait_timeout(int(limit_ns), _ptr(ok), _stream(stream)))
+    return ok
 
 
 def fp4_probe_cvt(start: int, count: int, kind: int, out=None, stream=None):

@@ -61,12 +61,13 @@ enum : unsigned { kDevErrTimeout = 1u };
 // Device error word (one per device); read and cleared by fp4_status().
 __device__ unsigned g_fp4_err;
 
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity,
+                                         uint64_t limit_ns = kTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (*reinterpret_cast<volatile unsigned*>(&g_fp4_err) != 0u) return false;
-    if (globaltimer_ns() - t0 > kTimeoutNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       atomicOr(&g_fp4_err, kDevErrTimeout);
       return false;
     }
@@ -79,6 +80,18 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity))
     if (globaltimer_ns() - t0 > kTimeoutNs / 20) return;
+}
+
+// Test support: one thread waits, with the kernels' bounded wait and the given
+// limit, on an mbarrier that nothing arrives on; the wait expires, sets the
+// device error word and returns. *ok receives 0 (expired) or 1.
+__global__ void wait_timeout_kernel(uint64_t limit_ns, int* ok) {
+  __shared__ uint64_t b;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&b), 1);
+    fence_mbar_init();
+    *ok = wait_bar(smem_u32(&b), 0, limit_ns) ? 1 : 0;
+  }
 }
 
 struct AttnParams {

@@ -459,4 +459,16 @@ fp4_status_t fp4_probe_cvt(uint32_t start, int64_t count, int kind, uint8_t* out
   return FP4_OK;
 }
 
+fp4_status_t fp4_test_wait_timeout(uint64_t limit_ns, int* ok, void* stream) {
+  g_last_error.clear();
+  if (limit_ns == 0 || limit_ns > 5000000000ull || !ok)
+    return fail(FP4_ERR_INVALID_ARG, "limit must be in (0, 5 s] and ok non-null");
+  int dev, sms;
+  fp4_status_t s;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  fp4::wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, ok);
+  FP4_CUDA(cudaGetLastError());
+  return FP4_OK;
+}
+
 }  // extern "C"

@@ -214,6 +214,17 @@ const char* fp4_last_error(void);
  */
 fp4_status_t fp4_probe_cvt(uint32_t start, int64_t count, int kind, uint8_t* out, void* stream);
 
+/*
+ * Test support for failure detection: launches one thread that waits, with
+ * the same bounded wait the attention kernel uses and a limit of limit_ns
+ * (0 < limit_ns <= 5 s), on an mbarrier that nothing arrives on. The wait
+ * expires and sets the device error word, so the next fp4_status() returns
+ * FP4_ERR_TIMEOUT; *ok (device int) receives 0. Nothing faults or hangs, and
+ * the context stays usable. The pages have no counterpart; this exists so
+ * the timeout path can be exercised without breaking a real kernel.
+ */
+fp4_status_t fp4_test_wait_timeout(uint64_t limit_ns, int* ok, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
