@@ -29,7 +29,8 @@ FP4_BLOCK_ALONG_N_T = 1
 
 # Every symbol include/fp4attn.h declares.
 EXPORTS = ("fp4_codes_bytes", "fp4_scales_bytes", "fp4_attn_workspace_bytes", "fp4_quantize",
-           "fp4_amax", "fp4_quantize_scaled", "fp4_attn_fwd", "fp4_attn_fwd_quantized",
+           "fp4_amax", "fp4_quantize_scaled", "fp4_scales_to_canonical", "fp4_attn_fwd",
+           "fp4_attn_fwd_quantized",
            "fp4_attn_fwd_efq", "fp4_attn_fwd_quantized_efq", "fp4_attn_fwd_noalloc",
            "fp4_status", "fp4_last_error", "fp4_probe_cvt", "fp4_test_wait_timeout")
 FP4_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -87,6 +88,8 @@ def lib():
         L.fp4_amax.restype = i32
         L.fp4_quantize_scaled.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp]
         L.fp4_quantize_scaled.restype = i32
+        L.fp4_scales_to_canonical.argtypes = [vp, i32, i32, i32, i32, vp, vp]
+        L.fp4_scales_to_canonical.restype = i32
         L.fp4_attn_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, sz]
         L.fp4_attn_fwd.restype = i32
         L.fp4_attn_fwd_quantized.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
@@ -182,6 +185,18 @@ def fp4_quantize(x, axis: int = FP4_BLOCK_ALONG_D, stream=None, amax=None) -> Fp
         _check(lib().fp4_quantize_scaled(_ptr(x), G, N, D, axis, _ptr(amax), _ptr(codes),
                                          _ptr(scales), _stream(stream)))
     return Fp4Tensor(codes, scales, amax, G, N, D, axis)
+
+
+def fp4_scales_to_canonical(t: Fp4Tensor, stream=None):
+    """t's block scales in their logical layout: [G][N][D/16] (blocks along D)
+    or [G][D][Npad/16] (blocks along tokens), a uint8 CUDA tensor."""
+    import torch
+    npad = (t.N + 127) // 128 * 128
+    shape = (t.G, t.N, t.D // 16) if t.axis == FP4_BLOCK_ALONG_D else (t.G, t.D, npad // 16)
+    out = torch.empty(shape, dtype=torch.uint8, device=t.scales.device)
+    _check(lib().fp4_scales_to_canonical(_ptr(t.scales), t.G, t.N, t.D, t.axis, _ptr(out),
+                                         _stream(stream)))
+    return out
 
 
 def fp4_amax(x, out=None, stream=None):

@@ -459,6 +459,22 @@ fp4_status_t fp4_probe_cvt(uint32_t start, int64_t count, int kind, uint8_t* out
   return FP4_OK;
 }
 
+fp4_status_t fp4_scales_to_canonical(const uint8_t* native, int G, int N, int D,
+                                     fp4_axis_t axis, uint8_t* canonical, void* stream) {
+  g_last_error.clear();
+  fp4_status_t s;
+  if ((s = check_shape(1, G, G, N, D)) != FP4_OK) return s;
+  if (axis != FP4_BLOCK_ALONG_D && axis != FP4_BLOCK_ALONG_N_T)
+    return fail(FP4_ERR_INVALID_ARG, "axis %d", (int)axis);
+  if (!native || !canonical) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  int dev, sms;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  fp4::scales_canonical_kernel<<<sms * 4, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      native, G, N, D, (int)axis, canonical);
+  FP4_CUDA(cudaGetLastError());
+  return FP4_OK;
+}
+
 fp4_status_t fp4_test_wait_timeout(uint64_t limit_ns, int* ok, void* stream) {
   g_last_error.clear();
   if (limit_ns == 0 || limit_ns > 5000000000ull || !ok)

@@ -217,4 +217,34 @@ __global__ void probe_cvt_kernel(uint32_t start, int64_t count, int kind, uint8_
   }
 }
 
+// Block scales from the tensor-core atom layout to the logical one.
+//   along D   (axis 0): canonical [G][N][D/16]; row n, block b sits in atom
+//             (g * Npad/128 + n/128) * D/64 + b/4 at (n%128 % 32) * 16 +
+//             (n%128 / 32) * 4 + b % 4
+//   along N^T (axis 1): canonical [G][D][Npad/16]; channel d, token block tb
+//             sits in atom g * Npad/64 + tb/4 at (d % 32) * 16 + (d / 32) * 4 + tb % 4
+__global__ void scales_canonical_kernel(const uint8_t* __restrict__ native, int64_t G, int N,
+                                        int D, int axis, uint8_t* __restrict__ out) {
+  const int64_t Npad = (N + 127) / 128 * 128;
+  const int64_t per_g = axis == 0 ? (int64_t)N * (D / 16) : (int64_t)D * (Npad / 16);
+  const int64_t total = G * per_g;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t g = i / per_g, rem = i % per_g;
+    int64_t atom, r, k;
+    if (axis == 0) {
+      const int64_t n = rem / (D / 16), b = rem % (D / 16);
+      atom = (g * (Npad / 128) + n / 128) * (D / 64) + b / 4;
+      r = n % 128;
+      k = b % 4;
+    } else {
+      const int64_t d = rem / (Npad / 16), tb = rem % (Npad / 16);
+      atom = g * (Npad / 64) + tb / 4;
+      r = d;
+      k = tb % 4;
+    }
+    out[i] = native[atom * 512 + (r % 32) * 16 + (r / 32) * 4 + k];
+  }
+}
+
 }  // namespace fp4

@@ -134,6 +134,19 @@ fp4_status_t fp4_quantize_scaled(const void* x, int G, int N, int D, fp4_axis_t 
                                  void* stream);
 
 /*
+ * The block scales fp4_quantize() wrote (tensor-core atom layout, above) in
+ * their logical layout, for callers that inspect or compare them:
+ *   FP4_BLOCK_ALONG_D:   canonical [G][N][D/16], byte (g, n, b) = scale of
+ *                        row n, block b (16 elements along D)
+ *   FP4_BLOCK_ALONG_N_T: canonical [G][D][Npad/16], byte (g, d, t) = scale of
+ *                        channel d, token block t (tokens >= N have zero codes)
+ * native and canonical are device pointers; canonical holds G*N*D/16 or
+ * G*D*Npad/16 bytes. The pages define no layout; this is the plain one.
+ */
+fp4_status_t fp4_scales_to_canonical(const uint8_t* native, int G, int N, int D,
+                                     fp4_axis_t axis, uint8_t* canonical, void* stream);
+
+/*
  * The NVFP4 attention forward: quantises q and k along D and v along tokens
  * into the workspace, then runs the fused forward. softmax_scale <= 0 (or NaN)
  * selects 1/sqrt(D). out may not alias q, k, v or the workspace.

@@ -76,6 +76,9 @@ def test_argument_errors_launch_nothing(L):
     assert L.fp4_quantize_scaled(vp(16), 0, 8, 128, 1, vp(4), vp(16), vp(16), vp(0)) == \
         fa.FP4_ERR_INVALID_ARG
     assert L.fp4_probe_cvt(0xFFFFFFF0, 64, 0, vp(16), vp(0)) == fa.FP4_ERR_INVALID_ARG
+    assert L.fp4_scales_to_canonical(vp(16), 1, 8, 128, 5, vp(16), vp(0)) == fa.FP4_ERR_INVALID_ARG
+    assert L.fp4_scales_to_canonical(vp(0), 1, 8, 128, 0, vp(16), vp(0)) == fa.FP4_ERR_INVALID_ARG
+    assert L.fp4_scales_to_canonical(vp(16), 1, 8, 96, 0, vp(16), vp(0)) == fa.FP4_ERR_UNSUPPORTED
     assert L.fp4_test_wait_timeout(0, vp(16), vp(0)) == fa.FP4_ERR_INVALID_ARG
     assert L.fp4_test_wait_timeout(6_000_000_000, vp(16), vp(0)) == fa.FP4_ERR_INVALID_ARG
     assert L.fp4_test_wait_timeout(1000, vp(0), vp(0)) == fa.FP4_ERR_INVALID_ARG

@@ -13,16 +13,18 @@ def _gpu_quant(x_u16, axis):
     import torch
     G, N, D = x_u16.shape
     t = fa.fp4_quantize(to_dev(x_u16), axis)
+    canon = fa.fp4_scales_to_canonical(t)  # the C ABI's logical view of the scales
     torch.cuda.synchronize()
     fa.fp4_status()
-    return t.codes.cpu().numpy(), t.scales.cpu().numpy(), float(t.amax[0].item())
+    return t.codes.cpu().numpy(), t.scales.cpu().numpy(), float(t.amax[0].item()), \
+        canon.cpu().numpy()
 
 
 def check_rows(ora, x):
     """x: uint16 [G, N, D]; blocks along D."""
     G, N, D = x.shape
     Npad = (N + 127) // 128 * 128
-    codes, scales, amax = _gpu_quant(x, fa.FP4_BLOCK_ALONG_D)
+    codes, scales, amax, canon = _gpu_quant(x, fa.FP4_BLOCK_ALONG_D)
     a = ora.amax_bf16(x)
     assert amax == a
     s_enc, _ = ora.tensor_scale(a)
@@ -31,6 +33,7 @@ def check_rows(ora, x):
     np.testing.assert_array_equal(codes[:, :N], oc.reshape(G, N, D // 2))
     assert not codes[:, N:].any()
     np.testing.assert_array_equal(scales_rows_logical(scales, G, N, D), os_.reshape(G, N, D // 16))
+    np.testing.assert_array_equal(canon, os_.reshape(G, N, D // 16))
 
 
 def check_tokens(ora, x):
@@ -38,7 +41,7 @@ def check_tokens(ora, x):
     G, N, D = x.shape
     Npad = (N + 127) // 128 * 128
     n16 = (N + 15) // 16 * 16
-    codes, scales, amax = _gpu_quant(x, fa.FP4_BLOCK_ALONG_N_T)
+    codes, scales, amax, canon = _gpu_quant(x, fa.FP4_BLOCK_ALONG_N_T)
     a = ora.amax_bf16(x)
     assert amax == a
     s_enc, _ = ora.tensor_scale(a)
@@ -51,6 +54,7 @@ def check_tokens(ora, x):
         assert not codes[g, :, n16 // 2:].any()
         np.testing.assert_array_equal(sc[g, :, :n16 // 16], os_)
         assert not sc[g, :, n16 // 16:].any()
+        np.testing.assert_array_equal(canon[g], sc[g])
 
 
 CASES = [(1, 1, 64), (2, 37, 128), (3, 300, 64), (1, 128, 128), (2, 1000, 128), (5, 257, 64)]
