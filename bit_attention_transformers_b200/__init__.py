@@ -299,6 +299,57 @@ def fp4_attn_fwd_host(q, k, v, causal: bool = False, softmax_scale: float | None
     return out
 
 
+def fp4_attn_fwd_host_many(batches, outs, causal: bool = False,
+                           softmax_scale: float | None = None, device="cuda", efq: bool = False,
+                           return_ms: bool = False):
+    """End-to-end over a sequence of host batches: batches = [(q, k, v), ...]
+    pinned CPU bf16 tensors of one shape, outs = pinned CPU tensors for the
+    outputs. Two sets of device buffers and three streams (copies in, compute,
+    copies out) let batch i+1's host-to-device copies and batch i-1's
+    device-to-host copy run while batch i is computed. Returns outs (and the
+    device time in ms from the first copy in to the last copy out, measured
+    with CUDA events, when return_ms) once everything has finished."""
+    import torch
+    if not batches:
+        return (outs, 0.0) if return_ms else outs
+    q0, k0, _ = batches[0]
+    B, H, N, D = q0.shape
+    Hkv = k0.shape[1]
+    dev = torch.device(device)
+    s_in, s_run, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    bufs = [tuple(torch.empty(t.shape, dtype=torch.bfloat16, device=dev) for t in (q0, k0, k0, q0))
+            for _ in range(2)]
+    ws = workspace(B, H, Hkv, N, D, dev)
+    free = [None, None]  # event: slot's last device-to-host copy done
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(s_in)
+    for i, (hq, hk, hv) in enumerate(batches):
+        slot = i % 2
+        dq, dk, dv, do = bufs[slot]
+        with torch.cuda.stream(s_in):
+            if free[slot] is not None:
+                s_in.wait_event(free[slot])
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            loaded = torch.cuda.Event()
+            loaded.record(s_in)
+        s_run.wait_event(loaded)
+        fp4_attn_fwd(dq, dk, dv, causal, softmax_scale, out=do, stream=s_run, ws=ws, efq=efq)
+        done = torch.cuda.Event()
+        done.record(s_run)
+        s_out.wait_event(done)
+        with torch.cuda.stream(s_out):
+            outs[i].copy_(do, non_blocking=True)
+            free[slot] = torch.cuda.Event()
+            free[slot].record(s_out)
+    end.record(s_out)
+    end.synchronize()  # every stream is done with the device buffers
+    if return_ms:
+        return outs, start.elapsed_time(end)
+    return outs
+
+
 def fp4_status(stream=None):
     """Synchronise and raise if a kernel reported an expired wait."""
     _check(lib().fp4_status(_stream(stream)))
