@@ -24,6 +24,7 @@ FLAG_QP_DENOMINATOR = 1
 FLAG_FLIP_BOUND = 2
 FLAG_PERTURB_P = 4
 FLAG_EFQ = 8  # EFQ-Softmax P generation (exp-free), denominator from its p~
+FLAG_FP8PV = 16  # P and V quantised to FP8 E4M3 for the PV product
 
 
 def build(force: bool = False) -> str:
@@ -65,6 +66,10 @@ def _load():
         lib.ora_quantize_rows.restype = None
         lib.ora_quantize_tokens_T.argtypes = [vp, i32, i32, f32, vp, vp, i32]
         lib.ora_quantize_tokens_T.restype = None
+        lib.ora_fp8_tensor_scale.argtypes = [f32, vp, vp]
+        lib.ora_fp8_tensor_scale.restype = None
+        lib.ora_quantize_fp8_tokens_T.argtypes = [vp, i32, i32, f32, vp, i32]
+        lib.ora_quantize_fp8_tokens_T.restype = None
         lib.ora_efq_block.argtypes = [vp, i32, vp, vp]
         lib.ora_efq_block.restype = i32
         lib.ora_scores_head.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32]
@@ -161,6 +166,23 @@ def quantize_tokens_T(x_bf16: np.ndarray, s_enc: float, npad: int | None = None)
     _load().ora_quantize_tokens_T(x.ctypes.data, N, D, float(s_enc), codes.ctypes.data,
                                   scales.ctypes.data, npad)
     return codes, scales
+
+
+def fp8_tensor_scale(amax: float) -> tuple[float, float]:
+    """(s8, d8) of the FP8 V recipe: s8 = 448 / amax."""
+    s, d = ctypes.c_float(), ctypes.c_float()
+    _load().ora_fp8_tensor_scale(float(amax), ctypes.byref(s), ctypes.byref(d))
+    return s.value, d.value
+
+
+def quantize_fp8_tokens_T(x_bf16: np.ndarray, s8: float, npad: int | None = None) -> np.ndarray:
+    """x [N, D] bf16 bits -> E4M3 codes [D, npad] (tokens >= N zero)."""
+    x = _c(x_bf16, np.uint16)
+    N, D = x.shape
+    npad = npad or N
+    codes = np.empty((D, npad), dtype=np.uint8)
+    _load().ora_quantize_fp8_tokens_T(x.ctypes.data, N, D, float(s8), codes.ctypes.data, npad)
+    return codes
 
 
 def efq_block(z) -> tuple[np.ndarray, int, int | None]:

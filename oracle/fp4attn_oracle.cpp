@@ -227,6 +227,27 @@ void quantize_tokens_T(const uint16_t* x, int N, int D, float s_enc, uint8_t* co
 
 // Dequantised value in the contraction's own units: E2M1 value times the E4M3
 // block scale. The tensor scale d is applied after the contraction.
+// FP8 variant of V (flag 16) [SageAttention2 abstract, searcharxiv.com author
+// page "Pengle Zhang": P~ and V quantised to FP8 for the PV product]. The page
+// gives no recipe; the reading: one fp32 scale per tensor mapping its absolute
+// maximum onto E4M3's largest value 448, s8 = fl(448 / amax) (1 if amax == 0,
+// FLT_MAX on overflow), code = E4M3(fl(v s8)) round to nearest even,
+// saturating; v~ = dec(code) / s8.
+void fp8_tensor_scale(float amax, float* s8, float* d8) {
+  float s = (amax > 0.0f) ? 448.0f / amax : 1.0f;
+  if (!std::isfinite(s)) s = FLT_MAX;
+  *s8 = s;
+  *d8 = 1.0f / s;
+}
+
+// x [N][D] -> codes [D][npad] (channel-major, tokens >= N zero).
+void quantize_fp8_tokens_T(const uint16_t* x, int N, int D, float s8, uint8_t* codes, int npad) {
+  for (int d = 0; d < D; ++d)
+    for (int n = 0; n < npad; ++n)
+      codes[(int64_t)d * npad + n] =
+          n < N ? e4m3_encode(bf16_to_f32(x[(int64_t)n * D + d]) * s8) : (uint8_t)0;
+}
+
 inline double deq(uint8_t code, uint8_t scale) {
   return (double)e2m1_decode(code) * (double)e4m3_decode(scale);
 }
@@ -237,6 +258,7 @@ struct Tensors {
   const uint16_t *q, *k, *v;
   int B, H, Hkv, N, D;
   float sq, dq, sk, dk, sv, dv;
+  bool fp8v;  // V in FP8 (flag 16): sv, dv are s8, d8
 };
 
 // K and V of one (b, kv-head), dequantised to contraction units, [N][D].
@@ -258,6 +280,13 @@ KVGroup make_group(const Tensors& T, int b, int hk) {
       uint8_t c = (d & 1) ? (byte >> 4) : (byte & 15);
       g.K[n * D + d] = deq(c, ks[n * (D / 16) + d / 16]);
     }
+  if (T.fp8v) {  // FP8 V: contraction units dec(code), d8 applied at the end
+    std::vector<uint8_t> v8((size_t)D * N);
+    quantize_fp8_tokens_T(T.v + off, N, D, T.sv, v8.data(), N);
+    for (int d = 0; d < D; ++d)
+      for (int64_t n = 0; n < N; ++n) g.V[n * D + d] = (double)e4m3_decode(v8[d * N + n]);
+    return g;
+  }
   const int npad = (N + 15) / 16 * 16;
   std::vector<uint8_t> vc((size_t)D * npad / 2), vs((size_t)D * npad / 16);
   quantize_tokens_T(T.v + off, N, D, T.sv, vc.data(), vs.data(), npad);
@@ -270,7 +299,14 @@ KVGroup make_group(const Tensors& T, int b, int hk) {
   return g;
 }
 
-enum { FLAG_QP_DENOMINATOR = 1, FLAG_FLIP_BOUND = 2, FLAG_PERTURB_P = 4, FLAG_EFQ = 8 };
+enum { FLAG_QP_DENOMINATOR = 1, FLAG_FLIP_BOUND = 2, FLAG_PERTURB_P = 4, FLAG_EFQ = 8,
+       FLAG_FP8PV = 16 };
+
+// FP8 P (flag 16): p~ = E4M3(fl(p * 256)) / 256, round to nearest even; p <= 1
+// so p * 256 <= 256 stays inside E4M3's range (largest 448) and the scaling is
+// exact; d_P = 2^-8. The reading matches V's: one tensor scale, here a power
+// of two.
+const float kFp8PScale = 256.0f;
 
 // EFQ-Softmax P generation for one block of n <= 16 keys of one row
 // [EFQ-Softmax abstract, scholarbro.com page "AVQ Attention: Adaptive
@@ -450,9 +486,11 @@ void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float 
     qd[d] = deq((d & 1) ? (byte >> 4) : (byte & 15), qs[d / 16]);
   }
   const bool efq = (flags & FLAG_EFQ) != 0;
+  const bool fp8 = (flags & FLAG_FP8PV) != 0;
   float sP, dP;
   tensor_scale(1.0f, &sP, &dP);  // P: a-priori amax 1, so s_enc = 2688
   if (efq) dP = std::ldexp(1.0f, -kEfqScaleExp);
+  if (fp8) dP = 1.0f / kFp8PScale;
   std::vector<double> O(D, 0.0), F(D, 0.0);
   std::vector<float> x(Bc), p(Bc);
   std::vector<double> pq(Bc), A(Bc, 0.0), eps(Bc, 0.0), dlt(Bc, 0.0), z(Bc);
@@ -497,7 +535,8 @@ void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float 
         if (live && want_flip) {
           const double u = std::ldexp(1.0, -22);
           eps[jj] = std::log(2.0) * ((double)c * u * (A[jj] + amx) +
-                                     u * (std::fabs((double)x[jj]) + std::fabs(m_new))) +
+                                     u * (std::fabs((double)x[jj]) + std::fabs(m_new) +
+                                          (fp8 ? 8.0 : 0.0))) +
                     std::ldexp(1.0, -21);
           if (flags & FLAG_PERTURB_P) {
             double uu = (double)(mix64(rowkey ^ mix64((uint64_t)j)) >> 11) * std::ldexp(1.0, -53);
@@ -507,8 +546,25 @@ void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float 
           epsmax = std::max(epsmax, eps[jj]);
         }
       }
-      // P quantisation, blocks of 16 keys from the tile start
-      for (int b0 = 0; b0 < Bc; b0 += 16) {
+      // P quantisation: FP8 per key (flag 16), else NVFP4 blocks of 16 keys
+      if (fp8) {
+        for (int jj = 0; jj < Bc; ++jj) {
+          const float y = p[jj] * kFp8PScale;
+          const uint8_t code = e4m3_encode(y);
+          pq[jj] = (double)e4m3_decode(code);
+          dlt[jj] = 0.0;
+          if (!(flags & FLAG_FLIP_BOUND) || y == 0.0f) continue;
+          // a neighbouring code whose rounding midpoint lies within eps of y
+          for (int nb = -1; nb <= 1; nb += 2) {
+            const int c2 = (int)code + nb;
+            if (c2 < 0 || c2 > 126) continue;
+            const double v2 = (double)e4m3_decode((uint8_t)c2);
+            if (std::fabs((double)y - 0.5 * (pq[jj] + v2)) <= eps[jj] * (double)y + 1e-30)
+              dlt[jj] = std::max(dlt[jj], std::fabs(v2 - pq[jj]));
+          }
+        }
+      }
+      for (int b0 = 0; !fp8 && b0 < Bc; b0 += 16) {
         int n = std::min(16, Bc - b0);
         uint8_t codes[16], e;
         quantize_block(&p[b0], n, sP, codes, &e);
@@ -651,13 +707,22 @@ int ora_efq_block(const double* z, int n, uint8_t* codes, uint8_t* scale) {
   return efq_block(z, n, codes, scale);
 }
 
+// FP8 V (flag 16's quantiser): x [N][D] bf16 -> codes [D][npad]; the scale
+// comes from ora_fp8_tensor_scale of the whole tensor's maximum.
+void ora_fp8_tensor_scale(float amax, float* s8, float* d8) { fp8_tensor_scale(amax, s8, d8); }
+void ora_quantize_fp8_tokens_T(const uint16_t* x, int N, int D, float s8, uint8_t* codes,
+                               int npad) {
+  e4m3_encode(0.0f);
+  quantize_fp8_tokens_T(x, N, D, s8, codes, npad);
+}
+
 // Unscaled scores of one head: S[i][j] = fl32(exact q~_i . k~_j), contraction
 // units (before d_Q d_K), no mask. S is [N][N].
 int ora_scores_head(const uint16_t* q, const uint16_t* k, int B, int H, int Hkv, int N, int D,
                     int b, int h, float* S, int nthreads) {
   if (B <= 0 || H <= 0 || Hkv <= 0 || H % Hkv || N <= 0 || D % 16 || b >= B || h >= H) return -1;
   e4m3_encode(0.0f);
-  Tensors T{q, k, k, B, H, Hkv, N, D, 0, 0, 0, 0, 0, 0};
+  Tensors T{q, k, k, B, H, Hkv, N, D, 0, 0, 0, 0, 0, 0, false};
   tensor_scale(amax_bf16(q, (int64_t)B * H * N * D), &T.sq, &T.dq);
   tensor_scale(amax_bf16(k, (int64_t)B * Hkv * N * D), &T.sk, &T.dk);
   const int hk = h / (H / Hkv);
@@ -687,7 +752,8 @@ int ora_scores_head(const uint16_t* q, const uint16_t* k, int B, int H, int Hkv,
 //   Bc: key tile (128 on the path); flags: 1 = denominator from p~,
 //   2 = flip bound into out_flip ([nrows][D], may be NULL otherwise),
 //   4 = perturb p within the flip bound's uncertainty (tests the bound),
-//   8 = EFQ-Softmax P generation (efq_block), denominator from its p~.
+//   8 = EFQ-Softmax P generation (efq_block), denominator from its p~,
+//   16 = P and V in FP8 E4M3 (not with 8).
 // Returns 0, or -1 on bad arguments.
 int ora_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H, int Hkv,
                  int N, int D, int causal, float softmax_scale, int Bc, int flags,
@@ -697,10 +763,14 @@ int ora_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B,
       Bc % 16)
     return -1;
   e4m3_encode(0.0f);
-  Tensors T{q, k, v, B, H, Hkv, N, D, 0, 0, 0, 0, 0, 0};
+  if ((flags & FLAG_FP8PV) && (flags & FLAG_EFQ)) return -1;
+  Tensors T{q, k, v, B, H, Hkv, N, D, 0, 0, 0, 0, 0, 0, (flags & FLAG_FP8PV) != 0};
   tensor_scale(amax_bf16(q, (int64_t)B * H * N * D), &T.sq, &T.dq);
   tensor_scale(amax_bf16(k, (int64_t)B * Hkv * N * D), &T.sk, &T.dk);
-  tensor_scale(amax_bf16(v, (int64_t)B * Hkv * N * D), &T.sv, &T.dv);
+  if (T.fp8v)
+    fp8_tensor_scale(amax_bf16(v, (int64_t)B * Hkv * N * D), &T.sv, &T.dv);
+  else
+    tensor_scale(amax_bf16(v, (int64_t)B * Hkv * N * D), &T.sv, &T.dv);
   if (!(softmax_scale > 0.0f)) softmax_scale = 1.0f / std::sqrt((float)D);
   float c = T.dq * T.dk;
   c = c * softmax_scale;
