@@ -49,8 +49,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="video_dit")
     ap.add_argument("--impl", default="fp4attn", choices=["fp4attn", "reference"])
-    ap.add_argument("--variant", default="exp", choices=["exp", "efq"],
-                    help="P generation: exp-then-quantize (the default path) or EFQ-Softmax")
+    ap.add_argument("--variant", default="exp", choices=["exp", "efq", "fp8pv"],
+                    help="P generation: exp-then-quantize (the default path), EFQ-Softmax, "
+                         "or exp-then-quantize to FP8 with V in FP8 (PV as an FP8 contraction)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0,
                     help="override H and Hkv (keeping their ratio) for a smaller profiling case")
@@ -124,7 +125,12 @@ def flush_l2(buf):
     buf.add_(1)
 
 
-def cpu_baseline(wl, q, k, v, rows_total: int):
+def oracle_flags(variant: str) -> int:
+    import oracle
+    return {"exp": 0, "efq": oracle.FLAG_EFQ, "fp8pv": oracle.FLAG_FP8PV}[variant]
+
+
+def cpu_baseline(wl, q, k, v, rows_total: int, variant: str = "exp"):
     """The oracle, as it stands, on a bounded sample: `rows_total` seeded query
     rows spread over the heads (plus the quantisation of K and V it needs)."""
     import numpy as np
@@ -135,7 +141,8 @@ def cpu_baseline(wl, q, k, v, rows_total: int):
     rows = synth.sample_rows(wl, per_head)
     threads = os.cpu_count() or 1
     t0 = time.perf_counter()
-    oracle.attn_fwd(q, k, v, causal=wl.causal, rows=rows, threads=threads)
+    oracle.attn_fwd(q, k, v, causal=wl.causal, rows=rows, threads=threads,
+                    flags=oracle_flags(variant))
     dt = time.perf_counter() - t0
     keys = (rows[:, 2] + 1).astype(np.float64) if wl.causal else np.full(len(rows), wl.N, np.float64)
     flops = float((4.0 * wl.D * keys).sum())
@@ -157,7 +164,7 @@ def run_reference(args, wl):
     rows_total = args.cpu_rows or wl.B * wl.H
     times, res = [], None
     for i in range(args.warmup + args.steps):
-        res = cpu_baseline(wl, q, k, v, rows_total)
+        res = cpu_baseline(wl, q, k, v, rows_total, args.variant)
         if i >= args.warmup:
             times.append(res["seconds"])
     flops = res["value"] * res["seconds"] * 1e12
@@ -212,18 +219,18 @@ def main():
     q, k, v = hq.to(dev), hk.to(dev), hv.to(dev)
     out = torch.empty_like(q)
     qf, kf, vf, outf = (t.view(-1, wl.N, wl.D) for t in (q, k, v, out))
-    ws = fa.workspace(wl.B, wl.H, wl.Hkv, wl.N, wl.D, dev)
+    efq, fp8pv = args.variant == "efq", args.variant == "fp8pv"
+    ws = fa.workspace(wl.B, wl.H, wl.Hkv, wl.N, wl.D, dev, fp8pv)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
     flops = wl.flops
 
-    efq = args.variant == "efq"
-
     def step():
         if world > 1:
-            fa.fp4_attn_fwd_sharded(qf, kf, vf, causal=wl.causal, out=outf, efq=efq)
+            fa.fp4_attn_fwd_sharded(qf, kf, vf, causal=wl.causal, out=outf, efq=efq,
+                                    fp8pv=fp8pv)
         else:
-            fa.fp4_attn_fwd(q, k, v, causal=wl.causal, out=out, ws=ws, efq=efq)
+            fa.fp4_attn_fwd(q, k, v, causal=wl.causal, out=out, ws=ws, efq=efq, fp8pv=fp8pv)
 
     def barrier():
         if world > 1:
@@ -261,11 +268,11 @@ def main():
     # the fused attention kernel alone (same inputs, already quantised)
     qq = fa.fp4_quantize(q, fa.FP4_BLOCK_ALONG_D)
     kq = fa.fp4_quantize(k, fa.FP4_BLOCK_ALONG_D)
-    vq = fa.fp4_quantize(v, fa.FP4_BLOCK_ALONG_N_T)
+    vq = fa.fp4_quantize_fp8(v) if fp8pv else fa.fp4_quantize(v, fa.FP4_BLOCK_ALONG_N_T)
 
     def kernel():
         fa.fp4_attn_fwd_quantized(qq, kq, vq, wl.B, wl.H, wl.Hkv, causal=wl.causal, out=out,
-                                  efq=efq)
+                                  efq=efq, fp8pv=fp8pv)
 
     for _ in range(args.warmup):
         kernel()
@@ -279,11 +286,13 @@ def main():
         if world > 1:
             for d, h in ((q, hq), (k, hk), (v, hv)):
                 d.copy_(h, non_blocking=True)
-            fa.fp4_attn_fwd_sharded(qf, kf, vf, causal=wl.causal, out=outf, efq=efq)
+            fa.fp4_attn_fwd_sharded(qf, kf, vf, causal=wl.causal, out=outf, efq=efq,
+                                    fp8pv=fp8pv)
             hout.copy_(out, non_blocking=True)
             stream.synchronize()
         else:
-            fa.fp4_attn_fwd_host(hq, hk, hv, causal=wl.causal, out=hout, device=dev, efq=efq)
+            fa.fp4_attn_fwd_host(hq, hk, hv, causal=wl.causal, out=hout, device=dev, efq=efq,
+                                 fp8pv=fp8pv)
 
     houts = [hout, torch.empty(shape_q, dtype=torch.bfloat16, pin_memory=True)]
     n_e2e = max(2, args.steps)
@@ -298,10 +307,11 @@ def main():
         # inputs in and its output out, overlapped with the neighbouring steps'
         # compute
         batches = [(hq, hk, hv)] * n_e2e
-        fa.fp4_attn_fwd_host_many(batches[:2], houts, causal=wl.causal, device=dev, efq=efq)
+        fa.fp4_attn_fwd_host_many(batches[:2], houts, causal=wl.causal, device=dev, efq=efq,
+                                  fp8pv=fp8pv)
         _, total = fa.fp4_attn_fwd_host_many(batches, [houts[i % 2] for i in range(n_e2e)],
                                              causal=wl.causal, device=dev, efq=efq,
-                                             return_ms=True)
+                                             fp8pv=fp8pv, return_ms=True)
         e_ms = [total / n_e2e] * n_e2e
     e_total = sum(e_ms)
     if world > 1:
@@ -312,21 +322,27 @@ def main():
     fa.fp4_status()
 
     peaks, src = measured_peaks()
-    fp4_peak = 4.0 * peaks["bf16_tflops"]  # dense FP4 = 4x dense bf16 (nominal 9 vs 2.25 PF)
+    # dense FP4 = 4x dense bf16 (nominal 9 vs 2.25 PF); with FP8 P and V half the
+    # flops (PV) run at FP8's 2x: the time-weighted peak is 1 / (0.5/4 + 0.5/2) = 8/3 x
+    peak_ratio = 8.0 / 3.0 if fp8pv else 4.0
+    fp4_peak = peak_ratio * peaks["bf16_tflops"]
     achieved = flops / (k_ms * 1e-3) / 1e12
     traffic = None
     kernel_src = os.path.join(ROOT, "bit_attention_transformers_b200", "csrc", "attn_fwd.cuh")
     with open(kernel_src, "rb") as f:
-        if (wl.name == ATTN_TRAFFIC["workload"] and not args.heads and not efq and
+        if (wl.name == ATTN_TRAFFIC["workload"] and not args.heads and args.variant == "exp" and
                 hashlib.sha256(f.read()).hexdigest() == ATTN_TRAFFIC["attn_fwd_sha256"]):
             traffic = ATTN_TRAFFIC["bytes"]
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 (P and V: e4m3)" if fp8pv else "nvfp4",
         "data": "synthetic",
         "config": {**wl.describe(),
-                   "p_generation": "EFQ-Softmax" if efq else "exp-then-quantize",
+                   "p_generation": {"exp": "exp-then-quantize", "efq": "EFQ-Softmax",
+                                    "fp8pv": "exp-then-quantize to FP8 E4M3, V in FP8 E4M3"}[
+                                        args.variant],
                    "parallelism": (f"heads sharded over {world} ranks ({world} x B*Hkv units, "
                                    "one all-reduce MAX of 3 floats per step)") if world > 1
                    else "1 GPU",
@@ -339,7 +355,8 @@ def main():
         "attn_kernel_ms": k_ms,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak,
                      "unit": "TFLOP/s", "frac": achieved / fp4_peak, "traffic": traffic,
-                     "peak_source": f"4 x measured dense bf16 ({peaks['bf16_tflops']} TFLOP/s, "
+                     "peak_source": f"{peak_ratio:.3g} x measured dense bf16 "
+                                    f"({peaks['bf16_tflops']} TFLOP/s, "
                                     f"{src}); fraction of measured"},
         "e2e": {"value": e2e_value, "unit": "TFLOPS",
                 "h2d_bytes_per_step": (hq.numel() + hk.numel() + hv.numel()) * 2,
@@ -355,7 +372,8 @@ def main():
                                 cpu_baseline(wl, hq.view(torch.int16).numpy().view(np.uint16),
                                              hk.view(torch.int16).numpy().view(np.uint16),
                                              hv.view(torch.int16).numpy().view(np.uint16),
-                                             args.cpu_rows or wl.B * wl.H).items()
+                                             args.cpu_rows or wl.B * wl.H,
+                                             args.variant).items()
                                 if k2 != "seconds"}
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -26,12 +26,15 @@ FP4_ERR_CUDA = 4
 FP4_ERR_TIMEOUT = 5
 FP4_BLOCK_ALONG_D = 0
 FP4_BLOCK_ALONG_N_T = 1
+FP8_TOKENS_T = -1  # Fp4Tensor.axis of E4M3 V codes [G][D][Npad] (no block scales)
 
 # Every symbol include/fp4attn.h declares.
 EXPORTS = ("fp4_codes_bytes", "fp4_scales_bytes", "fp4_attn_workspace_bytes", "fp4_quantize",
            "fp4_amax", "fp4_quantize_scaled", "fp4_scales_to_canonical", "fp4_attn_fwd",
            "fp4_attn_fwd_quantized",
-           "fp4_attn_fwd_efq", "fp4_attn_fwd_quantized_efq", "fp4_attn_fwd_noalloc",
+           "fp4_attn_fwd_efq", "fp4_attn_fwd_quantized_efq", "fp4_fp8_codes_bytes",
+           "fp4_quantize_fp8", "fp4_quantize_fp8_scaled", "fp4_attn_workspace_bytes_fp8pv",
+           "fp4_attn_fwd_fp8pv", "fp4_attn_fwd_quantized_fp8pv", "fp4_attn_fwd_noalloc",
            "fp4_status", "fp4_last_error", "fp4_probe_cvt", "fp4_test_wait_timeout")
 FP4_NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -98,6 +101,18 @@ def lib():
         L.fp4_attn_fwd_efq.restype = i32
         L.fp4_attn_fwd_quantized_efq.argtypes = L.fp4_attn_fwd_quantized.argtypes
         L.fp4_attn_fwd_quantized_efq.restype = i32
+        L.fp4_fp8_codes_bytes.argtypes = [i32, i32, i32]
+        L.fp4_fp8_codes_bytes.restype = sz
+        L.fp4_quantize_fp8.argtypes = [vp, i32, i32, i32, vp, vp, vp]
+        L.fp4_quantize_fp8.restype = i32
+        L.fp4_quantize_fp8_scaled.argtypes = [vp, i32, i32, i32, vp, vp, vp]
+        L.fp4_quantize_fp8_scaled.restype = i32
+        L.fp4_attn_workspace_bytes_fp8pv.argtypes = [i32, i32, i32, i32, i32]
+        L.fp4_attn_workspace_bytes_fp8pv.restype = sz
+        L.fp4_attn_fwd_fp8pv.argtypes = L.fp4_attn_fwd.argtypes
+        L.fp4_attn_fwd_fp8pv.restype = i32
+        L.fp4_attn_fwd_quantized_fp8pv.argtypes = L.fp4_attn_fwd_quantized.argtypes
+        L.fp4_attn_fwd_quantized_fp8pv.restype = i32
         L.fp4_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
         L.fp4_attn_fwd_noalloc.restype = i32
         L.fp4_status.argtypes = [vp]
@@ -187,6 +202,32 @@ def fp4_quantize(x, axis: int = FP4_BLOCK_ALONG_D, stream=None, amax=None) -> Fp
     return Fp4Tensor(codes, scales, amax, G, N, D, axis)
 
 
+def fp4_fp8_codes_bytes(G: int, N: int, D: int) -> int:
+    return lib().fp4_fp8_codes_bytes(G, N, D)
+
+
+def fp4_attn_workspace_bytes_fp8pv(B: int, H: int, Hkv: int, N: int, D: int) -> int:
+    return lib().fp4_attn_workspace_bytes_fp8pv(B, H, Hkv, N, D)
+
+
+def fp4_quantize_fp8(x, stream=None, amax=None) -> Fp4Tensor:
+    """E4M3 quantisation of V for the FP8 P/V variant: x bf16 CUDA [..., N, D]
+    -> codes [G][D][Npad] (one byte each), no block scales (scales is None,
+    axis FP8_TOKENS_T). With `amax` (float32 CUDA, first element the tensor
+    maximum) fp4_quantize_fp8_scaled runs; otherwise max |x| is computed first."""
+    import torch
+    G, N, D = _gnd(x)
+    codes = torch.empty(fp4_fp8_codes_bytes(G, N, D), dtype=torch.uint8, device=x.device)
+    if amax is None:
+        amax = torch.empty(4, dtype=torch.float32, device=x.device)
+        _check(lib().fp4_quantize_fp8(_ptr(x), G, N, D, _ptr(codes), _ptr(amax), _stream(stream)))
+    else:
+        assert amax.is_cuda and amax.dtype == torch.float32
+        _check(lib().fp4_quantize_fp8_scaled(_ptr(x), G, N, D, _ptr(amax), _ptr(codes),
+                                             _stream(stream)))
+    return Fp4Tensor(codes, None, amax, G, N, D, FP8_TOKENS_T)
+
+
 def fp4_scales_to_canonical(t: Fp4Tensor, stream=None):
     """t's block scales in their logical layout: [G][N][D/16] (blocks along D)
     or [G][D][Npad/16] (blocks along tokens), a uint8 CUDA tensor."""
@@ -213,10 +254,11 @@ def fp4_amax(x, out=None, stream=None):
 _ws_cache: dict = {}
 
 
-def workspace(B, H, Hkv, N, D, device):
-    """A cached device workspace large enough for fp4_attn_fwd on this shape."""
+def workspace(B, H, Hkv, N, D, device, fp8pv: bool = False):
+    """A cached device workspace large enough for fp4_attn_fwd (or, with
+    fp8pv, fp4_attn_fwd_fp8pv) on this shape."""
     import torch
-    need = fp4_attn_workspace_bytes(B, H, Hkv, N, D)
+    need = (fp4_attn_workspace_bytes_fp8pv if fp8pv else fp4_attn_workspace_bytes)(B, H, Hkv, N, D)
     key = (str(device),)
     ws = _ws_cache.get(key)
     if ws is None or ws.numel() < need:
@@ -225,11 +267,19 @@ def workspace(B, H, Hkv, N, D, device):
     return ws
 
 
+def _attn_fn(efq: bool, fp8pv: bool, quantized: bool):
+    if efq and fp8pv:
+        raise ValueError("efq and fp8pv are two different P generations; pick one")
+    name = "fp4_attn_fwd_quantized" if quantized else "fp4_attn_fwd"
+    return getattr(lib(), name + ("_efq" if efq else "_fp8pv" if fp8pv else ""))
+
+
 def fp4_attn_fwd(q, k, v, causal: bool = False, softmax_scale: float | None = None, out=None,
-                 stream=None, ws=None, efq: bool = False):
+                 stream=None, ws=None, efq: bool = False, fp8pv: bool = False):
     """NVFP4 attention forward. q [B,H,N,D], k/v [B,Hkv,N,D]: contiguous bf16
     CUDA tensors. Returns out [B,H,N,D] bf16. efq=True calls fp4_attn_fwd_efq
-    (P from EFQ-Softmax instead of exp-then-quantize)."""
+    (P from EFQ-Softmax instead of exp-then-quantize); fp8pv=True calls
+    fp4_attn_fwd_fp8pv (P and V in E4M3)."""
     import torch
     B, H, N, D = q.shape
     Hkv = k.shape[1]
@@ -238,9 +288,9 @@ def fp4_attn_fwd(q, k, v, causal: bool = False, softmax_scale: float | None = No
     assert k.shape == (B, Hkv, N, D) and v.shape == (B, Hkv, N, D)
     if out is None:
         out = torch.empty_like(q)
+    fn = _attn_fn(efq, fp8pv, False)
     if ws is None:
-        ws = workspace(B, H, Hkv, N, D, q.device)
-    fn = lib().fp4_attn_fwd_efq if efq else lib().fp4_attn_fwd
+        ws = workspace(B, H, Hkv, N, D, q.device, fp8pv)
     _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, Hkv, N, D, int(bool(causal)),
               float(softmax_scale or 0.0), _stream(stream), _ptr(ws), ws.numel()))
     return out
@@ -268,22 +318,27 @@ def fp4_attn_fwd_noalloc(q, k, v, causal: bool = False, softmax_scale: float | N
 
 def fp4_attn_fwd_quantized(qq: Fp4Tensor, kq: Fp4Tensor, vq: Fp4Tensor, B: int, H: int,
                            Hkv: int, causal: bool = False, softmax_scale: float | None = None,
-                           out=None, stream=None, efq: bool = False):
+                           out=None, stream=None, efq: bool = False, fp8pv: bool = False):
     """The fused forward alone on tensors fp4_quantize() produced
-    (fp4_attn_fwd_quantized_efq with efq=True)."""
+    (fp4_attn_fwd_quantized_efq with efq=True; fp4_attn_fwd_quantized_fp8pv
+    with fp8pv=True, vq from fp4_quantize_fp8)."""
     import torch
     N, D = qq.N, qq.D
     if out is None:
         out = torch.empty((B, H, N, D), dtype=torch.bfloat16, device=qq.codes.device)
-    ts = [_Tensor(t.codes.data_ptr(), t.scales.data_ptr(), t.amax.data_ptr()) for t in (qq, kq, vq)]
-    fn = lib().fp4_attn_fwd_quantized_efq if efq else lib().fp4_attn_fwd_quantized
+    fn = _attn_fn(efq, fp8pv, True)
+    if (vq.axis == FP8_TOKENS_T) != bool(fp8pv):
+        raise ValueError("vq must come from fp4_quantize_fp8 exactly when fp8pv is set")
+    ts = [_Tensor(t.codes.data_ptr(), 0 if t.scales is None else t.scales.data_ptr(),
+                  t.amax.data_ptr()) for t in (qq, kq, vq)]
     _check(fn(ctypes.byref(ts[0]), ctypes.byref(ts[1]), ctypes.byref(ts[2]), _ptr(out), B, H,
               Hkv, N, D, int(bool(causal)), float(softmax_scale or 0.0), _stream(stream)))
     return out
 
 
 def fp4_attn_fwd_host(q, k, v, causal: bool = False, softmax_scale: float | None = None,
-                      out=None, device="cuda", stream=None, efq: bool = False):
+                      out=None, device="cuda", stream=None, efq: bool = False,
+                      fp8pv: bool = False):
     """End-to-end call on host buffers: copies q, k, v (pinned CPU bf16
     tensors) to the device, runs fp4_attn_fwd, copies the output back into
     `out` (a pinned CPU tensor) and returns it once the stream has finished."""
@@ -291,7 +346,7 @@ def fp4_attn_fwd_host(q, k, v, causal: bool = False, softmax_scale: float | None
     dq = q.to(device, non_blocking=True)
     dk = k.to(device, non_blocking=True)
     dv = v.to(device, non_blocking=True)
-    o = fp4_attn_fwd(dq, dk, dv, causal, softmax_scale, stream=stream, efq=efq)
+    o = fp4_attn_fwd(dq, dk, dv, causal, softmax_scale, stream=stream, efq=efq, fp8pv=fp8pv)
     if out is None:
         out = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
     out.copy_(o, non_blocking=True)
@@ -301,7 +356,7 @@ def fp4_attn_fwd_host(q, k, v, causal: bool = False, softmax_scale: float | None
 
 def fp4_attn_fwd_host_many(batches, outs, causal: bool = False,
                            softmax_scale: float | None = None, device="cuda", efq: bool = False,
-                           return_ms: bool = False):
+                           return_ms: bool = False, fp8pv: bool = False):
     """End-to-end over a sequence of host batches: batches = [(q, k, v), ...]
     pinned CPU bf16 tensors of one shape, outs = pinned CPU tensors for the
     outputs. Two sets of device buffers and three streams (copies in, compute,
@@ -319,7 +374,7 @@ def fp4_attn_fwd_host_many(batches, outs, causal: bool = False,
     s_in, s_run, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     bufs = [tuple(torch.empty(t.shape, dtype=torch.bfloat16, device=dev) for t in (q0, k0, k0, q0))
             for _ in range(2)]
-    ws = workspace(B, H, Hkv, N, D, dev)
+    ws = workspace(B, H, Hkv, N, D, dev, fp8pv)
     free = [None, None]  # event: slot's last device-to-host copy done
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(s_in)
@@ -335,7 +390,8 @@ def fp4_attn_fwd_host_many(batches, outs, causal: bool = False,
             loaded = torch.cuda.Event()
             loaded.record(s_in)
         s_run.wait_event(loaded)
-        fp4_attn_fwd(dq, dk, dv, causal, softmax_scale, out=do, stream=s_run, ws=ws, efq=efq)
+        fp4_attn_fwd(dq, dk, dv, causal, softmax_scale, out=do, stream=s_run, ws=ws, efq=efq,
+                     fp8pv=fp8pv)
         done = torch.cuda.Event()
         done.record(s_run)
         s_out.wait_event(done)

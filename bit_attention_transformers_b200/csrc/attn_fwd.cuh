@@ -106,12 +106,16 @@ struct AttnParams {
   float softmax_scale;
 };
 
-template <int D>
+// P generation: exp-then-quantize to NVFP4 (the method), EFQ-Softmax, or
+// exp-then-quantize to FP8 E4M3 with V in FP8 as well.
+enum : int { kPgExp = 0, kPgEfq = 1, kPgFp8 = 2 };
+
+template <int D, bool FP8 = false>
 struct AttnSmem {
   static constexpr int kQ = kBM * D / 2;   // Q codes tile
   static constexpr int kK = kBN * D / 2;   // K codes tile
-  static constexpr int kV = D * kBN / 2;   // V^T codes tile
-  static constexpr int kP = kBM * kBN / 2; // P codes tile
+  static constexpr int kV = FP8 ? D * kBN : D * kBN / 2;    // V^T codes tile
+  static constexpr int kP = FP8 ? kBM * kBN : kBM * kBN / 2;  // P codes tile
   static constexpr int kSfQK = (D / 64) * 512;
   static constexpr int oQ = 0;
   static constexpr int oK = oQ + kQ;
@@ -159,11 +163,12 @@ struct TmemCols {
 constexpr float kInv7 = 1.0f / 7.0f;
 constexpr float kRound = 8388608.0f;  // 2^23: x + 2^23 rounds x (0 <= x < 2^22) to an integer
 
-template <int D, bool CAUSAL, bool EFQ>
+template <int D, bool CAUSAL, int PG>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
-  using L = AttnSmem<D>;
+  constexpr bool EFQ = PG == kPgEfq, FP8 = PG == kPgFp8;
+  using L = AttnSmem<D, FP8>;
   using TC = TmemCols<EFQ>;
   constexpr uint32_t kColQsf = TC::kQsf, kColKsf = TC::kKsf, kColPsf = TC::kPsf,
                      kColVsf = TC::kVsf, kColL = kColO + D;
@@ -249,10 +254,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                   p.k_sf + ((int64_t)gk * (p.Npad / kBN) + j) * L::kSfQK, L::kSfQK,
                   bar(kBarKFull + st));
         if (j >= kStages && !(ok = wait_bar(bar(kBarVEmpty + st), pe))) break;
-        mbar_arrive_expect_tx(bar(kBarVFull + st), L::kV + 1024);
-        tma_load_2d(sb + L::oV + st * L::kV, &tmV, j * (kBN / 2), gk * D, bar(kBarVFull + st));
-        bulk_load(sb + L::oVsf + st * 1024, p.v_sf + ((int64_t)gk * (p.Npad / 64) + 2 * j) * 512,
-                  1024, bar(kBarVFull + st));
+        mbar_arrive_expect_tx(bar(kBarVFull + st), L::kV + (FP8 ? 0 : 1024));
+        tma_load_2d(sb + L::oV + st * L::kV, &tmV, j * (FP8 ? kBN : kBN / 2), gk * D,
+                    bar(kBarVFull + st));
+        if (!FP8)
+          bulk_load(sb + L::oVsf + st * 1024, p.v_sf + ((int64_t)gk * (p.Npad / 64) + 2 * j) * 512,
+                    1024, bar(kBarVFull + st));
       }
     }
   } else if (warp == 1 || warp == 2) {
@@ -305,16 +312,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (!(ok = wait_bar(bar(kBarVFull + st), (t / kStages) & 1))) break;
           if (!(ok = wait_bar(bar(kBarPFull + (t & 1)), (t >> 1) & 1))) break;
           tc_fence_after();
+          if constexpr (FP8) {
+            // E4M3 P (128 bytes per row) times E4M3 V^T, 128-byte swizzle, K = 32 per MMA
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            tc_cp_32x128b_x4(tPsf + 4 * c, smem_desc(sb + L::oPsf + (t & 1) * 1024 + 512 * c, 0, 128, 0));
-            tc_cp_32x128b_x4(tVsf + 4 * c, smem_desc(sb + L::oVsf + st * 1024 + 512 * c, 0, 128, 0));
+            for (int c = 0; c < 4; ++c)
+              mma_f8e4m3(tO, smem_desc(sb + L::oP + (t & 1) * L::kP + 32 * c, 16, 1024, 2),
+                         smem_desc(sb + L::oV + st * L::kV + 32 * c, 16, 1024, 2),
+                         idesc_f8e4m3(kBM, D), (t > 0 || c > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              tc_cp_32x128b_x4(tPsf + 4 * c,
+                               smem_desc(sb + L::oPsf + (t & 1) * 1024 + 512 * c, 0, 128, 0));
+              tc_cp_32x128b_x4(tVsf + 4 * c, smem_desc(sb + L::oVsf + st * 1024 + 512 * c, 0, 128, 0));
+            }
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              mma_mxf4nvf4(tO, smem_desc(sb + L::oP + (t & 1) * L::kP + 32 * c, 16, 512, 4),
+                           smem_desc(sb + L::oV + st * L::kV + 32 * c, 16, 512, 4), kIdO,
+                           tPsf + 4 * c, tVsf + 4 * c, (t > 0 || c > 0) ? 1u : 0u);
           }
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-            mma_mxf4nvf4(tO, smem_desc(sb + L::oP + (t & 1) * L::kP + 32 * c, 16, 512, 4),
-                         smem_desc(sb + L::oV + st * L::kV + 32 * c, 16, 512, 4), kIdO,
-                         tPsf + 4 * c, tVsf + 4 * c, (t > 0 || c > 0) ? 1u : 0u);
           if (EFQ) {
 #pragma unroll
             for (int c = 0; c < 2; ++c)
@@ -344,10 +361,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float* mval = reinterpret_cast<float*>(sm + L::oRed);  // [2][128]: running max after tile t, slot t & 1
     float* lval = mval + 2 * kBM;                          // [2][128]: each stream's row sum
     const float sq = tensor_senc(*p.amax_q), sk = tensor_senc(*p.amax_k),
-                sv = tensor_senc(*p.amax_v);
+                sv = FP8 ? fp8_senc(*p.amax_v) : tensor_senc(*p.amax_v);
     const float dq = __fdiv_rn(1.0f, sq), dk = __fdiv_rn(1.0f, sk), dv = __fdiv_rn(1.0f, sv);
     const float c = __fmul_rn(__fmul_rn(__fmul_rn(dq, dk), p.softmax_scale), kLog2e);
-    const float fpv = __fmul_rn(__fdiv_rn(1.0f, kTensorRange), dv);  // d_P * d_V
+    // d_P d_V; with FP8 P the row sum is kept in units of 256 p, so d_V alone
+    const float fpv = FP8 ? dv : __fmul_rn(__fdiv_rn(1.0f, kTensorRange), dv);
     const uint64_t c2 = pk(c, c);
     const float c27 = __fdiv_rn(__fmul_rn(2.0f, c), 7.0f);  // EFQ: slope of the affine rule / 7
     float m_own = -INFINITY;   // running max after this stream's previous tile
@@ -402,10 +420,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float alpha = (m_prev == -INFINITY) ? 0.0f : ex2_approx(m_prev - m_new);
       const float neg_m = (m_new == -INFINITY) ? 0.0f : -m_new;
       const uint64_t nm2 = pk(neg_m, neg_m);
-      uint32_t pc[16];
+      uint32_t pc[FP8 ? 32 : 16];
       uint32_t sfw[2] = {0u, 0u};
       float lsum = 0.0f;
-      if constexpr (EFQ) {
+      if constexpr (FP8) {
+        // FP8 P: p' = 2^(x - m + 8) = 256 p, E4M3 per key (round to nearest
+        // even, the 256 keeps p' inside E4M3's range); the row sum of p'
+        const float nm8 = (m_new == -INFINITY) ? 0.0f : __fsub_rn(8.0f, m_new);
+        const uint64_t n8 = pk(nm8, nm8);
+#pragma unroll
+        for (int bk = 0; bk < 8; ++bk) {
+          uint64_t acc = 0;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float u0, u1;
+            upk(fma2(pk(s[16 * bk + 2 * i], s[16 * bk + 2 * i + 1]), c2, n8), u0, u1);
+            const float p0 = ex2_approx(u0), p1 = ex2_approx(u1);
+            const uint64_t pp = pk(p0, p1);
+            acc = (i == 0) ? pp : add2(acc, pp);
+            const uint32_t h = cvt_e4m3x2(p0, p1);
+            if (i & 1)
+              pc[4 * bk + (i >> 1)] |= h << 16;
+            else
+              pc[4 * bk + (i >> 1)] = h;
+          }
+          float a0, a1;
+          upk(acc, a0, a1);
+          lsum += a0 + a1;
+        }
+      } else if constexpr (EFQ) {
         // EFQ-Softmax: per block, E = floor(max z) - 2 and scale byte 2^(E + 10);
         // per score, code = rne(7 sat((2 (z - E) + 2) / 7)) from the bits of
         // fma(sat(s c' + o), 7, 2^23); eight codes per word by shift-and-add
@@ -497,15 +540,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         tmem_wait_st();
       }
-      // codes: the row's 64 bytes (64-byte swizzle); scales: two 4-block atoms
-      uint8_t* pbuf = sm + L::oP + stream * L::kP + row * 64;
+      if constexpr (FP8) {
+        // codes: the row's 128 bytes (128-byte swizzle)
+        uint8_t* pbuf = sm + L::oP + stream * L::kP + row * 128;
 #pragma unroll
-      for (int k2 = 0; k2 < 4; ++k2)
-        *reinterpret_cast<uint4*>(pbuf + ((k2 ^ ((row >> 1) & 3)) * 16)) =
-            make_uint4(pc[4 * k2], pc[4 * k2 + 1], pc[4 * k2 + 2], pc[4 * k2 + 3]);
-      uint8_t* psf = sm + L::oPsf + stream * 1024 + (row & 31) * 16 + (row >> 5) * 4;
-      *reinterpret_cast<uint32_t*>(psf) = sfw[0];
-      *reinterpret_cast<uint32_t*>(psf + 512) = sfw[1];
+        for (int k2 = 0; k2 < 8; ++k2)
+          *reinterpret_cast<uint4*>(pbuf + ((k2 ^ (row & 7)) * 16)) =
+              make_uint4(pc[4 * k2], pc[4 * k2 + 1], pc[4 * k2 + 2], pc[4 * k2 + 3]);
+      } else {
+        // codes: the row's 64 bytes (64-byte swizzle); scales: two 4-block atoms
+        uint8_t* pbuf = sm + L::oP + stream * L::kP + row * 64;
+#pragma unroll
+        for (int k2 = 0; k2 < 4; ++k2)
+          *reinterpret_cast<uint4*>(pbuf + ((k2 ^ ((row >> 1) & 3)) * 16)) =
+              make_uint4(pc[4 * k2], pc[4 * k2 + 1], pc[4 * k2 + 2], pc[4 * k2 + 3]);
+        uint8_t* psf = sm + L::oPsf + stream * 1024 + (row & 31) * 16 + (row >> 5) * 4;
+        *reinterpret_cast<uint32_t*>(psf) = sfw[0];
+        *reinterpret_cast<uint32_t*>(psf + 512) = sfw[1];
+      }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();

@@ -51,16 +51,24 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 using AttnKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
                             const fp4::AttnParams);
 
-// The fused kernel for head dim D and causal masking.
-AttnKernel attn_kernel(int D, int causal, int efq) {
-  if (efq) {
-    if (D == 128)
-      return causal ? fp4::attn_fwd_kernel<128, true, true> : fp4::attn_fwd_kernel<128, false, true>;
-    return causal ? fp4::attn_fwd_kernel<64, true, true> : fp4::attn_fwd_kernel<64, false, true>;
-  }
+template <int PG>
+AttnKernel attn_kernel_pg(int D, int causal) {
   if (D == 128)
-    return causal ? fp4::attn_fwd_kernel<128, true, false> : fp4::attn_fwd_kernel<128, false, false>;
-  return causal ? fp4::attn_fwd_kernel<64, true, false> : fp4::attn_fwd_kernel<64, false, false>;
+    return causal ? fp4::attn_fwd_kernel<128, true, PG> : fp4::attn_fwd_kernel<128, false, PG>;
+  return causal ? fp4::attn_fwd_kernel<64, true, PG> : fp4::attn_fwd_kernel<64, false, PG>;
+}
+
+// The fused kernel for head dim D, causal masking and P generation pg
+// (fp4::kPgExp, kPgEfq, kPgFp8).
+AttnKernel attn_kernel(int D, int causal, int pg) {
+  if (pg == fp4::kPgEfq) return attn_kernel_pg<fp4::kPgEfq>(D, causal);
+  if (pg == fp4::kPgFp8) return attn_kernel_pg<fp4::kPgFp8>(D, causal);
+  return attn_kernel_pg<fp4::kPgExp>(D, causal);
+}
+
+int attn_smem_bytes(int D, int pg) {
+  if (pg == fp4::kPgFp8) return D == 128 ? fp4::AttnSmem<128, true>::kBytes : fp4::AttnSmem<64, true>::kBytes;
+  return D == 128 ? fp4::AttnSmem<128>::kBytes : fp4::AttnSmem<64>::kBytes;
 }
 
 // sm_100 check, per-device one-time kernel attributes, SM count.
@@ -79,10 +87,10 @@ fp4_status_t device_setup(int* dev_out, int* sms_out) {
                   dev, major, minor);
     for (int d = 0; d < 2; ++d)
       for (int causal = 0; causal < 2; ++causal)
-        for (int efq = 0; efq < 2; ++efq)
-          FP4_CUDA(cudaFuncSetAttribute(attn_kernel(d ? 128 : 64, causal, efq),
+        for (int pg = 0; pg < 3; ++pg)
+          FP4_CUDA(cudaFuncSetAttribute(attn_kernel(d ? 128 : 64, causal, pg),
                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        d ? fp4::AttnSmem<128>::kBytes : fp4::AttnSmem<64>::kBytes));
+                                        attn_smem_bytes(d ? 128 : 64, pg)));
     if (!g_encode) {
       cudaDriverEntryPointQueryResult q;
       void* fn = nullptr;
@@ -123,7 +131,10 @@ size_t scales_bytes(int64_t G, int64_t N, int64_t D, fp4_axis_t axis) {
   return axis == FP4_BLOCK_ALONG_D ? (size_t)(G * Npad * D / 16) : (size_t)(G * (Npad / 64) * 512);
 }
 
-WsLayout ws_layout(int B, int H, int Hkv, int N, int D) {
+size_t fp8_codes_bytes(int64_t G, int64_t N, int64_t D) { return (size_t)(G * D * round_up(N, 128)); }
+
+// Workspace of the quantizing forwards; fp8v: V as E4M3 codes, no V scales.
+WsLayout ws_layout(int B, int H, int Hkv, int N, int D, bool fp8v = false) {
   WsLayout w;
   size_t off = 0;
   auto take = [&](size_t n) {
@@ -137,8 +148,8 @@ WsLayout ws_layout(int B, int H, int Hkv, int N, int D) {
   w.qs = take(scales_bytes(Gq, N, D, FP4_BLOCK_ALONG_D));
   w.kc = take(codes_bytes(Gk, N, D));
   w.ks = take(scales_bytes(Gk, N, D, FP4_BLOCK_ALONG_D));
-  w.vc = take(codes_bytes(Gk, N, D));
-  w.vs = take(scales_bytes(Gk, N, D, FP4_BLOCK_ALONG_N_T));
+  w.vc = take(fp8v ? fp8_codes_bytes(Gk, N, D) : codes_bytes(Gk, N, D));
+  w.vs = take(fp8v ? 0 : scales_bytes(Gk, N, D, FP4_BLOCK_ALONG_N_T));
   w.total = off;
   return w;
 }
@@ -200,10 +211,27 @@ fp4_status_t launch_quant(const void* x, int64_t G, int N, int D, fp4_axis_t axi
   return FP4_OK;
 }
 
+// V [G][N][D] bf16 -> E4M3 codes [G][D][Npad] with the tensor maximum *amax.
+fp4_status_t launch_quant_fp8(const void* x, int64_t G, int N, int D, uint8_t* codes,
+                              const float* amax, cudaStream_t stream) {
+  const int64_t Npad = round_up(N, 128);
+  const int64_t blocks = G * (Npad / 128);
+  if (blocks > INT32_MAX) return fail(FP4_ERR_INVALID_ARG, "problem too large");
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  if (D == 128)
+    fp4::quant_fp8_tokens_T_kernel<128><<<(unsigned)blocks, 128, 0, stream>>>(xb, (int)G, N,
+                                                                              (int)Npad, amax, codes);
+  else
+    fp4::quant_fp8_tokens_T_kernel<64><<<(unsigned)blocks, 128, 0, stream>>>(xb, (int)G, N,
+                                                                             (int)Npad, amax, codes);
+  FP4_CUDA(cudaGetLastError());
+  return FP4_OK;
+}
+
 fp4_status_t launch_attn(const uint8_t* qc, const uint8_t* qs, const float* qa, const uint8_t* kc,
                          const uint8_t* ks, const float* ka, const uint8_t* vc, const uint8_t* vs,
                          const float* va, void* out, int B, int H, int Hkv, int N, int D,
-                         int causal, float softmax_scale, int efq, cudaStream_t stream) {
+                         int causal, float softmax_scale, int pg, cudaStream_t stream) {
   const int64_t Npad = round_up(N, 128);
   const int64_t Gq = (int64_t)B * H, Gk = (int64_t)B * Hkv;
   const CUtensorMapSwizzle swQK =
@@ -212,8 +240,12 @@ fp4_status_t launch_attn(const uint8_t* qc, const uint8_t* qs, const float* qa, 
   fp4_status_t s;
   if ((s = tmap_2d(&tq, qc, D / 2, Gq * Npad, D / 2, 128, swQK)) != FP4_OK) return s;
   if ((s = tmap_2d(&tk, kc, D / 2, Gk * Npad, D / 2, 128, swQK)) != FP4_OK) return s;
-  if ((s = tmap_2d(&tv, vc, Npad / 2, Gk * D, 64, D, CU_TENSOR_MAP_SWIZZLE_64B)) != FP4_OK)
+  if (pg == fp4::kPgFp8) {  // E4M3 V^T: 128 one-byte keys per row, 128-byte swizzle
+    if ((s = tmap_2d(&tv, vc, Npad, Gk * D, 128, D, CU_TENSOR_MAP_SWIZZLE_128B)) != FP4_OK)
+      return s;
+  } else if ((s = tmap_2d(&tv, vc, Npad / 2, Gk * D, 64, D, CU_TENSOR_MAP_SWIZZLE_64B)) != FP4_OK) {
     return s;
+  }
   fp4::AttnParams p;
   p.q_sf = qs;
   p.k_sf = ks;
@@ -231,22 +263,22 @@ fp4_status_t launch_attn(const uint8_t* qc, const uint8_t* qs, const float* qa, 
                         ? softmax_scale
                         : 1.0f / std::sqrt((float)D);
   dim3 grid(p.ntq, H, B);
-  const int smem = D == 128 ? fp4::AttnSmem<128>::kBytes : fp4::AttnSmem<64>::kBytes;
-  attn_kernel(D, causal, efq)<<<grid, fp4::kAttnThreads, smem, stream>>>(tq, tk, tv, p);
+  attn_kernel(D, causal, pg)<<<grid, fp4::kAttnThreads, attn_smem_bytes(D, pg), stream>>>(tq, tk, tv,
+                                                                                       p);
   FP4_CUDA(cudaGetLastError());
   return FP4_OK;
 }
 
 fp4_status_t attn_fwd_any(const void* q, const void* k, const void* v, void* out, int B, int H,
                           int Hkv, int N, int D, int causal, float softmax_scale, void* stream,
-                          void* workspace, size_t workspace_bytes, int efq) {
+                          void* workspace, size_t workspace_bytes, int pg) {
   g_last_error.clear();
   fp4_status_t s;
   if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
   if (!q || !k || !v || !out || !workspace) return fail(FP4_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace))
     return fail(FP4_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
-  const WsLayout w = ws_layout(B, H, Hkv, N, D);
+  const WsLayout w = ws_layout(B, H, Hkv, N, D, pg == fp4::kPgFp8);
   if (workspace_bytes < w.total)
     return fail(FP4_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, w.total);
   int dev, sms;
@@ -263,25 +295,31 @@ fp4_status_t attn_fwd_any(const void* q, const void* k, const void* v, void* out
   if ((s = launch_quant(k, (int64_t)B * Hkv, N, D, FP4_BLOCK_ALONG_D, ws + w.kc, ws + w.ks,
                         amax + 1, sms, st)) != FP4_OK)
     return s;
-  if ((s = launch_quant(v, (int64_t)B * Hkv, N, D, FP4_BLOCK_ALONG_N_T, ws + w.vc, ws + w.vs,
-                        amax + 2, sms, st)) != FP4_OK)
-    return s;
+  if (pg == fp4::kPgFp8)
+    s = launch_quant_fp8(v, (int64_t)B * Hkv, N, D, ws + w.vc, amax + 2, st);
+  else
+    s = launch_quant(v, (int64_t)B * Hkv, N, D, FP4_BLOCK_ALONG_N_T, ws + w.vc, ws + w.vs,
+                     amax + 2, sms, st);
+  if (s != FP4_OK) return s;
   return launch_attn(ws + w.qc, ws + w.qs, amax, ws + w.kc, ws + w.ks, amax + 1, ws + w.vc,
-                     ws + w.vs, amax + 2, out, B, H, Hkv, N, D, causal, softmax_scale, efq, st);
+                     ws + w.vs, amax + 2, out, B, H, Hkv, N, D, causal, softmax_scale, pg, st);
 }
 
 fp4_status_t attn_fwd_quantized_any(const fp4_tensor_t* q, const fp4_tensor_t* k,
                                     const fp4_tensor_t* v, void* out, int B, int H, int Hkv,
                                     int N, int D, int causal, float softmax_scale, void* stream,
-                                    int efq) {
+                                    int pg) {
   g_last_error.clear();
   fp4_status_t s;
   if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
   if (!q || !k || !v || !out) return fail(FP4_ERR_INVALID_ARG, "null pointer");
   const fp4_tensor_t* t[3] = {q, k, v};
-  for (auto* x : t) {
-    if (!x->codes || !x->scales || !x->amax) return fail(FP4_ERR_INVALID_ARG, "null pointer");
-    if (!aligned16(x->codes) || !aligned16(x->scales) ||
+  for (int i = 0; i < 3; ++i) {
+    const fp4_tensor_t* x = t[i];
+    const bool no_scales = i == 2 && pg == fp4::kPgFp8;  // E4M3 V has no block scales
+    if (!x->codes || (!x->scales && !no_scales) || !x->amax)
+      return fail(FP4_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(x->codes) || (!no_scales && !aligned16(x->scales)) ||
         (reinterpret_cast<uintptr_t>(x->amax) & 3u))
       return fail(FP4_ERR_INVALID_ARG, "codes/scales must be 16-byte aligned");
   }
@@ -289,7 +327,7 @@ fp4_status_t attn_fwd_quantized_any(const fp4_tensor_t* q, const fp4_tensor_t* k
   int dev, sms;
   if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
   return launch_attn(q->codes, q->scales, q->amax, k->codes, k->scales, k->amax, v->codes,
-                     v->scales, v->amax, out, B, H, Hkv, N, D, causal, softmax_scale, efq,
+                     v->scales, v->amax, out, B, H, Hkv, N, D, causal, softmax_scale, pg,
                      static_cast<cudaStream_t>(stream));
 }
 
@@ -310,6 +348,46 @@ size_t fp4_scales_bytes(int G, int N, int D, fp4_axis_t axis) {
 size_t fp4_attn_workspace_bytes(int B, int H, int Hkv, int N, int D) {
   if (check_shape(B, H, Hkv, N, D) != FP4_OK) return 0;
   return ws_layout(B, H, Hkv, N, D).total;
+}
+
+size_t fp4_attn_workspace_bytes_fp8pv(int B, int H, int Hkv, int N, int D) {
+  if (check_shape(B, H, Hkv, N, D) != FP4_OK) return 0;
+  return ws_layout(B, H, Hkv, N, D, true).total;
+}
+
+size_t fp4_fp8_codes_bytes(int G, int N, int D) {
+  if (G < 1 || N < 1 || D < 16) return 0;
+  return fp8_codes_bytes(G, N, D);
+}
+
+fp4_status_t fp4_quantize_fp8(const void* x, int G, int N, int D, uint8_t* codes, float* amax,
+                              void* stream) {
+  g_last_error.clear();
+  fp4_status_t s;
+  if ((s = check_shape(1, G, G, N, D)) != FP4_OK) return s;
+  if (!x || !codes || !amax) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(amax) & 3u))
+    return fail(FP4_ERR_INVALID_ARG, "x and codes must be 16-byte aligned, amax 4-byte aligned");
+  int dev, sms;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = launch_amax(x, (int64_t)G * N * D, nullptr, 0, nullptr, 0, amax, nullptr, nullptr, sms,
+                       st)) != FP4_OK)
+    return s;
+  return launch_quant_fp8(x, G, N, D, codes, amax, st);
+}
+
+fp4_status_t fp4_quantize_fp8_scaled(const void* x, int G, int N, int D, const float* amax,
+                                     uint8_t* codes, void* stream) {
+  g_last_error.clear();
+  fp4_status_t s;
+  if ((s = check_shape(1, G, G, N, D)) != FP4_OK) return s;
+  if (!x || !codes || !amax) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(amax) & 3u))
+    return fail(FP4_ERR_INVALID_ARG, "x and codes must be 16-byte aligned, amax 4-byte aligned");
+  int dev, sms;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  return launch_quant_fp8(x, G, N, D, codes, amax, static_cast<cudaStream_t>(stream));
 }
 
 fp4_status_t fp4_quantize(const void* x, int G, int N, int D, fp4_axis_t axis, uint8_t* codes,
@@ -388,6 +466,20 @@ fp4_status_t fp4_attn_fwd_quantized_efq(const fp4_tensor_t* q, const fp4_tensor_
                                         int N, int D, int causal, float softmax_scale,
                                         void* stream) {
   return attn_fwd_quantized_any(q, k, v, out, B, H, Hkv, N, D, causal, softmax_scale, stream, 1);
+}
+
+fp4_status_t fp4_attn_fwd_fp8pv(const void* q, const void* k, const void* v, void* out, int B,
+                                int H, int Hkv, int N, int D, int causal, float softmax_scale,
+                                void* stream, void* workspace, size_t workspace_bytes) {
+  return attn_fwd_any(q, k, v, out, B, H, Hkv, N, D, causal, softmax_scale, stream, workspace,
+                      workspace_bytes, 2);
+}
+
+fp4_status_t fp4_attn_fwd_quantized_fp8pv(const fp4_tensor_t* q, const fp4_tensor_t* k,
+                                          const fp4_tensor_t* v, void* out, int B, int H, int Hkv,
+                                          int N, int D, int causal, float softmax_scale,
+                                          void* stream) {
+  return attn_fwd_quantized_any(q, k, v, out, B, H, Hkv, N, D, causal, softmax_scale, stream, 2);
 }
 
 

@@ -97,8 +97,8 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 
 // Shared-memory matrix descriptor (tcgen05 format, version 1).
-//   layout: 0 = no swizzle (core matrices 8 rows x 16 B), 4 = 64-byte swizzle,
-//   6 = 32-byte swizzle. lbo/sbo in bytes.
+//   layout: 0 = no swizzle (core matrices 8 rows x 16 B), 2 = 128-byte swizzle,
+//   4 = 64-byte swizzle, 6 = 32-byte swizzle. lbo/sbo in bytes.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
                                               uint32_t layout) {
   uint64_t d = 0;
@@ -126,6 +126,23 @@ __device__ __forceinline__ void mma_mxf4nvf4(uint32_t d_tmem, uint64_t a_desc, u
       "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X"
       " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Instruction descriptor of kind::f8f6f4 with E4M3 A and B (both K-major),
+// FP32 accumulation, K = 32 per instruction.
+__host__ __device__ constexpr uint32_t idesc_f8e4m3(uint32_t M, uint32_t N) {
+  return (1u << 4) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, E4M3 operands, no block scales.
+__device__ __forceinline__ void mma_f8e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -195,6 +212,13 @@ __device__ __forceinline__ uint32_t cvt_e4m3(float x) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
   return r & 0xFFu;
+}
+// Two values -> two E4M3 bytes (round to nearest even, saturating to +-448),
+// lo in the low byte.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 // Exact value of an E4M3 byte.
 __device__ __forceinline__ float e4m3_to_f32(uint32_t e) {

@@ -207,6 +207,55 @@ __global__ void __launch_bounds__(128) quant_tokens_T_kernel(const __nv_bfloat16
   }
 }
 
+// FP8 (E4M3) V for the FP8 P/V variant [SageAttention2 abstract: P~ and V in
+// FP8]: one fp32 scale per tensor, s8 = 448 / amax (1 if amax == 0, FLT_MAX on
+// overflow), code = E4M3(fl(v s8)), round to nearest even, saturating.
+__device__ __forceinline__ float fp8_senc(float amax) {
+  float s = (amax > 0.0f) ? __fdiv_rn(448.0f, amax) : 1.0f;
+  if (!isfinite(s)) s = FLT_MAX;
+  return s;
+}
+
+// v [G][N][D] bf16 -> codes [G][D][Npad] (channel-major, tokens >= N zero):
+// one CTA per 128-token tile, staged in shared memory, one thread per channel
+// writing its 128 codes.
+template <int D>
+__global__ void __launch_bounds__(128) quant_fp8_tokens_T_kernel(const __nv_bfloat16* __restrict__ v,
+                                                                 int G, int N, int Npad,
+                                                                 const float* __restrict__ amax,
+                                                                 uint8_t* __restrict__ codes) {
+  __shared__ __align__(16) uint16_t tile[128 * D];
+  const int ntile = Npad >> 7;
+  const int64_t g = blockIdx.x / ntile;
+  const int t = blockIdx.x % ntile;
+  const float s8 = fp8_senc(*amax);
+  constexpr int VEC = D / 8;  // uint4 per token row
+  for (int idx = threadIdx.x; idx < 128 * VEC; idx += blockDim.x) {
+    const int tok = idx / VEC, c = idx % VEC;
+    const int n = t * 128 + tok;
+    uint4 w = make_uint4(0, 0, 0, 0);
+    if (n < N) w = ld_nc_v4(v + ((g * N + n) * D + c * 8));
+    *reinterpret_cast<uint4*>(&tile[tok * D + c * 8]) = w;
+  }
+  __syncthreads();
+  const int d = threadIdx.x;
+  if (d < D) {
+    uint32_t out[32];
+#pragma unroll
+    for (int w4 = 0; w4 < 32; ++w4) {
+      float x[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        x[i] = __fmul_rn(__uint_as_float((uint32_t)tile[(w4 * 4 + i) * D + d] << 16), s8);
+      out[w4] = cvt_e4m3x2(x[0], x[1]) | (cvt_e4m3x2(x[2], x[3]) << 16);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(codes + (g * D + d) * (int64_t)Npad + t * 128);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      dst[k] = make_uint4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
+  }
+}
+
 // Hardware conversion probe over fp32 bit patterns start + i: kind 0 gives
 // the E2M1 code (one per byte), kind 1 the E4M3 byte.
 __global__ void probe_cvt_kernel(uint32_t start, int64_t count, int kind, uint8_t* __restrict__ out) {

@@ -55,7 +55,8 @@ def allreduce_max_(t, group=None):
 
 
 def fp4_attn_fwd_sharded(q, k, v, causal: bool = False, softmax_scale: float | None = None,
-                         group=None, out=None, stream=None, efq: bool = False):
+                         group=None, out=None, stream=None, efq: bool = False,
+                         fp8pv: bool = False):
     """This rank's part of a head-sharded NVFP4 attention forward.
 
     q: this rank's query heads, a contiguous bf16 CUDA tensor [..., N, D] whose
@@ -63,10 +64,11 @@ def fp4_attn_fwd_sharded(q, k, v, causal: bool = False, softmax_scale: float | N
     heads, [..., N, D]. Every rank of `group` calls this with the same N, D,
     G, causal and softmax_scale, an empty shard (U = 0) included: it still
     takes part in the all-reduce. Returns `out` (like q) with this rank's
-    output heads. efq selects the EFQ-Softmax P generation."""
+    output heads. efq selects the EFQ-Softmax P generation, fp8pv the FP8 P
+    and V variant."""
     import torch
     from . import (FP4_BLOCK_ALONG_D, FP4_BLOCK_ALONG_N_T, fp4_amax, fp4_attn_fwd_quantized,
-                   fp4_quantize)
+                   fp4_quantize, fp4_quantize_fp8)
     N, D = q.shape[-2], q.shape[-1]
     if k.shape[-2:] != (N, D) or v.shape != k.shape:
         raise ValueError("q, k, v must share N and D, and k and v their shape")
@@ -85,7 +87,10 @@ def fp4_attn_fwd_sharded(q, k, v, causal: bool = False, softmax_scale: float | N
         return out
     qq = fp4_quantize(q, FP4_BLOCK_ALONG_D, stream, amax=amax[0:1])
     kq = fp4_quantize(k, FP4_BLOCK_ALONG_D, stream, amax=amax[1:2])
-    vq = fp4_quantize(v, FP4_BLOCK_ALONG_N_T, stream, amax=amax[2:3])
+    if fp8pv:
+        vq = fp4_quantize_fp8(v, stream, amax=amax[2:3])
+    else:
+        vq = fp4_quantize(v, FP4_BLOCK_ALONG_N_T, stream, amax=amax[2:3])
     fp4_attn_fwd_quantized(qq, kq, vq, 1, gq, gkv, causal, softmax_scale, out=out, stream=stream,
-                           efq=efq)
+                           efq=efq, fp8pv=fp8pv)
     return out

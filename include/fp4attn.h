@@ -189,6 +189,46 @@ fp4_status_t fp4_attn_fwd_quantized_efq(const fp4_tensor_t* q, const fp4_tensor_
                                         void* stream);
 
 /*
+ * FP8 V (the FP8 P/V variant below): x [G][N][D] bf16 -> E4M3 codes
+ * [G][D][Npad] (one byte per element, channel-major, keys >= N zero; Npad = N
+ * rounded up to 128). SageAttention2 abstract (searcharxiv.com author page
+ * "Pengle Zhang": P~ and V in FP8 for the PV product) gives no recipe; the
+ * reading: one fp32 scale per tensor, s8 = 448 / amax (1 if amax == 0, FLT_MAX
+ * if the quotient overflows), code = E4M3(fl(v s8)), round to nearest even,
+ * saturating; v~ = dec(code) / s8. Steps: *amax = max |x| (written, stream
+ * order), then the codes. fp4_fp8_codes_bytes gives the size of codes (0 for a
+ * bad shape). x and codes 16-byte aligned, amax 4-byte aligned, all device
+ * memory, caller-owned. Errors: as fp4_quantize.
+ */
+size_t fp4_fp8_codes_bytes(int G, int N, int D);
+fp4_status_t fp4_quantize_fp8(const void* x, int G, int N, int D, uint8_t* codes, float* amax,
+                              void* stream);
+/* The codes step alone, with a given tensor maximum *amax (device memory, read
+ * only; e.g. combined over shards as for fp4_quantize_scaled). */
+fp4_status_t fp4_quantize_fp8_scaled(const void* x, int G, int N, int D, const float* amax,
+                                     uint8_t* codes, void* stream);
+
+/*
+ * The FP8 P/V variant of fp4_attn_fwd / fp4_attn_fwd_quantized (same
+ * arguments, layouts and errors, except as stated). Q and K and S = QK^T as in
+ * the method; V quantised by fp4_quantize_fp8; P per key in E4M3 without block
+ * scales: p~ = E4M3(fl(256 p)) / 256 with p = 2^(x - m) (the 256 keeps every
+ * p <= 1 inside E4M3's range and its subnormals below 2^-17); O = P~ V~ as a
+ * tcgen05 kind::f8f6f4 contraction; l sums the unquantised p; out = O / l.
+ * fp4_attn_fwd_fp8pv needs fp4_attn_workspace_bytes_fp8pv bytes of workspace.
+ * fp4_attn_fwd_quantized_fp8pv takes v->codes from fp4_quantize_fp8 and
+ * v->amax its maximum; v->scales is not read and may be NULL.
+ */
+size_t fp4_attn_workspace_bytes_fp8pv(int B, int H, int Hkv, int N, int D);
+fp4_status_t fp4_attn_fwd_fp8pv(const void* q, const void* k, const void* v, void* out, int B,
+                                int H, int Hkv, int N, int D, int causal, float softmax_scale,
+                                void* stream, void* workspace, size_t workspace_bytes);
+fp4_status_t fp4_attn_fwd_quantized_fp8pv(const fp4_tensor_t* q, const fp4_tensor_t* k,
+                                          const fp4_tensor_t* v, void* out, int B, int H, int Hkv,
+                                          int N, int D, int causal, float softmax_scale,
+                                          void* stream);
+
+/*
  * fp4_attn_fwd without a caller-supplied workspace, for callers that cannot
  * allocate device memory: code whose device memory is owned by a host
  * framework that hands it no allocator, or code that must not call

@@ -42,6 +42,13 @@ def test_sizes(L):
     assert ws >= 2 * 8 * 1024 * 64 + 2 * 2 * 1024 * 64 * 2
     assert fa.fp4_attn_workspace_bytes(1, 3, 2, 10, 128) == 0  # H % Hkv != 0
     assert fa.fp4_attn_workspace_bytes(1, 1, 1, 10, 96) == 0   # unsupported D
+    # FP8 V: one byte per element, channel-major over Npad tokens, no scales
+    assert fa.fp4_fp8_codes_bytes(3, 300, 64) == 3 * 64 * 384
+    assert fa.fp4_fp8_codes_bytes(0, 300, 64) == 0
+    ws8 = fa.fp4_attn_workspace_bytes_fp8pv(2, 8, 2, 1000, 128)
+    assert ws8 >= 2 * 8 * 1024 * 64 + 2 * 1024 * 64 * 2 + 2 * 2 * 128 * 1024
+    assert ws8 > ws  # V codes twice as large, V block scales dropped
+    assert fa.fp4_attn_workspace_bytes_fp8pv(1, 3, 2, 10, 128) == 0
 
 
 def _call_fwd(L, q=16, k=16, v=16, out=16, B=1, H=1, Hkv=1, N=8, D=128, ws=1 << 20,
@@ -83,6 +90,30 @@ def test_argument_errors_launch_nothing(L):
     assert L.fp4_test_wait_timeout(6_000_000_000, vp(16), vp(0)) == fa.FP4_ERR_INVALID_ARG
     assert L.fp4_test_wait_timeout(1000, vp(0), vp(0)) == fa.FP4_ERR_INVALID_ARG
     assert L.fp4_probe_cvt(0, 16, 3, vp(16), vp(0)) == fa.FP4_ERR_INVALID_ARG
+    # the FP8 P/V entries: same checks, before any launch
+    assert L.fp4_attn_fwd_fp8pv(vp(16), vp(16), vp(16), vp(16), 1, 1, 1, 8, 96, 0, 0.0, vp(0),
+                                vp(16), 1 << 30) == fa.FP4_ERR_UNSUPPORTED
+    need = fa.fp4_attn_workspace_bytes_fp8pv(1, 1, 1, 8, 128)
+    assert L.fp4_attn_fwd_fp8pv(vp(16), vp(16), vp(16), vp(16), 1, 1, 1, 8, 128, 0, 0.0, vp(0),
+                                vp(16), need - 1) == fa.FP4_ERR_WORKSPACE
+    assert L.fp4_quantize_fp8(vp(16), 1, 8, 128, vp(0), vp(16), vp(0)) == fa.FP4_ERR_INVALID_ARG
+    assert L.fp4_quantize_fp8(vp(16), 1, 8, 128, vp(24), vp(16), vp(0)) == fa.FP4_ERR_INVALID_ARG
+    assert L.fp4_quantize_fp8(vp(16), 1, 8, 96, vp(16), vp(16), vp(0)) == fa.FP4_ERR_UNSUPPORTED
+    assert L.fp4_quantize_fp8_scaled(vp(16), 1, 8, 128, vp(18), vp(16), vp(0)) == \
+        fa.FP4_ERR_INVALID_ARG
+    assert L.fp4_quantize_fp8_scaled(vp(16), 1, 0, 128, vp(16), vp(16), vp(0)) == \
+        fa.FP4_ERR_INVALID_ARG
+    t = fa._Tensor(16, 16, 16)
+    t0 = fa._Tensor(16, 0, 16)  # FP8 V: scales not read, may be NULL
+    assert L.fp4_attn_fwd_quantized_fp8pv(ctypes.byref(t), ctypes.byref(t), ctypes.byref(t0),
+                                          vp(16), 1, 3, 2, 8, 128, 0, 0.0, vp(0)) == \
+        fa.FP4_ERR_INVALID_ARG  # H % Hkv
+    assert L.fp4_attn_fwd_quantized_fp8pv(ctypes.byref(t0), ctypes.byref(t), ctypes.byref(t0),
+                                          vp(16), 1, 1, 1, 8, 128, 0, 0.0, vp(0)) == \
+        fa.FP4_ERR_INVALID_ARG  # Q without scales
+    assert L.fp4_attn_fwd_quantized(ctypes.byref(t), ctypes.byref(t), ctypes.byref(t0),
+                                    vp(16), 1, 1, 1, 8, 128, 0, 0.0, vp(0)) == \
+        fa.FP4_ERR_INVALID_ARG  # NVFP4 V without scales
 
 
 def test_product_path_does_not_touch_the_oracle():
