@@ -25,6 +25,8 @@ FLAG_FLIP_BOUND = 2
 FLAG_PERTURB_P = 4
 FLAG_EFQ = 8  # EFQ-Softmax P generation (exp-free), denominator from its p~
 FLAG_FP8PV = 16  # P and V quantised to FP8 E4M3 for the PV product
+FLAG_SMOOTH_K = 32  # K smoothed: channel mean over tokens subtracted before quantisation
+FLAG_SMOOTH_Q = 64  # Q smoothed likewise, the score correction mean_Q . k_j added back
 
 
 def build(force: bool = False) -> str:
@@ -64,6 +66,14 @@ def _load():
         lib.ora_quantize_block.restype = None
         lib.ora_quantize_rows.argtypes = [vp, i64, i32, f32, vp, vp, i32]
         lib.ora_quantize_rows.restype = None
+        lib.ora_quantize_rows_smoothed.argtypes = [vp, i64, i32, f32, vp, vp, vp, i32]
+        lib.ora_quantize_rows_smoothed.restype = None
+        lib.ora_channel_mean.argtypes = [vp, i32, i32, f32, vp]
+        lib.ora_channel_mean.restype = None
+        lib.ora_smoothed_amax.argtypes = [vp, i64, i32, i32, vp]
+        lib.ora_smoothed_amax.restype = f32
+        lib.ora_score_bias.argtypes = [vp, vp, vp, i32, i32, f32, vp]
+        lib.ora_score_bias.restype = None
         lib.ora_quantize_tokens_T.argtypes = [vp, i32, i32, f32, vp, vp, i32]
         lib.ora_quantize_tokens_T.restype = None
         lib.ora_fp8_tensor_scale.argtypes = [f32, vp, vp]
@@ -153,6 +163,55 @@ def quantize_rows(x_bf16: np.ndarray, s_enc: float, threads: int | None = None):
     _load().ora_quantize_rows(x.ctypes.data, rows, D, float(s_enc), codes.ctypes.data,
                               scales.ctypes.data, _threads(threads))
     return codes, scales
+
+
+def quantize_rows_smoothed(x_bf16: np.ndarray, s_enc: float, mean, threads: int | None = None):
+    """quantize_rows of the smoothed values fl32(x - mean) (mean: D fp32 values,
+    one per column). Returns (codes, scales)."""
+    x = _c(x_bf16, np.uint16)
+    D = x.shape[-1]
+    mean = _c(mean, np.float32)
+    assert mean.size == D
+    codes = np.empty(x.shape[:-1] + (D // 2,), dtype=np.uint8)
+    scales = np.empty(x.shape[:-1] + (D // 16,), dtype=np.uint8)
+    _load().ora_quantize_rows_smoothed(x.ctypes.data, x.size // D, D, float(s_enc),
+                                       mean.ctypes.data, codes.ctypes.data, scales.ctypes.data,
+                                       _threads(threads))
+    return codes, scales
+
+
+def channel_mean(x_bf16: np.ndarray, amax: float) -> np.ndarray:
+    """Smoothing means of one head's slab x [N, D] (bf16 bits): D fp32 values,
+    on the fixed-point grid set by `amax` (max |x| of the whole raw tensor)."""
+    x = _c(x_bf16, np.uint16)
+    N, D = x.shape
+    mean = np.empty(D, dtype=np.float32)
+    _load().ora_channel_mean(x.ctypes.data, N, D, float(amax), mean.ctypes.data)
+    return mean
+
+
+def smoothed_amax(x_bf16: np.ndarray, means: np.ndarray) -> float:
+    """max |fl32(x - mean)| over slabs x [G, N, D] with means [G, D]."""
+    x = _c(x_bf16, np.uint16)
+    G, N, D = x.shape
+    means = _c(means, np.float32)
+    assert means.shape == (G, D)
+    return float(_load().ora_smoothed_amax(x.ctypes.data, G, N, D, means.ctypes.data))
+
+
+def score_bias(qmean, k_bf16: np.ndarray, kmean, cs: float) -> np.ndarray:
+    """Score correction of one query head: fl32(delta_j cs), delta_j = qmean . k'_j
+    (an fp32 fma chain; k' = fl32(k - kmean), or k when kmean is None).
+    k [N, D] bf16 bits; returns N fp32 values."""
+    k = _c(k_bf16, np.uint16)
+    N, D = k.shape
+    qmean = _c(qmean, np.float32)
+    km = None if kmean is None else _c(kmean, np.float32)
+    out = np.empty(N, dtype=np.float32)
+    _load().ora_score_bias(qmean.ctypes.data, k.ctypes.data,
+                           None if km is None else km.ctypes.data, N, D, float(cs),
+                           out.ctypes.data)
+    return out
 
 
 def quantize_tokens_T(x_bf16: np.ndarray, s_enc: float, npad: int | None = None):

@@ -22,6 +22,10 @@
 //    from the shifted scores by an exponent-only block scale and one affine
 //    rule, the same operand in numerator and denominator [EFQ-Softmax
 //    abstract]; the reading is at efq_block.
+//  * Flags 32 and 64 smooth K and Q before quantisation (mean subtraction per
+//    channel, with the score correction that keeps the softmax exact)
+//    [SageAttention2 abstract, searcharxiv.com author page "Pengle Zhang"];
+//    the reading is at channel_mean.
 // The pages give no formula for any of these steps. Where this file fixes one
 // (format constants, scale recipe, rounding, masking, GQA mapping, the
 // denominator) it states the reading it takes.
@@ -191,14 +195,19 @@ void parallel_for(int64_t n, int nthreads, F&& f) {
 // Rows of `cols` values, blocks of 16 along the row (Q and K: along D).
 // codes [rows][cols/2]: element 2i in the low nibble of byte i.
 // scales [rows][cols/16].
+// With `mean` (one fp32 per column; the smoothing of flags 32 and 64) the
+// quantised values are the smoothed fl32(x - mean[col]).
 void quantize_rows(const uint16_t* x, int64_t rows, int cols, float s_enc, uint8_t* codes,
-                   uint8_t* scales, int nthreads) {
+                   uint8_t* scales, int nthreads, const float* mean = nullptr) {
   const int nb = cols / 16;
   parallel_for(rows, nthreads, [&](int64_t r) {
     float blk[16];
     uint8_t c[16];
     for (int b = 0; b < nb; ++b) {
-      for (int i = 0; i < 16; ++i) blk[i] = bf16_to_f32(x[r * cols + b * 16 + i]);
+      for (int i = 0; i < 16; ++i) {
+        blk[i] = bf16_to_f32(x[r * cols + b * 16 + i]);
+        if (mean) blk[i] = blk[i] - mean[b * 16 + i];
+      }
       quantize_block(blk, 16, s_enc, c, &scales[r * nb + b]);
       for (int i = 0; i < 8; ++i)
         codes[r * (cols / 2) + b * 8 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
@@ -254,11 +263,77 @@ inline double deq(uint8_t code, uint8_t scale) {
 
 const float kLog2e = 1.44269504088896340736f;  // fl32(1 / ln 2)
 
+// -------------------------------------------- smoothing (flags 32, 64) ----
+// Outlier smoothing [SageAttention2 abstract, searcharxiv.com author page
+// "Pengle Zhang": Q is smoothed to make the low-bit QK^T more accurate]. The
+// page gives no formula; the reading taken here:
+//   per (batch, head) and channel d, the mean over the head's N tokens,
+//   x'_nd = fl32(x_nd - mean_d), quantised as usual (tensor scale from
+//   max |x'| over the whole smoothed tensor).
+//   K (flag 32): S_ij changes by -q_i . mean_K, the same for every key of
+//   row i, which the softmax cancels: nothing is added back.
+//   Q (flag 64): q_i . k_j = q'_i . k_j + mean_Q . k_j; the second term
+//   depends on the key, so it is added back to the scores in fp32:
+//   delta_j = mean_Q . k'_j (k' the smoothed K under flag 32, else K), and
+//   x_ij = fl32(S'_ij c + fl32(delta_j cs)) with one rounding (fma),
+//   cs = fl32(softmax_scale log2 e).
+// The mean is made independent of summation order so that it is one value on
+// any machine: every element is truncated toward zero to the fixed-point
+// grid 2^-s with s = 44 - E, 2^(E-1) <= amax < 2^E (amax of the raw tensor),
+// the integers are summed exactly (|x| 2^s < 2^44, so N <= 2^19 tokens fit in
+// 64 bits), and mean = fl32(fl64(fl64(T) 2^-s) / N); amax == 0 gives 0.
+// delta_j is a sequential fp32 fma chain over d = 0 .. D-1 from 0.
+const int kMeanGridBits = 44;
+
+void channel_mean(const uint16_t* x, int N, int D, float amax, float* mean) {
+  if (!(amax > 0.0f)) {
+    for (int d = 0; d < D; ++d) mean[d] = 0.0f;
+    return;
+  }
+  int E;
+  std::frexp(amax, &E);
+  const int s = kMeanGridBits - E;
+  for (int d = 0; d < D; ++d) {
+    int64_t T = 0;
+    for (int64_t n = 0; n < N; ++n)
+      T += (int64_t)std::trunc(std::ldexp((double)bf16_to_f32(x[n * D + d]), s));
+    mean[d] = (float)(std::ldexp((double)T, -s) / (double)N);
+  }
+}
+
+// max |fl32(x - mean)| over G slabs [N][D] with means [G][D].
+float smoothed_amax(const uint16_t* x, int64_t G, int N, int D, const float* mean) {
+  float a = 0.0f;
+  for (int64_t g = 0; g < G; ++g)
+    for (int64_t n = 0; n < N; ++n)
+      for (int d = 0; d < D; ++d)
+        a = std::max(a, std::fabs(bf16_to_f32(x[(g * N + n) * D + d]) - mean[g * D + d]));
+  return a;
+}
+
+// delta_j cs for the N keys of one head: qmean [D]; k [N][D] bf16; kmean [D]
+// (NULL: K not smoothed).
+void score_bias(const float* qmean, const uint16_t* k, const float* kmean, int N, int D, float cs,
+                float* out) {
+  for (int64_t j = 0; j < N; ++j) {
+    float delta = 0.0f;
+    for (int d = 0; d < D; ++d) {
+      float kv = bf16_to_f32(k[j * D + d]);
+      if (kmean) kv = kv - kmean[d];
+      delta = std::fmaf(qmean[d], kv, delta);
+    }
+    out[j] = delta * cs;
+  }
+}
+
 struct Tensors {
   const uint16_t *q, *k, *v;
   int B, H, Hkv, N, D;
   float sq, dq, sk, dk, sv, dv;
-  bool fp8v;  // V in FP8 (flag 16): sv, dv are s8, d8
+  bool fp8v;                   // V in FP8 (flag 16): sv, dv are s8, d8
+  const float* qmean = nullptr;  // flag 64: [B*H][D]
+  const float* kmean = nullptr;  // flag 32: [B*Hkv][D]
+  const float* bias = nullptr;   // flag 64: [B*H][N], delta_j cs
 };
 
 // K and V of one (b, kv-head), dequantised to contraction units, [N][D].
@@ -273,7 +348,8 @@ KVGroup make_group(const Tensors& T, int b, int hk) {
   g.K.resize((size_t)N * D);
   g.V.resize((size_t)N * D);
   std::vector<uint8_t> kc((size_t)N * D / 2), ks((size_t)N * D / 16);
-  quantize_rows(T.k + off, N, D, T.sk, kc.data(), ks.data(), 1);
+  quantize_rows(T.k + off, N, D, T.sk, kc.data(), ks.data(), 1,
+                T.kmean ? T.kmean + ((int64_t)b * T.Hkv + hk) * D : nullptr);
   for (int64_t n = 0; n < N; ++n)
     for (int d = 0; d < D; ++d) {
       uint8_t byte = kc[n * (D / 2) + d / 2];
@@ -300,6 +376,7 @@ KVGroup make_group(const Tensors& T, int b, int hk) {
 }
 
 enum { FLAG_QP_DENOMINATOR = 1, FLAG_FLIP_BOUND = 2, FLAG_PERTURB_P = 4, FLAG_EFQ = 8,
+       FLAG_SMOOTH_K = 32, FLAG_SMOOTH_Q = 64,
        FLAG_FP8PV = 16 };
 
 // FP8 P (flag 16): p~ = E4M3(fl(p * 256)) / 256, round to nearest even; p <= 1
@@ -448,6 +525,7 @@ void efq_tile(const std::vector<float>& x, const std::vector<double>& A, double 
 // One query row: the tiled forward over key tiles of Bc keys.
 //   S_ij = fl32(exact dot product of dequantised q_i, k_j)
 //   x_ij = fl32(S_ij * c), c = fl32(fl32(fl32(d_Q d_K) * softmax_scale) * log2 e)
+//          (flag 64: fl32(S_ij * c + bias_j) with one rounding)
 //   masked (causal j > i, top-left aligned) -> -inf
 // per tile: m_new = max(m, max_j x_ij); alpha = exp2(m - m_new) (0 while m is -inf)
 //   p_ij = fl32(exp2(x_ij - m_new)) (double exp2, rounded once)
@@ -479,7 +557,9 @@ void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float 
   // quantise the query row
   const uint16_t* qrow = T.q + (((int64_t)b * T.H + h) * N + i) * D;
   std::vector<uint8_t> qc(D / 2), qs(D / 16);
-  quantize_rows(qrow, 1, D, T.sq, qc.data(), qs.data(), 1);
+  quantize_rows(qrow, 1, D, T.sq, qc.data(), qs.data(), 1,
+                T.qmean ? T.qmean + ((int64_t)b * T.H + h) * D : nullptr);
+  const float* brow = T.bias ? T.bias + ((int64_t)b * T.H + h) * N : nullptr;
   std::vector<double> qd(D);
   for (int d = 0; d < D; ++d) {
     uint8_t byte = qc[d / 2];
@@ -513,7 +593,7 @@ void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float 
         if (want_flip)
           for (int d = 0; d < D; ++d) aj += std::fabs(qd[d] * kr[d]);
         float sf = (float)s;
-        xv = sf * c;
+        xv = brow ? std::fmaf(sf, c, brow[j]) : sf * c;
       }
       x[j - j0] = xv;
       A[j - j0] = aj;
@@ -694,6 +774,27 @@ void ora_quantize_rows(const uint16_t* x, int64_t rows, int cols, float s_enc, u
   quantize_rows(x, rows, cols, s_enc, codes, scales, nthreads);
 }
 
+// Smoothed rows: the values fl32(x - mean[col]) (mean: one fp32 per column).
+void ora_quantize_rows_smoothed(const uint16_t* x, int64_t rows, int cols, float s_enc,
+                                const float* mean, uint8_t* codes, uint8_t* scales, int nthreads) {
+  e4m3_encode(0.0f);
+  quantize_rows(x, rows, cols, s_enc, codes, scales, nthreads, mean);
+}
+
+// Smoothing (flags 32, 64): the channel means of one head's slab x [N][D]
+// (amax: max |x| of the whole raw tensor), max |x - mean| over G slabs, and
+// the score bias delta_j cs of one query head (kmean may be NULL).
+void ora_channel_mean(const uint16_t* x, int N, int D, float amax, float* mean) {
+  channel_mean(x, N, D, amax, mean);
+}
+float ora_smoothed_amax(const uint16_t* x, int64_t G, int N, int D, const float* mean) {
+  return smoothed_amax(x, G, N, D, mean);
+}
+void ora_score_bias(const float* qmean, const uint16_t* k, const float* kmean, int N, int D,
+                    float cs, float* out) {
+  score_bias(qmean, k, kmean, N, D, cs, out);
+}
+
 void ora_quantize_tokens_T(const uint16_t* x, int N, int D, float s_enc, uint8_t* codes,
                            uint8_t* scales, int npad) {
   quantize_tokens_T(x, N, D, s_enc, codes, scales, npad);
@@ -753,7 +854,8 @@ int ora_scores_head(const uint16_t* q, const uint16_t* k, int B, int H, int Hkv,
 //   2 = flip bound into out_flip ([nrows][D], may be NULL otherwise),
 //   4 = perturb p within the flip bound's uncertainty (tests the bound),
 //   8 = EFQ-Softmax P generation (efq_block), denominator from its p~,
-//   16 = P and V in FP8 E4M3 (not with 8).
+//   16 = P and V in FP8 E4M3 (not with 8), 32 = smooth K, 64 = smooth Q
+//   (channel_mean; N <= 2^19 with either).
 // Returns 0, or -1 on bad arguments.
 int ora_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int H, int Hkv,
                  int N, int D, int causal, float softmax_scale, int Bc, int flags,
@@ -764,14 +866,38 @@ int ora_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B,
     return -1;
   e4m3_encode(0.0f);
   if ((flags & FLAG_FP8PV) && (flags & FLAG_EFQ)) return -1;
+  if ((flags & (FLAG_SMOOTH_K | FLAG_SMOOTH_Q)) && N > (1 << 19)) return -1;
   Tensors T{q, k, v, B, H, Hkv, N, D, 0, 0, 0, 0, 0, 0, (flags & FLAG_FP8PV) != 0};
-  tensor_scale(amax_bf16(q, (int64_t)B * H * N * D), &T.sq, &T.dq);
-  tensor_scale(amax_bf16(k, (int64_t)B * Hkv * N * D), &T.sk, &T.dk);
+  if (!(softmax_scale > 0.0f)) softmax_scale = 1.0f / std::sqrt((float)D);
+  const int64_t Gq = (int64_t)B * H, Gk = (int64_t)B * Hkv;
+  std::vector<float> qmean, kmean, bias;
+  float amax_q = amax_bf16(q, Gq * N * D), amax_k = amax_bf16(k, Gk * N * D);
+  if (flags & FLAG_SMOOTH_K) {
+    kmean.resize((size_t)(Gk * D));
+    for (int64_t g = 0; g < Gk; ++g) channel_mean(k + g * N * D, N, D, amax_k, &kmean[g * D]);
+    amax_k = smoothed_amax(k, Gk, N, D, kmean.data());
+    T.kmean = kmean.data();
+  }
+  if (flags & FLAG_SMOOTH_Q) {
+    qmean.resize((size_t)(Gq * D));
+    for (int64_t g = 0; g < Gq; ++g) channel_mean(q + g * N * D, N, D, amax_q, &qmean[g * D]);
+    amax_q = smoothed_amax(q, Gq, N, D, qmean.data());
+    T.qmean = qmean.data();
+    const float cs = softmax_scale * kLog2e;
+    bias.resize((size_t)(Gq * N));
+    parallel_for(Gq, nthreads, [&](int64_t g) {
+      const int64_t gk = (g / H) * Hkv + (g % H) / (H / Hkv);
+      score_bias(&qmean[g * D], k + gk * N * D, T.kmean ? T.kmean + gk * D : nullptr, N, D, cs,
+                 &bias[g * N]);
+    });
+    T.bias = bias.data();
+  }
+  tensor_scale(amax_q, &T.sq, &T.dq);
+  tensor_scale(amax_k, &T.sk, &T.dk);
   if (T.fp8v)
     fp8_tensor_scale(amax_bf16(v, (int64_t)B * Hkv * N * D), &T.sv, &T.dv);
   else
     tensor_scale(amax_bf16(v, (int64_t)B * Hkv * N * D), &T.sv, &T.dv);
-  if (!(softmax_scale > 0.0f)) softmax_scale = 1.0f / std::sqrt((float)D);
   float c = T.dq * T.dk;
   c = c * softmax_scale;
   c = c * kLog2e;
