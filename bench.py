@@ -49,9 +49,10 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="video_dit")
     ap.add_argument("--impl", default="fp4attn", choices=["fp4attn", "reference"])
-    ap.add_argument("--variant", default="exp", choices=["exp", "efq", "fp8pv"],
+    ap.add_argument("--variant", default="exp", choices=["exp", "efq", "fp8pv", "smooth"],
                     help="P generation: exp-then-quantize (the default path), EFQ-Softmax, "
-                         "or exp-then-quantize to FP8 with V in FP8 (PV as an FP8 contraction)")
+                         "or exp-then-quantize to FP8 with V in FP8 (PV as an FP8 contraction); "
+                         "smooth: the default path with Q and K smoothed")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0,
                     help="override H and Hkv (keeping their ratio) for a smaller profiling case")
@@ -127,7 +128,8 @@ def flush_l2(buf):
 
 def oracle_flags(variant: str) -> int:
     import oracle
-    return {"exp": 0, "efq": oracle.FLAG_EFQ, "fp8pv": oracle.FLAG_FP8PV}[variant]
+    return {"exp": 0, "efq": oracle.FLAG_EFQ, "fp8pv": oracle.FLAG_FP8PV,
+            "smooth": oracle.FLAG_SMOOTH_K | oracle.FLAG_SMOOTH_Q}[variant]
 
 
 def cpu_baseline(wl, q, k, v, rows_total: int, variant: str = "exp"):
@@ -220,7 +222,8 @@ def main():
     out = torch.empty_like(q)
     qf, kf, vf, outf = (t.view(-1, wl.N, wl.D) for t in (q, k, v, out))
     efq, fp8pv = args.variant == "efq", args.variant == "fp8pv"
-    ws = fa.workspace(wl.B, wl.H, wl.Hkv, wl.N, wl.D, dev, fp8pv)
+    smooth = (fa.FP4_SMOOTH_K | fa.FP4_SMOOTH_Q) if args.variant == "smooth" else 0
+    ws = fa.workspace(wl.B, wl.H, wl.Hkv, wl.N, wl.D, dev, fp8pv, smooth)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
     flops = wl.flops
@@ -228,9 +231,10 @@ def main():
     def step():
         if world > 1:
             fa.fp4_attn_fwd_sharded(qf, kf, vf, causal=wl.causal, out=outf, efq=efq,
-                                    fp8pv=fp8pv)
+                                    fp8pv=fp8pv, smooth=smooth)
         else:
-            fa.fp4_attn_fwd(q, k, v, causal=wl.causal, out=out, ws=ws, efq=efq, fp8pv=fp8pv)
+            fa.fp4_attn_fwd(q, k, v, causal=wl.causal, out=out, ws=ws, efq=efq, fp8pv=fp8pv,
+                            smooth=smooth)
 
     def barrier():
         if world > 1:
@@ -266,13 +270,24 @@ def main():
     value = world * flops / (ms_per_step * 1e-3) / 1e12
 
     # the fused attention kernel alone (same inputs, already quantised)
-    qq = fa.fp4_quantize(q, fa.FP4_BLOCK_ALONG_D)
-    kq = fa.fp4_quantize(k, fa.FP4_BLOCK_ALONG_D)
     vq = fa.fp4_quantize_fp8(v) if fp8pv else fa.fp4_quantize(v, fa.FP4_BLOCK_ALONG_N_T)
+    if smooth:
+        kmean = fa.fp4_channel_mean(k, fa.fp4_amax(k))
+        qmean = fa.fp4_channel_mean(q, fa.fp4_amax(q))
+        kq = fa.fp4_quantize_smoothed(k, kmean, fa.fp4_amax_smoothed(k, kmean))
+        qq = fa.fp4_quantize_smoothed(q, qmean, fa.fp4_amax_smoothed(q, qmean))
+        bias = fa.fp4_score_bias(qmean, k, kmean, wl.H)
+    else:
+        qq = fa.fp4_quantize(q, fa.FP4_BLOCK_ALONG_D)
+        kq = fa.fp4_quantize(k, fa.FP4_BLOCK_ALONG_D)
 
     def kernel():
-        fa.fp4_attn_fwd_quantized(qq, kq, vq, wl.B, wl.H, wl.Hkv, causal=wl.causal, out=out,
-                                  efq=efq, fp8pv=fp8pv)
+        if smooth:
+            fa.fp4_attn_fwd_quantized_bias(qq, kq, vq, bias, wl.B, wl.H, wl.Hkv, causal=wl.causal,
+                                           out=out)
+        else:
+            fa.fp4_attn_fwd_quantized(qq, kq, vq, wl.B, wl.H, wl.Hkv, causal=wl.causal, out=out,
+                                      efq=efq, fp8pv=fp8pv)
 
     for _ in range(args.warmup):
         kernel()
@@ -287,12 +302,12 @@ def main():
             for d, h in ((q, hq), (k, hk), (v, hv)):
                 d.copy_(h, non_blocking=True)
             fa.fp4_attn_fwd_sharded(qf, kf, vf, causal=wl.causal, out=outf, efq=efq,
-                                    fp8pv=fp8pv)
+                                    fp8pv=fp8pv, smooth=smooth)
             hout.copy_(out, non_blocking=True)
             stream.synchronize()
         else:
             fa.fp4_attn_fwd_host(hq, hk, hv, causal=wl.causal, out=hout, device=dev, efq=efq,
-                                 fp8pv=fp8pv)
+                                 fp8pv=fp8pv, smooth=smooth)
 
     houts = [hout, torch.empty(shape_q, dtype=torch.bfloat16, pin_memory=True)]
     n_e2e = max(2, args.steps)
@@ -308,10 +323,10 @@ def main():
         # compute
         batches = [(hq, hk, hv)] * n_e2e
         fa.fp4_attn_fwd_host_many(batches[:2], houts, causal=wl.causal, device=dev, efq=efq,
-                                  fp8pv=fp8pv)
+                                  fp8pv=fp8pv, smooth=smooth)
         _, total = fa.fp4_attn_fwd_host_many(batches, [houts[i % 2] for i in range(n_e2e)],
                                              causal=wl.causal, device=dev, efq=efq,
-                                             fp8pv=fp8pv, return_ms=True)
+                                             fp8pv=fp8pv, smooth=smooth, return_ms=True)
         e_ms = [total / n_e2e] * n_e2e
     e_total = sum(e_ms)
     if world > 1:
@@ -341,7 +356,8 @@ def main():
         "data": "synthetic",
         "config": {**wl.describe(),
                    "p_generation": {"exp": "exp-then-quantize", "efq": "EFQ-Softmax",
-                                    "fp8pv": "exp-then-quantize to FP8 E4M3, V in FP8 E4M3"}[
+                                    "fp8pv": "exp-then-quantize to FP8 E4M3, V in FP8 E4M3",
+                                    "smooth": "exp-then-quantize, Q and K smoothed"}[
                                         args.variant],
                    "parallelism": (f"heads sharded over {world} ranks ({world} x B*Hkv units, "
                                    "one all-reduce MAX of 3 floats per step)") if world > 1
@@ -361,8 +377,10 @@ def main():
         "e2e": {"value": e2e_value, "unit": "TFLOPS",
                 "h2d_bytes_per_step": (hq.numel() + hk.numel() + hv.numel()) * 2,
                 "d2h_bytes_per_step": hout.numel() * 2},
-        # per step: amax (1, or 3 when sharded), 3 quantisations, the fused forward
-        "gpu_launches": (7 if world > 1 else 5) * args.steps,
+        # per step: amax (1, or 3 when sharded), 3 quantisations, the fused forward;
+        # smoothing adds per smoothed tensor the sums, the means and the smoothed
+        # maximum, plus Q's score correction
+        "gpu_launches": ((7 if world > 1 else 5) + (7 if smooth else 0)) * args.steps,
     }
     c = clk.summary()
     if c:

@@ -27,6 +27,8 @@ FP4_ERR_TIMEOUT = 5
 FP4_BLOCK_ALONG_D = 0
 FP4_BLOCK_ALONG_N_T = 1
 FP8_TOKENS_T = -1  # Fp4Tensor.axis of E4M3 V codes [G][D][Npad] (no block scales)
+FP4_SMOOTH_K = 1
+FP4_SMOOTH_Q = 2
 
 # Every symbol include/fp4attn.h declares.
 EXPORTS = ("fp4_codes_bytes", "fp4_scales_bytes", "fp4_attn_workspace_bytes", "fp4_quantize",
@@ -34,7 +36,9 @@ EXPORTS = ("fp4_codes_bytes", "fp4_scales_bytes", "fp4_attn_workspace_bytes", "f
            "fp4_attn_fwd_quantized",
            "fp4_attn_fwd_efq", "fp4_attn_fwd_quantized_efq", "fp4_fp8_codes_bytes",
            "fp4_quantize_fp8", "fp4_quantize_fp8_scaled", "fp4_attn_workspace_bytes_fp8pv",
-           "fp4_attn_fwd_fp8pv", "fp4_attn_fwd_quantized_fp8pv", "fp4_attn_fwd_noalloc",
+           "fp4_attn_fwd_fp8pv", "fp4_attn_fwd_quantized_fp8pv", "fp4_attn_workspace_bytes_smooth",
+           "fp4_attn_fwd_smooth", "fp4_channel_mean", "fp4_amax_smoothed", "fp4_quantize_smoothed",
+           "fp4_score_bias", "fp4_attn_fwd_quantized_bias", "fp4_attn_fwd_noalloc",
            "fp4_status", "fp4_last_error", "fp4_probe_cvt", "fp4_test_wait_timeout")
 FP4_NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -113,6 +117,22 @@ def lib():
         L.fp4_attn_fwd_fp8pv.restype = i32
         L.fp4_attn_fwd_quantized_fp8pv.argtypes = L.fp4_attn_fwd_quantized.argtypes
         L.fp4_attn_fwd_quantized_fp8pv.restype = i32
+        L.fp4_attn_workspace_bytes_smooth.argtypes = [i32, i32, i32, i32, i32]
+        L.fp4_attn_workspace_bytes_smooth.restype = sz
+        L.fp4_attn_fwd_smooth.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32,
+                                          vp, vp, sz]
+        L.fp4_attn_fwd_smooth.restype = i32
+        L.fp4_channel_mean.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
+        L.fp4_channel_mean.restype = i32
+        L.fp4_amax_smoothed.argtypes = [vp, i32, i32, i32, vp, vp, vp]
+        L.fp4_amax_smoothed.restype = i32
+        L.fp4_quantize_smoothed.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp]
+        L.fp4_quantize_smoothed.restype = i32
+        L.fp4_score_bias.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp]
+        L.fp4_score_bias.restype = i32
+        L.fp4_attn_fwd_quantized_bias.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                                  f32, vp]
+        L.fp4_attn_fwd_quantized_bias.restype = i32
         L.fp4_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
         L.fp4_attn_fwd_noalloc.restype = i32
         L.fp4_status.argtypes = [vp]
@@ -254,11 +274,13 @@ def fp4_amax(x, out=None, stream=None):
 _ws_cache: dict = {}
 
 
-def workspace(B, H, Hkv, N, D, device, fp8pv: bool = False):
+def workspace(B, H, Hkv, N, D, device, fp8pv: bool = False, smooth: int = 0):
     """A cached device workspace large enough for fp4_attn_fwd (or, with
-    fp8pv, fp4_attn_fwd_fp8pv) on this shape."""
+    fp8pv, fp4_attn_fwd_fp8pv; with smooth, fp4_attn_fwd_smooth) on this shape."""
     import torch
-    need = (fp4_attn_workspace_bytes_fp8pv if fp8pv else fp4_attn_workspace_bytes)(B, H, Hkv, N, D)
+    fn = (fp4_attn_workspace_bytes_smooth if smooth else
+          fp4_attn_workspace_bytes_fp8pv if fp8pv else fp4_attn_workspace_bytes)
+    need = fn(B, H, Hkv, N, D)
     key = (str(device),)
     ws = _ws_cache.get(key)
     if ws is None or ws.numel() < need:
@@ -275,11 +297,17 @@ def _attn_fn(efq: bool, fp8pv: bool, quantized: bool):
 
 
 def fp4_attn_fwd(q, k, v, causal: bool = False, softmax_scale: float | None = None, out=None,
-                 stream=None, ws=None, efq: bool = False, fp8pv: bool = False):
+                 stream=None, ws=None, efq: bool = False, fp8pv: bool = False, smooth: int = 0):
     """NVFP4 attention forward. q [B,H,N,D], k/v [B,Hkv,N,D]: contiguous bf16
     CUDA tensors. Returns out [B,H,N,D] bf16. efq=True calls fp4_attn_fwd_efq
     (P from EFQ-Softmax instead of exp-then-quantize); fp8pv=True calls
-    fp4_attn_fwd_fp8pv (P and V in E4M3)."""
+    fp4_attn_fwd_fp8pv (P and V in E4M3); smooth (FP4_SMOOTH_K | FP4_SMOOTH_Q)
+    calls fp4_attn_fwd_smooth."""
+    if smooth:
+        if efq or fp8pv:
+            raise ValueError("smoothing is built for the exp-then-quantize NVFP4 path")
+        return fp4_attn_fwd_smooth(q, k, v, smooth, causal, softmax_scale, out=out, stream=stream,
+                                   ws=ws)
     import torch
     B, H, N, D = q.shape
     Hkv = k.shape[1]
@@ -293,6 +321,104 @@ def fp4_attn_fwd(q, k, v, causal: bool = False, softmax_scale: float | None = No
         ws = workspace(B, H, Hkv, N, D, q.device, fp8pv)
     _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, Hkv, N, D, int(bool(causal)),
               float(softmax_scale or 0.0), _stream(stream), _ptr(ws), ws.numel()))
+    return out
+
+
+def fp4_attn_workspace_bytes_smooth(B: int, H: int, Hkv: int, N: int, D: int) -> int:
+    return lib().fp4_attn_workspace_bytes_smooth(B, H, Hkv, N, D)
+
+
+_ws_smooth: dict = {}
+
+
+def fp4_attn_fwd_smooth(q, k, v, smooth: int = FP4_SMOOTH_K | FP4_SMOOTH_Q, causal: bool = False,
+                        softmax_scale: float | None = None, out=None, stream=None, ws=None):
+    """NVFP4 attention forward with Q and/or K smoothed before quantisation
+    (smooth = FP4_SMOOTH_K | FP4_SMOOTH_Q; the reading in include/fp4attn.h).
+    Same tensors as fp4_attn_fwd."""
+    import torch
+    B, H, N, D = q.shape
+    Hkv = k.shape[1]
+    for t in (q, k, v):
+        assert t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()
+    assert k.shape == (B, Hkv, N, D) and v.shape == (B, Hkv, N, D)
+    if out is None:
+        out = torch.empty_like(q)
+    if ws is None:
+        need = fp4_attn_workspace_bytes_smooth(B, H, Hkv, N, D)
+        key = (str(q.device),)
+        ws = _ws_smooth.get(key)
+        if ws is None or ws.numel() < need:
+            ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+            _ws_smooth[key] = ws
+    _check(lib().fp4_attn_fwd_smooth(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, Hkv, N, D,
+                                     int(bool(causal)), float(softmax_scale or 0.0), int(smooth),
+                                     _stream(stream), _ptr(ws), ws.numel()))
+    return out
+
+
+def fp4_channel_mean(x, amax, stream=None):
+    """Smoothing means [G, D] fp32 of x [..., N, D] (bf16 CUDA) on the grid of
+    amax (float32 CUDA tensor, first element the raw tensor's maximum)."""
+    import torch
+    G, N, D = _gnd(x)
+    mean = torch.empty((G, D), dtype=torch.float32, device=x.device)
+    sums = torch.empty((G, D), dtype=torch.int64, device=x.device)
+    _check(lib().fp4_channel_mean(_ptr(x), G, N, D, _ptr(amax), _ptr(mean), _ptr(sums),
+                                  _stream(stream)))
+    return mean
+
+
+def fp4_amax_smoothed(x, mean, stream=None):
+    """max |fl32(x - mean)| (float32 CUDA tensor of one element)."""
+    import torch
+    G, N, D = _gnd(x)
+    out = torch.empty(1, dtype=torch.float32, device=x.device)
+    _check(lib().fp4_amax_smoothed(_ptr(x), G, N, D, _ptr(mean), _ptr(out), _stream(stream)))
+    return out
+
+
+def fp4_quantize_smoothed(x, mean, amax, stream=None) -> Fp4Tensor:
+    """NVFP4 (blocks along D) of fl32(x - mean) with the smoothed tensor's
+    maximum amax (float32 CUDA)."""
+    import torch
+    G, N, D = _gnd(x)
+    codes = torch.empty(fp4_codes_bytes(G, N, D, FP4_BLOCK_ALONG_D), dtype=torch.uint8,
+                        device=x.device)
+    scales = torch.empty(fp4_scales_bytes(G, N, D, FP4_BLOCK_ALONG_D), dtype=torch.uint8,
+                         device=x.device)
+    _check(lib().fp4_quantize_smoothed(_ptr(x), G, N, D, _ptr(mean), _ptr(amax), _ptr(codes),
+                                       _ptr(scales), _stream(stream)))
+    return Fp4Tensor(codes, scales, amax, G, N, D, FP4_BLOCK_ALONG_D)
+
+
+def fp4_score_bias(qmean, k, kmean, H: int, softmax_scale: float | None = None, stream=None):
+    """Smoothed Q's score correction [B*H, Npad] fp32: qmean [B*H, D], k
+    [B, Hkv, N, D] bf16, kmean [B*Hkv, D] or None."""
+    import torch
+    B, Hkv, N, D = k.shape
+    npad = (N + 127) // 128 * 128
+    bias = torch.empty((B * H, npad), dtype=torch.float32, device=k.device)
+    _check(lib().fp4_score_bias(_ptr(qmean), _ptr(k), None if kmean is None else _ptr(kmean), B, H,
+                                Hkv, N, D, float(softmax_scale or 0.0), _ptr(bias),
+                                _stream(stream)))
+    return bias
+
+
+def fp4_attn_fwd_quantized_bias(qq: Fp4Tensor, kq: Fp4Tensor, vq: Fp4Tensor, bias, B: int, H: int,
+                                Hkv: int, causal: bool = False,
+                                softmax_scale: float | None = None, out=None, stream=None):
+    """The fused forward on quantised tensors with the per-key score
+    correction bias [B*H, Npad] (exp-then-quantize P)."""
+    import torch
+    N, D = qq.N, qq.D
+    if out is None:
+        out = torch.empty((B, H, N, D), dtype=torch.bfloat16, device=qq.codes.device)
+    ts = [_Tensor(t.codes.data_ptr(), t.scales.data_ptr(), t.amax.data_ptr()) for t in (qq, kq, vq)]
+    _check(lib().fp4_attn_fwd_quantized_bias(ctypes.byref(ts[0]), ctypes.byref(ts[1]),
+                                             ctypes.byref(ts[2]), _ptr(bias), _ptr(out), B, H, Hkv,
+                                             N, D, int(bool(causal)), float(softmax_scale or 0.0),
+                                             _stream(stream)))
     return out
 
 
@@ -338,7 +464,7 @@ def fp4_attn_fwd_quantized(qq: Fp4Tensor, kq: Fp4Tensor, vq: Fp4Tensor, B: int, 
 
 def fp4_attn_fwd_host(q, k, v, causal: bool = False, softmax_scale: float | None = None,
                       out=None, device="cuda", stream=None, efq: bool = False,
-                      fp8pv: bool = False):
+                      fp8pv: bool = False, smooth: int = 0):
     """End-to-end call on host buffers: copies q, k, v (pinned CPU bf16
     tensors) to the device, runs fp4_attn_fwd, copies the output back into
     `out` (a pinned CPU tensor) and returns it once the stream has finished."""
@@ -346,7 +472,8 @@ def fp4_attn_fwd_host(q, k, v, causal: bool = False, softmax_scale: float | None
     dq = q.to(device, non_blocking=True)
     dk = k.to(device, non_blocking=True)
     dv = v.to(device, non_blocking=True)
-    o = fp4_attn_fwd(dq, dk, dv, causal, softmax_scale, stream=stream, efq=efq, fp8pv=fp8pv)
+    o = fp4_attn_fwd(dq, dk, dv, causal, softmax_scale, stream=stream, efq=efq, fp8pv=fp8pv,
+                     smooth=smooth)
     if out is None:
         out = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
     out.copy_(o, non_blocking=True)
@@ -356,7 +483,7 @@ def fp4_attn_fwd_host(q, k, v, causal: bool = False, softmax_scale: float | None
 
 def fp4_attn_fwd_host_many(batches, outs, causal: bool = False,
                            softmax_scale: float | None = None, device="cuda", efq: bool = False,
-                           return_ms: bool = False, fp8pv: bool = False):
+                           return_ms: bool = False, fp8pv: bool = False, smooth: int = 0):
     """End-to-end over a sequence of host batches: batches = [(q, k, v), ...]
     pinned CPU bf16 tensors of one shape, outs = pinned CPU tensors for the
     outputs. Two sets of device buffers and three streams (copies in, compute,
@@ -374,7 +501,7 @@ def fp4_attn_fwd_host_many(batches, outs, causal: bool = False,
     s_in, s_run, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     bufs = [tuple(torch.empty(t.shape, dtype=torch.bfloat16, device=dev) for t in (q0, k0, k0, q0))
             for _ in range(2)]
-    ws = workspace(B, H, Hkv, N, D, dev, fp8pv)
+    ws = workspace(B, H, Hkv, N, D, dev, fp8pv, smooth)
     free = [None, None]  # event: slot's last device-to-host copy done
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(s_in)
@@ -391,7 +518,7 @@ def fp4_attn_fwd_host_many(batches, outs, causal: bool = False,
             loaded.record(s_in)
         s_run.wait_event(loaded)
         fp4_attn_fwd(dq, dk, dv, causal, softmax_scale, out=do, stream=s_run, ws=ws, efq=efq,
-                     fp8pv=fp8pv)
+                     fp8pv=fp8pv, smooth=smooth)
         done = torch.cuda.Event()
         done.record(s_run)
         s_out.wait_event(done)

@@ -54,7 +54,6 @@ constexpr int kAttnThreads = 384;  // 12 warps = 3 warpgroups
 // the 384 x 168 registers the block is launched with.
 constexpr uint32_t kRegsCtl = 56, kRegsSoftmax = 224;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
-constexpr float kLog2e = 1.44269504088896340736f;
 
 enum : unsigned { kDevErrTimeout = 1u };
 
@@ -102,6 +101,7 @@ struct AttnParams {
   const float* amax_k;
   const float* amax_v;
   __nv_bfloat16* out;  // [B][H][N][D]
+  const float* bias;   // [B*H][Npad]: per-key score correction (smoothed Q), or unused
   int H, Hkv, N, Npad, ntq;
   float softmax_scale;
 };
@@ -129,7 +129,8 @@ struct AttnSmem {
   static constexpr int oPsf = oVsf + kStages * 1024;
   static constexpr int oRed = oPsf + 2 * 1024;  // float [2][128] running max per stream, [2][128] l
   static constexpr int oPtab = oRed + 2048;     // float [128]
-  static constexpr int oBar = oPtab + 512;      // mbarriers
+  static constexpr int oBias = oPtab + 512;     // float [kStages][128]: score correction per key
+  static constexpr int oBar = oBias + kStages * 512;  // mbarriers
   static constexpr int oTmem = oBar + 256;
   static constexpr int kBytes = oTmem + 16 + 1024;  // + alignment slack
 };
@@ -163,11 +164,16 @@ struct TmemCols {
 constexpr float kInv7 = 1.0f / 7.0f;
 constexpr float kRound = 8388608.0f;  // 2^23: x + 2^23 rounds x (0 <= x < 2^22) to an integer
 
-template <int D, bool CAUSAL, int PG>
+// BIAS: add a per-key fp32 correction to the scores, x = fma(S, c, bias_j)
+// (the smoothed-Q path; exp-then-quantize P only). The key tile's 128 values
+// travel with its V tile, so they stay in shared memory until PV of the tile
+// has completed, after the softmax has read them.
+template <int D, bool CAUSAL, int PG, bool BIAS = false>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   constexpr bool EFQ = PG == kPgEfq, FP8 = PG == kPgFp8;
+  static_assert(!BIAS || PG == kPgExp, "the score correction is built for exp-then-quantize P");
   using L = AttnSmem<D, FP8>;
   using TC = TmemCols<EFQ>;
   constexpr uint32_t kColQsf = TC::kQsf, kColKsf = TC::kKsf, kColPsf = TC::kPsf,
@@ -254,12 +260,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                   p.k_sf + ((int64_t)gk * (p.Npad / kBN) + j) * L::kSfQK, L::kSfQK,
                   bar(kBarKFull + st));
         if (j >= kStages && !(ok = wait_bar(bar(kBarVEmpty + st), pe))) break;
-        mbar_arrive_expect_tx(bar(kBarVFull + st), L::kV + (FP8 ? 0 : 1024));
+        mbar_arrive_expect_tx(bar(kBarVFull + st), L::kV + (FP8 ? 0 : 1024) + (BIAS ? 512 : 0));
         tma_load_2d(sb + L::oV + st * L::kV, &tmV, j * (FP8 ? kBN : kBN / 2), gk * D,
                     bar(kBarVFull + st));
         if (!FP8)
           bulk_load(sb + L::oVsf + st * 1024, p.v_sf + ((int64_t)gk * (p.Npad / 64) + 2 * j) * 512,
                     1024, bar(kBarVFull + st));
+        if (BIAS)
+          bulk_load(sb + L::oBias + st * 512, p.bias + (int64_t)gq * p.Npad + j * kBN, 512,
+                    bar(kBarVFull + st));
       }
     }
   } else if (warp == 1 || warp == 2) {
@@ -363,7 +372,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const float sq = tensor_senc(*p.amax_q), sk = tensor_senc(*p.amax_k),
                 sv = FP8 ? fp8_senc(*p.amax_v) : tensor_senc(*p.amax_v);
     const float dq = __fdiv_rn(1.0f, sq), dk = __fdiv_rn(1.0f, sk), dv = __fdiv_rn(1.0f, sv);
-    const float c = __fmul_rn(__fmul_rn(__fmul_rn(dq, dk), p.softmax_scale), kLog2e);
+    const float c_s = __fmul_rn(__fmul_rn(__fmul_rn(dq, dk), p.softmax_scale), kLog2e);
+    // with the score correction x = fma(S, c_s, bias) is formed first and the
+    // steps below take x with the unit multiplier
+    const float c = BIAS ? 1.0f : c_s;
     // d_P d_V; with FP8 P the row sum is kept in units of 256 p, so d_V alone
     const float fpv = FP8 ? dv : __fmul_rn(__fdiv_rn(1.0f, kTensorRange), dv);
     const uint64_t c2 = pk(c, c);
@@ -390,6 +402,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int i = 0; i < kBN; ++i)
           if (key0 + i >= p.N || (CAUSAL && key0 + i > qrow)) s[i] = -INFINITY;
+      }
+      if constexpr (BIAS) {
+        // the tile's corrections arrived with its V tile (same stage and phase)
+        if (ok)
+          ok = __all_sync(0xFFFFFFFFu, wait_bar(bar(kBarVFull + t % kStages), (t / kStages) & 1));
+        const float4* bb = reinterpret_cast<const float4*>(sm + L::oBias + (t % kStages) * 512);
+        const uint64_t cs2 = pk(c_s, c_s);
+#pragma unroll
+        for (int i4 = 0; i4 < kBN / 4; ++i4) {
+          const float4 b4 = bb[i4];
+          upk(fma2(pk(s[4 * i4], s[4 * i4 + 1]), cs2, pk(b4.x, b4.y)), s[4 * i4], s[4 * i4 + 1]);
+          upk(fma2(pk(s[4 * i4 + 2], s[4 * i4 + 3]), cs2, pk(b4.z, b4.w)), s[4 * i4 + 2],
+              s[4 * i4 + 3]);
+        }
       }
       float bm[8];
 #pragma unroll

@@ -59,8 +59,16 @@ AttnKernel attn_kernel_pg(int D, int causal) {
 }
 
 // The fused kernel for head dim D, causal masking and P generation pg
-// (fp4::kPgExp, kPgEfq, kPgFp8).
-AttnKernel attn_kernel(int D, int causal, int pg) {
+// (fp4::kPgExp, kPgEfq, kPgFp8); bias: with the per-key score correction of
+// smoothed Q (exp-then-quantize only).
+AttnKernel attn_kernel(int D, int causal, int pg, bool bias = false) {
+  if (bias) {
+    if (D == 128)
+      return causal ? fp4::attn_fwd_kernel<128, true, fp4::kPgExp, true>
+                    : fp4::attn_fwd_kernel<128, false, fp4::kPgExp, true>;
+    return causal ? fp4::attn_fwd_kernel<64, true, fp4::kPgExp, true>
+                  : fp4::attn_fwd_kernel<64, false, fp4::kPgExp, true>;
+  }
   if (pg == fp4::kPgEfq) return attn_kernel_pg<fp4::kPgEfq>(D, causal);
   if (pg == fp4::kPgFp8) return attn_kernel_pg<fp4::kPgFp8>(D, causal);
   return attn_kernel_pg<fp4::kPgExp>(D, causal);
@@ -87,10 +95,10 @@ fp4_status_t device_setup(int* dev_out, int* sms_out) {
                   dev, major, minor);
     for (int d = 0; d < 2; ++d)
       for (int causal = 0; causal < 2; ++causal)
-        for (int pg = 0; pg < 3; ++pg)
-          FP4_CUDA(cudaFuncSetAttribute(attn_kernel(d ? 128 : 64, causal, pg),
+        for (int pg = 0; pg < 4; ++pg)  // pg 3: exp-then-quantize with the score correction
+          FP4_CUDA(cudaFuncSetAttribute(attn_kernel(d ? 128 : 64, causal, pg % 3, pg == 3),
                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        attn_smem_bytes(d ? 128 : 64, pg)));
+                                        attn_smem_bytes(d ? 128 : 64, pg % 3)));
     if (!g_encode) {
       cudaDriverEntryPointQueryResult q;
       void* fn = nullptr;
@@ -122,7 +130,7 @@ fp4_status_t tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t 
 }
 
 struct WsLayout {
-  size_t amax, qc, qs, kc, ks, vc, vs, total;
+  size_t amax, qc, qs, kc, ks, vc, vs, sums, qmean, kmean, bias, total;
 };
 
 size_t codes_bytes(int64_t G, int64_t N, int64_t D) { return (size_t)(G * round_up(N, 128) * D / 2); }
@@ -133,8 +141,9 @@ size_t scales_bytes(int64_t G, int64_t N, int64_t D, fp4_axis_t axis) {
 
 size_t fp8_codes_bytes(int64_t G, int64_t N, int64_t D) { return (size_t)(G * D * round_up(N, 128)); }
 
-// Workspace of the quantizing forwards; fp8v: V as E4M3 codes, no V scales.
-WsLayout ws_layout(int B, int H, int Hkv, int N, int D, bool fp8v = false) {
+// Workspace of the quantizing forwards; fp8v: V as E4M3 codes, no V scales;
+// smooth: the smoothing sums, means and Q's score correction as well.
+WsLayout ws_layout(int B, int H, int Hkv, int N, int D, bool fp8v = false, bool smooth = false) {
   WsLayout w;
   size_t off = 0;
   auto take = [&](size_t n) {
@@ -150,6 +159,11 @@ WsLayout ws_layout(int B, int H, int Hkv, int N, int D, bool fp8v = false) {
   w.ks = take(scales_bytes(Gk, N, D, FP4_BLOCK_ALONG_D));
   w.vc = take(fp8v ? fp8_codes_bytes(Gk, N, D) : codes_bytes(Gk, N, D));
   w.vs = take(fp8v ? 0 : scales_bytes(Gk, N, D, FP4_BLOCK_ALONG_N_T));
+  const int64_t Npad = round_up(N, 128);
+  w.sums = take(smooth ? (size_t)((Gq + Gk) * D * 8) : 0);
+  w.qmean = take(smooth ? (size_t)(Gq * D * 4) : 0);
+  w.kmean = take(smooth ? (size_t)(Gk * D * 4) : 0);
+  w.bias = take(smooth ? (size_t)(Gq * Npad * 4) : 0);
   w.total = off;
   return w;
 }
@@ -185,18 +199,26 @@ fp4_status_t launch_amax(const void* x0, int64_t n0, const void* x1, int64_t n1,
 }
 
 fp4_status_t launch_quant(const void* x, int64_t G, int N, int D, fp4_axis_t axis, uint8_t* codes,
-                          uint8_t* scales, const float* amax, int sms, cudaStream_t stream) {
+                          uint8_t* scales, const float* amax, int sms, cudaStream_t stream,
+                          const float* mean = nullptr) {
   const int64_t Npad = round_up(N, 128);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (axis == FP4_BLOCK_ALONG_D) {
     const int64_t total = G * Npad * (D / 16);
     const int64_t blocks = std::min<int64_t>((total + 255) / 256, (int64_t)sms * 16);
-    if (D == 128)
-      fp4::quant_rows_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(xb, (int)G, N, (int)Npad,
-                                                                       amax, codes, scales);
+    const unsigned nb = (unsigned)blocks;
+    if (mean && D == 128)
+      fp4::quant_rows_kernel<128, true><<<nb, 256, 0, stream>>>(xb, (int)G, N, (int)Npad, amax,
+                                                                codes, scales, mean);
+    else if (mean)
+      fp4::quant_rows_kernel<64, true><<<nb, 256, 0, stream>>>(xb, (int)G, N, (int)Npad, amax,
+                                                               codes, scales, mean);
+    else if (D == 128)
+      fp4::quant_rows_kernel<128><<<nb, 256, 0, stream>>>(xb, (int)G, N, (int)Npad, amax, codes,
+                                                          scales);
     else
-      fp4::quant_rows_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(xb, (int)G, N, (int)Npad,
-                                                                      amax, codes, scales);
+      fp4::quant_rows_kernel<64><<<nb, 256, 0, stream>>>(xb, (int)G, N, (int)Npad, amax, codes,
+                                                         scales);
   } else {
     const int64_t blocks = G * (Npad / 128);
     if (blocks > INT32_MAX) return fail(FP4_ERR_INVALID_ARG, "problem too large");
@@ -207,6 +229,65 @@ fp4_status_t launch_quant(const void* x, int64_t G, int N, int D, fp4_axis_t axi
       fp4::quant_tokens_T_kernel<64><<<(unsigned)blocks, 128, 0, stream>>>(
           xb, (int)G, N, (int)Npad, amax, codes, scales);
   }
+  FP4_CUDA(cudaGetLastError());
+  return FP4_OK;
+}
+
+float resolve_scale(float softmax_scale, int D) {
+  return (softmax_scale > 0.0f && std::isfinite(softmax_scale)) ? softmax_scale
+                                                                 : 1.0f / std::sqrt((float)D);
+}
+
+// Smoothing means of x [G][N][D]: sums [G][D] (zeroed here) on the grid of
+// *amax, then mean [G][D].
+fp4_status_t launch_mean(const void* x, int64_t G, int N, int D, const float* amax,
+                         unsigned long long* sums, float* mean, cudaStream_t stream) {
+  if (G > 65535) return fail(FP4_ERR_INVALID_ARG, "more than 65535 heads");
+  FP4_CUDA(cudaMemsetAsync(sums, 0, (size_t)(G * D * 8), stream));
+  dim3 grid((unsigned)((N + fp4::kSumRows - 1) / fp4::kSumRows), (unsigned)G);
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  if (D == 128)
+    fp4::colsum_fixed_kernel<128><<<grid, 256, 0, stream>>>(xb, N, amax, sums);
+  else
+    fp4::colsum_fixed_kernel<64><<<grid, 256, 0, stream>>>(xb, N, amax, sums);
+  FP4_CUDA(cudaGetLastError());
+  const int64_t n = G * D;
+  fp4::mean_from_sums_kernel<<<(unsigned)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, stream>>>(
+      sums, n, N, amax, mean);
+  FP4_CUDA(cudaGetLastError());
+  return FP4_OK;
+}
+
+// *out = max |fl32(x - mean)| (zeroed here).
+fp4_status_t launch_amax_smoothed(const void* x, int64_t G, int N, int D, const float* mean,
+                                  float* out, int sms, cudaStream_t stream) {
+  FP4_CUDA(cudaMemsetAsync(out, 0, sizeof(float), stream));
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  if (D == 128)
+    fp4::amax_smoothed_kernel<128><<<sms * 4, 256, 0, stream>>>(xb, G, N, mean,
+                                                                reinterpret_cast<unsigned*>(out));
+  else
+    fp4::amax_smoothed_kernel<64><<<sms * 4, 256, 0, stream>>>(xb, G, N, mean,
+                                                               reinterpret_cast<unsigned*>(out));
+  FP4_CUDA(cudaGetLastError());
+  return FP4_OK;
+}
+
+// Q's score correction bias [B*H][Npad].
+fp4_status_t launch_score_bias(const float* qmean, const void* k, const float* kmean, int B, int H,
+                               int Hkv, int N, int D, float softmax_scale, float* bias,
+                               cudaStream_t stream) {
+  const int64_t Npad = round_up(N, 128);
+  if ((int64_t)B * Hkv > 65535) return fail(FP4_ERR_INVALID_ARG, "more than 65535 key/value heads");
+  dim3 grid((unsigned)(Npad / 128), (unsigned)(B * Hkv));
+  const float sc = resolve_scale(softmax_scale, D);
+  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
+  if (D == 128)
+    fp4::score_bias_kernel<128><<<grid, 128, 0, stream>>>(qmean, kb, kmean, H, Hkv, N, (int)Npad, sc,
+                                                          bias);
+  else
+    fp4::score_bias_kernel<64><<<grid, 128, 0, stream>>>(qmean, kb, kmean, H, Hkv, N, (int)Npad, sc,
+                                                         bias);
   FP4_CUDA(cudaGetLastError());
   return FP4_OK;
 }
@@ -231,7 +312,8 @@ fp4_status_t launch_quant_fp8(const void* x, int64_t G, int N, int D, uint8_t* c
 fp4_status_t launch_attn(const uint8_t* qc, const uint8_t* qs, const float* qa, const uint8_t* kc,
                          const uint8_t* ks, const float* ka, const uint8_t* vc, const uint8_t* vs,
                          const float* va, void* out, int B, int H, int Hkv, int N, int D,
-                         int causal, float softmax_scale, int pg, cudaStream_t stream) {
+                         int causal, float softmax_scale, int pg, cudaStream_t stream,
+                         const float* bias = nullptr) {
   const int64_t Npad = round_up(N, 128);
   const int64_t Gq = (int64_t)B * H, Gk = (int64_t)B * Hkv;
   const CUtensorMapSwizzle swQK =
@@ -259,12 +341,13 @@ fp4_status_t launch_attn(const uint8_t* qc, const uint8_t* qs, const float* qa, 
   p.N = N;
   p.Npad = (int)Npad;
   p.ntq = (int)(Npad / 128);
-  p.softmax_scale = (softmax_scale > 0.0f && std::isfinite(softmax_scale))
-                        ? softmax_scale
-                        : 1.0f / std::sqrt((float)D);
+  p.bias = bias;
+  p.softmax_scale = resolve_scale(softmax_scale, D);
   dim3 grid(p.ntq, H, B);
-  attn_kernel(D, causal, pg)<<<grid, fp4::kAttnThreads, attn_smem_bytes(D, pg), stream>>>(tq, tk, tv,
-                                                                                       p);
+  if (bias && pg != fp4::kPgExp)
+    return fail(FP4_ERR_UNSUPPORTED, "the score correction needs exp-then-quantize P");
+  attn_kernel(D, causal, pg, bias != nullptr)<<<grid, fp4::kAttnThreads, attn_smem_bytes(D, pg),
+                                                stream>>>(tq, tk, tv, p);
   FP4_CUDA(cudaGetLastError());
   return FP4_OK;
 }
@@ -305,10 +388,72 @@ fp4_status_t attn_fwd_any(const void* q, const void* k, const void* v, void* out
                      ws + w.vs, amax + 2, out, B, H, Hkv, N, D, causal, softmax_scale, pg, st);
 }
 
+// The smoothed forward: smooth bit 0 = K, bit 1 = Q (FP4_SMOOTH_K / _Q).
+fp4_status_t attn_fwd_smooth_any(const void* q, const void* k, const void* v, void* out, int B,
+                                 int H, int Hkv, int N, int D, int causal, float softmax_scale,
+                                 int smooth, void* stream, void* workspace,
+                                 size_t workspace_bytes) {
+  g_last_error.clear();
+  fp4_status_t s;
+  if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
+  if (smooth & ~3) return fail(FP4_ERR_INVALID_ARG, "smooth flags %d", smooth);
+  if (N > (1 << 19)) return fail(FP4_ERR_INVALID_ARG, "smoothing takes N <= 2^19 (got %d)", N);
+  if (!q || !k || !v || !out || !workspace) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(workspace))
+    return fail(FP4_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const WsLayout w = ws_layout(B, H, Hkv, N, D, false, true);
+  if (workspace_bytes < w.total)
+    return fail(FP4_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, w.total);
+  int dev, sms;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* amax = reinterpret_cast<float*>(ws + w.amax);  // raw Q, K, V; smoothed Q, K
+  const int64_t Gq = (int64_t)B * H, Gk = (int64_t)B * Hkv;
+  auto* sums = reinterpret_cast<unsigned long long*>(ws + w.sums);
+  float* qmean = reinterpret_cast<float*>(ws + w.qmean);
+  float* kmean = reinterpret_cast<float*>(ws + w.kmean);
+  float* bias = reinterpret_cast<float*>(ws + w.bias);
+  if ((s = launch_amax(q, Gq * N * D, k, Gk * N * D, v, Gk * N * D, amax, amax + 1, amax + 2, sms,
+                       st)) != FP4_OK)
+    return s;
+  const float* ak = amax + 1;
+  const float* kmean_used = nullptr;
+  if (smooth & 1) {
+    if ((s = launch_mean(k, Gk, N, D, amax + 1, sums + Gq * D, kmean, st)) != FP4_OK) return s;
+    if ((s = launch_amax_smoothed(k, Gk, N, D, kmean, amax + 4, sms, st)) != FP4_OK) return s;
+    ak = amax + 4;
+    kmean_used = kmean;
+  }
+  if ((s = launch_quant(k, Gk, N, D, FP4_BLOCK_ALONG_D, ws + w.kc, ws + w.ks, ak, sms, st,
+                        kmean_used)) != FP4_OK)
+    return s;
+  const float* aq = amax;
+  const float* qmean_used = nullptr;
+  if (smooth & 2) {
+    if ((s = launch_mean(q, Gq, N, D, amax, sums, qmean, st)) != FP4_OK) return s;
+    if ((s = launch_amax_smoothed(q, Gq, N, D, qmean, amax + 3, sms, st)) != FP4_OK) return s;
+    if ((s = launch_score_bias(qmean, k, kmean_used, B, H, Hkv, N, D, softmax_scale, bias, st)) !=
+        FP4_OK)
+      return s;
+    aq = amax + 3;
+    qmean_used = qmean;
+  }
+  if ((s = launch_quant(q, Gq, N, D, FP4_BLOCK_ALONG_D, ws + w.qc, ws + w.qs, aq, sms, st,
+                        qmean_used)) != FP4_OK)
+    return s;
+  if ((s = launch_quant(v, Gk, N, D, FP4_BLOCK_ALONG_N_T, ws + w.vc, ws + w.vs, amax + 2, sms,
+                        st)) != FP4_OK)
+    return s;
+  return launch_attn(ws + w.qc, ws + w.qs, aq, ws + w.kc, ws + w.ks, ak, ws + w.vc, ws + w.vs,
+                     amax + 2, out, B, H, Hkv, N, D, causal, softmax_scale, fp4::kPgExp, st,
+                     (smooth & 2) ? bias : nullptr);
+}
+
 fp4_status_t attn_fwd_quantized_any(const fp4_tensor_t* q, const fp4_tensor_t* k,
                                     const fp4_tensor_t* v, void* out, int B, int H, int Hkv,
                                     int N, int D, int causal, float softmax_scale, void* stream,
-                                    int pg) {
+                                    int pg, const float* bias = nullptr) {
   g_last_error.clear();
   fp4_status_t s;
   if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
@@ -324,11 +469,12 @@ fp4_status_t attn_fwd_quantized_any(const fp4_tensor_t* q, const fp4_tensor_t* k
       return fail(FP4_ERR_INVALID_ARG, "codes/scales must be 16-byte aligned");
   }
   if (!aligned16(out)) return fail(FP4_ERR_INVALID_ARG, "out must be 16-byte aligned");
+  if (bias && !aligned16(bias)) return fail(FP4_ERR_INVALID_ARG, "bias must be 16-byte aligned");
   int dev, sms;
   if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
   return launch_attn(q->codes, q->scales, q->amax, k->codes, k->scales, k->amax, v->codes,
                      v->scales, v->amax, out, B, H, Hkv, N, D, causal, softmax_scale, pg,
-                     static_cast<cudaStream_t>(stream));
+                     static_cast<cudaStream_t>(stream), bias);
 }
 
 }  // namespace
@@ -348,6 +494,91 @@ size_t fp4_scales_bytes(int G, int N, int D, fp4_axis_t axis) {
 size_t fp4_attn_workspace_bytes(int B, int H, int Hkv, int N, int D) {
   if (check_shape(B, H, Hkv, N, D) != FP4_OK) return 0;
   return ws_layout(B, H, Hkv, N, D).total;
+}
+
+size_t fp4_attn_workspace_bytes_smooth(int B, int H, int Hkv, int N, int D) {
+  if (check_shape(B, H, Hkv, N, D) != FP4_OK || N > (1 << 19)) return 0;
+  return ws_layout(B, H, Hkv, N, D, false, true).total;
+}
+
+fp4_status_t fp4_channel_mean(const void* x, int G, int N, int D, const float* amax,
+                              float* mean, unsigned long long* sums, void* stream) {
+  g_last_error.clear();
+  fp4_status_t s;
+  if ((s = check_shape(1, G, G, N, D)) != FP4_OK) return s;
+  if (N > (1 << 19)) return fail(FP4_ERR_INVALID_ARG, "N <= 2^19 (got %d)", N);
+  if (!x || !amax || !mean || !sums) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(mean) || !aligned16(sums) ||
+      (reinterpret_cast<uintptr_t>(amax) & 3u))
+    return fail(FP4_ERR_INVALID_ARG, "x, mean and sums 16-byte aligned, amax 4-byte aligned");
+  int dev, sms;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  return launch_mean(x, G, N, D, amax, sums, mean, static_cast<cudaStream_t>(stream));
+}
+
+fp4_status_t fp4_amax_smoothed(const void* x, int G, int N, int D, const float* mean, float* amax,
+                               void* stream) {
+  g_last_error.clear();
+  fp4_status_t s;
+  if ((s = check_shape(1, G, G, N, D)) != FP4_OK) return s;
+  if (!x || !mean || !amax) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(mean) || (reinterpret_cast<uintptr_t>(amax) & 3u))
+    return fail(FP4_ERR_INVALID_ARG, "x and mean 16-byte aligned, amax 4-byte aligned");
+  int dev, sms;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  return launch_amax_smoothed(x, G, N, D, mean, amax, sms, static_cast<cudaStream_t>(stream));
+}
+
+fp4_status_t fp4_quantize_smoothed(const void* x, int G, int N, int D, const float* mean,
+                                   const float* amax, uint8_t* codes, uint8_t* scales,
+                                   void* stream) {
+  g_last_error.clear();
+  fp4_status_t s;
+  if ((s = check_shape(1, G, G, N, D)) != FP4_OK) return s;
+  if (!x || !mean || !amax || !codes || !scales) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(mean) || !aligned16(codes) || !aligned16(scales) ||
+      (reinterpret_cast<uintptr_t>(amax) & 3u))
+    return fail(FP4_ERR_INVALID_ARG,
+                "x, mean, codes and scales 16-byte aligned, amax 4-byte aligned");
+  int dev, sms;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  return launch_quant(x, G, N, D, FP4_BLOCK_ALONG_D, codes, scales, amax, sms,
+                      static_cast<cudaStream_t>(stream), mean);
+}
+
+fp4_status_t fp4_score_bias(const float* qmean, const void* k, const float* kmean, int B, int H,
+                            int Hkv, int N, int D, float softmax_scale, float* bias,
+                            void* stream) {
+  g_last_error.clear();
+  fp4_status_t s;
+  if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
+  if (!qmean || !k || !bias) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(qmean) || !aligned16(k) || !aligned16(bias) || (kmean && !aligned16(kmean)))
+    return fail(FP4_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  int dev, sms;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  return launch_score_bias(qmean, k, kmean, B, H, Hkv, N, D, softmax_scale, bias,
+                           static_cast<cudaStream_t>(stream));
+}
+
+fp4_status_t fp4_attn_fwd_smooth(const void* q, const void* k, const void* v, void* out, int B,
+                                 int H, int Hkv, int N, int D, int causal, float softmax_scale,
+                                 int smooth, void* stream, void* workspace,
+                                 size_t workspace_bytes) {
+  return attn_fwd_smooth_any(q, k, v, out, B, H, Hkv, N, D, causal, softmax_scale, smooth, stream,
+                             workspace, workspace_bytes);
+}
+
+fp4_status_t fp4_attn_fwd_quantized_bias(const fp4_tensor_t* q, const fp4_tensor_t* k,
+                                         const fp4_tensor_t* v, const float* bias, void* out,
+                                         int B, int H, int Hkv, int N, int D, int causal,
+                                         float softmax_scale, void* stream) {
+  if (!bias) {
+    g_last_error.clear();
+    return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  }
+  return attn_fwd_quantized_any(q, k, v, out, B, H, Hkv, N, D, causal, softmax_scale, stream, 0,
+                                bias);
 }
 
 size_t fp4_attn_workspace_bytes_fp8pv(int B, int H, int Hkv, int N, int D) {

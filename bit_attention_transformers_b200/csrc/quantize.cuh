@@ -112,12 +112,15 @@ __global__ void __launch_bounds__(256) amax3_kernel(const uint4* __restrict__ x0
 
 // Blocks of 16 along D (Q and K). One thread per block; the four scales of a
 // row's consecutive blocks are gathered with shuffles into one 32-bit store.
-template <int D>
+// With `mean` ([G][D] fp32, the smoothing means) the quantised values are the
+// smoothed fl32(x - mean) of rows < N.
+template <int D, bool SMOOTH = false>
 __global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16* __restrict__ x, int G,
                                                          int N, int Npad,
                                                          const float* __restrict__ amax,
                                                          uint8_t* __restrict__ codes,
-                                                         uint8_t* __restrict__ sf) {
+                                                         uint8_t* __restrict__ sf,
+                                                         const float* __restrict__ mean = nullptr) {
   constexpr int NB = D / 16;
   const float s_enc = tensor_senc(*amax);
   const int64_t total = (int64_t)G * Npad * NB;  // a multiple of 32
@@ -135,6 +138,17 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16* __
       const __nv_bfloat16* src = x + ((g * N + n) * D + kb * 16);
       bf16x8_to_f32(ld_nc_v4(src), xv);
       bf16x8_to_f32(ld_nc_v4(src + 8), xv + 8);
+      if constexpr (SMOOTH) {
+        const float4* mu = reinterpret_cast<const float4*>(mean + g * D + kb * 16);
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const float4 m4 = __ldg(mu + k4);
+          xv[4 * k4] = __fsub_rn(xv[4 * k4], m4.x);
+          xv[4 * k4 + 1] = __fsub_rn(xv[4 * k4 + 1], m4.y);
+          xv[4 * k4 + 2] = __fsub_rn(xv[4 * k4 + 2], m4.z);
+          xv[4 * k4 + 3] = __fsub_rn(xv[4 * k4 + 3], m4.w);
+        }
+      }
     } else {
 #pragma unroll
       for (int k = 0; k < 16; ++k) xv[k] = 0.0f;
@@ -253,6 +267,170 @@ __global__ void __launch_bounds__(128) quant_fp8_tokens_T_kernel(const __nv_bflo
 #pragma unroll
     for (int k = 0; k < 8; ++k)
       dst[k] = make_uint4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
+  }
+}
+
+// ------------------------------------------------------------- smoothing
+// Outlier smoothing of Q and K [SageAttention2 abstract, searcharxiv.com author
+// page "Pengle Zhang": smoothing Q for a more accurate low-bit QK^T]. The page
+// gives no formula; the reading implemented:
+//   mean_d per (batch, head) and channel over the head's N tokens, on a
+//   fixed-point grid so that it is one value whatever the summation order:
+//   every element truncated toward zero to a multiple of 2^-s, s = 44 - E with
+//   2^(E-1) <= amax < 2^E (amax of the raw tensor), the integers summed
+//   exactly in 64 bits (N <= 2^19), mean = fl32(fl64(fl64(T) 2^-s) / N);
+//   x' = fl32(x - mean) is quantised as usual, with the tensor scale from
+//   max |x'| over the whole smoothed tensor.
+//   K: the correction -q_i . mean_K is the same for every key of a row and
+//   cancels in the softmax. Q: the correction mean_Q . k'_j depends on the key;
+//   it is added to the scores: bias_j = fl32(delta_j fl32(softmax_scale log2 e)),
+//   delta_j an fp32 fma chain over d = 0 .. D-1 from 0, k' = fl32(k - mean_K)
+//   when K is smoothed, else k; x_ij = fma(S'_ij, c, bias_j).
+
+constexpr int kMeanGridBits = 44;
+
+// s = 44 - E for amax in [2^(E-1), 2^E) (amax > 0).
+__device__ __forceinline__ int mean_grid_shift(float amax) {
+  int E;
+  frexpf(amax, &E);
+  return kMeanGridBits - E;
+}
+
+// trunc(x 2^s) of a bf16 bit pattern, exactly, from its integer significand
+// (|x| < 2^E keeps the result below 2^44).
+__device__ __forceinline__ long long bf16_fixed(uint32_t b, int s) {
+  const uint32_t ex = (b >> 7) & 0xFFu, man = b & 0x7Fu;
+  const long long M = ex ? (long long)(0x80u | man) : (long long)man;
+  const int sh = (ex ? (int)ex : 1) - 134 + s;  // x = M 2^(ex - 134), subnormals 2^-133
+  long long v = sh >= 0 ? (M << min(sh, 55)) : (sh > -16 ? (M >> -sh) : 0ll);
+  return (b & 0x8000u) ? -v : v;
+}
+
+// Per (group, channel) integer sums T of x [G][N][D] on the grid of amax
+// (blockIdx.y = group, blockIdx.x = a chunk of kSumRows tokens). sums [G][D]
+// must be zeroed first; 64-bit integer addition makes the result independent
+// of the order of the atomics.
+constexpr int kSumRows = 256;
+template <int D>
+__global__ void __launch_bounds__(256) colsum_fixed_kernel(const __nv_bfloat16* __restrict__ x,
+                                                           int N, const float* __restrict__ amax,
+                                                           unsigned long long* __restrict__ sums) {
+  constexpr int VEC = D / 8;         // uint4 per row
+  constexpr int R = 256 / VEC;       // rows per pass
+  __shared__ long long red[R][D];
+  const float a = *amax;
+  const int64_t g = blockIdx.y;
+  const int c8 = threadIdx.x % VEC, r0 = threadIdx.x / VEC;
+  long long acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (a > 0.0f) {
+    const int s = mean_grid_shift(a);
+    const int n1 = min(N, (int)(blockIdx.x + 1) * kSumRows);
+    for (int n = blockIdx.x * kSumRows + r0; n < n1; n += R) {
+      const uint4 w = ld_nc_v4(x + ((g * N + n) * D + c8 * 8));
+      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] += bf16_fixed(u[i] & 0xFFFFu, s);
+        acc[2 * i + 1] += bf16_fixed(u[i] >> 16, s);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) red[r0][c8 * 8 + i] = acc[i];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    long long t = 0;
+#pragma unroll 4
+    for (int r = 0; r < R; ++r) t += red[r][threadIdx.x];
+    if (t) atomicAdd(sums + g * D + threadIdx.x, (unsigned long long)t);
+  }
+}
+
+// mean = fl32(fl64(fl64(T) 2^-s) / N), 0 when amax == 0; n = G * D values.
+__global__ void mean_from_sums_kernel(const unsigned long long* __restrict__ sums, int64_t n, int N,
+                                      const float* __restrict__ amax, float* __restrict__ mean) {
+  const float a = *amax;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float m = 0.0f;
+    if (a > 0.0f) {
+      const double t = ldexp(__ll2double_rn((long long)sums[i]), -mean_grid_shift(a));
+      m = __double2float_rn(__ddiv_rn(t, (double)N));
+    }
+    mean[i] = m;
+  }
+}
+
+// max |fl32(x - mean)| over x [G][N][D] with means [G][D], as fp32 bits
+// (non-negative floats order like their bit patterns); out zeroed first.
+template <int D>
+__global__ void __launch_bounds__(256) amax_smoothed_kernel(const __nv_bfloat16* __restrict__ x,
+                                                            int64_t G, int N,
+                                                            const float* __restrict__ mean,
+                                                            unsigned* __restrict__ out) {
+  constexpr int VEC = D / 8;
+  const int64_t total = G * N * VEC;
+  uint32_t m = 0;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int c8 = (int)(i % VEC);
+    const int64_t g = i / ((int64_t)N * VEC);
+    float xv[8];
+    bf16x8_to_f32(ld_nc_v4(x + i * 8), xv);
+    const float4* mu = reinterpret_cast<const float4*>(mean + g * D + c8 * 8);
+    const float4 m0 = __ldg(mu), m1 = __ldg(mu + 1);
+    const float mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m = max(m, __float_as_uint(fabsf(__fsub_rn(xv[k], mv[k]))));
+  }
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  __shared__ uint32_t wm[8];
+  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t r = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r = max(r, wm[w]);
+    if (r) atomicMax(out, r);
+  }
+}
+
+// Q's score correction: bias [B*H][Npad] with bias_j = fl32(delta_j cs) for
+// keys j < N (0 beyond), delta_j = fma chain of qmean [B*H][D] with k'_j
+// (k [B*Hkv][N][D]; k' = fl32(k - kmean) when kmean [B*Hkv][D] is given).
+// Grid (Npad / 128, B * Hkv); thread = key, looping over the key/value head's
+// G = H / Hkv query heads.
+constexpr float kLog2e = 1.44269504088896340736f;  // fl32(1 / ln 2)
+template <int D>
+__global__ void __launch_bounds__(128) score_bias_kernel(const float* __restrict__ qmean,
+                                                         const __nv_bfloat16* __restrict__ k,
+                                                         const float* __restrict__ kmean, int H,
+                                                         int Hkv, int N, int Npad,
+                                                         float softmax_scale,
+                                                         float* __restrict__ bias) {
+  const int64_t gk = blockIdx.y;
+  const int j = blockIdx.x * 128 + threadIdx.x;
+  const int G = H / Hkv;
+  const int64_t gq0 = (gk / Hkv) * H + (gk % Hkv) * G;
+  const float cs = __fmul_rn(softmax_scale, kLog2e);
+  float kv[D];
+  if (j < N) {
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) bf16x8_to_f32(ld_nc_v4(k + ((gk * N + j) * D + c * 8)), kv + 8 * c);
+    if (kmean) {
+#pragma unroll
+      for (int d = 0; d < D; ++d) kv[d] = __fsub_rn(kv[d], __ldg(kmean + gk * D + d));
+    }
+  }
+  for (int g2 = 0; g2 < G; ++g2) {
+    float r = 0.0f;
+    if (j < N) {
+      const float* qm = qmean + (gq0 + g2) * D;
+      float delta = 0.0f;
+#pragma unroll
+      for (int d = 0; d < D; ++d) delta = __fmaf_rn(__ldg(qm + d), kv[d], delta);
+      r = __fmul_rn(delta, cs);
+    }
+    bias[(gq0 + g2) * Npad + j] = r;
   }
 }
 

@@ -56,7 +56,7 @@ def allreduce_max_(t, group=None):
 
 def fp4_attn_fwd_sharded(q, k, v, causal: bool = False, softmax_scale: float | None = None,
                          group=None, out=None, stream=None, efq: bool = False,
-                         fp8pv: bool = False):
+                         fp8pv: bool = False, smooth: int = 0):
     """This rank's part of a head-sharded NVFP4 attention forward.
 
     q: this rank's query heads, a contiguous bf16 CUDA tensor [..., N, D] whose
@@ -65,10 +65,16 @@ def fp4_attn_fwd_sharded(q, k, v, causal: bool = False, softmax_scale: float | N
     G, causal and softmax_scale, an empty shard (U = 0) included: it still
     takes part in the all-reduce. Returns `out` (like q) with this rank's
     output heads. efq selects the EFQ-Softmax P generation, fp8pv the FP8 P
-    and V variant."""
+    and V variant, smooth (FP4_SMOOTH_K | FP4_SMOOTH_Q) Q/K smoothing: the
+    means are per head, so local; their grid comes from the global raw
+    maxima, and a second all-reduce (MAX) makes the smoothed maxima global."""
     import torch
-    from . import (FP4_BLOCK_ALONG_D, FP4_BLOCK_ALONG_N_T, fp4_amax, fp4_attn_fwd_quantized,
-                   fp4_quantize, fp4_quantize_fp8)
+    from . import (FP4_BLOCK_ALONG_D, FP4_BLOCK_ALONG_N_T, FP4_SMOOTH_K, FP4_SMOOTH_Q,
+                   fp4_amax, fp4_amax_smoothed, fp4_attn_fwd_quantized,
+                   fp4_attn_fwd_quantized_bias, fp4_channel_mean, fp4_quantize, fp4_quantize_fp8,
+                   fp4_quantize_smoothed, fp4_score_bias)
+    if smooth and (efq or fp8pv):
+        raise ValueError("smoothing is built for the exp-then-quantize NVFP4 path")
     N, D = q.shape[-2], q.shape[-1]
     if k.shape[-2:] != (N, D) or v.shape != k.shape:
         raise ValueError("q, k, v must share N and D, and k and v their shape")
@@ -83,6 +89,32 @@ def fp4_attn_fwd_sharded(q, k, v, causal: bool = False, softmax_scale: float | N
     allreduce_max_(amax, group)
     if out is None:
         out = torch.empty_like(q)
+    if smooth:
+        # means with the global raw maxima; then the smoothed maxima, made global
+        sm = torch.zeros(2, dtype=torch.float32, device=q.device)
+        qmean = kmean = None
+        if gkv and smooth & FP4_SMOOTH_K:
+            kmean = fp4_channel_mean(k, amax[1:2], stream)
+            sm[1:2] = fp4_amax_smoothed(k, kmean, stream)
+        if gkv and smooth & FP4_SMOOTH_Q:
+            qmean = fp4_channel_mean(q, amax[0:1], stream)
+            sm[0:1] = fp4_amax_smoothed(q, qmean, stream)
+        allreduce_max_(sm, group)
+        if gkv == 0:
+            return out
+        qq = (fp4_quantize_smoothed(q, qmean, sm[0:1], stream) if qmean is not None else
+              fp4_quantize(q, FP4_BLOCK_ALONG_D, stream, amax=amax[0:1]))
+        kq = (fp4_quantize_smoothed(k, kmean, sm[1:2], stream) if kmean is not None else
+              fp4_quantize(k, FP4_BLOCK_ALONG_D, stream, amax=amax[1:2]))
+        vq = fp4_quantize(v, FP4_BLOCK_ALONG_N_T, stream, amax=amax[2:3])
+        if qmean is not None:
+            bias = fp4_score_bias(qmean, k.view(1, gkv, N, D), kmean, gq, softmax_scale, stream)
+            fp4_attn_fwd_quantized_bias(qq, kq, vq, bias, 1, gq, gkv, causal, softmax_scale,
+                                        out=out, stream=stream)
+        else:
+            fp4_attn_fwd_quantized(qq, kq, vq, 1, gq, gkv, causal, softmax_scale, out=out,
+                                   stream=stream)
+        return out
     if gkv == 0:
         return out
     qq = fp4_quantize(q, FP4_BLOCK_ALONG_D, stream, amax=amax[0:1])

@@ -219,6 +219,72 @@ fp4_status_t fp4_quantize_fp8_scaled(const void* x, int G, int N, int D, const f
  * fp4_attn_fwd_quantized_fp8pv takes v->codes from fp4_quantize_fp8 and
  * v->amax its maximum; v->scales is not read and may be NULL.
  */
+/*
+ * Outlier smoothing of Q and K before NVFP4 (SageAttention2 abstract,
+ * searcharxiv.com author page "Pengle Zhang": Q is smoothed to make the
+ * low-bit QK^T more accurate). The page gives no formula; the reading:
+ *   per (batch, head) and channel d, mean_d over the head's N tokens, on a
+ *   fixed-point grid so that it does not depend on summation order: each
+ *   element truncated toward zero to a multiple of 2^-s, s = 44 - E with
+ *   2^(E-1) <= amax < 2^E (amax: max |x| of the whole raw tensor), the
+ *   integers summed exactly in 64 bits (hence N <= 2^19), and
+ *   mean = fl32(fl64(fl64(T) * 2^-s) / N) (0 when amax == 0);
+ *   x' = fl32(x - mean) quantised as NVFP4 with the tensor scale taken from
+ *   max |x'| over the whole smoothed tensor.
+ *   Smoothing K changes every score of a query row by the same amount, which
+ *   the softmax cancels. Smoothing Q leaves the key-dependent term
+ *   mean_Q . k'_j, added back to the scores: bias_j = fl32(delta_j * cs),
+ *   cs = fl32(softmax_scale * log2(e)), delta_j = a sequential fp32 fma chain
+ *   over d = 0..D-1 from 0 of mean_Q[d] * k'_j[d] (k' = fl32(k - mean_K) if K
+ *   is smoothed, else k); the fused kernel forms x_ij = fma(S'_ij, c, bias_j).
+ */
+#define FP4_SMOOTH_K 1
+#define FP4_SMOOTH_Q 2
+
+/*
+ * The whole smoothed forward: fp4_attn_fwd with Q and/or K smoothed (smooth =
+ * FP4_SMOOTH_K | FP4_SMOOTH_Q, 0 gives the plain forward) and
+ * fp4_attn_workspace_bytes_smooth bytes of workspace (0 for a bad shape or
+ * N > 2^19). Same layouts and errors as fp4_attn_fwd; FP4_ERR_INVALID_ARG
+ * for unknown smooth bits or N > 2^19.
+ */
+size_t fp4_attn_workspace_bytes_smooth(int B, int H, int Hkv, int N, int D);
+fp4_status_t fp4_attn_fwd_smooth(const void* q, const void* k, const void* v, void* out, int B,
+                                 int H, int Hkv, int N, int D, int causal, float softmax_scale,
+                                 int smooth, void* stream, void* workspace,
+                                 size_t workspace_bytes);
+
+/*
+ * The steps of the smoothed forward, one by one.
+ * fp4_channel_mean: x [G][N][D] bf16 -> mean [G][D] fp32 on the grid of *amax
+ *   (the raw tensor's maximum, device memory); sums: G*D uint64 device scratch
+ *   (overwritten). N <= 2^19.
+ * fp4_amax_smoothed: *amax = max |fl32(x - mean)| over x [G][N][D].
+ * fp4_quantize_smoothed: NVFP4 codes and scales (FP4_BLOCK_ALONG_D layouts) of
+ *   fl32(x - mean) with the tensor scale 2688 / *amax (amax of the smoothed
+ *   tensor, device memory, read only).
+ * fp4_score_bias: bias [B*H][Npad] fp32 (keys >= N get 0) from qmean
+ *   [B*H][D], k [B][Hkv][N][D] bf16 and kmean [B*Hkv][D] (NULL when K is not
+ *   smoothed); softmax_scale <= 0 or NaN means 1/sqrt(D).
+ * fp4_attn_fwd_quantized_bias: fp4_attn_fwd_quantized (exp-then-quantize P)
+ *   with the per-key correction bias [B*H][Npad]: x_ij = fma(S_ij, c, bias_j).
+ * Pointers: device memory, 16-byte aligned (amax 4-byte aligned).
+ */
+fp4_status_t fp4_channel_mean(const void* x, int G, int N, int D, const float* amax,
+                              float* mean, unsigned long long* sums, void* stream);
+fp4_status_t fp4_amax_smoothed(const void* x, int G, int N, int D, const float* mean, float* amax,
+                               void* stream);
+fp4_status_t fp4_quantize_smoothed(const void* x, int G, int N, int D, const float* mean,
+                                   const float* amax, uint8_t* codes, uint8_t* scales,
+                                   void* stream);
+fp4_status_t fp4_score_bias(const float* qmean, const void* k, const float* kmean, int B, int H,
+                            int Hkv, int N, int D, float softmax_scale, float* bias,
+                            void* stream);
+fp4_status_t fp4_attn_fwd_quantized_bias(const fp4_tensor_t* q, const fp4_tensor_t* k,
+                                         const fp4_tensor_t* v, const float* bias, void* out,
+                                         int B, int H, int Hkv, int N, int D, int causal,
+                                         float softmax_scale, void* stream);
+
 size_t fp4_attn_workspace_bytes_fp8pv(int B, int H, int Hkv, int N, int D);
 fp4_status_t fp4_attn_fwd_fp8pv(const void* q, const void* k, const void* v, void* out, int B,
                                 int H, int Hkv, int N, int D, int causal, float softmax_scale,
