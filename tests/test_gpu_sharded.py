@@ -98,3 +98,53 @@ def test_emulated_shards_equal_unsharded(syn, case, world):
     torch.cuda.synchronize()
     fa.fp4_status()
     assert np.array_equal(from_dev(out).reshape(-1), from_dev(ref).reshape(-1))
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_one_rank_smooth_equals_unsharded(syn, case):
+    import torch
+    B, H, Hkv, N, D, causal = case
+    q, k, v, _ = _inputs(syn, B, H, Hkv, N, D, 700)
+    for smooth in (fa.FP4_SMOOTH_K, fa.FP4_SMOOTH_Q, fa.FP4_SMOOTH_K | fa.FP4_SMOOTH_Q):
+        ref = fa.fp4_attn_fwd_smooth(q, k, v, smooth=smooth, causal=causal)
+        got = fa.fp4_attn_fwd_sharded(q.view(B * H, N, D), k.view(B * Hkv, N, D),
+                                      v.view(B * Hkv, N, D), causal=causal, smooth=smooth)
+        torch.cuda.synchronize()
+        fa.fp4_status()
+        assert torch.equal(ref.view(-1), got.view(-1))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("case", CASES)
+def test_emulated_smoothed_shards_equal_unsharded(syn, case, world):
+    """Smoothing sharded by head: each shard's means come from the global raw
+    maxima; the smoothed maxima are combined by max (the second all-reduce);
+    each shard's output equals its slab of the unsharded smoothed run."""
+    import torch
+    B, H, Hkv, N, D, causal = case
+    q, k, v, _ = _inputs(syn, B, H, Hkv, N, D, 800 + world)
+    ref = fa.fp4_attn_fwd_smooth(q, k, v, causal=causal)
+    qf, kf, vf = q.view(B * H, N, D), k.view(B * Hkv, N, D), v.view(B * Hkv, N, D)
+    shards = [fa.shard_rows(B, H, Hkv, world, r) for r in range(world)
+              if fa.shard_rows(B, H, Hkv, world, r)[1].stop > fa.shard_rows(B, H, Hkv, world, r)[1].start]
+    amax = torch.zeros(3, dtype=torch.float32, device="cuda")
+    for sq, skv in shards:
+        part = torch.stack([fa.fp4_amax(qf[sq]), fa.fp4_amax(kf[skv]), fa.fp4_amax(vf[skv])]).view(3)
+        amax = torch.maximum(amax, part)
+    means = [(fa.fp4_channel_mean(qf[sq], amax[0:1]), fa.fp4_channel_mean(kf[skv], amax[1:2]))
+             for sq, skv in shards]
+    sm = torch.zeros(2, dtype=torch.float32, device="cuda")
+    for (sq, skv), (qm, km) in zip(shards, means):
+        part = torch.stack([fa.fp4_amax_smoothed(qf[sq], qm), fa.fp4_amax_smoothed(kf[skv], km)])
+        sm = torch.maximum(sm, part.view(2))
+    out = torch.empty_like(qf)
+    for (sq, skv), (qm, km) in zip(shards, means):
+        gq, gk = sq.stop - sq.start, skv.stop - skv.start
+        qs = fa.fp4_quantize_smoothed(qf[sq], qm, sm[0:1])
+        ks = fa.fp4_quantize_smoothed(kf[skv], km, sm[1:2])
+        vs = fa.fp4_quantize(vf[skv], fa.FP4_BLOCK_ALONG_N_T, amax=amax[2:3])
+        bias = fa.fp4_score_bias(qm, kf[skv].view(1, gk, N, D), km, gq)
+        fa.fp4_attn_fwd_quantized_bias(qs, ks, vs, bias, 1, gq, gk, causal=causal, out=out[sq])
+    torch.cuda.synchronize()
+    fa.fp4_status()
+    assert np.array_equal(from_dev(out).reshape(-1), from_dev(ref).reshape(-1))
