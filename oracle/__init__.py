@@ -87,6 +87,9 @@ def _load():
         lib.ora_attn_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, i32,
                                      vp, i64, vp, vp, vp, vp, i32]
         lib.ora_attn_fwd.restype = i32
+        lib.ora_attn_bwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, i64,
+                                     vp, i64, vp, vp, vp, vp, i32]
+        lib.ora_attn_bwd.restype = i32
         _lib = lib
     return _lib
 
@@ -314,3 +317,66 @@ def attn_fwd(q, k, v, causal: bool, softmax_scale: float = 0.0, rows=None, Bc: i
     if want_flip:
         res["flip"] = flip
     return res
+
+
+def attn_bwd(q, k, v, dout, causal: bool, softmax_scale: float = 0.0, q_rows=None,
+             kv_rows=None, want_D: bool = False, threads: int | None = None) -> dict:
+    """The FP4 attention backward (reading in the source, at bwd_row).
+    q, dout [B, H, N, D], k, v [B, Hkv, N, D] bf16 bits. q_rows / kv_rows:
+    int64 [n, 3] (b, h, i) / (b, hk, j) rows to compute, None for all, or an
+    empty array for none. Returns dq [.., D], dk, dv (fp64, shaped like the
+    inputs when every row is computed) and D [B, H, N] when want_D."""
+    q, k, v, dout = (_c(t, np.uint16) for t in (q, k, v, dout))
+    B, H, N, D = q.shape
+    Hkv = k.shape[1]
+    assert k.shape == (B, Hkv, N, D) and v.shape == k.shape and dout.shape == q.shape
+    out = {}
+    qr = None if q_rows is None else _c(q_rows, np.int64).reshape(-1, 3)
+    kr = None if kv_rows is None else _c(kv_rows, np.int64).reshape(-1, 3)
+    nq = B * H * N if qr is None else len(qr)
+    nkv = B * Hkv * N if kr is None else len(kr)
+    dq = np.zeros((nq, D))
+    dk = np.zeros((nkv, D))
+    dv = np.zeros((nkv, D))
+    Dv = np.zeros((B, H, N)) if want_D else None
+    rc = _load().ora_attn_bwd(
+        q.ctypes.data, k.ctypes.data, v.ctypes.data, dout.ctypes.data, B, H, Hkv, N, D,
+        int(bool(causal)), float(softmax_scale), None if qr is None else qr.ctypes.data, nq,
+        None if kr is None else kr.ctypes.data, nkv if (kr is None or len(kr)) else -1,
+        dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, None if Dv is None else Dv.ctypes.data,
+        _threads(threads))
+    if rc != 0:
+        raise ValueError("ora_attn_bwd: bad arguments")
+    out["dq"] = dq.reshape(B, H, N, D) if qr is None else dq
+    out["dk"] = dk.reshape(B, Hkv, N, D) if kr is None else dk
+    out["dv"] = dv.reshape(B, Hkv, N, D) if kr is None else dv
+    if want_D:
+        out["D"] = Dv
+    return out
+
+
+def dequantized(x_bf16: np.ndarray, axis: str) -> np.ndarray:
+    """Real values of x's NVFP4 quantisation (tensor scale from its own
+    maximum): axis "rows" (blocks along D, Q and K) or "tokens" (V).
+    x [..., N, D] bf16 bits -> float64 [..., N, D]."""
+    x = _c(x_bf16, np.uint16)
+    N, D = x.shape[-2:]
+    s_enc, dec = tensor_scale(amax_bf16(x))
+    flat = x.reshape(-1, N, D)
+    out = np.empty(flat.shape)
+    e2 = np.array([0, .5, 1, 1.5, 2, 3, 4, 6, -0., -.5, -1, -1.5, -2, -3, -4, -6])
+    for g in range(flat.shape[0]):
+        if axis == "rows":
+            c, sc = quantize_rows(flat[g], s_enc)
+            codes = np.stack([c & 15, c >> 4], -1).reshape(N, D)
+            scale = np.repeat(np.array([e4m3_decode(int(t)) for t in sc.ravel()]).reshape(N, D // 16),
+                              16, axis=1)
+            out[g] = e2[codes] * scale * dec
+        else:
+            c, sc = quantize_tokens_T(flat[g], s_enc)
+            npad = c.shape[1] * 2
+            codes = np.stack([c & 15, c >> 4], -1).reshape(D, npad)
+            scale = np.repeat(np.array([e4m3_decode(int(t)) for t in sc.ravel()]).reshape(D, npad // 16),
+                              16, axis=1)
+            out[g] = (e2[codes] * scale * dec)[:, :N].T
+    return out.reshape(x.shape)

@@ -26,6 +26,10 @@
 //    channel, with the score correction that keeps the softmax exact)
 //    [SageAttention2 abstract, searcharxiv.com author page "Pengle Zhang"];
 //    the reading is at channel_mean.
+//  * The backward (ora_attn_bwd) recomputes the scores from the forward's
+//    FP4 operands and takes D from its own P and V~ [Attn-QAT abstract, arxiv
+//    listing "Attn-QAT: 4-Bit Attention With Quantization-Aware Training"];
+//    the reading is at attn_bwd_group.
 // The pages give no formula for any of these steps. Where this file fixes one
 // (format constants, scale recipe, rounding, masking, GQA mapping, the
 // denominator) it states the reading it takes.
@@ -721,6 +725,116 @@ void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float 
   }
 }
 
+// ---------------------------------------------------------------- backward ----
+// FP4 attention backward [Attn-QAT abstract, arxiv listing "Attn-QAT: 4-Bit
+// Attention With Quantization-Aware Training": stable FP4 attention training
+// needs (1) the backward to recompute the attention scores in the same low
+// precision as the forward and (2) FlashAttention's gradient computation to be
+// freed of an implicit precision assumption]. The abstract gives no formula;
+// the reading taken here, for one (batch, key/value head) group:
+//   q~, k~, v~   the forward's NVFP4 operands, dequantised to real values
+//                (val(code) dec(e) d, d the tensor's decode scale)
+//   s_ij         q~_i . k~_j, exact; masked (causal j > i) -> -inf   (1)
+//   P_ij         exp(scale s_ij - lse_i), lse_i = log sum_j exp(scale s_ij):
+//                the forward's probabilities before their quantisation
+//   dP_ij        dO_i . v~_j
+//   D_i          sum_j P_ij dP_ij                                   (2)
+//                FlashAttention forms D from the forward output as dO_i . O_i,
+//                which equals sum_j P_ij dP_ij only when O = P V~ exactly in
+//                the backward's precision; the FP4 forward's O is P~ V~ / l with
+//                quantised P~, so D is taken from this P and v~ instead
+//   dS_ij        P_ij (dP_ij - D_i)
+//   dq_i         scale sum_j dS_ij k~_j
+//   dk_j         scale sum_{i, query heads of the group} dS_ij q~_i
+//   dv_j         sum_{i, query heads of the group} P_ij dO_i
+// The quantisers pass gradients straight through: dq, dk, dv are the
+// gradients with respect to q~, k~, v~ and serve as those of q, k, v.
+// Everything in double.
+struct BwdGroup {
+  int N, D, G;
+  std::vector<double> K, V;       // [N][D] real values
+  std::vector<double> Q, dO;      // [G][N][D]
+};
+
+BwdGroup make_bwd_group(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                        const uint16_t* dout, int B, int H, int Hkv, int N, int D, int b, int hk,
+                        const float* s_enc, const float* dec) {
+  (void)B;
+  BwdGroup g;
+  g.N = N;
+  g.D = D;
+  g.G = H / Hkv;
+  const int64_t nd = (int64_t)N * D;
+  g.K.resize(nd);
+  g.V.resize(nd);
+  g.Q.resize(g.G * nd);
+  g.dO.resize(g.G * nd);
+  std::vector<uint8_t> c((size_t)nd / 2), sc((size_t)nd / 16);
+  auto deq_rows = [&](const uint16_t* x, float se, float d, double* outp) {
+    quantize_rows(x, N, D, se, c.data(), sc.data(), 1);
+    for (int64_t n = 0; n < N; ++n)
+      for (int dd = 0; dd < D; ++dd) {
+        uint8_t byte = c[n * (D / 2) + dd / 2];
+        outp[n * D + dd] = deq((dd & 1) ? (byte >> 4) : (byte & 15), sc[n * (D / 16) + dd / 16]) *
+                           (double)d;
+      }
+  };
+  const int64_t kvoff = ((int64_t)b * Hkv + hk) * nd;
+  deq_rows(k + kvoff, s_enc[1], dec[1], g.K.data());
+  {
+    const int npad = (N + 15) / 16 * 16;
+    std::vector<uint8_t> vc((size_t)D * npad / 2), vs((size_t)D * npad / 16);
+    quantize_tokens_T(v + kvoff, N, D, s_enc[2], vc.data(), vs.data(), npad);
+    for (int dd = 0; dd < D; ++dd)
+      for (int64_t n = 0; n < N; ++n) {
+        uint8_t byte = vc[dd * (npad / 2) + n / 2];
+        g.V[n * D + dd] = deq((n & 1) ? (byte >> 4) : (byte & 15), vs[dd * (npad / 16) + n / 16]) *
+                          (double)dec[2];
+      }
+  }
+  for (int gg = 0; gg < g.G; ++gg) {
+    const int64_t qoff = ((int64_t)b * H + hk * g.G + gg) * nd;
+    deq_rows(q + qoff, s_enc[0], dec[0], &g.Q[gg * nd]);
+    for (int64_t e = 0; e < nd; ++e) g.dO[gg * nd + e] = (double)bf16_to_f32(dout[qoff + e]);
+  }
+  return g;
+}
+
+// One query row of head gg of the group: P (N), dS (N) and D; row masked to
+// keys <= i when causal.
+void bwd_row(const BwdGroup& g, int gg, int i, int causal, double scale, double* P, double* dS,
+             double* Dout) {
+  const int N = g.N, D = g.D;
+  const double* qi = &g.Q[((int64_t)gg * N + i) * D];
+  const double* di = &g.dO[((int64_t)gg * N + i) * D];
+  const int jmax = causal ? i + 1 : N;
+  double mx = -INFINITY;
+  for (int j = 0; j < jmax; ++j) {
+    double s = 0.0;
+    for (int d = 0; d < D; ++d) s += qi[d] * g.K[(int64_t)j * D + d];
+    P[j] = scale * s;
+    mx = std::max(mx, P[j]);
+  }
+  double sum = 0.0;
+  for (int j = 0; j < jmax; ++j) sum += std::exp(P[j] - mx);
+  const double lse = mx + std::log(sum);
+  double Dsum = 0.0;
+  for (int j = 0; j < N; ++j) {
+    if (j >= jmax) {
+      P[j] = 0.0;
+      dS[j] = 0.0;
+      continue;
+    }
+    P[j] = std::exp(P[j] - lse);
+    double dp = 0.0;
+    for (int d = 0; d < D; ++d) dp += di[d] * g.V[(int64_t)j * D + d];
+    dS[j] = dp;  // dP for now
+    Dsum += P[j] * dp;
+  }
+  for (int j = 0; j < jmax; ++j) dS[j] = P[j] * (dS[j] - Dsum);
+  *Dout = Dsum;
+}
+
 }  // namespace
 
 extern "C" {
@@ -841,6 +955,119 @@ int ora_scores_head(const uint16_t* q, const uint16_t* k, int B, int H, int Hkv,
       S[i * N + j] = (float)s;
     }
   });
+  return 0;
+}
+
+// The FP4 attention backward (reading at bwd_row / make_bwd_group).
+//   q, dout [B][H][N][D], k, v [B][Hkv][N][D] bf16 bit patterns.
+//   q_rows: nq (b, h, i) triples whose dq rows are wanted (NULL: every row);
+//   kv_rows: nkv (b, hk, j) triples whose dk and dv rows are wanted (NULL:
+//   every row; nkv < 0: none). dq_out [nq][D], dk_out / dv_out [nkv][D]
+//   (fp64, may be NULL), D_out [B][H][N] (may be NULL; computed for every
+//   row of a group that needs any).
+// Returns 0, or -1 on bad arguments.
+int ora_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                 int B, int H, int Hkv, int N, int D, int causal, float softmax_scale,
+                 const int64_t* q_rows, int64_t nq, const int64_t* kv_rows, int64_t nkv,
+                 double* dq_out, double* dk_out, double* dv_out, double* D_out, int nthreads) {
+  if (B <= 0 || H <= 0 || Hkv <= 0 || H % Hkv || N <= 0 || D <= 0 || D % 16) return -1;
+  e4m3_encode(0.0f);
+  float se[3], dc[3];
+  tensor_scale(amax_bf16(q, (int64_t)B * H * N * D), &se[0], &dc[0]);
+  tensor_scale(amax_bf16(k, (int64_t)B * Hkv * N * D), &se[1], &dc[1]);
+  tensor_scale(amax_bf16(v, (int64_t)B * Hkv * N * D), &se[2], &dc[2]);
+  if (!(softmax_scale > 0.0f)) softmax_scale = 1.0f / std::sqrt((float)D);
+  const double scale = (double)softmax_scale;
+  const int G = H / Hkv;
+  std::vector<int64_t> allq, allkv;
+  if (!q_rows) {
+    nq = (int64_t)B * H * N;
+    allq.resize((size_t)nq * 3);
+    for (int64_t r = 0; r < nq; ++r) {
+      allq[r * 3] = r / ((int64_t)H * N);
+      allq[r * 3 + 1] = (r / N) % H;
+      allq[r * 3 + 2] = r % N;
+    }
+    q_rows = allq.data();
+  }
+  if (!kv_rows && nkv >= 0) {
+    nkv = (int64_t)B * Hkv * N;
+    allkv.resize((size_t)nkv * 3);
+    for (int64_t r = 0; r < nkv; ++r) {
+      allkv[r * 3] = r / ((int64_t)Hkv * N);
+      allkv[r * 3 + 1] = (r / N) % Hkv;
+      allkv[r * 3 + 2] = r % N;
+    }
+    kv_rows = allkv.data();
+  }
+  if (nkv < 0) nkv = 0;
+  for (int64_t r = 0; r < nq; ++r)
+    if (q_rows[r * 3] < 0 || q_rows[r * 3] >= B || q_rows[r * 3 + 1] < 0 ||
+        q_rows[r * 3 + 1] >= H || q_rows[r * 3 + 2] < 0 || q_rows[r * 3 + 2] >= N)
+      return -1;
+  for (int64_t r = 0; r < nkv; ++r)
+    if (kv_rows[r * 3] < 0 || kv_rows[r * 3] >= B || kv_rows[r * 3 + 1] < 0 ||
+        kv_rows[r * 3 + 1] >= Hkv || kv_rows[r * 3 + 2] < 0 || kv_rows[r * 3 + 2] >= N)
+      return -1;
+  for (int b = 0; b < B; ++b)
+    for (int hk = 0; hk < Hkv; ++hk) {
+      std::vector<int64_t> mq, mkv;
+      for (int64_t r = 0; r < nq; ++r)
+        if (q_rows[r * 3] == b && q_rows[r * 3 + 1] / G == hk) mq.push_back(r);
+      for (int64_t r = 0; r < nkv; ++r)
+        if (kv_rows[r * 3] == b && kv_rows[r * 3 + 1] == hk) mkv.push_back(r);
+      if (mq.empty() && mkv.empty() && !D_out) continue;
+      const BwdGroup g = make_bwd_group(q, k, v, dout, B, H, Hkv, N, D, b, hk, se, dc);
+      // dq rows: one row's P and dS each
+      parallel_for((int64_t)mq.size(), nthreads, [&](int64_t u) {
+        const int64_t r = mq[u];
+        const int gg = (int)q_rows[r * 3 + 1] % G, i = (int)q_rows[r * 3 + 2];
+        std::vector<double> P(N), dS(N);
+        double Dv;
+        bwd_row(g, gg, i, causal, scale, P.data(), dS.data(), &Dv);
+        if (dq_out)
+          for (int d = 0; d < D; ++d) {
+            double acc = 0.0;
+            for (int j = 0; j < N; ++j) acc += dS[j] * g.K[(int64_t)j * D + d];
+            dq_out[r * D + d] = scale * acc;
+          }
+      });
+      if (mkv.empty() && !D_out) continue;
+      // dk, dv rows and D: every query row of every head of the group
+      std::vector<double> dK(mkv.size() * D, 0.0), dV(mkv.size() * D, 0.0);
+      std::vector<double> Dall((size_t)G * N);
+      std::vector<double> Pall, dSall;
+      if (!mkv.empty()) {
+        Pall.resize((size_t)G * N * mkv.size());
+        dSall.resize(Pall.size());
+      }
+      parallel_for((int64_t)G * N, nthreads, [&](int64_t rr) {
+        const int gg = (int)(rr / N), i = (int)(rr % N);
+        std::vector<double> P(N), dS(N);
+        bwd_row(g, gg, i, causal, scale, P.data(), dS.data(), &Dall[rr]);
+        for (size_t u = 0; u < mkv.size(); ++u) {
+          const int j = (int)kv_rows[mkv[u] * 3 + 2];
+          Pall[(size_t)rr * mkv.size() + u] = P[j];
+          dSall[(size_t)rr * mkv.size() + u] = dS[j];
+        }
+      });
+      if (D_out)
+        for (int gg = 0; gg < G; ++gg)
+          for (int i = 0; i < N; ++i)
+            D_out[((int64_t)b * H + hk * G + gg) * N + i] = Dall[(size_t)gg * N + i];
+      parallel_for((int64_t)mkv.size(), nthreads, [&](int64_t u) {
+        for (int d = 0; d < D; ++d) {
+          double ak = 0.0, av = 0.0;
+          for (int64_t rr = 0; rr < (int64_t)G * N; ++rr) {
+            const size_t at = (size_t)rr * mkv.size() + u;
+            ak += dSall[at] * g.Q[rr * D + d];
+            av += Pall[at] * g.dO[rr * D + d];
+          }
+          if (dk_out) dk_out[mkv[u] * D + d] = scale * ak;
+          if (dv_out) dv_out[mkv[u] * D + d] = av;
+        }
+      });
+    }
   return 0;
 }
 
