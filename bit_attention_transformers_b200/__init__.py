@@ -38,7 +38,8 @@ EXPORTS = ("fp4_codes_bytes", "fp4_scales_bytes", "fp4_attn_workspace_bytes", "f
            "fp4_quantize_fp8", "fp4_quantize_fp8_scaled", "fp4_attn_workspace_bytes_fp8pv",
            "fp4_attn_fwd_fp8pv", "fp4_attn_fwd_quantized_fp8pv", "fp4_attn_workspace_bytes_smooth",
            "fp4_attn_fwd_smooth", "fp4_channel_mean", "fp4_amax_smoothed", "fp4_quantize_smoothed",
-           "fp4_score_bias", "fp4_attn_fwd_quantized_bias", "fp4_attn_fwd_noalloc",
+           "fp4_score_bias", "fp4_attn_fwd_quantized_bias", "fp4_attn_fwd_lse",
+           "fp4_attn_bwd_workspace_bytes", "fp4_attn_bwd", "fp4_attn_fwd_noalloc",
            "fp4_status", "fp4_last_error", "fp4_probe_cvt", "fp4_test_wait_timeout")
 FP4_NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -133,6 +134,14 @@ def lib():
         L.fp4_attn_fwd_quantized_bias.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                                   f32, vp]
         L.fp4_attn_fwd_quantized_bias.restype = i32
+        L.fp4_attn_fwd_lse.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp,
+                                       vp, sz]
+        L.fp4_attn_fwd_lse.restype = i32
+        L.fp4_attn_bwd_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+        L.fp4_attn_bwd_workspace_bytes.restype = sz
+        L.fp4_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                   f32, vp, vp, sz]
+        L.fp4_attn_bwd.restype = i32
         L.fp4_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
         L.fp4_attn_fwd_noalloc.restype = i32
         L.fp4_status.argtypes = [vp]
@@ -322,6 +331,59 @@ def fp4_attn_fwd(q, k, v, causal: bool = False, softmax_scale: float | None = No
     _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, Hkv, N, D, int(bool(causal)),
               float(softmax_scale or 0.0), _stream(stream), _ptr(ws), ws.numel()))
     return out
+
+
+def fp4_attn_fwd_lse(q, k, v, causal: bool = False, softmax_scale: float | None = None,
+                     out=None, lse=None, stream=None, ws=None):
+    """fp4_attn_fwd that also returns lse [B, H, N] fp32 (log2 units) for the
+    backward. Returns (out, lse)."""
+    import torch
+    B, H, N, D = q.shape
+    Hkv = k.shape[1]
+    for t in (q, k, v):
+        assert t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()
+    assert k.shape == (B, Hkv, N, D) and v.shape == (B, Hkv, N, D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(B, H, Hkv, N, D, q.device)
+    _check(lib().fp4_attn_fwd_lse(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, N, D,
+                                  int(bool(causal)), float(softmax_scale or 0.0), _stream(stream),
+                                  _ptr(ws), ws.numel()))
+    return out, lse
+
+
+_ws_bwd: dict = {}
+
+
+def fp4_attn_bwd(q, k, v, dout, lse, causal: bool = False, softmax_scale: float | None = None,
+                 dq=None, dk=None, dv=None, stream=None, ws=None):
+    """The FP4 attention backward (reading in include/fp4attn.h): q, dout [B,H,N,D],
+    k, v [B,Hkv,N,D] bf16 CUDA, lse [B,H,N] from fp4_attn_fwd_lse. Returns
+    (dq, dk, dv) bf16."""
+    import torch
+    B, H, N, D = q.shape
+    Hkv = k.shape[1]
+    for t in (q, k, v, dout):
+        assert t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()
+    assert k.shape == (B, Hkv, N, D) and v.shape == k.shape and dout.shape == q.shape
+    assert lse.dtype == torch.float32 and lse.is_contiguous() and lse.numel() == B * H * N
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if ws is None:
+        need = lib().fp4_attn_bwd_workspace_bytes(B, H, Hkv, N, D)
+        key = (str(q.device),)
+        ws = _ws_bwd.get(key)
+        if ws is None or ws.numel() < need:
+            ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+            _ws_bwd[key] = ws
+    _check(lib().fp4_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                              _ptr(dv), B, H, Hkv, N, D, int(bool(causal)),
+                              float(softmax_scale or 0.0), _stream(stream), _ptr(ws), ws.numel()))
+    return dq, dk, dv
 
 
 def fp4_attn_workspace_bytes_smooth(B: int, H: int, Hkv: int, N: int, D: int) -> int:

@@ -1,0 +1,758 @@
+// FP4 attention backward on sm_100a.
+//
+// Reading [Attn-QAT abstract, arxiv listing "Attn-QAT: 4-Bit Attention With
+// Quantization-Aware Training": the backward recomputes the scores in the
+// forward's low precision, and FlashAttention's D = dO . O holds an implicit
+// precision assumption]:
+//   S = Q^ K^T from the forward's NVFP4 operands (Q^, K^, V^ = val(code) dec(e),
+//       contraction units, exact in bf16; the tensor scales d_Q, d_K, d_V are
+//       applied as fp32 factors), x = S c with the forward's c
+//   P_ij = 2^(x_ij - lse_i), lse from the forward (log2 units)
+//   dP = d_V dO V^T,  D_i = sum_j P_ij dP_ij  (from this P and V~, not dO . O)
+//   dS = P (dP - D),  dq = scale d_K dS K^,  dk = scale d_Q dS^T Q^,  dv = P^T dO
+// with straight-through quantisers (the gradients of q~, k~, v~ serve as
+// those of q, k, v).
+//
+// Kernels (all contractions on tcgen05 kind::f16, bf16 operands from shared
+// memory, fp32 accumulators in TMEM; every operand K-major with the 128-byte
+// swizzle, transposed copies prepared by the pre-kernels so that no MN-major
+// operand is needed):
+//   fq_rows_kernel / fq_tokens_kernel  the forward's quantisers, decoded to
+//       bf16 (Q^, K^ and their transposes; V^), bit-identical codes and scales
+//   pad_transpose_kernel  dO padded to Npad rows, and dO^T
+//   lse_pad_kernel        lse padded with +inf (padded rows get P = 0)
+//   bwd_dq_kernel   one CTA per 128 query rows: sweep 1 over the key tiles
+//       forms D, sweep 2 forms dS and accumulates dQ += dS K^ in TMEM
+//   bwd_dkdv_kernel one CTA per 128 keys: over the query tiles of every query
+//       head of its key/value head, dV += P^T dO and dK += dS^T Q^ in TMEM
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "attn_fwd.cuh"  // the bounded-wait limit and the device error word
+#include "ptx.cuh"
+#include "quantize.cuh"
+
+namespace fp4 {
+
+constexpr int kBwdThreads = 256;  // warp 0 loads, warp 1 issues MMAs, warps 4-7 compute
+constexpr int kBwdQ = 128;        // dq kernel: query rows per CTA
+constexpr int kBwdKt = 64;        // dq kernel: keys per tile
+constexpr int kBwdK = 128;        // dk/dv kernel: keys per CTA
+constexpr int kBwdQt = 64;        // dk/dv kernel: queries per tile
+
+// Instruction descriptor of kind::f16 with bf16 A and B (both K-major), fp32 D.
+__host__ __device__ constexpr uint32_t idesc_bf16(uint32_t M, uint32_t N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 operands, K = 16 per instruction.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// K-major bf16 operand with the 128-byte swizzle: `rows` rows, K split in
+// 64-element atoms stored one after another (rows x 128 bytes each). The
+// descriptor of K step s (16 elements) starts 32 bytes further inside an atom.
+__device__ __forceinline__ uint64_t kmaj_desc(uint32_t base, int rows, int s) {
+  return smem_desc(base + (s >> 2) * rows * 128 + (s & 3) * 32, 16, 1024, 2);
+}
+
+// Decoded E2M1 magnitude times the block scale: code c (sign bit 3), scale byte e.
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+  const uint32_t m = c & 7u;
+  const float mag = m < 4 ? 0.5f * (float)m : (m == 4 ? 2.0f : (m == 5 ? 3.0f : (m == 6 ? 4.0f : 6.0f)));
+  return (c & 8u) ? -mag : mag;
+}
+
+// 16 decoded values of one block from its codes (lo: elements 0..7, hi: 8..15).
+__device__ __forceinline__ void decode_block16(uint32_t lo, uint32_t hi, uint32_t e, float* out) {
+  const float de = e4m3_to_f32(e);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    out[i] = e2m1_value((lo >> (4 * i)) & 15u) * de;
+    out[8 + i] = e2m1_value((hi >> (4 * i)) & 15u) * de;
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ---------------------------------------------------------- pre-kernels ----
+// Q or K [G][N][D] -> Q^ [G][Npad][D] and Q^T [G][D][Npad] (bf16, decoded
+// NVFP4 with blocks of 16 along D, the forward's quantiser). One CTA per
+// (group, 128-row tile); thread = row.
+template <int D>
+__global__ void __launch_bounds__(128) fq_rows_kernel(const __nv_bfloat16* __restrict__ x, int N,
+                                                      int Npad, const float* __restrict__ amax,
+                                                      __nv_bfloat16* __restrict__ xh,
+                                                      __nv_bfloat16* __restrict__ xt) {
+  __shared__ __align__(16) uint16_t tile[128 * (D + 8)];  // +8: no bank conflicts on the transpose
+  constexpr int LD = D + 8;
+  const int ntile = Npad >> 7;
+  const int64_t g = blockIdx.x / ntile;
+  const int t = blockIdx.x % ntile;
+  const float s_enc = tensor_senc(*amax);
+  const int r = threadIdx.x, n = t * 128 + r;
+  __nv_bfloat16* dst = xh + (g * Npad + n) * D;
+#pragma unroll 1
+  for (int kb = 0; kb < D / 16; ++kb) {
+    float xv[16];
+    if (n < N) {
+      const __nv_bfloat16* src = x + ((g * N + n) * D + kb * 16);
+      bf16x8_to_f32(ld_nc_v4(src), xv);
+      bf16x8_to_f32(ld_nc_v4(src + 8), xv + 8);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) xv[i] = 0.0f;
+    }
+    uint32_t lo, hi;
+    const uint32_t e = quant_block16(xv, s_enc, lo, hi);
+    float yv[16];
+    decode_block16(lo, hi, e, yv);
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = pack_bf16(yv[2 * i], yv[2 * i + 1]);
+    uint4* d4 = reinterpret_cast<uint4*>(dst + kb * 16);
+    d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    uint32_t* s32 = reinterpret_cast<uint32_t*>(&tile[r * LD + kb * 16]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s32[i] = w[i];
+  }
+  __syncthreads();
+  // transpose: one channel per thread, 128 consecutive rows written as 256 bytes
+  for (int d = threadIdx.x; d < D; d += 128) {
+    uint32_t w[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i)
+      w[i] = (uint32_t)tile[(2 * i) * LD + d] | ((uint32_t)tile[(2 * i + 1) * LD + d] << 16);
+    uint4* d4 = reinterpret_cast<uint4*>(xt + (g * D + d) * (int64_t)Npad + t * 128);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) d4[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+  }
+}
+
+// V [G][N][D] -> V^ [G][Npad][D] (bf16, decoded NVFP4 with blocks of 16 tokens
+// per channel, the forward's quantiser). One CTA per (group, 128-token tile);
+// thread = channel.
+template <int D>
+__global__ void __launch_bounds__(128) fq_tokens_kernel(const __nv_bfloat16* __restrict__ v, int N,
+                                                        int Npad, const float* __restrict__ amax,
+                                                        __nv_bfloat16* __restrict__ vh) {
+  __shared__ __align__(16) uint16_t tile[128 * D];
+  const int ntile = Npad >> 7;
+  const int64_t g = blockIdx.x / ntile;
+  const int t = blockIdx.x % ntile;
+  const float s_enc = tensor_senc(*amax);
+  constexpr int VEC = D / 8;
+  for (int idx = threadIdx.x; idx < 128 * VEC; idx += blockDim.x) {
+    const int tok = idx / VEC, c = idx % VEC;
+    const int n = t * 128 + tok;
+    uint4 w = make_uint4(0, 0, 0, 0);
+    if (n < N) w = ld_nc_v4(v + ((g * N + n) * D + c * 8));
+    *reinterpret_cast<uint4*>(&tile[tok * D + c * 8]) = w;
+  }
+  __syncthreads();
+  const int d = threadIdx.x;
+  if (d < D) {
+#pragma unroll 1
+    for (int b = 0; b < 8; ++b) {
+      float xv[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        xv[i] = __uint_as_float((uint32_t)tile[(b * 16 + i) * D + d] << 16);
+      uint32_t lo, hi;
+      const uint32_t e = quant_block16(xv, s_enc, lo, hi);
+      float yv[16];
+      decode_block16(lo, hi, e, yv);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        __nv_bfloat16 h = __float2bfloat16_rn(yv[i]);
+        tile[(b * 16 + i) * D + d] = *reinterpret_cast<uint16_t*>(&h);
+      }
+    }
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < 128 * VEC; idx += blockDim.x) {
+    const int tok = idx / VEC, c = idx % VEC;
+    *reinterpret_cast<uint4*>(vh + ((g * Npad + t * 128 + tok) * D + c * 8)) =
+        *reinterpret_cast<const uint4*>(&tile[tok * D + c * 8]);
+  }
+}
+
+// dO [G][N][D] -> dO [G][Npad][D] (rows >= N zero) and dO^T [G][D][Npad].
+template <int D>
+__global__ void __launch_bounds__(128) pad_transpose_kernel(const __nv_bfloat16* __restrict__ x,
+                                                            int N, int Npad,
+                                                            __nv_bfloat16* __restrict__ xp,
+                                                            __nv_bfloat16* __restrict__ xt) {
+  __shared__ __align__(16) uint16_t tile[128 * (D + 8)];
+  constexpr int LD = D + 8, VEC = D / 8;
+  const int ntile = Npad >> 7;
+  const int64_t g = blockIdx.x / ntile;
+  const int t = blockIdx.x % ntile;
+  for (int idx = threadIdx.x; idx < 128 * VEC; idx += blockDim.x) {
+    const int tok = idx / VEC, c = idx % VEC;
+    const int n = t * 128 + tok;
+    uint4 w = make_uint4(0, 0, 0, 0);
+    if (n < N) w = ld_nc_v4(x + ((g * N + n) * D + c * 8));
+    *reinterpret_cast<uint4*>(xp + ((g * Npad + n) * D + c * 8)) = w;
+    uint32_t* s32 = reinterpret_cast<uint32_t*>(&tile[tok * LD + c * 8]);
+    s32[0] = w.x;
+    s32[1] = w.y;
+    s32[2] = w.z;
+    s32[3] = w.w;
+  }
+  __syncthreads();
+  for (int d = threadIdx.x; d < D; d += 128) {
+    uint32_t w[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i)
+      w[i] = (uint32_t)tile[(2 * i) * LD + d] | ((uint32_t)tile[(2 * i + 1) * LD + d] << 16);
+    uint4* d4 = reinterpret_cast<uint4*>(xt + (g * D + d) * (int64_t)Npad + t * 128);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) d4[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+  }
+}
+
+// lse [G][N] -> [G][Npad], +inf beyond N.
+__global__ void lse_pad_kernel(const float* __restrict__ lse, int64_t G, int N, int Npad,
+                               float* __restrict__ out) {
+  const int64_t total = G * Npad;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t g = i / Npad;
+    const int n = (int)(i % Npad);
+    out[i] = n < N ? lse[g * N + n] : INFINITY;
+  }
+}
+
+struct BwdParams {
+  const float* amax;   // [3]: Q, K, V maxima (the forward's tensor scales)
+  const float* lse;    // [B*H][Npad], +inf on padded rows
+  float* Dvec;         // [B*H][Npad]: D, written by the dq kernel
+  __nv_bfloat16* dq;   // [B][H][N][D]
+  __nv_bfloat16* dk;   // [B][Hkv][N][D]
+  __nv_bfloat16* dv;
+  int H, Hkv, N, Npad;
+  float softmax_scale;
+};
+
+struct BwdScales {
+  float c, dv, sdq, sdk;  // score multiplier, d_V, scale d_K (for dq), scale d_Q (for dk)
+};
+
+__device__ __forceinline__ BwdScales bwd_scales(const BwdParams& p) {
+  const float dq = __fdiv_rn(1.0f, tensor_senc(p.amax[0]));
+  const float dk = __fdiv_rn(1.0f, tensor_senc(p.amax[1]));
+  const float dv = __fdiv_rn(1.0f, tensor_senc(p.amax[2]));
+  BwdScales s;
+  s.c = __fmul_rn(__fmul_rn(__fmul_rn(dq, dk), p.softmax_scale), kLog2e);
+  s.dv = dv;
+  s.sdq = __fmul_rn(p.softmax_scale, dk);
+  s.sdk = __fmul_rn(p.softmax_scale, dq);
+  return s;
+}
+
+// Bounded wait (the forward's rule: a device error word and a time limit).
+__device__ __forceinline__ bool bwd_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*reinterpret_cast<volatile unsigned*>(&g_fp4_err) != 0u) return false;
+    if (globaltimer_ns() - t0 > kTimeoutNs) {
+      atomicOr(&g_fp4_err, kDevErrTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+// ------------------------------------------------------------- dq kernel ----
+template <int D>
+struct BwdDqSmem {
+  static constexpr int kQ = kBwdQ * D * 2;    // Q^ tile, bf16
+  static constexpr int kK = kBwdKt * D * 2;   // K^ tile
+  static constexpr int kKT = D * kBwdKt * 2;  // K^T tile (D rows x 64 keys)
+  static constexpr int kStage = 2 * kK + kKT; // K^, V^, K^T
+  static constexpr int oQ = 0;
+  static constexpr int oDO = oQ + kQ;
+  static constexpr int oStage = oDO + kQ;
+  static constexpr int oDS = oStage + 2 * kStage;  // dS tile: 128 rows x 64 keys, bf16
+  static constexpr int oBar = oDS + kBwdQ * kBwdKt * 2;
+  static constexpr int oTmem = oBar + 256;
+  static constexpr int kBytes = oTmem + 16 + 1024;
+};
+
+enum : int {
+  kDqBarQ = 0,
+  kDqBarFull = 1,     // [2]
+  kDqBarEmpty = 3,    // [2]
+  kDqBarSFull = 5,    // [2]
+  kDqBarSEmpty = 7,   // [2]
+  kDqBarDsFull = 9,
+  kDqBarDsEmpty = 10,
+  kDqBarDone = 11,
+  kDqBars = 12
+};
+
+// One CTA per (128-query tile, head, batch). TMEM: S[b] at 128 b, dP[b] at
+// 128 b + 64 (64 columns each, b = tile parity), dQ at 256 (D columns).
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const __grid_constant__ CUtensorMap tmKT, const BwdParams p) {
+  using L = BwdDqSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(sm);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int gq = b * p.H + h;
+  const int gk = b * p.Hkv + h / (p.H / p.Hkv);
+  const int nk_all = (p.N + kBwdKt - 1) / kBwdKt;
+  const int nkt = CAUSAL ? min(nk_all, (qt * kBwdQ + kBwdQ - 1) / kBwdKt + 1) : nk_all;
+  const int T = 2 * nkt;  // sweep 1 (D), then sweep 2 (dS, dQ)
+  auto bar = [&](int i) -> uint32_t { return sb + L::oBar + 8 * i; };
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kDqBarQ), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kDqBarFull + s), 1);
+      mbar_init(bar(kDqBarEmpty + s), 1);
+      mbar_init(bar(kDqBarSFull + s), 1);
+      mbar_init(bar(kDqBarSEmpty + s), 4);
+    }
+    mbar_init(bar(kDqBarDsFull), 4);
+    mbar_init(bar(kDqBarDsEmpty), 1);
+    mbar_init(bar(kDqBarDone), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sb + L::oTmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + L::oTmem);
+  constexpr int NA = D / 64;  // 64-element atoms along D
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool ok = true;
+      int issued = 0;
+      mbar_arrive_expect_tx(bar(kDqBarQ), 2 * L::kQ);
+      for (int a = 0; a < NA; ++a) {
+        tma_load_2d(sb + L::oQ + a * kBwdQ * 128, &tmQ, a * 64, gq * p.Npad + qt * kBwdQ, bar(kDqBarQ));
+        tma_load_2d(sb + L::oDO + a * kBwdQ * 128, &tmDO, a * 64, gq * p.Npad + qt * kBwdQ,
+                    bar(kDqBarQ));
+      }
+      for (int t = 0; t < T && ok; ++t) {
+        const int st = t & 1, j = t % nkt;
+        const bool sw2 = t >= nkt;
+        if (t >= 2 && !(ok = bwd_wait(bar(kDqBarEmpty + st), ((t >> 1) - 1) & 1))) break;
+        const uint32_t base = sb + L::oStage + st * L::kStage;
+        mbar_arrive_expect_tx(bar(kDqBarFull + st), 2 * L::kK + (sw2 ? L::kKT : 0));
+        for (int a = 0; a < NA; ++a) {
+          tma_load_2d(base + a * kBwdKt * 128, &tmK, a * 64, gk * p.Npad + j * kBwdKt,
+                      bar(kDqBarFull + st));
+          tma_load_2d(base + L::kK + a * kBwdKt * 128, &tmV, a * 64, gk * p.Npad + j * kBwdKt,
+                      bar(kDqBarFull + st));
+        }
+        if (sw2)
+          tma_load_2d(base + 2 * L::kK, &tmKT, j * kBwdKt, gk * D, bar(kDqBarFull + st));
+        issued = t + 1;
+      }
+      // copies still in flight after a failed wait land before the CTA exits
+      drain_wait(bar(kDqBarQ), 0);
+      for (int t = max(0, issued - 2); t < issued; ++t) drain_wait(bar(kDqBarFull + (t & 1)), (t >> 1) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = bwd_wait(bar(kDqBarQ), 0);
+      const uint32_t idS = idesc_bf16(kBwdQ, kBwdKt), idQ = idesc_bf16(kBwdQ, D);
+      auto issue_dq = [&](int t) {  // dQ += dS K^ of tile t (sweep 2)
+        const int st = t & 1, t2 = t - nkt;
+        ok = ok && bwd_wait(bar(kDqBarDsFull), t2 & 1);
+        if (!ok) return;
+        tc_fence_after();
+        const uint32_t kt = sb + L::oStage + st * L::kStage + 2 * L::kK;
+#pragma unroll
+        for (int s = 0; s < kBwdKt / 16; ++s)
+          mma_bf16(tmem + 256, kmaj_desc(sb + L::oDS, kBwdQ, s), kmaj_desc(kt, D, s), idQ,
+                   (t2 > 0 || s > 0) ? 1u : 0u);
+        tc_commit(bar(kDqBarEmpty + st));
+        tc_commit(bar(kDqBarDsEmpty));
+      };
+      for (int t = 0; t < T && ok; ++t) {
+        const int st = t & 1, buf = t & 1;
+        if (!(ok = bwd_wait(bar(kDqBarFull + st), (t >> 1) & 1))) break;
+        if (t >= 2 && !(ok = bwd_wait(bar(kDqBarSEmpty + buf), ((t >> 1) - 1) & 1))) break;
+        tc_fence_after();
+        const uint32_t base = sb + L::oStage + st * L::kStage;
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s) {
+          mma_bf16(tmem + buf * 128, kmaj_desc(sb + L::oQ, kBwdQ, s), kmaj_desc(base, kBwdKt, s),
+                   idS, s > 0 ? 1u : 0u);
+          mma_bf16(tmem + buf * 128 + 64, kmaj_desc(sb + L::oDO, kBwdQ, s),
+                   kmaj_desc(base + L::kK, kBwdKt, s), idS, s > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(kDqBarSFull + buf));
+        if (t < nkt) tc_commit(bar(kDqBarEmpty + st));
+        if (t > nkt) issue_dq(t - 1);  // the previous tile's dQ, one step behind
+      }
+      if (ok && T > nkt) issue_dq(T - 1);
+      tc_commit(bar(kDqBarDone));
+      drain_wait(bar(kDqBarDone), 0);  // every MMA complete before TMEM is freed
+    }
+  } else if (warp >= 4) {
+    const int quad = warp & 3, row = quad * 32 + lane, qrow = qt * kBwdQ + row;
+    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+    const BwdScales sc = bwd_scales(p);
+    const float lse = p.lse[(int64_t)gq * p.Npad + qrow];
+    float Dsum = 0.0f;
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      const int buf = t & 1, j = t % nkt;
+      float s[64], dp[64];
+      ok = ok && __all_sync(0xFFFFFFFFu, bwd_wait(bar(kDqBarSFull + buf), (t >> 1) & 1));
+      if (ok) {
+        tc_fence_after();
+        tmem_ld32(tl + buf * 128, s);
+        tmem_ld32(tl + buf * 128 + 32, s + 32);
+        tmem_ld32(tl + buf * 128 + 64, dp);
+        tmem_ld32(tl + buf * 128 + 96, dp + 32);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kDqBarSEmpty + buf));
+      if (!ok) break;
+      const int key0 = j * kBwdKt;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const int key = key0 + c;
+        const bool live = key < p.N && (!CAUSAL || key <= qrow);
+        s[c] = live ? ex2_approx(fmaf(s[c], sc.c, -lse)) : 0.0f;  // P
+      }
+      if (t < nkt) {
+        float acc = 0.0f;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) acc = fmaf(s[c], dp[c], acc);
+        Dsum = fmaf(acc, sc.dv, Dsum);
+        if (t == nkt - 1) p.Dvec[(int64_t)gq * p.Npad + qrow] = Dsum;
+        continue;
+      }
+      // dS = P (d_V dP - D) -> bf16, the row's 128 bytes (128-byte swizzle)
+      uint32_t w[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        w[c] = pack_bf16(s[2 * c] * fmaf(dp[2 * c], sc.dv, -Dsum),
+                         s[2 * c + 1] * fmaf(dp[2 * c + 1], sc.dv, -Dsum));
+      const int t2 = t - nkt;
+      if (t2 > 0) ok = __all_sync(0xFFFFFFFFu, bwd_wait(bar(kDqBarDsEmpty), (t2 - 1) & 1));
+      if (!ok) break;
+      uint8_t* dsr = sm + L::oDS + row * 128;
+#pragma unroll
+      for (int k2 = 0; k2 < 8; ++k2)
+        *reinterpret_cast<uint4*>(dsr + ((k2 ^ (row & 7)) * 16)) =
+            make_uint4(w[4 * k2], w[4 * k2 + 1], w[4 * k2 + 2], w[4 * k2 + 3]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kDqBarDsFull));
+    }
+    ok = ok && __all_sync(0xFFFFFFFFu, bwd_wait(bar(kDqBarDone), 0));
+    if (ok) {  // warp-uniform: tcgen05.ld is a whole-warp instruction; only the stores are per row
+      tc_fence_after();
+      __nv_bfloat16* dst = p.dq + ((int64_t)gq * p.N + qrow) * D;
+#pragma unroll
+      for (int cc = 0; cc < D; cc += 32) {
+        float o[32];
+        __syncwarp();
+        tmem_ld32(tl + 256 + cc, o);
+        tmem_wait_ld();
+        if (qrow < p.N) {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[i] = pack_bf16(o[2 * i] * sc.sdq, o[2 * i + 1] * sc.sdq);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + cc);
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4)
+            d4[k4] = make_uint4(w[4 * k4], w[4 * k4 + 1], w[4 * k4 + 2], w[4 * k4 + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ----------------------------------------------------------- dk/dv kernel ----
+template <int D>
+struct BwdDkvSmem {
+  static constexpr int kK = kBwdK * D * 2;     // K^ or V^ tile, bf16
+  static constexpr int kQ = kBwdQt * D * 2;    // Q^ or dO tile
+  static constexpr int kQT = D * kBwdQt * 2;   // Q^T or dO^T tile
+  static constexpr int kStage = 2 * kQ + 2 * kQT;  // Q^, dO, Q^T, dO^T
+  static constexpr int oK = 0;
+  static constexpr int oV = oK + kK;
+  static constexpr int oStage = oV + kK;
+  static constexpr int oP = oStage + 2 * kStage;      // P^T: 128 keys x 64 queries, bf16
+  static constexpr int oDS = oP + kBwdK * kBwdQt * 2; // dS^T
+  static constexpr int oLse = oDS + kBwdK * kBwdQt * 2;  // [2 stages]: lse[64], D[64]
+  static constexpr int oBar = oLse + 2 * 512;
+  static constexpr int oTmem = oBar + 256;
+  static constexpr int kBytes = oTmem + 16 + 1024;
+};
+
+enum : int {
+  kKvBarKV = 0,
+  kKvBarFull = 1,    // [2]
+  kKvBarEmpty = 3,   // [2]
+  kKvBarSFull = 5,   // [2]
+  kKvBarSEmpty = 7,  // [2]
+  kKvBarPFull = 9,
+  kKvBarPEmpty = 10,
+  kKvBarDone = 11,
+};
+
+// One CTA per (128-key tile, key/value head, batch); tiles of 64 queries of
+// every query head of the group. TMEM: S^T[b] at 128 b, dP^T[b] at 128 b + 64,
+// dV at 256, dK at 256 + D.
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                    const __grid_constant__ CUtensorMap tmQT,
+                    const __grid_constant__ CUtensorMap tmDOT, const BwdParams p) {
+  using L = BwdDkvSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(sm);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  const int gk = b * p.Hkv + hk;
+  const int G = p.H / p.Hkv;
+  const int nq_all = (p.N + kBwdQt - 1) / kBwdQt;
+  const int i0 = CAUSAL ? (kt * kBwdK) / kBwdQt : 0;  // first query tile that sees these keys
+  const int nqt = max(0, nq_all - i0);
+  const int T = G * nqt;
+  auto bar = [&](int i) -> uint32_t { return sb + L::oBar + 8 * i; };
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kKvBarKV), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kKvBarFull + s), 1);
+      mbar_init(bar(kKvBarEmpty + s), 1);
+      mbar_init(bar(kKvBarSFull + s), 1);
+      mbar_init(bar(kKvBarSEmpty + s), 4);
+    }
+    mbar_init(bar(kKvBarPFull), 4);
+    mbar_init(bar(kKvBarPEmpty), 1);
+    mbar_init(bar(kKvBarDone), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sb + L::oTmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + L::oTmem);
+  constexpr int NA = D / 64;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      bool ok = true;
+      int issued = 0;
+      mbar_arrive_expect_tx(bar(kKvBarKV), 2 * L::kK);
+      for (int a = 0; a < NA; ++a) {
+        tma_load_2d(sb + L::oK + a * kBwdK * 128, &tmK, a * 64, gk * p.Npad + kt * kBwdK,
+                    bar(kKvBarKV));
+        tma_load_2d(sb + L::oV + a * kBwdK * 128, &tmV, a * 64, gk * p.Npad + kt * kBwdK,
+                    bar(kKvBarKV));
+      }
+      for (int t = 0; t < T && ok; ++t) {
+        const int st = t & 1;
+        const int gq = b * p.H + hk * G + t / nqt, i = i0 + t % nqt;
+        if (t >= 2 && !(ok = bwd_wait(bar(kKvBarEmpty + st), ((t >> 1) - 1) & 1))) break;
+        const uint32_t base = sb + L::oStage + st * L::kStage;
+        mbar_arrive_expect_tx(bar(kKvBarFull + st), L::kStage + 512);
+        for (int a = 0; a < NA; ++a) {
+          tma_load_2d(base + a * kBwdQt * 128, &tmQ, a * 64, gq * p.Npad + i * kBwdQt,
+                      bar(kKvBarFull + st));
+          tma_load_2d(base + L::kQ + a * kBwdQt * 128, &tmDO, a * 64, gq * p.Npad + i * kBwdQt,
+                      bar(kKvBarFull + st));
+        }
+        tma_load_2d(base + 2 * L::kQ, &tmQT, i * kBwdQt, gq * D, bar(kKvBarFull + st));
+        tma_load_2d(base + 2 * L::kQ + L::kQT, &tmDOT, i * kBwdQt, gq * D, bar(kKvBarFull + st));
+        bulk_load(sb + L::oLse + st * 512, p.lse + (int64_t)gq * p.Npad + i * kBwdQt, 256,
+                  bar(kKvBarFull + st));
+        bulk_load(sb + L::oLse + st * 512 + 256, p.Dvec + (int64_t)gq * p.Npad + i * kBwdQt, 256,
+                  bar(kKvBarFull + st));
+        issued = t + 1;
+      }
+      drain_wait(bar(kKvBarKV), 0);
+      for (int t = max(0, issued - 2); t < issued; ++t) drain_wait(bar(kKvBarFull + (t & 1)), (t >> 1) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = bwd_wait(bar(kKvBarKV), 0);
+      const uint32_t idS = idesc_bf16(kBwdK, kBwdQt), idO = idesc_bf16(kBwdK, D);
+      auto issue_kv = [&](int t) {  // dV += P^T dO, dK += dS^T Q^ of tile t
+        const int st = t & 1;
+        ok = ok && bwd_wait(bar(kKvBarPFull), t & 1);
+        if (!ok) return;
+        tc_fence_after();
+        const uint32_t base = sb + L::oStage + st * L::kStage;
+#pragma unroll
+        for (int s = 0; s < kBwdQt / 16; ++s) {
+          const uint32_t acc = (t > 0 || s > 0) ? 1u : 0u;
+          mma_bf16(tmem + 256, kmaj_desc(sb + L::oP, kBwdK, s),
+                   kmaj_desc(base + 2 * L::kQ + L::kQT, D, s), idO, acc);
+          mma_bf16(tmem + 256 + D, kmaj_desc(sb + L::oDS, kBwdK, s),
+                   kmaj_desc(base + 2 * L::kQ, D, s), idO, acc);
+        }
+        tc_commit(bar(kKvBarEmpty + st));
+        tc_commit(bar(kKvBarPEmpty));
+      };
+      for (int t = 0; t < T && ok; ++t) {
+        const int st = t & 1, buf = t & 1;
+        if (!(ok = bwd_wait(bar(kKvBarFull + st), (t >> 1) & 1))) break;
+        if (t >= 2 && !(ok = bwd_wait(bar(kKvBarSEmpty + buf), ((t >> 1) - 1) & 1))) break;
+        tc_fence_after();
+        const uint32_t base = sb + L::oStage + st * L::kStage;
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s) {
+          mma_bf16(tmem + buf * 128, kmaj_desc(sb + L::oK, kBwdK, s), kmaj_desc(base, kBwdQt, s),
+                   idS, s > 0 ? 1u : 0u);
+          mma_bf16(tmem + buf * 128 + 64, kmaj_desc(sb + L::oV, kBwdK, s),
+                   kmaj_desc(base + L::kQ, kBwdQt, s), idS, s > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(kKvBarSFull + buf));
+        if (t > 0) issue_kv(t - 1);
+      }
+      if (ok && T > 0) issue_kv(T - 1);
+      tc_commit(bar(kKvBarDone));
+      drain_wait(bar(kKvBarDone), 0);
+    }
+  } else if (warp >= 4) {
+    const int quad = warp & 3, row = quad * 32 + lane, key = kt * kBwdK + row;
+    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+    const BwdScales sc = bwd_scales(p);
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      const int st = t & 1, buf = t & 1, i = i0 + t % nqt;
+      float s[64], dp[64];
+      ok = ok && __all_sync(0xFFFFFFFFu, bwd_wait(bar(kKvBarSFull + buf), (t >> 1) & 1));
+      if (ok) {
+        tc_fence_after();
+        tmem_ld32(tl + buf * 128, s);
+        tmem_ld32(tl + buf * 128 + 32, s + 32);
+        tmem_ld32(tl + buf * 128 + 64, dp);
+        tmem_ld32(tl + buf * 128 + 96, dp + 32);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kKvBarSEmpty + buf));
+      if (!ok) break;
+      // the stage's lse and D: its full barrier has completed (S^T was issued
+      // after it); the wait makes the bulk copies' data visible to this thread
+      ok = __all_sync(0xFFFFFFFFu, bwd_wait(bar(kKvBarFull + st), (t >> 1) & 1));
+      if (!ok) break;
+      const float* lq = reinterpret_cast<const float*>(sm + L::oLse + st * 512);
+      const float* dq = lq + 64;
+      uint32_t wp[32], wd[32];
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        float pv[2], dv2[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int q = i * kBwdQt + c + u;
+          const bool live = key < p.N && q < p.N && (!CAUSAL || key <= q);
+          pv[u] = live ? ex2_approx(fmaf(s[c + u], sc.c, -lq[c + u])) : 0.0f;
+          dv2[u] = pv[u] * fmaf(dp[c + u], sc.dv, -dq[c + u]);
+        }
+        wp[c >> 1] = pack_bf16(pv[0], pv[1]);
+        wd[c >> 1] = pack_bf16(dv2[0], dv2[1]);
+      }
+      if (t > 0) ok = __all_sync(0xFFFFFFFFu, bwd_wait(bar(kKvBarPEmpty), (t - 1) & 1));
+      if (!ok) break;
+      uint8_t* pr = sm + L::oP + row * 128;
+      uint8_t* dr = sm + L::oDS + row * 128;
+#pragma unroll
+      for (int k2 = 0; k2 < 8; ++k2) {
+        const int off = (k2 ^ (row & 7)) * 16;
+        *reinterpret_cast<uint4*>(pr + off) =
+            make_uint4(wp[4 * k2], wp[4 * k2 + 1], wp[4 * k2 + 2], wp[4 * k2 + 3]);
+        *reinterpret_cast<uint4*>(dr + off) =
+            make_uint4(wd[4 * k2], wd[4 * k2 + 1], wd[4 * k2 + 2], wd[4 * k2 + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kKvBarPFull));
+    }
+    ok = ok && __all_sync(0xFFFFFFFFu, bwd_wait(bar(kKvBarDone), 0));
+    if (ok) {  // warp-uniform: tcgen05.ld is a whole-warp instruction; only the stores are per row
+      tc_fence_after();
+      __nv_bfloat16* dvp = p.dv + ((int64_t)gk * p.N + key) * D;
+      __nv_bfloat16* dkp = p.dk + ((int64_t)gk * p.N + key) * D;
+#pragma unroll
+      for (int cc = 0; cc < D; cc += 32) {
+        float o[32], o2[32];
+        if (T > 0) {
+          __syncwarp();
+          tmem_ld32(tl + 256 + cc, o);
+          tmem_ld32(tl + 256 + D + cc, o2);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int u = 0; u < 32; ++u) o[u] = o2[u] = 0.0f;
+        }
+        if (key < p.N) {
+          uint32_t wv[16], wk[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            wv[u] = pack_bf16(o[2 * u], o[2 * u + 1]);
+            wk[u] = pack_bf16(o2[2 * u] * sc.sdk, o2[2 * u + 1] * sc.sdk);
+          }
+          uint4* v4 = reinterpret_cast<uint4*>(dvp + cc);
+          uint4* k4 = reinterpret_cast<uint4*>(dkp + cc);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            v4[u] = make_uint4(wv[4 * u], wv[4 * u + 1], wv[4 * u + 2], wv[4 * u + 3]);
+            k4[u] = make_uint4(wk[4 * u], wk[4 * u + 1], wk[4 * u + 2], wk[4 * u + 3]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fp4

@@ -102,6 +102,7 @@ struct AttnParams {
   const float* amax_v;
   __nv_bfloat16* out;  // [B][H][N][D]
   const float* bias;   // [B*H][Npad]: per-key score correction (smoothed Q), or unused
+  float* lse;          // [B*H][N]: log2 sum_j 2^(x_ij) per row for the backward, or NULL
   int H, Hkv, N, Npad, ntq;
   float softmax_scale;
 };
@@ -609,7 +610,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_wait_ld();
         inv = __fdiv_rn(dv, lq[0]);
       } else {
-        inv = __fdiv_rn(fpv, lval[row] + lval[kBM + row]);
+        const float lsum = lval[row] + lval[kBM + row];
+        inv = __fdiv_rn(fpv, lsum);
+        if (PG == kPgExp && p.lse && stream == 0 && qrow < p.N)
+          p.lse[(int64_t)gq * p.N + qrow] = m_fin + log2f(lsum);
       }
       constexpr int DH = D / 2;             // each stream writes half the channels
       __nv_bfloat16* dst = p.out + ((int64_t)gq * p.N + qrow) * D + stream * DH;

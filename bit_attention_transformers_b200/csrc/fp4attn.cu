@@ -14,6 +14,7 @@
 #include <string>
 
 #include "../../include/fp4attn.h"
+#include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
 #include "quantize.cuh"
 
@@ -79,6 +80,21 @@ int attn_smem_bytes(int D, int pg) {
   return D == 128 ? fp4::AttnSmem<128>::kBytes : fp4::AttnSmem<64>::kBytes;
 }
 
+using BwdKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                          const CUtensorMap, const CUtensorMap, const fp4::BwdParams);
+using BwdKvKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                             const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                             const fp4::BwdParams);
+
+BwdKernel bwd_dq_kernel_for(int D, int causal) {
+  if (D == 128) return causal ? fp4::bwd_dq_kernel<128, true> : fp4::bwd_dq_kernel<128, false>;
+  return causal ? fp4::bwd_dq_kernel<64, true> : fp4::bwd_dq_kernel<64, false>;
+}
+BwdKvKernel bwd_dkdv_kernel_for(int D, int causal) {
+  if (D == 128) return causal ? fp4::bwd_dkdv_kernel<128, true> : fp4::bwd_dkdv_kernel<128, false>;
+  return causal ? fp4::bwd_dkdv_kernel<64, true> : fp4::bwd_dkdv_kernel<64, false>;
+}
+
 // sm_100 check, per-device one-time kernel attributes, SM count.
 fp4_status_t device_setup(int* dev_out, int* sms_out) {
   int dev;
@@ -99,6 +115,15 @@ fp4_status_t device_setup(int* dev_out, int* sms_out) {
           FP4_CUDA(cudaFuncSetAttribute(attn_kernel(d ? 128 : 64, causal, pg % 3, pg == 3),
                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         attn_smem_bytes(d ? 128 : 64, pg % 3)));
+    for (int d = 0; d < 2; ++d)
+      for (int causal = 0; causal < 2; ++causal) {
+        FP4_CUDA(cudaFuncSetAttribute(bwd_dq_kernel_for(d ? 128 : 64, causal),
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      d ? fp4::BwdDqSmem<128>::kBytes : fp4::BwdDqSmem<64>::kBytes));
+        FP4_CUDA(cudaFuncSetAttribute(bwd_dkdv_kernel_for(d ? 128 : 64, causal),
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      d ? fp4::BwdDkvSmem<128>::kBytes : fp4::BwdDkvSmem<64>::kBytes));
+      }
     if (!g_encode) {
       cudaDriverEntryPointQueryResult q;
       void* fn = nullptr;
@@ -125,6 +150,21 @@ fp4_status_t tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t 
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FP4_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return FP4_OK;
+}
+
+// 2D bf16 tensor map: rows x inner elements, box rows x 64 elements, 128-byte swizzle.
+fp4_status_t tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                       uint32_t box_rows) {
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FP4_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return FP4_OK;
 }
@@ -164,6 +204,36 @@ WsLayout ws_layout(int B, int H, int Hkv, int N, int D, bool fp8v = false, bool 
   w.qmean = take(smooth ? (size_t)(Gq * D * 4) : 0);
   w.kmean = take(smooth ? (size_t)(Gk * D * 4) : 0);
   w.bias = take(smooth ? (size_t)(Gq * Npad * 4) : 0);
+  w.total = off;
+  return w;
+}
+
+// Workspace of the backward: the maxima, the decoded operands (Q^, Q^T, K^,
+// K^T, V^), dO padded and transposed, lse padded, D.
+struct BwdWs {
+  size_t amax, qh, qt, kh, kt, vh, dop, dot, lse, dvec, total;
+};
+
+BwdWs bwd_ws_layout(int B, int H, int Hkv, int N, int D) {
+  BwdWs w;
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    size_t o = off;
+    off += (size_t)round_up((int64_t)n, 1024);
+    return o;
+  };
+  const int64_t Npad = round_up(N, 128), Gq = (int64_t)B * H, Gk = (int64_t)B * Hkv;
+  const size_t q2 = (size_t)(Gq * Npad * D * 2), k2 = (size_t)(Gk * Npad * D * 2);
+  w.amax = take(256);
+  w.qh = take(q2);
+  w.qt = take(q2);
+  w.kh = take(k2);
+  w.kt = take(k2);
+  w.vh = take(k2);
+  w.dop = take(q2);
+  w.dot = take(q2);
+  w.lse = take((size_t)(Gq * Npad * 4));
+  w.dvec = take((size_t)(Gq * Npad * 4));
   w.total = off;
   return w;
 }
@@ -313,7 +383,7 @@ fp4_status_t launch_attn(const uint8_t* qc, const uint8_t* qs, const float* qa, 
                          const uint8_t* ks, const float* ka, const uint8_t* vc, const uint8_t* vs,
                          const float* va, void* out, int B, int H, int Hkv, int N, int D,
                          int causal, float softmax_scale, int pg, cudaStream_t stream,
-                         const float* bias = nullptr) {
+                         const float* bias = nullptr, float* lse = nullptr) {
   const int64_t Npad = round_up(N, 128);
   const int64_t Gq = (int64_t)B * H, Gk = (int64_t)B * Hkv;
   const CUtensorMapSwizzle swQK =
@@ -342,6 +412,7 @@ fp4_status_t launch_attn(const uint8_t* qc, const uint8_t* qs, const float* qa, 
   p.Npad = (int)Npad;
   p.ntq = (int)(Npad / 128);
   p.bias = bias;
+  p.lse = lse;
   p.softmax_scale = resolve_scale(softmax_scale, D);
   dim3 grid(p.ntq, H, B);
   if (bias && pg != fp4::kPgExp)
@@ -354,7 +425,7 @@ fp4_status_t launch_attn(const uint8_t* qc, const uint8_t* qs, const float* qa, 
 
 fp4_status_t attn_fwd_any(const void* q, const void* k, const void* v, void* out, int B, int H,
                           int Hkv, int N, int D, int causal, float softmax_scale, void* stream,
-                          void* workspace, size_t workspace_bytes, int pg) {
+                          void* workspace, size_t workspace_bytes, int pg, float* lse = nullptr) {
   g_last_error.clear();
   fp4_status_t s;
   if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
@@ -385,7 +456,8 @@ fp4_status_t attn_fwd_any(const void* q, const void* k, const void* v, void* out
                      amax + 2, sms, st);
   if (s != FP4_OK) return s;
   return launch_attn(ws + w.qc, ws + w.qs, amax, ws + w.kc, ws + w.ks, amax + 1, ws + w.vc,
-                     ws + w.vs, amax + 2, out, B, H, Hkv, N, D, causal, softmax_scale, pg, st);
+                     ws + w.vs, amax + 2, out, B, H, Hkv, N, D, causal, softmax_scale, pg, st,
+                     nullptr, lse);
 }
 
 // The smoothed forward: smooth bit 0 = K, bit 1 = Q (FP4_SMOOTH_K / _Q).
@@ -450,6 +522,100 @@ fp4_status_t attn_fwd_smooth_any(const void* q, const void* k, const void* v, vo
                      (smooth & 2) ? bias : nullptr);
 }
 
+// The backward (attn_bwd.cuh): pre-kernels, then the dq kernel (D and dQ),
+// then the dk/dv kernel.
+fp4_status_t attn_bwd_any(const void* q, const void* k, const void* v, const void* dout,
+                          const float* lse, void* dq, void* dk, void* dv, int B, int H, int Hkv,
+                          int N, int D, int causal, float softmax_scale, void* stream,
+                          void* workspace, size_t workspace_bytes) {
+  g_last_error.clear();
+  fp4_status_t s;
+  if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
+  if (!q || !k || !v || !dout || !lse || !dq || !dk || !dv || !workspace)
+    return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return fail(FP4_ERR_INVALID_ARG, "pointers must be 16-byte aligned (lse 4-byte)");
+  const BwdWs w = bwd_ws_layout(B, H, Hkv, N, D);
+  if (workspace_bytes < w.total)
+    return fail(FP4_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, w.total);
+  int dev, sms;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* amax = reinterpret_cast<float*>(ws + w.amax);
+  const int64_t Npad = round_up(N, 128), Gq = (int64_t)B * H, Gk = (int64_t)B * Hkv;
+  if ((s = launch_amax(q, Gq * N * D, k, Gk * N * D, v, Gk * N * D, amax, amax + 1, amax + 2, sms,
+                       st)) != FP4_OK)
+    return s;
+  auto* qh = reinterpret_cast<__nv_bfloat16*>(ws + w.qh);
+  auto* qt = reinterpret_cast<__nv_bfloat16*>(ws + w.qt);
+  auto* kh = reinterpret_cast<__nv_bfloat16*>(ws + w.kh);
+  auto* kt = reinterpret_cast<__nv_bfloat16*>(ws + w.kt);
+  auto* vh = reinterpret_cast<__nv_bfloat16*>(ws + w.vh);
+  auto* dop = reinterpret_cast<__nv_bfloat16*>(ws + w.dop);
+  auto* dot = reinterpret_cast<__nv_bfloat16*>(ws + w.dot);
+  float* lsep = reinterpret_cast<float*>(ws + w.lse);
+  float* dvec = reinterpret_cast<float*>(ws + w.dvec);
+  const auto* qb = static_cast<const __nv_bfloat16*>(q);
+  const auto* kb = static_cast<const __nv_bfloat16*>(k);
+  const auto* vb = static_cast<const __nv_bfloat16*>(v);
+  const auto* ob = static_cast<const __nv_bfloat16*>(dout);
+  const unsigned tq = (unsigned)(Gq * (Npad / 128)), tk = (unsigned)(Gk * (Npad / 128));
+  if (D == 128) {
+    fp4::fq_rows_kernel<128><<<tq, 128, 0, st>>>(qb, N, (int)Npad, amax, qh, qt);
+    fp4::fq_rows_kernel<128><<<tk, 128, 0, st>>>(kb, N, (int)Npad, amax + 1, kh, kt);
+    fp4::fq_tokens_kernel<128><<<tk, 128, 0, st>>>(vb, N, (int)Npad, amax + 2, vh);
+    fp4::pad_transpose_kernel<128><<<tq, 128, 0, st>>>(ob, N, (int)Npad, dop, dot);
+  } else {
+    fp4::fq_rows_kernel<64><<<tq, 128, 0, st>>>(qb, N, (int)Npad, amax, qh, qt);
+    fp4::fq_rows_kernel<64><<<tk, 128, 0, st>>>(kb, N, (int)Npad, amax + 1, kh, kt);
+    fp4::fq_tokens_kernel<64><<<tk, 128, 0, st>>>(vb, N, (int)Npad, amax + 2, vh);
+    fp4::pad_transpose_kernel<64><<<tq, 128, 0, st>>>(ob, N, (int)Npad, dop, dot);
+  }
+  FP4_CUDA(cudaGetLastError());
+  fp4::lse_pad_kernel<<<(unsigned)std::min<int64_t>((Gq * Npad + 255) / 256, (int64_t)sms * 8), 256,
+                        0, st>>>(lse, Gq, N, (int)Npad, lsep);
+  FP4_CUDA(cudaGetLastError());
+  CUtensorMap mQ, mDO, mK64, mV64, mKT, mK128, mV128, mQ64, mDO64, mQT, mDOT;
+  if ((s = tmap_bf16(&mQ, qh, D, Gq * Npad, fp4::kBwdQ)) != FP4_OK) return s;
+  if ((s = tmap_bf16(&mDO, dop, D, Gq * Npad, fp4::kBwdQ)) != FP4_OK) return s;
+  if ((s = tmap_bf16(&mK64, kh, D, Gk * Npad, fp4::kBwdKt)) != FP4_OK) return s;
+  if ((s = tmap_bf16(&mV64, vh, D, Gk * Npad, fp4::kBwdKt)) != FP4_OK) return s;
+  if ((s = tmap_bf16(&mKT, kt, Npad, Gk * D, D)) != FP4_OK) return s;
+  if ((s = tmap_bf16(&mK128, kh, D, Gk * Npad, fp4::kBwdK)) != FP4_OK) return s;
+  if ((s = tmap_bf16(&mV128, vh, D, Gk * Npad, fp4::kBwdK)) != FP4_OK) return s;
+  if ((s = tmap_bf16(&mQ64, qh, D, Gq * Npad, fp4::kBwdQt)) != FP4_OK) return s;
+  if ((s = tmap_bf16(&mDO64, dop, D, Gq * Npad, fp4::kBwdQt)) != FP4_OK) return s;
+  if ((s = tmap_bf16(&mQT, qt, Npad, Gq * D, D)) != FP4_OK) return s;
+  if ((s = tmap_bf16(&mDOT, dot, Npad, Gq * D, D)) != FP4_OK) return s;
+  fp4::BwdParams p;
+  p.amax = amax;
+  p.lse = lsep;
+  p.Dvec = dvec;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.H = H;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.Npad = (int)Npad;
+  p.softmax_scale = resolve_scale(softmax_scale, D);
+  dim3 g1((unsigned)(Npad / fp4::kBwdQ), (unsigned)H, (unsigned)B);
+  bwd_dq_kernel_for(D, causal)<<<g1, fp4::kBwdThreads,
+                                 D == 128 ? fp4::BwdDqSmem<128>::kBytes : fp4::BwdDqSmem<64>::kBytes,
+                                 st>>>(mQ, mDO, mK64, mV64, mKT, p);
+  FP4_CUDA(cudaGetLastError());
+  dim3 g2((unsigned)(Npad / fp4::kBwdK), (unsigned)Hkv, (unsigned)B);
+  bwd_dkdv_kernel_for(D, causal)<<<g2, fp4::kBwdThreads,
+                                   D == 128 ? fp4::BwdDkvSmem<128>::kBytes
+                                            : fp4::BwdDkvSmem<64>::kBytes,
+                                   st>>>(mK128, mV128, mQ64, mDO64, mQT, mDOT, p);
+  FP4_CUDA(cudaGetLastError());
+  return FP4_OK;
+}
+
 fp4_status_t attn_fwd_quantized_any(const fp4_tensor_t* q, const fp4_tensor_t* k,
                                     const fp4_tensor_t* v, void* out, int B, int H, int Hkv,
                                     int N, int D, int causal, float softmax_scale, void* stream,
@@ -494,6 +660,31 @@ size_t fp4_scales_bytes(int G, int N, int D, fp4_axis_t axis) {
 size_t fp4_attn_workspace_bytes(int B, int H, int Hkv, int N, int D) {
   if (check_shape(B, H, Hkv, N, D) != FP4_OK) return 0;
   return ws_layout(B, H, Hkv, N, D).total;
+}
+
+size_t fp4_attn_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D) {
+  if (check_shape(B, H, Hkv, N, D) != FP4_OK) return 0;
+  return bwd_ws_layout(B, H, Hkv, N, D).total;
+}
+
+fp4_status_t fp4_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
+                          const float* lse, void* dq, void* dk, void* dv, int B, int H, int Hkv,
+                          int N, int D, int causal, float softmax_scale, void* stream,
+                          void* workspace, size_t workspace_bytes) {
+  return attn_bwd_any(q, k, v, dout, lse, dq, dk, dv, B, H, Hkv, N, D, causal, softmax_scale,
+                      stream, workspace, workspace_bytes);
+}
+
+fp4_status_t fp4_attn_fwd_lse(const void* q, const void* k, const void* v, void* out, float* lse,
+                              int B, int H, int Hkv, int N, int D, int causal,
+                              float softmax_scale, void* stream, void* workspace,
+                              size_t workspace_bytes) {
+  if (!lse || (reinterpret_cast<uintptr_t>(lse) & 3u)) {
+    g_last_error.clear();
+    return fail(FP4_ERR_INVALID_ARG, "lse must be a 4-byte aligned device pointer");
+  }
+  return attn_fwd_any(q, k, v, out, B, H, Hkv, N, D, causal, softmax_scale, stream, workspace,
+                      workspace_bytes, 0, lse);
 }
 
 size_t fp4_attn_workspace_bytes_smooth(int B, int H, int Hkv, int N, int D) {

@@ -285,6 +285,42 @@ fp4_status_t fp4_attn_fwd_quantized_bias(const fp4_tensor_t* q, const fp4_tensor
                                          int B, int H, int Hkv, int N, int D, int causal,
                                          float softmax_scale, void* stream);
 
+/*
+ * Training support: the forward of fp4_attn_fwd that also writes, per query
+ * row, lse [B*H][N] fp32 = log2 sum_j 2^(x_ij) with x_ij = S_ij * c (the
+ * scores in log2 units, the quantity the backward needs to re-form P). Same
+ * arguments as fp4_attn_fwd plus lse (device memory, 4-byte aligned).
+ */
+fp4_status_t fp4_attn_fwd_lse(const void* q, const void* k, const void* v, void* out, float* lse,
+                              int B, int H, int Hkv, int N, int D, int causal,
+                              float softmax_scale, void* stream, void* workspace,
+                              size_t workspace_bytes);
+
+/*
+ * The FP4 attention backward. The Attn-QAT abstract (arxiv listing "Attn-QAT:
+ * 4-Bit Attention With Quantization-Aware Training") asks that (1) the
+ * backward recompute the attention scores in the forward's low precision and
+ * (2) FlashAttention's gradient lose an implicit precision assumption; it
+ * gives no formula. The reading implemented:
+ *   q~, k~, v~  the forward's NVFP4 operands (same tensor scales, codes and
+ *               block scales as fp4_attn_fwd), dequantised
+ *   P_ij = 2^(S_ij c - lse_i)   scores recomputed from q~, k~ (1)
+ *   dP_ij = dO_i . v~_j,  D_i = sum_j P_ij dP_ij   (2): D from this P and v~,
+ *               not FlashAttention's dO . O, which assumes O = P V exactly
+ *   dS = P (dP - D),  dq = scale dS k~,  dk = scale dS^T q~,  dv = P^T dO
+ *   (dk, dv summed over the query heads of each key/value head)
+ * with straight-through quantisers. Inputs: q, k, v as fp4_attn_fwd; dout
+ * [B][H][N][D] bf16; lse from fp4_attn_fwd_lse. Outputs (bf16): dq
+ * [B][H][N][D], dk and dv [B][Hkv][N][D]. The contractions run on the tensor
+ * cores in bf16 with fp32 accumulation (P and dS rounded to bf16 for theirs).
+ * workspace: fp4_attn_bwd_workspace_bytes(B, H, Hkv, N, D) bytes.
+ */
+size_t fp4_attn_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D);
+fp4_status_t fp4_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
+                          const float* lse, void* dq, void* dk, void* dv, int B, int H, int Hkv,
+                          int N, int D, int causal, float softmax_scale, void* stream,
+                          void* workspace, size_t workspace_bytes);
+
 size_t fp4_attn_workspace_bytes_fp8pv(int B, int H, int Hkv, int N, int D);
 fp4_status_t fp4_attn_fwd_fp8pv(const void* q, const void* k, const void* v, void* out, int B,
                                 int H, int Hkv, int N, int D, int causal, float softmax_scale,

@@ -335,21 +335,26 @@ def attn_bwd(q, k, v, dout, causal: bool, softmax_scale: float = 0.0, q_rows=Non
     kr = None if kv_rows is None else _c(kv_rows, np.int64).reshape(-1, 3)
     nq = B * H * N if qr is None else len(qr)
     nkv = B * Hkv * N if kr is None else len(kr)
-    dq = np.zeros((nq, D))
-    dk = np.zeros((nkv, D))
-    dv = np.zeros((nkv, D))
+    dummy = np.zeros((1, 3), np.int64)  # a valid pointer for an empty selection
+    if qr is not None and not len(qr):
+        qr = dummy
+    if kr is not None and not len(kr):
+        kr = dummy
+    dq = np.zeros((max(nq, 1), D))
+    dk = np.zeros((max(nkv, 1), D))
+    dv = np.zeros((max(nkv, 1), D))
     Dv = np.zeros((B, H, N)) if want_D else None
     rc = _load().ora_attn_bwd(
         q.ctypes.data, k.ctypes.data, v.ctypes.data, dout.ctypes.data, B, H, Hkv, N, D,
         int(bool(causal)), float(softmax_scale), None if qr is None else qr.ctypes.data, nq,
-        None if kr is None else kr.ctypes.data, nkv if (kr is None or len(kr)) else -1,
+        None if kr is None else kr.ctypes.data, nkv if (kr is None or nkv) else -1,
         dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, None if Dv is None else Dv.ctypes.data,
         _threads(threads))
     if rc != 0:
         raise ValueError("ora_attn_bwd: bad arguments")
-    out["dq"] = dq.reshape(B, H, N, D) if qr is None else dq
-    out["dk"] = dk.reshape(B, Hkv, N, D) if kr is None else dk
-    out["dv"] = dv.reshape(B, Hkv, N, D) if kr is None else dv
+    out["dq"] = dq.reshape(B, H, N, D) if qr is None else dq[:nq]
+    out["dk"] = dk.reshape(B, Hkv, N, D) if kr is None else dk[:nkv]
+    out["dv"] = dv.reshape(B, Hkv, N, D) if kr is None else dv[:nkv]
     if want_D:
         out["D"] = Dv
     return out
