@@ -49,10 +49,11 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="video_dit")
     ap.add_argument("--impl", default="fp4attn", choices=["fp4attn", "reference"])
-    ap.add_argument("--variant", default="exp", choices=["exp", "efq", "fp8pv", "smooth"],
+    ap.add_argument("--variant", default="exp", choices=["exp", "efq", "fp8pv", "smooth", "bwd"],
                     help="P generation: exp-then-quantize (the default path), EFQ-Softmax, "
                          "or exp-then-quantize to FP8 with V in FP8 (PV as an FP8 contraction); "
-                         "smooth: the default path with Q and K smoothed")
+                         "smooth: the default path with Q and K smoothed; bwd: the FP4 attention "
+                         "backward (one GPU; its own metric)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0,
                     help="override H and Hkv (keeping their ratio) for a smaller profiling case")
@@ -156,6 +157,9 @@ def cpu_baseline(wl, q, k, v, rows_total: int, variant: str = "exp"):
 
 def run_reference(args, wl):
     """The reference arm: the CPU oracle on a bounded sample per step."""
+    if args.variant == "bwd":
+        raise SystemExit("the reference arm times the forward; bench --variant bwd reports the "
+                         "oracle backward as its cpu_baseline")
     import numpy as np
     import synth
     rank = int(os.environ.get("RANK", "0"))
@@ -182,6 +186,115 @@ def run_reference(args, wl):
     print(json.dumps(line), flush=True)
 
 
+def run_bwd(args, wl):
+    """The FP4 attention backward on one GPU: fp4_attn_bwd timed with inputs
+    resident (lse from fp4_attn_fwd_lse), e2e through host buffers."""
+    import numpy as np
+    import torch
+    import bit_attention_transformers_b200 as fa
+    import synth
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--variant bwd runs on one GPU")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    fa.lib()
+    synth.build()
+    hq, hk, hv = (torch.empty(shape, dtype=torch.bfloat16, pin_memory=True) for shape in
+                  ((wl.B, wl.H, wl.N, wl.D), (wl.B, wl.Hkv, wl.N, wl.D), (wl.B, wl.Hkv, wl.N, wl.D)))
+    synth.workload_inputs(wl, outs=[t.view(torch.int16).numpy().view(np.uint16) for t in (hq, hk, hv)])
+    hdo = torch.empty_like(hq).pin_memory()
+    hdo.view(torch.int16).numpy().view(np.uint16)[...] = synth.normal_bf16(
+        hq.numel(), seed=wl.seed + 17, stream=5).reshape(hq.shape)
+    q, k, v, do = (t.to(dev) for t in (hq, hk, hv, hdo))
+    out, lse = fa.fp4_attn_fwd_lse(q, k, v, causal=wl.causal)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        fa.fp4_attn_bwd(q, k, v, do, lse, causal=wl.causal, dq=dq, dk=dk, dv=dv)
+
+    def timed(fn, n):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
+        for a, b in evs:
+            flush_l2(flush)
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in evs]
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    fa.fp4_status()
+    with Clocks(0) as clk:
+        ms = timed(step, args.steps)
+    fa.fp4_status()
+    ms_per_step = sum(ms) / len(ms)
+    fwd_flops = wl.flops
+    value = 2.5 * fwd_flops / (ms_per_step * 1e-3) / 1e12
+    # the kernels' own tensor work: the dq kernel's two sweeps (S, dP twice) and
+    # dQ, the dk/dv kernel's S, dP, dV, dK: 9 contractions of 2 N^2 D per head
+    tensor_flops = 9 * fwd_flops / 2
+    peaks, src = measured_peaks()
+    hlse = torch.empty(lse.shape, dtype=torch.float32, pin_memory=True)
+    hlse.copy_(lse)
+    hdq, hdk, hdv = (torch.empty(t.shape, dtype=torch.bfloat16, pin_memory=True)
+                     for t in (dq, dk, dv))
+
+    def e2e():
+        gq, gk, gv, gdo, gl = (t.to(dev, non_blocking=True) for t in (hq, hk, hv, hdo, hlse))
+        a, b, c = fa.fp4_attn_bwd(gq, gk, gv, gdo, gl, causal=wl.causal)
+        hdq.copy_(a, non_blocking=True)
+        hdk.copy_(b, non_blocking=True)
+        hdv.copy_(c, non_blocking=True)
+        stream.synchronize()
+
+    e2e()
+    e_ms = timed(e2e, max(1, args.steps // 2))
+    e_val = 2.5 * fwd_flops / (sum(e_ms) / len(e_ms) * 1e-3) / 1e12
+    line = {
+        "metric": "FP4 attention bwd TFLOPS at 1 B200 (2.5 x forward FLOPs)", "value": value,
+        "unit": "TFLOPS", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4 scores, bf16 gradient contractions",
+        "data": "synthetic",
+        "config": {**wl.describe(), "pass": "backward (fp4_attn_bwd)", "parallelism": "1 GPU",
+                   "l2": "L2 flushed (252 MB write) before every timed step"},
+        "roofline": {"bound": "tensor", "achieved": tensor_flops / (ms_per_step * 1e-3) / 1e12,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": tensor_flops / (ms_per_step * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                     "traffic": None,
+                     "peak_source": f"measured dense bf16 ({src}); the whole call, 9 bf16 "
+                                    "contractions of 2 N^2 D per head; fraction of measured"},
+        "e2e": {"value": e_val, "unit": "TFLOPS",
+                "h2d_bytes_per_step": (hq.numel() + hk.numel() + hv.numel() + hdo.numel()) * 2
+                                      + hlse.numel() * 4,
+                "d2h_bytes_per_step": (hdq.numel() + hdk.numel() + hdv.numel()) * 2},
+        # amax, Q^ and K^ decode, V^ decode, dO pad/transpose, lse pad, dq kernel, dk/dv kernel
+        "gpu_launches": 8 * args.steps,
+    }
+    c = clk.summary()
+    if c:
+        line["clocks"] = c
+    if not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        rows = synth.sample_rows(wl, max(1, (args.cpu_rows or wl.B * wl.H) // (wl.B * wl.H)))
+        a = [t.view(torch.int16).numpy().view(np.uint16) for t in (hq, hk, hv, hdo)]
+        t0 = time.perf_counter()
+        oracle.attn_bwd(*a, wl.causal, q_rows=rows, kv_rows=np.zeros((0, 3), np.int64))
+        dt = time.perf_counter() - t0
+        keys = (rows[:, 2] + 1).astype(np.float64) if wl.causal else np.full(len(rows), wl.N, np.float64)
+        line["cpu_baseline"] = {"value": 2.5 * float((4.0 * wl.D * keys).sum()) / dt / 1e12,
+                                "unit": "TFLOPS", "cores": os.cpu_count() or 1, "kind": "oracle",
+                                "sample": f"dq of {len(rows)} seeded query rows of {wl.name} "
+                                          f"(plus decoding K, V for them); {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     import synth
@@ -192,6 +305,9 @@ def main():
         wl = dataclasses.replace(wl, H=args.heads, Hkv=max(1, args.heads // g))
     if args.impl == "reference":
         run_reference(args, wl)
+        return
+    if args.variant == "bwd":
+        run_bwd(args, wl)
         return
 
     import numpy as np
