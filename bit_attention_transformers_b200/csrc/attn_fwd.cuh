@@ -169,12 +169,14 @@ constexpr float kRound = 8388608.0f;  // 2^23: x + 2^23 rounds x (0 <= x < 2^22)
 // (the smoothed-Q path; exp-then-quantize P only). The key tile's 128 values
 // travel with its V tile, so they stay in shared memory until PV of the tile
 // has completed, after the softmax has read them.
-template <int D, bool CAUSAL, int PG, bool BIAS = false>
+// LSE: also write lse = m + log2 l per row (the training forward).
+template <int D, bool CAUSAL, int PG, bool BIAS = false, bool LSE = false>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   constexpr bool EFQ = PG == kPgEfq, FP8 = PG == kPgFp8;
   static_assert(!BIAS || PG == kPgExp, "the score correction is built for exp-then-quantize P");
+  static_assert(!LSE || PG == kPgExp, "lse is written by the exp-then-quantize forward");
   using L = AttnSmem<D, FP8>;
   using TC = TmemCols<EFQ>;
   constexpr uint32_t kColQsf = TC::kQsf, kColKsf = TC::kKsf, kColPsf = TC::kPsf,
@@ -612,7 +614,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       } else {
         const float lsum = lval[row] + lval[kBM + row];
         inv = __fdiv_rn(fpv, lsum);
-        if (PG == kPgExp && p.lse && stream == 0 && qrow < p.N)
+        if (LSE && stream == 0 && qrow < p.N)
           p.lse[(int64_t)gq * p.N + qrow] = m_fin + log2f(lsum);
       }
       constexpr int DH = D / 2;             // each stream writes half the channels

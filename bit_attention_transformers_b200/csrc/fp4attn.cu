@@ -62,7 +62,14 @@ AttnKernel attn_kernel_pg(int D, int causal) {
 // The fused kernel for head dim D, causal masking and P generation pg
 // (fp4::kPgExp, kPgEfq, kPgFp8); bias: with the per-key score correction of
 // smoothed Q (exp-then-quantize only).
-AttnKernel attn_kernel(int D, int causal, int pg, bool bias = false) {
+AttnKernel attn_kernel(int D, int causal, int pg, bool bias = false, bool lse = false) {
+  if (lse) {
+    if (D == 128)
+      return causal ? fp4::attn_fwd_kernel<128, true, fp4::kPgExp, false, true>
+                    : fp4::attn_fwd_kernel<128, false, fp4::kPgExp, false, true>;
+    return causal ? fp4::attn_fwd_kernel<64, true, fp4::kPgExp, false, true>
+                  : fp4::attn_fwd_kernel<64, false, fp4::kPgExp, false, true>;
+  }
   if (bias) {
     if (D == 128)
       return causal ? fp4::attn_fwd_kernel<128, true, fp4::kPgExp, true>
@@ -111,8 +118,8 @@ fp4_status_t device_setup(int* dev_out, int* sms_out) {
                   dev, major, minor);
     for (int d = 0; d < 2; ++d)
       for (int causal = 0; causal < 2; ++causal)
-        for (int pg = 0; pg < 4; ++pg)  // pg 3: exp-then-quantize with the score correction
-          FP4_CUDA(cudaFuncSetAttribute(attn_kernel(d ? 128 : 64, causal, pg % 3, pg == 3),
+        for (int pg = 0; pg < 5; ++pg)  // 3: with the score correction, 4: writing lse
+          FP4_CUDA(cudaFuncSetAttribute(attn_kernel(d ? 128 : 64, causal, pg % 3, pg == 3, pg == 4),
                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         attn_smem_bytes(d ? 128 : 64, pg % 3)));
     for (int d = 0; d < 2; ++d)
@@ -415,10 +422,12 @@ fp4_status_t launch_attn(const uint8_t* qc, const uint8_t* qs, const float* qa, 
   p.lse = lse;
   p.softmax_scale = resolve_scale(softmax_scale, D);
   dim3 grid(p.ntq, H, B);
-  if (bias && pg != fp4::kPgExp)
-    return fail(FP4_ERR_UNSUPPORTED, "the score correction needs exp-then-quantize P");
-  attn_kernel(D, causal, pg, bias != nullptr)<<<grid, fp4::kAttnThreads, attn_smem_bytes(D, pg),
-                                                stream>>>(tq, tk, tv, p);
+  if ((bias || lse) && pg != fp4::kPgExp)
+    return fail(FP4_ERR_UNSUPPORTED, "the score correction and lse need exp-then-quantize P");
+  if (bias && lse) return fail(FP4_ERR_UNSUPPORTED, "lse with the score correction");
+  attn_kernel(D, causal, pg, bias != nullptr, lse != nullptr)<<<grid, fp4::kAttnThreads,
+                                                                attn_smem_bytes(D, pg), stream>>>(
+      tq, tk, tv, p);
   FP4_CUDA(cudaGetLastError());
   return FP4_OK;
 }
