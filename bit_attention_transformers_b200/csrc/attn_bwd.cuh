@@ -279,37 +279,43 @@ __device__ __forceinline__ bool bwd_wait(uint32_t bar, uint32_t parity) {
 }
 
 // ------------------------------------------------------------- dq kernel ----
+constexpr int kDqThreads = 384;  // warps 0-3 control (warp 0 loads, warp 1 issues), 4-11 compute
+constexpr uint32_t kDqRegsCtl = 56, kDqRegsCompute = 224;  // 128 x 56 + 256 x 224 = 384 x 168
+
 template <int D>
 struct BwdDqSmem {
   static constexpr int kQ = kBwdQ * D * 2;    // Q^ tile, bf16
   static constexpr int kK = kBwdKt * D * 2;   // K^ tile
   static constexpr int kKT = D * kBwdKt * 2;  // K^T tile (D rows x 64 keys)
   static constexpr int kStage = 2 * kK + kKT; // K^, V^, K^T
+  static constexpr int kDS = kBwdQ * kBwdKt * 2;  // one dS tile: 128 rows x 64 keys, bf16
   static constexpr int oQ = 0;
   static constexpr int oDO = oQ + kQ;
   static constexpr int oStage = oDO + kQ;
-  static constexpr int oDS = oStage + 2 * kStage;  // dS tile: 128 rows x 64 keys, bf16
-  static constexpr int oBar = oDS + kBwdQ * kBwdKt * 2;
+  static constexpr int oDS = oStage + 2 * kStage;  // [2]: one dS buffer per compute stream
+  static constexpr int oD = oDS + 2 * kDS;         // float [2][128]: each stream's partial D
+  static constexpr int oBar = oD + 1024;
   static constexpr int oTmem = oBar + 256;
   static constexpr int kBytes = oTmem + 16 + 1024;
 };
 
 enum : int {
   kDqBarQ = 0,
-  kDqBarFull = 1,     // [2]
+  kDqBarFull = 1,     // [2] stages
   kDqBarEmpty = 3,    // [2]
-  kDqBarSFull = 5,    // [2]
+  kDqBarSFull = 5,    // [2] S/dP buffers (= compute streams)
   kDqBarSEmpty = 7,   // [2]
-  kDqBarDsFull = 9,
-  kDqBarDsEmpty = 10,
-  kDqBarDone = 11,
-  kDqBars = 12
+  kDqBarDsFull = 9,   // [2] dS buffers
+  kDqBarDsEmpty = 11, // [2]
+  kDqBarDone = 13,
 };
 
-// One CTA per (128-query tile, head, batch). TMEM: S[b] at 128 b, dP[b] at
-// 128 b + 64 (64 columns each, b = tile parity), dQ at 256 (D columns).
+// One CTA per (128-query tile, head, batch). Two compute streams (warpgroups)
+// take alternate key tiles, so that one forms its P and dS while the tensor
+// core works for the other. TMEM: S[b] at 128 b, dP[b] at 128 b + 64 (64
+// columns each, b = tile parity = stream), dQ at 256 (D columns).
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kDqThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmKT, const BwdParams p) {
@@ -333,9 +339,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar(kDqBarEmpty + s), 1);
       mbar_init(bar(kDqBarSFull + s), 1);
       mbar_init(bar(kDqBarSEmpty + s), 4);
+      mbar_init(bar(kDqBarDsFull + s), 4);
+      mbar_init(bar(kDqBarDsEmpty + s), 1);
     }
-    mbar_init(bar(kDqBarDsFull), 4);
-    mbar_init(bar(kDqBarDsEmpty), 1);
     mbar_init(bar(kDqBarDone), 1);
     fence_mbar_init();
   }
@@ -349,8 +355,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + L::oTmem);
   constexpr int NA = D / 64;  // 64-element atoms along D
 
-  if (warp == 0) {
-    if (lane == 0) {
+  if (warp < 4) {
+    regs_dec<kDqRegsCtl>();
+    if (warp == 0 && lane == 0) {
       bool ok = true;
       int issued = 0;
       mbar_arrive_expect_tx(bar(kDqBarQ), 2 * L::kQ);
@@ -377,24 +384,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       // copies still in flight after a failed wait land before the CTA exits
       drain_wait(bar(kDqBarQ), 0);
-      for (int t = max(0, issued - 2); t < issued; ++t) drain_wait(bar(kDqBarFull + (t & 1)), (t >> 1) & 1);
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
+      for (int t = max(0, issued - 2); t < issued; ++t)
+        drain_wait(bar(kDqBarFull + (t & 1)), (t >> 1) & 1);
+    } else if (warp == 1 && lane == 0) {
       bool ok = bwd_wait(bar(kDqBarQ), 0);
       const uint32_t idS = idesc_bf16(kBwdQ, kBwdKt), idQ = idesc_bf16(kBwdQ, D);
       auto issue_dq = [&](int t) {  // dQ += dS K^ of tile t (sweep 2)
         const int st = t & 1, t2 = t - nkt;
-        ok = ok && bwd_wait(bar(kDqBarDsFull), t2 & 1);
+        ok = ok && bwd_wait(bar(kDqBarDsFull + (t & 1)), (t2 >> 1) & 1);
         if (!ok) return;
         tc_fence_after();
         const uint32_t kt = sb + L::oStage + st * L::kStage + 2 * L::kK;
+        const uint32_t ds = sb + L::oDS + (t & 1) * L::kDS;
 #pragma unroll
         for (int s = 0; s < kBwdKt / 16; ++s)
-          mma_bf16(tmem + 256, kmaj_desc(sb + L::oDS, kBwdQ, s), kmaj_desc(kt, D, s), idQ,
+          mma_bf16(tmem + 256, kmaj_desc(ds, kBwdQ, s), kmaj_desc(kt, D, s), idQ,
                    (t2 > 0 || s > 0) ? 1u : 0u);
         tc_commit(bar(kDqBarEmpty + st));
-        tc_commit(bar(kDqBarDsEmpty));
+        tc_commit(bar(kDqBarDsEmpty + (t & 1)));
       };
       for (int t = 0; t < T && ok; ++t) {
         const int st = t & 1, buf = t & 1;
@@ -417,14 +424,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_commit(bar(kDqBarDone));
       drain_wait(bar(kDqBarDone), 0);  // every MMA complete before TMEM is freed
     }
-  } else if (warp >= 4) {
-    const int quad = warp & 3, row = quad * 32 + lane, qrow = qt * kBwdQ + row;
+  } else {
+    regs_inc<kDqRegsCompute>();
+    const int stream = (warp - 4) >> 2, quad = warp & 3;
+    const int row = quad * 32 + lane, qrow = qt * kBwdQ + row;
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
     const BwdScales sc = bwd_scales(p);
     const float lse = p.lse[(int64_t)gq * p.Npad + qrow];
+    float* Dpart = reinterpret_cast<float*>(sm + L::oD);
     float Dsum = 0.0f;
-    bool ok = true;
-    for (int t = 0; t < T; ++t) {
+    bool ok = true, combined = false;
+    // both streams' partial D of the row, once every sweep-1 tile is done
+    auto combine = [&]() {
+      Dpart[stream * kBwdQ + row] = Dsum;
+      named_bar_sync(1, 256);
+      Dsum = Dpart[row] + Dpart[kBwdQ + row];
+      if (stream == 0) p.Dvec[(int64_t)gq * p.Npad + qrow] = Dsum;
+      combined = true;
+    };
+    for (int t = stream; t < T; t += 2) {
+      if (!combined && t >= nkt) combine();
       const int buf = t & 1, j = t % nkt;
       float s[64], dp[64];
       ok = ok && __all_sync(0xFFFFFFFFu, bwd_wait(bar(kDqBarSFull + buf), (t >> 1) & 1));
@@ -452,7 +471,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < 64; ++c) acc = fmaf(s[c], dp[c], acc);
         Dsum = fmaf(acc, sc.dv, Dsum);
-        if (t == nkt - 1) p.Dvec[(int64_t)gq * p.Npad + qrow] = Dsum;
         continue;
       }
       // dS = P (d_V dP - D) -> bf16, the row's 128 bytes (128-byte swizzle)
@@ -462,9 +480,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         w[c] = pack_bf16(s[2 * c] * fmaf(dp[2 * c], sc.dv, -Dsum),
                          s[2 * c + 1] * fmaf(dp[2 * c + 1], sc.dv, -Dsum));
       const int t2 = t - nkt;
-      if (t2 > 0) ok = __all_sync(0xFFFFFFFFu, bwd_wait(bar(kDqBarDsEmpty), (t2 - 1) & 1));
+      if (t2 >= 2)
+        ok = __all_sync(0xFFFFFFFFu, bwd_wait(bar(kDqBarDsEmpty + buf), ((t2 >> 1) - 1) & 1));
       if (!ok) break;
-      uint8_t* dsr = sm + L::oDS + row * 128;
+      uint8_t* dsr = sm + L::oDS + buf * L::kDS + row * 128;
 #pragma unroll
       for (int k2 = 0; k2 < 8; ++k2)
         *reinterpret_cast<uint4*>(dsr + ((k2 ^ (row & 7)) * 16)) =
@@ -472,17 +491,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kDqBarDsFull));
+      if (lane == 0) mbar_arrive(bar(kDqBarDsFull + buf));
     }
+    if (!combined) combine();
     ok = ok && __all_sync(0xFFFFFFFFu, bwd_wait(bar(kDqBarDone), 0));
     if (ok) {  // warp-uniform: tcgen05.ld is a whole-warp instruction; only the stores are per row
       tc_fence_after();
-      __nv_bfloat16* dst = p.dq + ((int64_t)gq * p.N + qrow) * D;
+      constexpr int DH = D / 2;  // each stream writes half the channels
+      __nv_bfloat16* dst = p.dq + ((int64_t)gq * p.N + qrow) * D + stream * DH;
 #pragma unroll
-      for (int cc = 0; cc < D; cc += 32) {
+      for (int cc = 0; cc < DH; cc += 32) {
         float o[32];
         __syncwarp();
-        tmem_ld32(tl + 256 + cc, o);
+        tmem_ld32(tl + 256 + stream * DH + cc, o);
         tmem_wait_ld();
         if (qrow < p.N) {
           uint32_t w[16];

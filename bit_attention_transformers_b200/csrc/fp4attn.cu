@@ -612,7 +612,7 @@ fp4_status_t attn_bwd_any(const void* q, const void* k, const void* v, const voi
   p.Npad = (int)Npad;
   p.softmax_scale = resolve_scale(softmax_scale, D);
   dim3 g1((unsigned)(Npad / fp4::kBwdQ), (unsigned)H, (unsigned)B);
-  bwd_dq_kernel_for(D, causal)<<<g1, fp4::kBwdThreads,
+  bwd_dq_kernel_for(D, causal)<<<g1, fp4::kDqThreads,
                                  D == 128 ? fp4::BwdDqSmem<128>::kBytes : fp4::BwdDqSmem<64>::kBytes,
                                  st>>>(mQ, mDO, mK64, mV64, mKT, p);
   FP4_CUDA(cudaGetLastError());
