@@ -282,17 +282,22 @@ __device__ __forceinline__ bool bwd_wait(uint32_t bar, uint32_t parity) {
 constexpr int kDqThreads = 384;  // warps 0-3 control (warp 0 loads, warp 1 issues), 4-11 compute
 constexpr uint32_t kDqRegsCtl = 56, kDqRegsCompute = 224;  // 128 x 56 + 256 x 224 = 384 x 168
 
+// Two rings of key tiles: ring A (K^, V^) feeds S and dP and is released as
+// soon as they complete; ring B (K^T) feeds dQ, needed a tile later, and has
+// its own producer warp, so that neither ring's loads wait on the other's.
+constexpr int kDqRingA = 2, kDqRingB = 3;
+
 template <int D>
 struct BwdDqSmem {
   static constexpr int kQ = kBwdQ * D * 2;    // Q^ tile, bf16
   static constexpr int kK = kBwdKt * D * 2;   // K^ tile
   static constexpr int kKT = D * kBwdKt * 2;  // K^T tile (D rows x 64 keys)
-  static constexpr int kStage = 2 * kK + kKT; // K^, V^, K^T
   static constexpr int kDS = kBwdQ * kBwdKt * 2;  // one dS tile: 128 rows x 64 keys, bf16
   static constexpr int oQ = 0;
   static constexpr int oDO = oQ + kQ;
-  static constexpr int oStage = oDO + kQ;
-  static constexpr int oDS = oStage + 2 * kStage;  // [2]: one dS buffer per compute stream
+  static constexpr int oA = oDO + kQ;              // [kDqRingA]: K^ then V^
+  static constexpr int oB = oA + kDqRingA * 2 * kK;  // [kDqRingB]: K^T
+  static constexpr int oDS = oB + kDqRingB * kKT;  // [2]: one dS buffer per compute stream
   static constexpr int oD = oDS + 2 * kDS;         // float [2][128]: each stream's partial D
   static constexpr int oBar = oD + 1024;
   static constexpr int oTmem = oBar + 256;
@@ -301,13 +306,15 @@ struct BwdDqSmem {
 
 enum : int {
   kDqBarQ = 0,
-  kDqBarFull = 1,     // [2] stages
-  kDqBarEmpty = 3,    // [2]
-  kDqBarSFull = 5,    // [2] S/dP buffers (= compute streams)
-  kDqBarSEmpty = 7,   // [2]
-  kDqBarDsFull = 9,   // [2] dS buffers
-  kDqBarDsEmpty = 11, // [2]
-  kDqBarDone = 13,
+  kDqBarFullA = 1,                     // [kDqRingA]
+  kDqBarEmptyA = kDqBarFullA + kDqRingA,  // [kDqRingA]
+  kDqBarFullB = kDqBarEmptyA + kDqRingA,  // [kDqRingB]
+  kDqBarEmptyB = kDqBarFullB + kDqRingB,  // [kDqRingB]
+  kDqBarSFull = kDqBarEmptyB + kDqRingB,  // [2] S/dP buffers (= compute streams)
+  kDqBarSEmpty = kDqBarSFull + 2,         // [2]
+  kDqBarDsFull = kDqBarSEmpty + 2,        // [2] dS buffers
+  kDqBarDsEmpty = kDqBarDsFull + 2,       // [2]
+  kDqBarDone = kDqBarDsEmpty + 2,
 };
 
 // One CTA per (128-query tile, head, batch). Two compute streams (warpgroups)
@@ -334,9 +341,15 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   auto bar = [&](int i) -> uint32_t { return sb + L::oBar + 8 * i; };
   if (threadIdx.x == 0) {
     mbar_init(bar(kDqBarQ), 1);
+    for (int s = 0; s < kDqRingA; ++s) {
+      mbar_init(bar(kDqBarFullA + s), 1);
+      mbar_init(bar(kDqBarEmptyA + s), 1);
+    }
+    for (int s = 0; s < kDqRingB; ++s) {
+      mbar_init(bar(kDqBarFullB + s), 1);
+      mbar_init(bar(kDqBarEmptyB + s), 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(kDqBarFull + s), 1);
-      mbar_init(bar(kDqBarEmpty + s), 1);
       mbar_init(bar(kDqBarSFull + s), 1);
       mbar_init(bar(kDqBarSEmpty + s), 4);
       mbar_init(bar(kDqBarDsFull + s), 4);
@@ -366,49 +379,61 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         tma_load_2d(sb + L::oDO + a * kBwdQ * 128, &tmDO, a * 64, gq * p.Npad + qt * kBwdQ,
                     bar(kDqBarQ));
       }
-      for (int t = 0; t < T && ok; ++t) {
-        const int st = t & 1, j = t % nkt;
-        const bool sw2 = t >= nkt;
-        if (t >= 2 && !(ok = bwd_wait(bar(kDqBarEmpty + st), ((t >> 1) - 1) & 1))) break;
-        const uint32_t base = sb + L::oStage + st * L::kStage;
-        mbar_arrive_expect_tx(bar(kDqBarFull + st), 2 * L::kK + (sw2 ? L::kKT : 0));
+      for (int t = 0; t < T && ok; ++t) {  // ring A: K^ and V^ of every tile of both sweeps
+        const int st = t % kDqRingA, j = t % nkt;
+        if (t >= kDqRingA && !(ok = bwd_wait(bar(kDqBarEmptyA + st), ((t / kDqRingA) - 1) & 1)))
+          break;
+        const uint32_t base = sb + L::oA + st * 2 * L::kK;
+        mbar_arrive_expect_tx(bar(kDqBarFullA + st), 2 * L::kK);
         for (int a = 0; a < NA; ++a) {
           tma_load_2d(base + a * kBwdKt * 128, &tmK, a * 64, gk * p.Npad + j * kBwdKt,
-                      bar(kDqBarFull + st));
+                      bar(kDqBarFullA + st));
           tma_load_2d(base + L::kK + a * kBwdKt * 128, &tmV, a * 64, gk * p.Npad + j * kBwdKt,
-                      bar(kDqBarFull + st));
+                      bar(kDqBarFullA + st));
         }
-        if (sw2)
-          tma_load_2d(base + 2 * L::kK, &tmKT, j * kBwdKt, gk * D, bar(kDqBarFull + st));
         issued = t + 1;
       }
       // copies still in flight after a failed wait land before the CTA exits
       drain_wait(bar(kDqBarQ), 0);
-      for (int t = max(0, issued - 2); t < issued; ++t)
-        drain_wait(bar(kDqBarFull + (t & 1)), (t >> 1) & 1);
+      for (int t = max(0, issued - kDqRingA); t < issued; ++t)
+        drain_wait(bar(kDqBarFullA + t % kDqRingA), (t / kDqRingA) & 1);
+    } else if (warp == 2 && lane == 0) {
+      bool ok = true;
+      int issued = 0;
+      for (int t2 = 0; t2 < nkt && ok; ++t2) {  // ring B: K^T of the sweep-2 tiles
+        const int st = t2 % kDqRingB;
+        if (t2 >= kDqRingB && !(ok = bwd_wait(bar(kDqBarEmptyB + st), ((t2 / kDqRingB) - 1) & 1)))
+          break;
+        mbar_arrive_expect_tx(bar(kDqBarFullB + st), L::kKT);
+        tma_load_2d(sb + L::oB + st * L::kKT, &tmKT, t2 * kBwdKt, gk * D, bar(kDqBarFullB + st));
+        issued = t2 + 1;
+      }
+      for (int t2 = max(0, issued - kDqRingB); t2 < issued; ++t2)
+        drain_wait(bar(kDqBarFullB + t2 % kDqRingB), (t2 / kDqRingB) & 1);
     } else if (warp == 1 && lane == 0) {
       bool ok = bwd_wait(bar(kDqBarQ), 0);
       const uint32_t idS = idesc_bf16(kBwdQ, kBwdKt), idQ = idesc_bf16(kBwdQ, D);
       auto issue_dq = [&](int t) {  // dQ += dS K^ of tile t (sweep 2)
-        const int st = t & 1, t2 = t - nkt;
+        const int t2 = t - nkt, sb2 = t2 % kDqRingB;
         ok = ok && bwd_wait(bar(kDqBarDsFull + (t & 1)), (t2 >> 1) & 1);
+        ok = ok && bwd_wait(bar(kDqBarFullB + sb2), (t2 / kDqRingB) & 1);
         if (!ok) return;
         tc_fence_after();
-        const uint32_t kt = sb + L::oStage + st * L::kStage + 2 * L::kK;
+        const uint32_t kt = sb + L::oB + sb2 * L::kKT;
         const uint32_t ds = sb + L::oDS + (t & 1) * L::kDS;
 #pragma unroll
         for (int s = 0; s < kBwdKt / 16; ++s)
           mma_bf16(tmem + 256, kmaj_desc(ds, kBwdQ, s), kmaj_desc(kt, D, s), idQ,
                    (t2 > 0 || s > 0) ? 1u : 0u);
-        tc_commit(bar(kDqBarEmpty + st));
+        tc_commit(bar(kDqBarEmptyB + sb2));
         tc_commit(bar(kDqBarDsEmpty + (t & 1)));
       };
       for (int t = 0; t < T && ok; ++t) {
-        const int st = t & 1, buf = t & 1;
-        if (!(ok = bwd_wait(bar(kDqBarFull + st), (t >> 1) & 1))) break;
+        const int st = t % kDqRingA, buf = t & 1;
+        if (!(ok = bwd_wait(bar(kDqBarFullA + st), (t / kDqRingA) & 1))) break;
         if (t >= 2 && !(ok = bwd_wait(bar(kDqBarSEmpty + buf), ((t >> 1) - 1) & 1))) break;
         tc_fence_after();
-        const uint32_t base = sb + L::oStage + st * L::kStage;
+        const uint32_t base = sb + L::oA + st * 2 * L::kK;
 #pragma unroll
         for (int s = 0; s < D / 16; ++s) {
           mma_bf16(tmem + buf * 128, kmaj_desc(sb + L::oQ, kBwdQ, s), kmaj_desc(base, kBwdKt, s),
@@ -417,7 +442,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                    kmaj_desc(base + L::kK, kBwdKt, s), idS, s > 0 ? 1u : 0u);
         }
         tc_commit(bar(kDqBarSFull + buf));
-        if (t < nkt) tc_commit(bar(kDqBarEmpty + st));
+        tc_commit(bar(kDqBarEmptyA + st));
         if (t > nkt) issue_dq(t - 1);  // the previous tile's dQ, one step behind
       }
       if (ok && T > nkt) issue_dq(T - 1);
@@ -531,27 +556,31 @@ struct BwdDkvSmem {
   static constexpr int kK = kBwdK * D * 2;     // K^ or V^ tile, bf16
   static constexpr int kQ = kBwdQt * D * 2;    // Q^ or dO tile
   static constexpr int kQT = D * kBwdQt * 2;   // Q^T or dO^T tile
-  static constexpr int kStage = 2 * kQ + 2 * kQT;  // Q^, dO, Q^T, dO^T
   static constexpr int oK = 0;
   static constexpr int oV = oK + kK;
-  static constexpr int oStage = oV + kK;
-  static constexpr int oP = oStage + 2 * kStage;      // P^T: 128 keys x 64 queries, bf16
+  static constexpr int oA = oV + kK;          // ring A [2]: Q^ then dO (S^T, dP^T)
+  static constexpr int oB = oA + 2 * 2 * kQ;  // ring B [2]: Q^T then dO^T (dK, dV)
+  static constexpr int oP = oB + 2 * 2 * kQT;         // P^T: 128 keys x 64 queries, bf16
   static constexpr int oDS = oP + kBwdK * kBwdQt * 2; // dS^T
-  static constexpr int oLse = oDS + kBwdK * kBwdQt * 2;  // [2 stages]: lse[64], D[64]
+  static constexpr int oLse = oDS + kBwdK * kBwdQt * 2;  // ring B [2]: lse[64], D[64]
   static constexpr int oBar = oLse + 2 * 512;
   static constexpr int oTmem = oBar + 256;
   static constexpr int kBytes = oTmem + 16 + 1024;
 };
 
+// Ring A (Q^, dO) is released when S^T and dP^T complete; ring B (Q^T, dO^T,
+// lse, D) when dV and dK complete; each has its own producer warp.
 enum : int {
   kKvBarKV = 0,
-  kKvBarFull = 1,    // [2]
-  kKvBarEmpty = 3,   // [2]
-  kKvBarSFull = 5,   // [2]
-  kKvBarSEmpty = 7,  // [2]
-  kKvBarPFull = 9,
-  kKvBarPEmpty = 10,
-  kKvBarDone = 11,
+  kKvBarFullA = 1,    // [2]
+  kKvBarEmptyA = 3,   // [2]
+  kKvBarFullB = 5,    // [2]
+  kKvBarEmptyB = 7,   // [2]
+  kKvBarSFull = 9,    // [2]
+  kKvBarSEmpty = 11,  // [2]
+  kKvBarPFull = 13,
+  kKvBarPEmpty = 14,
+  kKvBarDone = 15,
 };
 
 // One CTA per (128-key tile, key/value head, batch); tiles of 64 queries of
@@ -580,8 +609,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(kKvBarKV), 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(kKvBarFull + s), 1);
-      mbar_init(bar(kKvBarEmpty + s), 1);
+      mbar_init(bar(kKvBarFullA + s), 1);
+      mbar_init(bar(kKvBarEmptyA + s), 1);
+      mbar_init(bar(kKvBarFullB + s), 1);
+      mbar_init(bar(kKvBarEmptyB + s), 1);
       mbar_init(bar(kKvBarSFull + s), 1);
       mbar_init(bar(kKvBarSEmpty + s), 4);
     }
@@ -611,28 +642,44 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tma_load_2d(sb + L::oV + a * kBwdK * 128, &tmV, a * 64, gk * p.Npad + kt * kBwdK,
                     bar(kKvBarKV));
       }
-      for (int t = 0; t < T && ok; ++t) {
+      for (int t = 0; t < T && ok; ++t) {  // ring A: Q^ and dO
         const int st = t & 1;
         const int gq = b * p.H + hk * G + t / nqt, i = i0 + t % nqt;
-        if (t >= 2 && !(ok = bwd_wait(bar(kKvBarEmpty + st), ((t >> 1) - 1) & 1))) break;
-        const uint32_t base = sb + L::oStage + st * L::kStage;
-        mbar_arrive_expect_tx(bar(kKvBarFull + st), L::kStage + 512);
+        if (t >= 2 && !(ok = bwd_wait(bar(kKvBarEmptyA + st), ((t >> 1) - 1) & 1))) break;
+        const uint32_t base = sb + L::oA + st * 2 * L::kQ;
+        mbar_arrive_expect_tx(bar(kKvBarFullA + st), 2 * L::kQ);
         for (int a = 0; a < NA; ++a) {
           tma_load_2d(base + a * kBwdQt * 128, &tmQ, a * 64, gq * p.Npad + i * kBwdQt,
-                      bar(kKvBarFull + st));
+                      bar(kKvBarFullA + st));
           tma_load_2d(base + L::kQ + a * kBwdQt * 128, &tmDO, a * 64, gq * p.Npad + i * kBwdQt,
-                      bar(kKvBarFull + st));
+                      bar(kKvBarFullA + st));
         }
-        tma_load_2d(base + 2 * L::kQ, &tmQT, i * kBwdQt, gq * D, bar(kKvBarFull + st));
-        tma_load_2d(base + 2 * L::kQ + L::kQT, &tmDOT, i * kBwdQt, gq * D, bar(kKvBarFull + st));
-        bulk_load(sb + L::oLse + st * 512, p.lse + (int64_t)gq * p.Npad + i * kBwdQt, 256,
-                  bar(kKvBarFull + st));
-        bulk_load(sb + L::oLse + st * 512 + 256, p.Dvec + (int64_t)gq * p.Npad + i * kBwdQt, 256,
-                  bar(kKvBarFull + st));
         issued = t + 1;
       }
       drain_wait(bar(kKvBarKV), 0);
-      for (int t = max(0, issued - 2); t < issued; ++t) drain_wait(bar(kKvBarFull + (t & 1)), (t >> 1) & 1);
+      for (int t = max(0, issued - 2); t < issued; ++t)
+        drain_wait(bar(kKvBarFullA + (t & 1)), (t >> 1) & 1);
+    }
+  } else if (warp == 2) {
+    if (lane == 0) {
+      bool ok = true;
+      int issued = 0;
+      for (int t = 0; t < T && ok; ++t) {  // ring B: Q^T, dO^T, lse, D
+        const int st = t & 1;
+        const int gq = b * p.H + hk * G + t / nqt, i = i0 + t % nqt;
+        if (t >= 2 && !(ok = bwd_wait(bar(kKvBarEmptyB + st), ((t >> 1) - 1) & 1))) break;
+        const uint32_t base = sb + L::oB + st * 2 * L::kQT;
+        mbar_arrive_expect_tx(bar(kKvBarFullB + st), 2 * L::kQT + 512);
+        tma_load_2d(base, &tmQT, i * kBwdQt, gq * D, bar(kKvBarFullB + st));
+        tma_load_2d(base + L::kQT, &tmDOT, i * kBwdQt, gq * D, bar(kKvBarFullB + st));
+        bulk_load(sb + L::oLse + st * 512, p.lse + (int64_t)gq * p.Npad + i * kBwdQt, 256,
+                  bar(kKvBarFullB + st));
+        bulk_load(sb + L::oLse + st * 512 + 256, p.Dvec + (int64_t)gq * p.Npad + i * kBwdQt, 256,
+                  bar(kKvBarFullB + st));
+        issued = t + 1;
+      }
+      for (int t = max(0, issued - 2); t < issued; ++t)
+        drain_wait(bar(kKvBarFullB + (t & 1)), (t >> 1) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -641,26 +688,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       auto issue_kv = [&](int t) {  // dV += P^T dO, dK += dS^T Q^ of tile t
         const int st = t & 1;
         ok = ok && bwd_wait(bar(kKvBarPFull), t & 1);
+        ok = ok && bwd_wait(bar(kKvBarFullB + st), (t >> 1) & 1);
         if (!ok) return;
         tc_fence_after();
-        const uint32_t base = sb + L::oStage + st * L::kStage;
+        const uint32_t base = sb + L::oB + st * 2 * L::kQT;
 #pragma unroll
         for (int s = 0; s < kBwdQt / 16; ++s) {
           const uint32_t acc = (t > 0 || s > 0) ? 1u : 0u;
-          mma_bf16(tmem + 256, kmaj_desc(sb + L::oP, kBwdK, s),
-                   kmaj_desc(base + 2 * L::kQ + L::kQT, D, s), idO, acc);
-          mma_bf16(tmem + 256 + D, kmaj_desc(sb + L::oDS, kBwdK, s),
-                   kmaj_desc(base + 2 * L::kQ, D, s), idO, acc);
+          mma_bf16(tmem + 256, kmaj_desc(sb + L::oP, kBwdK, s), kmaj_desc(base + L::kQT, D, s),
+                   idO, acc);
+          mma_bf16(tmem + 256 + D, kmaj_desc(sb + L::oDS, kBwdK, s), kmaj_desc(base, D, s), idO,
+                   acc);
         }
-        tc_commit(bar(kKvBarEmpty + st));
+        tc_commit(bar(kKvBarEmptyB + st));
         tc_commit(bar(kKvBarPEmpty));
       };
       for (int t = 0; t < T && ok; ++t) {
         const int st = t & 1, buf = t & 1;
-        if (!(ok = bwd_wait(bar(kKvBarFull + st), (t >> 1) & 1))) break;
+        if (!(ok = bwd_wait(bar(kKvBarFullA + st), (t >> 1) & 1))) break;
         if (t >= 2 && !(ok = bwd_wait(bar(kKvBarSEmpty + buf), ((t >> 1) - 1) & 1))) break;
         tc_fence_after();
-        const uint32_t base = sb + L::oStage + st * L::kStage;
+        const uint32_t base = sb + L::oA + st * 2 * L::kQ;
 #pragma unroll
         for (int s = 0; s < D / 16; ++s) {
           mma_bf16(tmem + buf * 128, kmaj_desc(sb + L::oK, kBwdK, s), kmaj_desc(base, kBwdQt, s),
@@ -669,6 +717,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                    kmaj_desc(base + L::kQ, kBwdQt, s), idS, s > 0 ? 1u : 0u);
         }
         tc_commit(bar(kKvBarSFull + buf));
+        tc_commit(bar(kKvBarEmptyA + st));
         if (t > 0) issue_kv(t - 1);
       }
       if (ok && T > 0) issue_kv(T - 1);
@@ -698,7 +747,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ok) break;
       // the stage's lse and D: its full barrier has completed (S^T was issued
       // after it); the wait makes the bulk copies' data visible to this thread
-      ok = __all_sync(0xFFFFFFFFu, bwd_wait(bar(kKvBarFull + st), (t >> 1) & 1));
+      ok = __all_sync(0xFFFFFFFFu, bwd_wait(bar(kKvBarFullB + st), (t >> 1) & 1));
       if (!ok) break;
       const float* lq = reinterpret_cast<const float*>(sm + L::oLse + st * 512);
       const float* dq = lq + 64;
