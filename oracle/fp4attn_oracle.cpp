@@ -277,16 +277,36 @@ const float kLog2e = 1.44269504088896340736f;  // fl32(1 / ln 2)
 //   K (flag 32): S_ij changes by -q_i . mean_K, the same for every key of
 //   row i, which the softmax cancels: nothing is added back.
 //   Q (flag 64): q_i . k_j = q'_i . k_j + mean_Q . k_j; the second term
-//   depends on the key, so it is added back to the scores in fp32:
-//   delta_j = mean_Q . k'_j (k' the smoothed K under flag 32, else K), and
-//   x_ij = fl32(S'_ij c + fl32(delta_j cs)) with one rounding (fma),
-//   cs = fl32(softmax_scale log2 e).
+//   depends on the key, so it is added back to the scores:
+//   delta_j = mean_Q . k'_j (k' the smoothed K under flag 32, else K), taken
+//   to the contraction's units, beta_j = fl32(delta_j fl32(s_Q s_K)) (the
+//   encode scales of the quantised Q' and K), and split into two tf32 values
+//   hi_j = tf32_rz(beta_j), lo_j = tf32_rz(fl32(beta_j - hi_j)) (tf32_rz: the
+//   low 13 mantissa bits cleared), beta'_j = hi_j + lo_j; the scores are
+//   x_ij = fl32(fl32(S'_ij + beta'_j) c), the sum exact and rounded once (the
+//   kernel adds beta' to the S accumulator as a rank-1 tensor-core product).
 // The mean is made independent of summation order so that it is one value on
 // any machine: every element is truncated toward zero to the fixed-point
 // grid 2^-s with s = 44 - E, 2^(E-1) <= amax < 2^E (amax of the raw tensor),
 // the integers are summed exactly (|x| 2^s < 2^44, so N <= 2^19 tokens fit in
 // 64 bits), and mean = fl32(fl64(fl64(T) 2^-s) / N); amax == 0 gives 0.
 // delta_j is a sequential fp32 fma chain over d = 0 .. D-1 from 0.
+const uint32_t kTf32Mask = 0xFFFFE000u;  // tf32: sign, exponent and 10 mantissa bits
+
+float tf32_rz(float x) {
+  uint32_t u;
+  std::memcpy(&u, &x, 4);
+  u &= kTf32Mask;
+  std::memcpy(&x, &u, 4);
+  return x;
+}
+
+// beta' = hi + lo of beta = fl32(delta * sqsk) (see above).
+void bias_split(float delta, float sqsk, float* hi, float* lo) {
+  const float beta = delta * sqsk;
+  *hi = tf32_rz(beta);
+  *lo = tf32_rz(beta - *hi);
+}
 const int kMeanGridBits = 44;
 
 void channel_mean(const uint16_t* x, int N, int D, float amax, float* mean) {
@@ -315,9 +335,9 @@ float smoothed_amax(const uint16_t* x, int64_t G, int N, int D, const float* mea
   return a;
 }
 
-// delta_j cs for the N keys of one head: qmean [D]; k [N][D] bf16; kmean [D]
+// delta_j for the N keys of one head: qmean [D]; k [N][D] bf16; kmean [D]
 // (NULL: K not smoothed).
-void score_bias(const float* qmean, const uint16_t* k, const float* kmean, int N, int D, float cs,
+void score_bias(const float* qmean, const uint16_t* k, const float* kmean, int N, int D,
                 float* out) {
   for (int64_t j = 0; j < N; ++j) {
     float delta = 0.0f;
@@ -326,7 +346,7 @@ void score_bias(const float* qmean, const uint16_t* k, const float* kmean, int N
       if (kmean) kv = kv - kmean[d];
       delta = std::fmaf(qmean[d], kv, delta);
     }
-    out[j] = delta * cs;
+    out[j] = delta;
   }
 }
 
@@ -337,7 +357,7 @@ struct Tensors {
   bool fp8v;                   // V in FP8 (flag 16): sv, dv are s8, d8
   const float* qmean = nullptr;  // flag 64: [B*H][D]
   const float* kmean = nullptr;  // flag 32: [B*Hkv][D]
-  const float* bias = nullptr;   // flag 64: [B*H][N], delta_j cs
+  const double* bias = nullptr;  // flag 64: [B*H][N], beta'_j (contraction units)
 };
 
 // K and V of one (b, kv-head), dequantised to contraction units, [N][D].
@@ -529,7 +549,7 @@ void efq_tile(const std::vector<float>& x, const std::vector<double>& A, double 
 // One query row: the tiled forward over key tiles of Bc keys.
 //   S_ij = fl32(exact dot product of dequantised q_i, k_j)
 //   x_ij = fl32(S_ij * c), c = fl32(fl32(fl32(d_Q d_K) * softmax_scale) * log2 e)
-//          (flag 64: fl32(S_ij * c + bias_j) with one rounding)
+//          (flag 64: S_ij + beta'_j, exact, before the rounding to fp32)
 //   masked (causal j > i, top-left aligned) -> -inf
 // per tile: m_new = max(m, max_j x_ij); alpha = exp2(m - m_new) (0 while m is -inf)
 //   p_ij = fl32(exp2(x_ij - m_new)) (double exp2, rounded once)
@@ -563,7 +583,7 @@ void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float 
   std::vector<uint8_t> qc(D / 2), qs(D / 16);
   quantize_rows(qrow, 1, D, T.sq, qc.data(), qs.data(), 1,
                 T.qmean ? T.qmean + ((int64_t)b * T.H + h) * D : nullptr);
-  const float* brow = T.bias ? T.bias + ((int64_t)b * T.H + h) * N : nullptr;
+  const double* brow = T.bias ? T.bias + ((int64_t)b * T.H + h) * N : nullptr;
   std::vector<double> qd(D);
   for (int d = 0; d < D; ++d) {
     uint8_t byte = qc[d / 2];
@@ -596,8 +616,12 @@ void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float 
         for (int d = 0; d < D; ++d) s += qd[d] * kr[d];
         if (want_flip)
           for (int d = 0; d < D; ++d) aj += std::fabs(qd[d] * kr[d]);
+        if (brow) {  // the correction joins the accumulated sum, one rounding
+          s += brow[j];
+          aj += std::fabs(brow[j]);
+        }
         float sf = (float)s;
-        xv = brow ? std::fmaf(sf, c, brow[j]) : sf * c;
+        xv = sf * c;
       }
       x[j - j0] = xv;
       A[j - j0] = aj;
@@ -905,8 +929,11 @@ float ora_smoothed_amax(const uint16_t* x, int64_t G, int N, int D, const float*
   return smoothed_amax(x, G, N, D, mean);
 }
 void ora_score_bias(const float* qmean, const uint16_t* k, const float* kmean, int N, int D,
-                    float cs, float* out) {
-  score_bias(qmean, k, kmean, N, D, cs, out);
+                    float* out) {
+  score_bias(qmean, k, kmean, N, D, out);
+}
+void ora_bias_split(float delta, float sqsk, float* hi, float* lo) {
+  bias_split(delta, sqsk, hi, lo);
 }
 
 void ora_quantize_tokens_T(const uint16_t* x, int N, int D, float s_enc, uint8_t* codes,
@@ -1097,7 +1124,8 @@ int ora_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B,
   Tensors T{q, k, v, B, H, Hkv, N, D, 0, 0, 0, 0, 0, 0, (flags & FLAG_FP8PV) != 0};
   if (!(softmax_scale > 0.0f)) softmax_scale = 1.0f / std::sqrt((float)D);
   const int64_t Gq = (int64_t)B * H, Gk = (int64_t)B * Hkv;
-  std::vector<float> qmean, kmean, bias;
+  std::vector<float> qmean, kmean, delta;
+  std::vector<double> bias;
   float amax_q = amax_bf16(q, Gq * N * D), amax_k = amax_bf16(k, Gk * N * D);
   if (flags & FLAG_SMOOTH_K) {
     kmean.resize((size_t)(Gk * D));
@@ -1110,17 +1138,25 @@ int ora_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B,
     for (int64_t g = 0; g < Gq; ++g) channel_mean(q + g * N * D, N, D, amax_q, &qmean[g * D]);
     amax_q = smoothed_amax(q, Gq, N, D, qmean.data());
     T.qmean = qmean.data();
-    const float cs = softmax_scale * kLog2e;
-    bias.resize((size_t)(Gq * N));
+    delta.resize((size_t)(Gq * N));
     parallel_for(Gq, nthreads, [&](int64_t g) {
       const int64_t gk = (g / H) * Hkv + (g % H) / (H / Hkv);
-      score_bias(&qmean[g * D], k + gk * N * D, T.kmean ? T.kmean + gk * D : nullptr, N, D, cs,
-                 &bias[g * N]);
+      score_bias(&qmean[g * D], k + gk * N * D, T.kmean ? T.kmean + gk * D : nullptr, N, D,
+                 &delta[g * N]);
     });
-    T.bias = bias.data();
   }
   tensor_scale(amax_q, &T.sq, &T.dq);
   tensor_scale(amax_k, &T.sk, &T.dk);
+  if (flags & FLAG_SMOOTH_Q) {
+    const float sqsk = T.sq * T.sk;
+    bias.resize(delta.size());
+    for (size_t u = 0; u < delta.size(); ++u) {
+      float hi, lo;
+      bias_split(delta[u], sqsk, &hi, &lo);
+      bias[u] = (double)hi + (double)lo;
+    }
+    T.bias = bias.data();
+  }
   if (T.fp8v)
     fp8_tensor_scale(amax_bf16(v, (int64_t)B * Hkv * N * D), &T.sv, &T.dv);
   else
