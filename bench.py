@@ -38,8 +38,8 @@ L2_BYTES = 126 * 1024 * 1024
 # workload, from ncu (dram__bytes_read.sum + dram__bytes_write.sum, one pass;
 # profiles/attn_fwd_traffic_video_dit.md). They hold only for the kernel source
 # they were taken on, identified by its hash; otherwise traffic is reported null.
-ATTN_TRAFFIC = {"workload": "video_dit", "bytes": 170.08e6 + 155.86e6,
-                "attn_fwd_sha256": "d1f520670fe34a2b5a5f613a5ed9f996b304785a670cef48f4dabe1994c93bd4"}
+ATTN_TRAFFIC = {"workload": "video_dit", "bytes": 170.74e6 + 155.99e6,
+                "attn_fwd_sha256": "4ba75167b948effd1fcb7ab048793bbf8cc2c85c9d49ceb35ec10c49dfc001c0"}
 
 
 def parse():
@@ -392,7 +392,7 @@ def main():
         qmean = fa.fp4_channel_mean(q, fa.fp4_amax(q))
         kq = fa.fp4_quantize_smoothed(k, kmean, fa.fp4_amax_smoothed(k, kmean))
         qq = fa.fp4_quantize_smoothed(q, qmean, fa.fp4_amax_smoothed(q, qmean))
-        bias = fa.fp4_score_bias(qmean, k, kmean, wl.H)
+        bias = fa.fp4_score_bias(qmean, k, kmean, wl.H, qq.amax, kq.amax)
     else:
         qq = fa.fp4_quantize(q, fa.FP4_BLOCK_ALONG_D)
         kq = fa.fp4_quantize(k, fa.FP4_BLOCK_ALONG_D)

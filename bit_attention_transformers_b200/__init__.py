@@ -129,7 +129,7 @@ def lib():
         L.fp4_amax_smoothed.restype = i32
         L.fp4_quantize_smoothed.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp]
         L.fp4_quantize_smoothed.restype = i32
-        L.fp4_score_bias.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, vp]
+        L.fp4_score_bias.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp]
         L.fp4_score_bias.restype = i32
         L.fp4_attn_fwd_quantized_bias.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                                   f32, vp]
@@ -454,15 +454,16 @@ def fp4_quantize_smoothed(x, mean, amax, stream=None) -> Fp4Tensor:
     return Fp4Tensor(codes, scales, amax, G, N, D, FP4_BLOCK_ALONG_D)
 
 
-def fp4_score_bias(qmean, k, kmean, H: int, softmax_scale: float | None = None, stream=None):
-    """Smoothed Q's score correction [B*H, Npad] fp32: qmean [B*H, D], k
-    [B, Hkv, N, D] bf16, kmean [B*Hkv, D] or None."""
+def fp4_score_bias(qmean, k, kmean, H: int, q_amax, k_amax, stream=None):
+    """Smoothed Q's score correction [B*H, Npad, 8] fp32 (hi, lo, 0...): qmean
+    [B*H, D], k [B, Hkv, N, D] bf16, kmean [B*Hkv, D] or None, q_amax / k_amax
+    the maxima (float32 CUDA, first element) the quantised Q' and K use."""
     import torch
     B, Hkv, N, D = k.shape
     npad = (N + 127) // 128 * 128
-    bias = torch.empty((B * H, npad), dtype=torch.float32, device=k.device)
+    bias = torch.empty((B * H, npad, 8), dtype=torch.float32, device=k.device)
     _check(lib().fp4_score_bias(_ptr(qmean), _ptr(k), None if kmean is None else _ptr(kmean), B, H,
-                                Hkv, N, D, float(softmax_scale or 0.0), _ptr(bias),
+                                Hkv, N, D, _ptr(q_amax), _ptr(k_amax), _ptr(bias),
                                 _stream(stream)))
     return bias
 
@@ -471,7 +472,7 @@ def fp4_attn_fwd_quantized_bias(qq: Fp4Tensor, kq: Fp4Tensor, vq: Fp4Tensor, bia
                                 Hkv: int, causal: bool = False,
                                 softmax_scale: float | None = None, out=None, stream=None):
     """The fused forward on quantised tensors with the per-key score
-    correction bias [B*H, Npad] (exp-then-quantize P)."""
+    correction bias [B*H, Npad, 8] from fp4_score_bias (exp-then-quantize P)."""
     import torch
     N, D = qq.N, qq.D
     if out is None:

@@ -101,7 +101,6 @@ struct AttnParams {
   const float* amax_k;
   const float* amax_v;
   __nv_bfloat16* out;  // [B][H][N][D]
-  const float* bias;   // [B*H][Npad]: per-key score correction (smoothed Q), or unused
   float* lse;          // [B*H][N]: log2 sum_j 2^(x_ij) per row for the backward, or NULL
   int H, Hkv, N, Npad, ntq;
   float softmax_scale;
@@ -111,7 +110,7 @@ struct AttnParams {
 // exp-then-quantize to FP8 E4M3 with V in FP8 as well.
 enum : int { kPgExp = 0, kPgEfq = 1, kPgFp8 = 2 };
 
-template <int D, bool FP8 = false>
+template <int D, bool FP8 = false, bool BIAS = false>
 struct AttnSmem {
   static constexpr int kQ = kBM * D / 2;   // Q codes tile
   static constexpr int kK = kBN * D / 2;   // K codes tile
@@ -130,10 +129,13 @@ struct AttnSmem {
   static constexpr int oPsf = oVsf + kStages * 1024;
   static constexpr int oRed = oPsf + 2 * 1024;  // float [2][128] running max per stream, [2][128] l
   static constexpr int oPtab = oRed + 2048;     // float [128]
-  static constexpr int oBias = oPtab + 512;     // float [kStages][128]: score correction per key
-  static constexpr int oBar = oBias + kStages * 512;  // mbarriers
+  static constexpr int oBar = oPtab + 512;      // mbarriers
   static constexpr int oTmem = oBar + 256;
-  static constexpr int kBytes = oTmem + 16 + 1024;  // + alignment slack
+  // BIAS: the rank-1 score correction, 128 keys x (hi, lo, 0, 0, 0, 0, 0, 0)
+  // tf32 per K stage (32-byte swizzle), and its all-ones A operand
+  static constexpr int oBiasB = (oTmem + 16 + 1023) / 1024 * 1024;
+  static constexpr int oOnesT = oBiasB + kStages * 4096;
+  static constexpr int kBytes = (BIAS ? oOnesT + 4096 : oTmem + 16) + 1024;  // + alignment slack
 };
 
 // Barrier indices (8 bytes each).
@@ -165,19 +167,21 @@ struct TmemCols {
 constexpr float kInv7 = 1.0f / 7.0f;
 constexpr float kRound = 8388608.0f;  // 2^23: x + 2^23 rounds x (0 <= x < 2^22) to an integer
 
-// BIAS: add a per-key fp32 correction to the scores, x = fma(S, c, bias_j)
-// (the smoothed-Q path; exp-then-quantize P only). The key tile's 128 values
-// travel with its V tile, so they stay in shared memory until PV of the tile
-// has completed, after the softmax has read them.
+// BIAS: add a per-key correction beta'_j = hi_j + lo_j (two tf32 values, in the
+// contraction's units) to the S accumulator as a rank-1 tensor-core product,
+// ones[128 x 8] x [hi, lo, 0, ...]^T (kind::tf32, K = 8) after the FP4 MMAs
+// of the tile (the smoothed-Q path; exp-then-quantize P only). The key tile's
+// corrections travel with its K tile (tmB) and the softmax is unchanged.
 // LSE: also write lse = m + log2 l per row (the training forward).
 template <int D, bool CAUSAL, int PG, bool BIAS = false, bool LSE = false>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmB,
+                    const AttnParams p) {
   constexpr bool EFQ = PG == kPgEfq, FP8 = PG == kPgFp8;
   static_assert(!BIAS || PG == kPgExp, "the score correction is built for exp-then-quantize P");
   static_assert(!LSE || PG == kPgExp, "lse is written by the exp-then-quantize forward");
-  using L = AttnSmem<D, FP8>;
+  using L = AttnSmem<D, FP8, BIAS>;
   using TC = TmemCols<EFQ>;
   constexpr uint32_t kColQsf = TC::kQsf, kColKsf = TC::kKsf, kColPsf = TC::kPsf,
                      kColVsf = TC::kVsf, kColL = kColO + D;
@@ -229,6 +233,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const float de = e4m3_to_f32(e);
     ptab[e] = (e >= 127u || de == 0.0f) ? 0.0f : __fdiv_rn(kTensorRange, de);
   }
+  if (BIAS && threadIdx.x >= 128 && threadIdx.x < 384) {
+    // the rank-1 correction's A operand: every row [1, 1, 0, 0 | 1, 1, 0, 0]
+    // (both 16-byte halves alike, so the 32-byte swizzle leaves it unchanged)
+    const int i = threadIdx.x - 128;  // 256 threads x 16 bytes = 4 KB
+    *reinterpret_cast<uint4*>(sm + L::oOnesT + 16 * i) =
+        make_uint4(0x3F800000u, 0x3F800000u, 0u, 0u);
+    fence_proxy_async_smem();
+  }
   if (EFQ && threadIdx.x >= 192 && threadIdx.x < 288) {
     // the all-ones B operand of P~1 (every code 2 = 1.0) and its scales (1.0)
     const int i = threadIdx.x - 192;  // 96 threads x 16 bytes = 1536 bytes
@@ -257,21 +269,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int st = j % kStages;
         const uint32_t pe = ((j / kStages) - 1) & 1;
         if (j >= kStages && !(ok = wait_bar(bar(kBarKEmpty + st), pe))) break;
-        mbar_arrive_expect_tx(bar(kBarKFull + st), L::kK + L::kSfQK);
+        mbar_arrive_expect_tx(bar(kBarKFull + st), L::kK + L::kSfQK + (BIAS ? 4096 : 0));
         tma_load_2d(sb + L::oK + st * L::kK, &tmK, 0, gk * p.Npad + j * kBN, bar(kBarKFull + st));
+        if (BIAS)
+          tma_load_2d(sb + L::oBiasB + st * 4096, &tmB, 0, gq * p.Npad + j * kBN,
+                      bar(kBarKFull + st));
         bulk_load(sb + L::oKsf + st * 1024,
                   p.k_sf + ((int64_t)gk * (p.Npad / kBN) + j) * L::kSfQK, L::kSfQK,
                   bar(kBarKFull + st));
         if (j >= kStages && !(ok = wait_bar(bar(kBarVEmpty + st), pe))) break;
-        mbar_arrive_expect_tx(bar(kBarVFull + st), L::kV + (FP8 ? 0 : 1024) + (BIAS ? 512 : 0));
+        mbar_arrive_expect_tx(bar(kBarVFull + st), L::kV + (FP8 ? 0 : 1024));
         tma_load_2d(sb + L::oV + st * L::kV, &tmV, j * (FP8 ? kBN : kBN / 2), gk * D,
                     bar(kBarVFull + st));
         if (!FP8)
           bulk_load(sb + L::oVsf + st * 1024, p.v_sf + ((int64_t)gk * (p.Npad / 64) + 2 * j) * 512,
                     1024, bar(kBarVFull + st));
-        if (BIAS)
-          bulk_load(sb + L::oBias + st * 512, p.bias + (int64_t)gq * p.Npad + j * kBN, 512,
-                    bar(kBarVFull + st));
       }
     }
   } else if (warp == 1 || warp == 2) {
@@ -299,6 +311,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mma_mxf4nvf4(tmem + kColS + (t & 1) * kBN, smem_desc(sb + L::oQ + 32 * kc, 16, kSboQK, kSw),
                          smem_desc(sb + L::oK + st * L::kK + 32 * kc, 16, kSboQK, kSw), kIdS,
                          tQsf + 4 * kc, tKsf + 4 * kc, kc > 0 ? 1u : 0u);
+          if constexpr (BIAS)  // S += ones x (hi + lo)^T: the correction, in the same accumulator
+            mma_tf32(tmem + kColS + (t & 1) * kBN, smem_desc(sb + L::oOnesT, 16, 256, 6),
+                     smem_desc(sb + L::oBiasB + st * 4096, 16, 256, 6), idesc_tf32(kBM, kBN), 1u);
           tc_commit(bar(kBarSFull + (t & 1)));
           tc_commit(bar(kBarKEmpty + st));
           return true;
@@ -375,10 +390,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const float sq = tensor_senc(*p.amax_q), sk = tensor_senc(*p.amax_k),
                 sv = FP8 ? fp8_senc(*p.amax_v) : tensor_senc(*p.amax_v);
     const float dq = __fdiv_rn(1.0f, sq), dk = __fdiv_rn(1.0f, sk), dv = __fdiv_rn(1.0f, sv);
-    const float c_s = __fmul_rn(__fmul_rn(__fmul_rn(dq, dk), p.softmax_scale), kLog2e);
-    // with the score correction x = fma(S, c_s, bias) is formed first and the
-    // steps below take x with the unit multiplier
-    const float c = BIAS ? 1.0f : c_s;
+    const float c = __fmul_rn(__fmul_rn(__fmul_rn(dq, dk), p.softmax_scale), kLog2e);
     // d_P d_V; with FP8 P the row sum is kept in units of 256 p, so d_V alone
     const float fpv = FP8 ? dv : __fmul_rn(__fdiv_rn(1.0f, kTensorRange), dv);
     const uint64_t c2 = pk(c, c);
@@ -405,20 +417,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int i = 0; i < kBN; ++i)
           if (key0 + i >= p.N || (CAUSAL && key0 + i > qrow)) s[i] = -INFINITY;
-      }
-      if constexpr (BIAS) {
-        // the tile's corrections arrived with its V tile (same stage and phase)
-        if (ok)
-          ok = __all_sync(0xFFFFFFFFu, wait_bar(bar(kBarVFull + t % kStages), (t / kStages) & 1));
-        const float4* bb = reinterpret_cast<const float4*>(sm + L::oBias + (t % kStages) * 512);
-        const uint64_t cs2 = pk(c_s, c_s);
-#pragma unroll
-        for (int i4 = 0; i4 < kBN / 4; ++i4) {
-          const float4 b4 = bb[i4];
-          upk(fma2(pk(s[4 * i4], s[4 * i4 + 1]), cs2, pk(b4.x, b4.y)), s[4 * i4], s[4 * i4 + 1]);
-          upk(fma2(pk(s[4 * i4 + 2], s[4 * i4 + 3]), cs2, pk(b4.z, b4.w)), s[4 * i4 + 2],
-              s[4 * i4 + 3]);
-        }
       }
       float bm[8];
 #pragma unroll

@@ -50,7 +50,7 @@ int g_num_sms[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 using AttnKernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
-                            const fp4::AttnParams);
+                            const CUtensorMap, const fp4::AttnParams);
 
 template <int PG>
 AttnKernel attn_kernel_pg(int D, int causal) {
@@ -82,8 +82,10 @@ AttnKernel attn_kernel(int D, int causal, int pg, bool bias = false, bool lse = 
   return attn_kernel_pg<fp4::kPgExp>(D, causal);
 }
 
-int attn_smem_bytes(int D, int pg) {
+int attn_smem_bytes(int D, int pg, bool bias = false) {
   if (pg == fp4::kPgFp8) return D == 128 ? fp4::AttnSmem<128, true>::kBytes : fp4::AttnSmem<64, true>::kBytes;
+  if (bias)
+    return D == 128 ? fp4::AttnSmem<128, false, true>::kBytes : fp4::AttnSmem<64, false, true>::kBytes;
   return D == 128 ? fp4::AttnSmem<128>::kBytes : fp4::AttnSmem<64>::kBytes;
 }
 
@@ -121,7 +123,7 @@ fp4_status_t device_setup(int* dev_out, int* sms_out) {
         for (int pg = 0; pg < 5; ++pg)  // 3: with the score correction, 4: writing lse
           FP4_CUDA(cudaFuncSetAttribute(attn_kernel(d ? 128 : 64, causal, pg % 3, pg == 3, pg == 4),
                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        attn_smem_bytes(d ? 128 : 64, pg % 3)));
+                                        attn_smem_bytes(d ? 128 : 64, pg % 3, pg == 3)));
     for (int d = 0; d < 2; ++d)
       for (int causal = 0; causal < 2; ++causal) {
         FP4_CUDA(cudaFuncSetAttribute(bwd_dq_kernel_for(d ? 128 : 64, causal),
@@ -210,7 +212,7 @@ WsLayout ws_layout(int B, int H, int Hkv, int N, int D, bool fp8v = false, bool 
   w.sums = take(smooth ? (size_t)((Gq + Gk) * D * 8) : 0);
   w.qmean = take(smooth ? (size_t)(Gq * D * 4) : 0);
   w.kmean = take(smooth ? (size_t)(Gk * D * 4) : 0);
-  w.bias = take(smooth ? (size_t)(Gq * Npad * 4) : 0);
+  w.bias = take(smooth ? (size_t)(Gq * Npad * 32) : 0);  // (hi, lo, 0 x 6) per key
   w.total = off;
   return w;
 }
@@ -350,21 +352,21 @@ fp4_status_t launch_amax_smoothed(const void* x, int64_t G, int N, int D, const 
   return FP4_OK;
 }
 
-// Q's score correction bias [B*H][Npad].
+// Q's score correction bias [B*H][Npad][8] (hi, lo, 0 ...), with the maxima
+// the quantised Q' and K were encoded with.
 fp4_status_t launch_score_bias(const float* qmean, const void* k, const float* kmean, int B, int H,
-                               int Hkv, int N, int D, float softmax_scale, float* bias,
-                               cudaStream_t stream) {
+                               int Hkv, int N, int D, const float* amax_q, const float* amax_k,
+                               float* bias, cudaStream_t stream) {
   const int64_t Npad = round_up(N, 128);
   if ((int64_t)B * Hkv > 65535) return fail(FP4_ERR_INVALID_ARG, "more than 65535 key/value heads");
   dim3 grid((unsigned)(Npad / 128), (unsigned)(B * Hkv));
-  const float sc = resolve_scale(softmax_scale, D);
   const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
   if (D == 128)
-    fp4::score_bias_kernel<128><<<grid, 128, 0, stream>>>(qmean, kb, kmean, H, Hkv, N, (int)Npad, sc,
-                                                          bias);
+    fp4::score_bias_kernel<128><<<grid, 128, 0, stream>>>(qmean, kb, kmean, H, Hkv, N, (int)Npad,
+                                                          amax_q, amax_k, bias);
   else
-    fp4::score_bias_kernel<64><<<grid, 128, 0, stream>>>(qmean, kb, kmean, H, Hkv, N, (int)Npad, sc,
-                                                         bias);
+    fp4::score_bias_kernel<64><<<grid, 128, 0, stream>>>(qmean, kb, kmean, H, Hkv, N, (int)Npad,
+                                                         amax_q, amax_k, bias);
   FP4_CUDA(cudaGetLastError());
   return FP4_OK;
 }
@@ -395,9 +397,13 @@ fp4_status_t launch_attn(const uint8_t* qc, const uint8_t* qs, const float* qa, 
   const int64_t Gq = (int64_t)B * H, Gk = (int64_t)B * Hkv;
   const CUtensorMapSwizzle swQK =
       D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, tb;
+  std::memset(&tb, 0, sizeof(tb));
   fp4_status_t s;
   if ((s = tmap_2d(&tq, qc, D / 2, Gq * Npad, D / 2, 128, swQK)) != FP4_OK) return s;
+  // the rank-1 correction: 128 keys x 32 bytes per K tile, 32-byte swizzle
+  if (bias && (s = tmap_2d(&tb, bias, 32, Gq * Npad, 32, 128, CU_TENSOR_MAP_SWIZZLE_32B)) != FP4_OK)
+    return s;
   if ((s = tmap_2d(&tk, kc, D / 2, Gk * Npad, D / 2, 128, swQK)) != FP4_OK) return s;
   if (pg == fp4::kPgFp8) {  // E4M3 V^T: 128 one-byte keys per row, 128-byte swizzle
     if ((s = tmap_2d(&tv, vc, Npad, Gk * D, 128, D, CU_TENSOR_MAP_SWIZZLE_128B)) != FP4_OK)
@@ -418,16 +424,14 @@ fp4_status_t launch_attn(const uint8_t* qc, const uint8_t* qs, const float* qa, 
   p.N = N;
   p.Npad = (int)Npad;
   p.ntq = (int)(Npad / 128);
-  p.bias = bias;
   p.lse = lse;
   p.softmax_scale = resolve_scale(softmax_scale, D);
   dim3 grid(p.ntq, H, B);
   if ((bias || lse) && pg != fp4::kPgExp)
     return fail(FP4_ERR_UNSUPPORTED, "the score correction and lse need exp-then-quantize P");
   if (bias && lse) return fail(FP4_ERR_UNSUPPORTED, "lse with the score correction");
-  attn_kernel(D, causal, pg, bias != nullptr, lse != nullptr)<<<grid, fp4::kAttnThreads,
-                                                                attn_smem_bytes(D, pg), stream>>>(
-      tq, tk, tv, p);
+  attn_kernel(D, causal, pg, bias != nullptr, lse != nullptr)<<<
+      grid, fp4::kAttnThreads, attn_smem_bytes(D, pg, bias != nullptr), stream>>>(tq, tk, tv, tb, p);
   FP4_CUDA(cudaGetLastError());
   return FP4_OK;
 }
@@ -514,7 +518,7 @@ fp4_status_t attn_fwd_smooth_any(const void* q, const void* k, const void* v, vo
   if (smooth & 2) {
     if ((s = launch_mean(q, Gq, N, D, amax, sums, qmean, st)) != FP4_OK) return s;
     if ((s = launch_amax_smoothed(q, Gq, N, D, qmean, amax + 3, sms, st)) != FP4_OK) return s;
-    if ((s = launch_score_bias(qmean, k, kmean_used, B, H, Hkv, N, D, softmax_scale, bias, st)) !=
+    if ((s = launch_score_bias(qmean, k, kmean_used, B, H, Hkv, N, D, amax + 3, ak, bias, st)) !=
         FP4_OK)
       return s;
     aq = amax + 3;
@@ -747,17 +751,18 @@ fp4_status_t fp4_quantize_smoothed(const void* x, int G, int N, int D, const flo
 }
 
 fp4_status_t fp4_score_bias(const float* qmean, const void* k, const float* kmean, int B, int H,
-                            int Hkv, int N, int D, float softmax_scale, float* bias,
-                            void* stream) {
+                            int Hkv, int N, int D, const float* q_amax, const float* k_amax,
+                            float* bias, void* stream) {
   g_last_error.clear();
   fp4_status_t s;
   if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
-  if (!qmean || !k || !bias) return fail(FP4_ERR_INVALID_ARG, "null pointer");
-  if (!aligned16(qmean) || !aligned16(k) || !aligned16(bias) || (kmean && !aligned16(kmean)))
-    return fail(FP4_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (!qmean || !k || !bias || !q_amax || !k_amax) return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(qmean) || !aligned16(k) || !aligned16(bias) || (kmean && !aligned16(kmean)) ||
+      (reinterpret_cast<uintptr_t>(q_amax) & 3u) || (reinterpret_cast<uintptr_t>(k_amax) & 3u))
+    return fail(FP4_ERR_INVALID_ARG, "pointers must be 16-byte aligned (maxima 4-byte)");
   int dev, sms;
   if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
-  return launch_score_bias(qmean, k, kmean, B, H, Hkv, N, D, softmax_scale, bias,
+  return launch_score_bias(qmean, k, kmean, B, H, Hkv, N, D, q_amax, k_amax, bias,
                            static_cast<cudaStream_t>(stream));
 }
 

@@ -146,6 +146,22 @@ __device__ __forceinline__ void mma_f8e4m3(uint32_t d_tmem, uint64_t a_desc, uin
       : "memory");
 }
 
+// Instruction descriptor of kind::tf32 (A and B tf32, both K-major), fp32 D, K = 8.
+__host__ __device__ constexpr uint32_t idesc_tf32(uint32_t M, uint32_t N) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, tf32 operands (fp32 containers).
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on bar when every tcgen05 operation this thread issued before completes.
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile(

@@ -283,9 +283,12 @@ __global__ void __launch_bounds__(128) quant_fp8_tokens_T_kernel(const __nv_bflo
 //   max |x'| over the whole smoothed tensor.
 //   K: the correction -q_i . mean_K is the same for every key of a row and
 //   cancels in the softmax. Q: the correction mean_Q . k'_j depends on the key;
-//   it is added to the scores: bias_j = fl32(delta_j fl32(softmax_scale log2 e)),
-//   delta_j an fp32 fma chain over d = 0 .. D-1 from 0, k' = fl32(k - mean_K)
-//   when K is smoothed, else k; x_ij = fma(S'_ij, c, bias_j).
+//   delta_j is an fp32 fma chain over d = 0 .. D-1 from 0 (k' = fl32(k -
+//   mean_K) when K is smoothed, else k), taken to the contraction's units,
+//   beta_j = fl32(delta_j fl32(s_Q s_K)), and split into two tf32 parts
+//   hi = tf32_rz(beta), lo = tf32_rz(fl32(beta - hi)) (the low 13 mantissa bits
+//   cleared) that the fused kernel adds to the S accumulator as a rank-1
+//   tensor-core product: S'' = S' + hi + lo before the scores are scaled.
 
 constexpr int kMeanGridBits = 44;
 
@@ -394,24 +397,27 @@ __global__ void __launch_bounds__(256) amax_smoothed_kernel(const __nv_bfloat16*
   }
 }
 
-// Q's score correction: bias [B*H][Npad] with bias_j = fl32(delta_j cs) for
-// keys j < N (0 beyond), delta_j = fma chain of qmean [B*H][D] with k'_j
-// (k [B*Hkv][N][D]; k' = fl32(k - kmean) when kmean [B*Hkv][D] is given).
-// Grid (Npad / 128, B * Hkv); thread = key, looping over the key/value head's
-// G = H / Hkv query heads.
+// Q's score correction: bias [B*H][Npad][8] fp32 with (hi_j, lo_j, 0, 0, 0,
+// 0, 0, 0) for keys j < N (0 beyond), from delta_j = fma chain of qmean
+// [B*H][D] with k'_j (k [B*Hkv][N][D]; k' = fl32(k - kmean) when kmean
+// [B*Hkv][D] is given) and the encode scales of the quantised Q' and K
+// (their maxima *amax_q, *amax_k). Grid (Npad / 128, B * Hkv); thread = key,
+// looping over the key/value head's G = H / Hkv query heads.
 constexpr float kLog2e = 1.44269504088896340736f;  // fl32(1 / ln 2)
+constexpr uint32_t kTf32Mask = 0xFFFFE000u;        // sign, exponent, 10 mantissa bits
 template <int D>
 __global__ void __launch_bounds__(128) score_bias_kernel(const float* __restrict__ qmean,
                                                          const __nv_bfloat16* __restrict__ k,
                                                          const float* __restrict__ kmean, int H,
                                                          int Hkv, int N, int Npad,
-                                                         float softmax_scale,
+                                                         const float* __restrict__ amax_q,
+                                                         const float* __restrict__ amax_k,
                                                          float* __restrict__ bias) {
   const int64_t gk = blockIdx.y;
   const int j = blockIdx.x * 128 + threadIdx.x;
   const int G = H / Hkv;
   const int64_t gq0 = (gk / Hkv) * H + (gk % Hkv) * G;
-  const float cs = __fmul_rn(softmax_scale, kLog2e);
+  const float sqsk = __fmul_rn(tensor_senc(*amax_q), tensor_senc(*amax_k));
   float kv[D];
   if (j < N) {
 #pragma unroll
@@ -422,15 +428,19 @@ __global__ void __launch_bounds__(128) score_bias_kernel(const float* __restrict
     }
   }
   for (int g2 = 0; g2 < G; ++g2) {
-    float r = 0.0f;
+    uint32_t hi = 0u, lo = 0u;
     if (j < N) {
       const float* qm = qmean + (gq0 + g2) * D;
       float delta = 0.0f;
 #pragma unroll
       for (int d = 0; d < D; ++d) delta = __fmaf_rn(__ldg(qm + d), kv[d], delta);
-      r = __fmul_rn(delta, cs);
+      const float beta = __fmul_rn(delta, sqsk);
+      hi = __float_as_uint(beta) & kTf32Mask;
+      lo = __float_as_uint(__fsub_rn(beta, __uint_as_float(hi))) & kTf32Mask;
     }
-    bias[(gq0 + g2) * Npad + j] = r;
+    uint4* dst = reinterpret_cast<uint4*>(bias + ((gq0 + g2) * Npad + j) * 8);
+    dst[0] = make_uint4(hi, lo, 0u, 0u);
+    dst[1] = make_uint4(0u, 0u, 0u, 0u);
   }
 }
 

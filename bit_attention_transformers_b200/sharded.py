@@ -108,7 +108,8 @@ def fp4_attn_fwd_sharded(q, k, v, causal: bool = False, softmax_scale: float | N
               fp4_quantize(k, FP4_BLOCK_ALONG_D, stream, amax=amax[1:2]))
         vq = fp4_quantize(v, FP4_BLOCK_ALONG_N_T, stream, amax=amax[2:3])
         if qmean is not None:
-            bias = fp4_score_bias(qmean, k.view(1, gkv, N, D), kmean, gq, softmax_scale, stream)
+            bias = fp4_score_bias(qmean, k.view(1, gkv, N, D), kmean, gq, sm[0:1],
+                                  sm[1:2] if kmean is not None else amax[1:2], stream)
             fp4_attn_fwd_quantized_bias(qq, kq, vq, bias, 1, gq, gkv, causal, softmax_scale,
                                         out=out, stream=stream)
         else:

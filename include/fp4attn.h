@@ -233,10 +233,13 @@ fp4_status_t fp4_quantize_fp8_scaled(const void* x, int G, int N, int D, const f
  *   max |x'| over the whole smoothed tensor.
  *   Smoothing K changes every score of a query row by the same amount, which
  *   the softmax cancels. Smoothing Q leaves the key-dependent term
- *   mean_Q . k'_j, added back to the scores: bias_j = fl32(delta_j * cs),
- *   cs = fl32(softmax_scale * log2(e)), delta_j = a sequential fp32 fma chain
- *   over d = 0..D-1 from 0 of mean_Q[d] * k'_j[d] (k' = fl32(k - mean_K) if K
- *   is smoothed, else k); the fused kernel forms x_ij = fma(S'_ij, c, bias_j).
+ *   mean_Q . k'_j, added back to the scores: delta_j = a sequential fp32 fma
+ *   chain over d = 0..D-1 from 0 of mean_Q[d] * k'_j[d] (k' = fl32(k - mean_K)
+ *   if K is smoothed, else k). In the contraction's units beta_j = fl32(delta_j *
+ *   fl32(s_Q * s_K)) (the encode scales of the quantised Q' and K), split in
+ *   two tf32 parts hi = tf32_rz(beta), lo = tf32_rz(fl32(beta - hi)) (low 13
+ *   mantissa bits cleared); the fused kernel adds hi + lo to the S
+ *   accumulator as a rank-1 tensor-core product before the scores are scaled.
  */
 #define FP4_SMOOTH_K 1
 #define FP4_SMOOTH_Q 2
@@ -263,11 +266,12 @@ fp4_status_t fp4_attn_fwd_smooth(const void* q, const void* k, const void* v, vo
  * fp4_quantize_smoothed: NVFP4 codes and scales (FP4_BLOCK_ALONG_D layouts) of
  *   fl32(x - mean) with the tensor scale 2688 / *amax (amax of the smoothed
  *   tensor, device memory, read only).
- * fp4_score_bias: bias [B*H][Npad] fp32 (keys >= N get 0) from qmean
- *   [B*H][D], k [B][Hkv][N][D] bf16 and kmean [B*Hkv][D] (NULL when K is not
- *   smoothed); softmax_scale <= 0 or NaN means 1/sqrt(D).
+ * fp4_score_bias: bias [B*H][Npad][8] fp32, per key (hi, lo, 0, 0, 0, 0, 0,
+ *   0) (keys >= N all 0), from qmean [B*H][D], k [B][Hkv][N][D] bf16, kmean
+ *   [B*Hkv][D] (NULL when K is not smoothed) and the maxima q_amax, k_amax
+ *   (one fp32 each, device) the quantised Q' and K are encoded with.
  * fp4_attn_fwd_quantized_bias: fp4_attn_fwd_quantized (exp-then-quantize P)
- *   with the per-key correction bias [B*H][Npad]: x_ij = fma(S_ij, c, bias_j).
+ *   with that correction: S_ij + hi_j + lo_j before the scores are scaled.
  * Pointers: device memory, 16-byte aligned (amax 4-byte aligned).
  */
 fp4_status_t fp4_channel_mean(const void* x, int G, int N, int D, const float* amax,
@@ -278,8 +282,8 @@ fp4_status_t fp4_quantize_smoothed(const void* x, int G, int N, int D, const flo
                                    const float* amax, uint8_t* codes, uint8_t* scales,
                                    void* stream);
 fp4_status_t fp4_score_bias(const float* qmean, const void* k, const float* kmean, int B, int H,
-                            int Hkv, int N, int D, float softmax_scale, float* bias,
-                            void* stream);
+                            int Hkv, int N, int D, const float* q_amax, const float* k_amax,
+                            float* bias, void* stream);
 fp4_status_t fp4_attn_fwd_quantized_bias(const fp4_tensor_t* q, const fp4_tensor_t* k,
                                          const fp4_tensor_t* v, const float* bias, void* out,
                                          int B, int H, int Hkv, int N, int D, int causal,

@@ -143,7 +143,7 @@ def test_emulated_smoothed_shards_equal_unsharded(syn, case, world):
         qs = fa.fp4_quantize_smoothed(qf[sq], qm, sm[0:1])
         ks = fa.fp4_quantize_smoothed(kf[skv], km, sm[1:2])
         vs = fa.fp4_quantize(vf[skv], fa.FP4_BLOCK_ALONG_N_T, amax=amax[2:3])
-        bias = fa.fp4_score_bias(qm, kf[skv].view(1, gk, N, D), km, gq)
+        bias = fa.fp4_score_bias(qm, kf[skv].view(1, gk, N, D), km, gq, sm[0:1], sm[1:2])
         fa.fp4_attn_fwd_quantized_bias(qs, ks, vs, bias, 1, gq, gk, causal=causal, out=out[sq])
     torch.cuda.synchronize()
     fa.fp4_status()

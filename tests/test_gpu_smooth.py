@@ -69,22 +69,24 @@ def test_score_bias_bit_exact(ora, syn, B, H, Hkv, N, D, smooth_k):
     qmean = bf16_bits_to_f32(syn.normal_bf16(B * H * D, seed=801, scale=3.0)).reshape(B * H, D)
     kmean = (bf16_bits_to_f32(syn.normal_bf16(B * Hkv * D, seed=802, scale=2.0))
              .reshape(B * Hkv, D) if smooth_k else None)
-    scale = 0.0883883461356163
+    amax_q, amax_k = np.float32(7.3125), np.float32(11.5)  # the quantised Q', K maxima
     got = fa.fp4_score_bias(torch.from_numpy(qmean).cuda(), to_dev(k),
                             None if kmean is None else torch.from_numpy(kmean).cuda(), H,
-                            softmax_scale=scale)
+                            torch.tensor([amax_q], device="cuda"), torch.tensor([amax_k], device="cuda"))
     torch.cuda.synchronize()
     fa.fp4_status()
     got = got.cpu().numpy()
-    cs = np.float32(np.float32(scale) * np.float32(1.44269504088896340736))
+    sqsk = np.float32(np.float32(ora.tensor_scale(amax_q)[0]) * np.float32(ora.tensor_scale(amax_k)[0]))
     G = H // Hkv
     for b in range(B):
         for h in range(H):
             gk = b * Hkv + h // G
-            want = ora.score_bias(qmean[b * H + h], k[b, h // G],
-                                  None if kmean is None else kmean[gk], cs)
-            np.testing.assert_array_equal(got[b * H + h, :N].view(np.uint32), want.view(np.uint32))
-            assert not got[b * H + h, N:].any()
+            delta = ora.score_bias(qmean[b * H + h], k[b, h // G],
+                                   None if kmean is None else kmean[gk])
+            want = np.array([ora.bias_split(d, sqsk) for d in delta], np.float32)  # [N, 2]
+            row = got[b * H + h]
+            np.testing.assert_array_equal(row[:N, :2].view(np.uint32), want.view(np.uint32))
+            assert not row[:N, 2:].any() and not row[N:].any()
 
 
 def run_smooth(ora, q, k, v, causal, smooth, label, rows=None):
@@ -149,7 +151,7 @@ def test_steps_compose_to_the_fused_call(syn):
         kq = fa.fp4_quantize_smoothed(k, kmean, fa.fp4_amax_smoothed(k, kmean))
         qq = fa.fp4_quantize_smoothed(q, qmean, fa.fp4_amax_smoothed(q, qmean))
         vq = fa.fp4_quantize(v, fa.FP4_BLOCK_ALONG_N_T)
-        bias = fa.fp4_score_bias(qmean, k, kmean, H)
+        bias = fa.fp4_score_bias(qmean, k, kmean, H, qq.amax, kq.amax)
         got = fa.fp4_attn_fwd_quantized_bias(qq, kq, vq, bias, B, H, Hkv, causal=causal)
         torch.cuda.synchronize()
         fa.fp4_status()
