@@ -120,3 +120,86 @@ def test_gloo_sharded_quantisation_matches_whole(ora, syn, tmp_path, world, B, H
             assert np.array_equal(got, want[skv])
         for u, (c, s) in zip(range(skv.start, skv.stop), res["v"]):
             assert np.array_equal(c, wv[u][0]) and np.array_equal(s, wv[u][1])
+
+
+def _rank_smooth_main(rank, world, port, shapes, arrays, out_dir):
+    """The smoothed sharded path's exchanges: the raw maxima (MAX), the
+    per-head means on the global raw maxima's grid, the smoothed maxima (a
+    second MAX), then the shard's smoothed codes and Q's correction."""
+    import torch
+    import torch.distributed as dist
+    import oracle
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        B, H, Hkv, N, D = shapes
+        q, k = arrays
+        sq, skv = sh.shard_rows(B, H, Hkv, world, rank)
+        qs, ks = q.reshape(B * H, N, D)[sq], k.reshape(B * Hkv, N, D)[skv]
+        amax = torch.tensor([oracle.amax_bf16(t) if t.size else 0.0 for t in (qs, ks)],
+                            dtype=torch.float32)
+        sh.allreduce_max_(amax)
+        qm = np.stack([oracle.channel_mean(x, float(amax[0])) for x in qs]) if qs.size else \
+            np.zeros((0, D), np.float32)
+        km = np.stack([oracle.channel_mean(x, float(amax[1])) for x in ks]) if ks.size else \
+            np.zeros((0, D), np.float32)
+        sm = torch.tensor([oracle.smoothed_amax(qs, qm) if qs.size else 0.0,
+                           oracle.smoothed_amax(ks, km) if ks.size else 0.0], dtype=torch.float32)
+        sh.allreduce_max_(sm)
+        s_q, s_k = oracle.tensor_scale(float(sm[0]))[0], oracle.tensor_scale(float(sm[1]))[0]
+        res = {"sm": sm.numpy(), "q": [], "k": [], "bias": []}
+        for x, m in zip(qs, qm):
+            res["q"].append(oracle.quantize_rows_smoothed(x, s_q, m))
+        for x, m in zip(ks, km):
+            res["k"].append(oracle.quantize_rows_smoothed(x, s_k, m))
+        G = H // Hkv
+        sqsk = np.float32(np.float32(s_q) * np.float32(s_k))
+        for i in range(sq.stop - sq.start):
+            u = i // G  # the shard's key/value head of this query head
+            delta = oracle.score_bias(qm[i], ks[u], km[u])
+            res["bias"].append(np.array([oracle.bias_split(d, sqsk) for d in delta]))
+        np.save(os.path.join(out_dir, f"rank{rank}.npy"), np.array(res, dtype=object),
+                allow_pickle=True)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,B,H,Hkv", [(2, 2, 4, 2), (3, 1, 4, 2)])
+def test_gloo_smoothed_sharding_matches_whole(ora, syn, tmp_path, world, B, H, Hkv):
+    """Smoothing sharded by head: every rank's smoothed codes and Q correction
+    equal the whole tensors' slabs, with two MAX all-reduces (raw maxima for the
+    means' grid, smoothed maxima for the tensor scales)."""
+    import torch.multiprocessing as mp
+    N, D = 40, 32
+    rng = np.random.default_rng(5)
+    q = syn.normal_bf16(B * H * N * D, 21, 0).reshape(B, H, N, D)
+    k = syn.normal_bf16(B * Hkv * N * D, 21, 1, scale=2.0).reshape(B, Hkv, N, D)
+    from _util import bf16_bits_to_f32, f32_to_bf16_bits
+    q = f32_to_bf16_bits(bf16_bits_to_f32(q) + rng.normal(scale=4, size=(B, H, 1, D)).astype(np.float32))
+    k = f32_to_bf16_bits(bf16_bits_to_f32(k) + rng.normal(scale=4, size=(B, Hkv, 1, D)).astype(np.float32))
+    mp.start_processes(_rank_smooth_main, args=(world, _free_port(), (B, H, Hkv, N, D), (q, k),
+                                                str(tmp_path)),
+                       nprocs=world, join=True, start_method="spawn")
+    qf, kf = q.reshape(B * H, N, D), k.reshape(B * Hkv, N, D)
+    aq, ak = ora.amax_bf16(q), ora.amax_bf16(k)
+    qm = np.stack([ora.channel_mean(x, aq) for x in qf])
+    km = np.stack([ora.channel_mean(x, ak) for x in kf])
+    sm = [ora.smoothed_amax(qf, qm), ora.smoothed_amax(kf, km)]
+    s_q, s_k = ora.tensor_scale(sm[0])[0], ora.tensor_scale(sm[1])[0]
+    sqsk = np.float32(np.float32(s_q) * np.float32(s_k))
+    G = H // Hkv
+    for r in range(world):
+        res = np.load(tmp_path / f"rank{r}.npy", allow_pickle=True).item()
+        assert list(res["sm"]) == sm  # the second all-reduce: global smoothed maxima
+        sq, skv = sh.shard_rows(B, H, Hkv, world, r)
+        for i, got in zip(range(sq.start, sq.stop), res["q"]):
+            want = ora.quantize_rows_smoothed(qf[i], s_q, qm[i])
+            assert np.array_equal(got[0], want[0]) and np.array_equal(got[1], want[1])
+            delta = ora.score_bias(qm[i], kf[(i // H) * Hkv + (i % H) // G], km[(i // H) * Hkv + (i % H) // G])
+            wb = np.array([ora.bias_split(d, sqsk) for d in delta])
+            assert np.array_equal(res["bias"][i - sq.start], wb)
+        for u, got in zip(range(skv.start, skv.stop), res["k"]):
+            want = ora.quantize_rows_smoothed(kf[u], s_k, km[u])
+            assert np.array_equal(got[0], want[0]) and np.array_equal(got[1], want[1])
