@@ -92,6 +92,8 @@ class Clocks:
         return self
 
     def __exit__(self, *a):
+        if getattr(self, "lines", None) is not None and self.proc is None:
+            return
         self.lines = []
         if self.proc:
             self.proc.terminate()
@@ -101,6 +103,7 @@ class Clocks:
                 self.proc.kill()
                 out, _ = self.proc.communicate()
             self.lines = [l for l in out.splitlines() if l.strip()]
+            self.proc = None
 
     def summary(self):
         mhz, maxes, reasons = [], [], set()
@@ -376,6 +379,8 @@ def main():
     # clocks sampled from the timed steps through the kernel-only and the
     # end-to-end timing below (10 steps alone last ~0.1 s, under one sample)
     clk = Clocks(local).__enter__()
+    import atexit
+    atexit.register(clk.__exit__, None, None, None)  # the sampler ends even if the run fails
     step_ms = timed(step, args.steps)
     barrier()
     fa.fp4_status()
