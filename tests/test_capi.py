@@ -114,6 +114,34 @@ def test_argument_errors_launch_nothing(L):
     assert L.fp4_attn_fwd_quantized(ctypes.byref(t), ctypes.byref(t), ctypes.byref(t0),
                                     vp(16), 1, 1, 1, 8, 128, 0, 0.0, vp(0)) == \
         fa.FP4_ERR_INVALID_ARG  # NVFP4 V without scales
+    # smoothing: unknown flags, N beyond the exact sums' range, workspace, misaligned maxima
+    need = fa.fp4_attn_workspace_bytes_smooth(1, 1, 1, 8, 128)
+    assert need > fa.fp4_attn_workspace_bytes(1, 1, 1, 8, 128)
+    assert fa.fp4_attn_workspace_bytes_smooth(1, 1, 1, (1 << 19) + 1, 64) == 0
+    smooth = lambda fl, N=8, wsz=1 << 30: L.fp4_attn_fwd_smooth(
+        vp(16), vp(16), vp(16), vp(16), 1, 1, 1, N, 128, 0, 0.0, fl, vp(0), vp(16), wsz)
+    assert smooth(4) == fa.FP4_ERR_INVALID_ARG
+    assert smooth(3, N=(1 << 19) + 1) == fa.FP4_ERR_INVALID_ARG
+    assert smooth(3, wsz=need - 1) == fa.FP4_ERR_WORKSPACE
+    assert L.fp4_channel_mean(vp(16), 1, 8, 128, vp(16), vp(16), vp(0), vp(0)) == \
+        fa.FP4_ERR_INVALID_ARG
+    assert L.fp4_score_bias(vp(16), vp(16), vp(0), 1, 1, 1, 8, 128, vp(18), vp(16), vp(16),
+                            vp(0)) == fa.FP4_ERR_INVALID_ARG
+    assert L.fp4_attn_fwd_quantized_bias(ctypes.byref(t), ctypes.byref(t), ctypes.byref(t),
+                                         vp(0), vp(16), 1, 1, 1, 8, 128, 0, 0.0, vp(0)) == \
+        fa.FP4_ERR_INVALID_ARG
+    # backward: workspace size, null lse, misaligned output, too small a workspace
+    wb = fa.lib().fp4_attn_bwd_workspace_bytes(1, 2, 1, 300, 128)
+    assert wb >= 2 * 384 * 128 * 2 * 4  # Q^, Q^T, dO, dO^T at least
+    assert fa.lib().fp4_attn_bwd_workspace_bytes(1, 3, 2, 300, 128) == 0
+    bwd = lambda lse=16, dq=16, wsz=1 << 34: L.fp4_attn_bwd(
+        vp(16), vp(16), vp(16), vp(16), vp(lse), vp(dq), vp(16), vp(16), 1, 2, 1, 300, 128, 0,
+        0.0, vp(0), vp(16), wsz)
+    assert bwd(lse=0) == fa.FP4_ERR_INVALID_ARG
+    assert bwd(dq=24) == fa.FP4_ERR_INVALID_ARG
+    assert bwd(wsz=wb - 1) == fa.FP4_ERR_WORKSPACE
+    assert L.fp4_attn_fwd_lse(vp(16), vp(16), vp(16), vp(16), vp(0), 1, 1, 1, 8, 128, 0, 0.0,
+                              vp(0), vp(16), 1 << 30) == fa.FP4_ERR_INVALID_ARG
 
 
 def test_product_path_does_not_touch_the_oracle():
