@@ -34,6 +34,16 @@
 // more MMAs per tile multiply P~ by a constant all-ones FP4 tile into 16 TMEM
 // columns beside O (L [256+D, 256+D+16)), so the same rescaling applies to
 // it; the scale columns then start at 400.
+//
+// FP8 variant (PG = kPgFp8) [SageAttention2 abstract, searcharxiv.com author
+// page "Pengle Zhang": P~ and V in FP8]: P~ = E4M3(256 p) per key (no block
+// scales), V in E4M3 with one tensor scale, PV as four kind::f8f6f4 MMAs
+// (K = 32) over 128-byte-swizzled tiles; l sums 256 p.
+// BIAS (smoothed Q, same page): the per-key correction hi + lo (tf32) joins
+// the S accumulator as a rank-1 product ones x [hi, lo]^T (kind::tf32) after
+// the tile's FP4 MMAs; the softmax is unchanged.
+// LSE (the training forward): the epilogue also writes m + log2 l per row.
+//
 // Every wait is bounded (2 s of %globaltimer); on expiry the kernel sets the
 // device error word, stops issuing, drains its tensor-core work and returns.
 #pragma once
