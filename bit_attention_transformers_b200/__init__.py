@@ -39,7 +39,8 @@ EXPORTS = ("fp4_codes_bytes", "fp4_scales_bytes", "fp4_attn_workspace_bytes", "f
            "fp4_attn_fwd_fp8pv", "fp4_attn_fwd_quantized_fp8pv", "fp4_attn_workspace_bytes_smooth",
            "fp4_attn_fwd_smooth", "fp4_channel_mean", "fp4_amax_smoothed", "fp4_quantize_smoothed",
            "fp4_score_bias", "fp4_attn_fwd_quantized_bias", "fp4_attn_fwd_lse",
-           "fp4_attn_bwd_workspace_bytes", "fp4_attn_bwd", "fp4_attn_fwd_noalloc",
+           "fp4_attn_bwd_workspace_bytes", "fp4_attn_bwd", "fp4_attn_bwd_scaled",
+           "fp4_attn_fwd_quantized_lse", "fp4_attn_fwd_noalloc",
            "fp4_status", "fp4_last_error", "fp4_probe_cvt", "fp4_test_wait_timeout")
 FP4_NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -142,6 +143,12 @@ def lib():
         L.fp4_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                    f32, vp, vp, sz]
         L.fp4_attn_bwd.restype = i32
+        L.fp4_attn_bwd_scaled.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                          i32, i32, f32, vp, vp, sz]
+        L.fp4_attn_bwd_scaled.restype = i32
+        L.fp4_attn_fwd_quantized_lse.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                                 f32, vp]
+        L.fp4_attn_fwd_quantized_lse.restype = i32
         L.fp4_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
         L.fp4_attn_fwd_noalloc.restype = i32
         L.fp4_status.argtypes = [vp]
@@ -359,10 +366,11 @@ _ws_bwd: dict = {}
 
 
 def fp4_attn_bwd(q, k, v, dout, lse, causal: bool = False, softmax_scale: float | None = None,
-                 dq=None, dk=None, dv=None, stream=None, ws=None):
+                 dq=None, dk=None, dv=None, stream=None, ws=None, amax=None):
     """The FP4 attention backward (reading in include/fp4attn.h): q, dout [B,H,N,D],
-    k, v [B,Hkv,N,D] bf16 CUDA, lse [B,H,N] from fp4_attn_fwd_lse. Returns
-    (dq, dk, dv) bf16."""
+    k, v [B,Hkv,N,D] bf16 CUDA, lse [B,H,N] from fp4_attn_fwd_lse. With `amax`
+    (float32 CUDA [3]: the maxima of Q, K, V, e.g. combined over shards)
+    fp4_attn_bwd_scaled quantises with them. Returns (dq, dk, dv) bf16."""
     import torch
     B, H, N, D = q.shape
     Hkv = k.shape[1]
@@ -380,6 +388,13 @@ def fp4_attn_bwd(q, k, v, dout, lse, causal: bool = False, softmax_scale: float 
         if ws is None or ws.numel() < need:
             ws = torch.empty(need, dtype=torch.uint8, device=q.device)
             _ws_bwd[key] = ws
+    if amax is not None:
+        assert amax.is_cuda and amax.dtype == torch.float32 and amax.numel() >= 3
+        _check(lib().fp4_attn_bwd_scaled(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lse),
+                                         _ptr(amax), _ptr(dq), _ptr(dk), _ptr(dv), B, H, Hkv, N, D,
+                                         int(bool(causal)), float(softmax_scale or 0.0),
+                                         _stream(stream), _ptr(ws), ws.numel()))
+        return dq, dk, dv
     _check(lib().fp4_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
                               _ptr(dv), B, H, Hkv, N, D, int(bool(causal)),
                               float(softmax_scale or 0.0), _stream(stream), _ptr(ws), ws.numel()))
@@ -507,10 +522,12 @@ def fp4_attn_fwd_noalloc(q, k, v, causal: bool = False, softmax_scale: float | N
 
 def fp4_attn_fwd_quantized(qq: Fp4Tensor, kq: Fp4Tensor, vq: Fp4Tensor, B: int, H: int,
                            Hkv: int, causal: bool = False, softmax_scale: float | None = None,
-                           out=None, stream=None, efq: bool = False, fp8pv: bool = False):
+                           out=None, stream=None, efq: bool = False, fp8pv: bool = False,
+                           lse=None):
     """The fused forward alone on tensors fp4_quantize() produced
     (fp4_attn_fwd_quantized_efq with efq=True; fp4_attn_fwd_quantized_fp8pv
-    with fp8pv=True, vq from fp4_quantize_fp8)."""
+    with fp8pv=True, vq from fp4_quantize_fp8; fp4_attn_fwd_quantized_lse,
+    writing lse [B, H, N] fp32, when lse is given)."""
     import torch
     N, D = qq.N, qq.D
     if out is None:
@@ -520,6 +537,15 @@ def fp4_attn_fwd_quantized(qq: Fp4Tensor, kq: Fp4Tensor, vq: Fp4Tensor, B: int, 
         raise ValueError("vq must come from fp4_quantize_fp8 exactly when fp8pv is set")
     ts = [_Tensor(t.codes.data_ptr(), 0 if t.scales is None else t.scales.data_ptr(),
                   t.amax.data_ptr()) for t in (qq, kq, vq)]
+    if lse is not None:
+        if efq or fp8pv:
+            raise ValueError("lse is written by the exp-then-quantize forward")
+        assert lse.dtype == torch.float32 and lse.is_contiguous()
+        _check(lib().fp4_attn_fwd_quantized_lse(ctypes.byref(ts[0]), ctypes.byref(ts[1]),
+                                                ctypes.byref(ts[2]), _ptr(out), _ptr(lse), B, H,
+                                                Hkv, N, D, int(bool(causal)),
+                                                float(softmax_scale or 0.0), _stream(stream)))
+        return out
     _check(fn(ctypes.byref(ts[0]), ctypes.byref(ts[1]), ctypes.byref(ts[2]), _ptr(out), B, H,
               Hkv, N, D, int(bool(causal)), float(softmax_scale or 0.0), _stream(stream)))
     return out
@@ -619,4 +645,5 @@ def fp4_probe_cvt(start: int, count: int, kind: int, out=None, stream=None):
     return out
 
 
-from .sharded import allreduce_max_, fp4_attn_fwd_sharded, shard_rows, shard_units  # noqa: E402
+from .sharded import (allreduce_max_, fp4_attn_bwd_sharded, fp4_attn_fwd_sharded,  # noqa: E402
+                      shard_rows, shard_units)

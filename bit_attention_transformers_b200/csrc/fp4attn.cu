@@ -537,10 +537,13 @@ fp4_status_t attn_fwd_smooth_any(const void* q, const void* k, const void* v, vo
 
 // The backward (attn_bwd.cuh): pre-kernels, then the dq kernel (D and dQ),
 // then the dk/dv kernel.
+// amax_in: the three tensor maxima (Q, K, V) to quantise with, e.g. combined
+// over shards, or NULL to compute them from q, k, v.
 fp4_status_t attn_bwd_any(const void* q, const void* k, const void* v, const void* dout,
                           const float* lse, void* dq, void* dk, void* dv, int B, int H, int Hkv,
                           int N, int D, int causal, float softmax_scale, void* stream,
-                          void* workspace, size_t workspace_bytes) {
+                          void* workspace, size_t workspace_bytes,
+                          const float* amax_in = nullptr) {
   g_last_error.clear();
   fp4_status_t s;
   if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
@@ -553,15 +556,20 @@ fp4_status_t attn_bwd_any(const void* q, const void* k, const void* v, const voi
   const BwdWs w = bwd_ws_layout(B, H, Hkv, N, D);
   if (workspace_bytes < w.total)
     return fail(FP4_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, w.total);
+  if (amax_in && (reinterpret_cast<uintptr_t>(amax_in) & 3u))
+    return fail(FP4_ERR_INVALID_ARG, "amax must be 4-byte aligned");
   int dev, sms;
   if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* amax = reinterpret_cast<float*>(ws + w.amax);
   const int64_t Npad = round_up(N, 128), Gq = (int64_t)B * H, Gk = (int64_t)B * Hkv;
-  if ((s = launch_amax(q, Gq * N * D, k, Gk * N * D, v, Gk * N * D, amax, amax + 1, amax + 2, sms,
-                       st)) != FP4_OK)
+  if (amax_in) {
+    FP4_CUDA(cudaMemcpyAsync(amax, amax_in, 3 * sizeof(float), cudaMemcpyDeviceToDevice, st));
+  } else if ((s = launch_amax(q, Gq * N * D, k, Gk * N * D, v, Gk * N * D, amax, amax + 1,
+                              amax + 2, sms, st)) != FP4_OK) {
     return s;
+  }
   auto* qh = reinterpret_cast<__nv_bfloat16*>(ws + w.qh);
   auto* qt = reinterpret_cast<__nv_bfloat16*>(ws + w.qt);
   auto* kh = reinterpret_cast<__nv_bfloat16*>(ws + w.kh);
@@ -632,7 +640,7 @@ fp4_status_t attn_bwd_any(const void* q, const void* k, const void* v, const voi
 fp4_status_t attn_fwd_quantized_any(const fp4_tensor_t* q, const fp4_tensor_t* k,
                                     const fp4_tensor_t* v, void* out, int B, int H, int Hkv,
                                     int N, int D, int causal, float softmax_scale, void* stream,
-                                    int pg, const float* bias = nullptr) {
+                                    int pg, const float* bias = nullptr, float* lse = nullptr) {
   g_last_error.clear();
   fp4_status_t s;
   if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
@@ -649,11 +657,13 @@ fp4_status_t attn_fwd_quantized_any(const fp4_tensor_t* q, const fp4_tensor_t* k
   }
   if (!aligned16(out)) return fail(FP4_ERR_INVALID_ARG, "out must be 16-byte aligned");
   if (bias && !aligned16(bias)) return fail(FP4_ERR_INVALID_ARG, "bias must be 16-byte aligned");
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return fail(FP4_ERR_INVALID_ARG, "lse must be 4-byte aligned");
   int dev, sms;
   if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
   return launch_attn(q->codes, q->scales, q->amax, k->codes, k->scales, k->amax, v->codes,
                      v->scales, v->amax, out, B, H, Hkv, N, D, causal, softmax_scale, pg,
-                     static_cast<cudaStream_t>(stream), bias);
+                     static_cast<cudaStream_t>(stream), bias, lse);
 }
 
 }  // namespace
@@ -686,6 +696,31 @@ fp4_status_t fp4_attn_bwd(const void* q, const void* k, const void* v, const voi
                           void* workspace, size_t workspace_bytes) {
   return attn_bwd_any(q, k, v, dout, lse, dq, dk, dv, B, H, Hkv, N, D, causal, softmax_scale,
                       stream, workspace, workspace_bytes);
+}
+
+fp4_status_t fp4_attn_bwd_scaled(const void* q, const void* k, const void* v, const void* dout,
+                                 const float* lse, const float* amax, void* dq, void* dk, void* dv,
+                                 int B, int H, int Hkv, int N, int D, int causal,
+                                 float softmax_scale, void* stream, void* workspace,
+                                 size_t workspace_bytes) {
+  if (!amax) {
+    g_last_error.clear();
+    return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  }
+  return attn_bwd_any(q, k, v, dout, lse, dq, dk, dv, B, H, Hkv, N, D, causal, softmax_scale,
+                      stream, workspace, workspace_bytes, amax);
+}
+
+fp4_status_t fp4_attn_fwd_quantized_lse(const fp4_tensor_t* q, const fp4_tensor_t* k,
+                                        const fp4_tensor_t* v, void* out, float* lse, int B,
+                                        int H, int Hkv, int N, int D, int causal,
+                                        float softmax_scale, void* stream) {
+  if (!lse) {
+    g_last_error.clear();
+    return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  }
+  return attn_fwd_quantized_any(q, k, v, out, B, H, Hkv, N, D, causal, softmax_scale, stream, 0,
+                                nullptr, lse);
 }
 
 fp4_status_t fp4_attn_fwd_lse(const void* q, const void* k, const void* v, void* out, float* lse,

@@ -56,7 +56,7 @@ def allreduce_max_(t, group=None):
 
 def fp4_attn_fwd_sharded(q, k, v, causal: bool = False, softmax_scale: float | None = None,
                          group=None, out=None, stream=None, efq: bool = False,
-                         fp8pv: bool = False, smooth: int = 0):
+                         fp8pv: bool = False, smooth: int = 0, lse=None):
     """This rank's part of a head-sharded NVFP4 attention forward.
 
     q: this rank's query heads, a contiguous bf16 CUDA tensor [..., N, D] whose
@@ -67,7 +67,9 @@ def fp4_attn_fwd_sharded(q, k, v, causal: bool = False, softmax_scale: float | N
     output heads. efq selects the EFQ-Softmax P generation, fp8pv the FP8 P
     and V variant, smooth (FP4_SMOOTH_K | FP4_SMOOTH_Q) Q/K smoothing: the
     means are per head, so local; their grid comes from the global raw
-    maxima, and a second all-reduce (MAX) makes the smoothed maxima global."""
+    maxima, and a second all-reduce (MAX) makes the smoothed maxima global.
+    lse (float32, this rank's Gq * N values): the training forward also
+    writes the rows' lse for fp4_attn_bwd_sharded."""
     import torch
     from . import (FP4_BLOCK_ALONG_D, FP4_BLOCK_ALONG_N_T, FP4_SMOOTH_K, FP4_SMOOTH_Q,
                    fp4_amax, fp4_amax_smoothed, fp4_attn_fwd_quantized,
@@ -75,6 +77,8 @@ def fp4_attn_fwd_sharded(q, k, v, causal: bool = False, softmax_scale: float | N
                    fp4_quantize_smoothed, fp4_score_bias)
     if smooth and (efq or fp8pv):
         raise ValueError("smoothing is built for the exp-then-quantize NVFP4 path")
+    if lse is not None and (smooth or efq or fp8pv):
+        raise ValueError("lse is written by the plain exp-then-quantize forward")
     N, D = q.shape[-2], q.shape[-1]
     if k.shape[-2:] != (N, D) or v.shape != k.shape:
         raise ValueError("q, k, v must share N and D, and k and v their shape")
@@ -125,5 +129,37 @@ def fp4_attn_fwd_sharded(q, k, v, causal: bool = False, softmax_scale: float | N
     else:
         vq = fp4_quantize(v, FP4_BLOCK_ALONG_N_T, stream, amax=amax[2:3])
     fp4_attn_fwd_quantized(qq, kq, vq, 1, gq, gkv, causal, softmax_scale, out=out, stream=stream,
-                           efq=efq, fp8pv=fp8pv)
+                           efq=efq, fp8pv=fp8pv, lse=lse)
     return out
+
+
+def fp4_attn_bwd_sharded(q, k, v, dout, lse, causal: bool = False,
+                         softmax_scale: float | None = None, group=None, dq=None, dk=None,
+                         dv=None, stream=None):
+    """This rank's part of the head-sharded FP4 attention backward: the same
+    units as fp4_attn_fwd_sharded (q, dout, lse: this rank's query heads; k,
+    v: its key/value heads), one all-reduce (MAX) of the three maxima so that
+    the operands are quantised as the whole tensors' are, then fp4_attn_bwd
+    on the shard. Every rank of `group` calls it, an empty shard included.
+    Returns (dq, dk, dv) for the shard."""
+    import torch
+    from . import fp4_amax, fp4_attn_bwd
+    N, D = q.shape[-2], q.shape[-1]
+    gq, gkv = q.numel() // (N * D), k.numel() // (N * D)
+    if (gkv == 0) != (gq == 0) or (gkv and gq % gkv):
+        raise ValueError(f"{gq} query heads for {gkv} key/value heads")
+    amax = torch.zeros(3, dtype=torch.float32, device=q.device)
+    if gkv:
+        fp4_amax(q, amax[0:1], stream)
+        fp4_amax(k, amax[1:2], stream)
+        fp4_amax(v, amax[2:3], stream)
+    allreduce_max_(amax, group)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if gkv == 0:
+        return dq, dk, dv
+    as4 = lambda t: t.view(1, -1, N, D)
+    fp4_attn_bwd(as4(q), as4(k), as4(v), as4(dout), lse.reshape(1, gq, N), causal, softmax_scale,
+                 dq=as4(dq), dk=as4(dk), dv=as4(dv), stream=stream, amax=amax)
+    return dq, dk, dv

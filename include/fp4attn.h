@@ -320,6 +320,23 @@ fp4_status_t fp4_attn_fwd_lse(const void* q, const void* k, const void* v, void*
  * workspace: fp4_attn_bwd_workspace_bytes(B, H, Hkv, N, D) bytes.
  */
 size_t fp4_attn_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D);
+/*
+ * For tensors held in shards (by head, one shard per GPU): the backward with
+ * the three tensor maxima given, amax[3] = {max|q|, max|k|, max|v|} of the
+ * whole tensors (device memory, 4-byte aligned; e.g. each shard's maxima
+ * from fp4_amax combined by max across the shards), so that every shard's
+ * operands are quantised as the whole tensors' are; and the training forward
+ * on quantised tensors (fp4_quantize_scaled with the same maxima) writing lse.
+ */
+fp4_status_t fp4_attn_bwd_scaled(const void* q, const void* k, const void* v, const void* dout,
+                                 const float* lse, const float* amax, void* dq, void* dk, void* dv,
+                                 int B, int H, int Hkv, int N, int D, int causal,
+                                 float softmax_scale, void* stream, void* workspace,
+                                 size_t workspace_bytes);
+fp4_status_t fp4_attn_fwd_quantized_lse(const fp4_tensor_t* q, const fp4_tensor_t* k,
+                                        const fp4_tensor_t* v, void* out, float* lse, int B,
+                                        int H, int Hkv, int N, int D, int causal,
+                                        float softmax_scale, void* stream);
 fp4_status_t fp4_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
                           const float* lse, void* dq, void* dk, void* dv, int B, int H, int Hkv,
                           int N, int D, int causal, float softmax_scale, void* stream,

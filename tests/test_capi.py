@@ -142,6 +142,15 @@ def test_argument_errors_launch_nothing(L):
     assert bwd(wsz=wb - 1) == fa.FP4_ERR_WORKSPACE
     assert L.fp4_attn_fwd_lse(vp(16), vp(16), vp(16), vp(16), vp(0), 1, 1, 1, 8, 128, 0, 0.0,
                               vp(0), vp(16), 1 << 30) == fa.FP4_ERR_INVALID_ARG
+    assert L.fp4_attn_bwd_scaled(vp(16), vp(16), vp(16), vp(16), vp(16), vp(0), vp(16), vp(16),
+                                 vp(16), 1, 2, 1, 300, 128, 0, 0.0, vp(0), vp(16), 1 << 34) == \
+        fa.FP4_ERR_INVALID_ARG  # no maxima
+    assert L.fp4_attn_fwd_quantized_lse(ctypes.byref(t), ctypes.byref(t), ctypes.byref(t), vp(16),
+                                        vp(0), 1, 1, 1, 8, 128, 0, 0.0, vp(0)) == \
+        fa.FP4_ERR_INVALID_ARG  # no lse
+    assert L.fp4_attn_fwd_quantized_lse(ctypes.byref(t), ctypes.byref(t), ctypes.byref(t), vp(16),
+                                        vp(18), 1, 1, 1, 8, 128, 0, 0.0, vp(0)) == \
+        fa.FP4_ERR_INVALID_ARG  # misaligned lse
 
 
 def test_product_path_does_not_touch_the_oracle():

@@ -148,3 +148,65 @@ def test_emulated_smoothed_shards_equal_unsharded(syn, case, world):
     torch.cuda.synchronize()
     fa.fp4_status()
     assert np.array_equal(from_dev(out).reshape(-1), from_dev(ref).reshape(-1))
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_training_pass_one_rank_equals_unsharded(syn, case):
+    """fp4_attn_fwd_sharded with lse and fp4_attn_bwd_sharded on one rank:
+    the same outputs, lse and gradients as fp4_attn_fwd_lse / fp4_attn_bwd."""
+    import torch
+    B, H, Hkv, N, D, causal = case
+    q, k, v, _ = _inputs(syn, B, H, Hkv, N, D, 900)
+    do = to_dev(syn.normal_bf16(B * H * N * D, 901, 4).reshape(B, H, N, D))
+    out, lse = fa.fp4_attn_fwd_lse(q, k, v, causal=causal)
+    grads = fa.fp4_attn_bwd(q, k, v, do, lse, causal=causal)
+    lse_s = torch.empty(B * H * N, dtype=torch.float32, device="cuda")
+    out_s = fa.fp4_attn_fwd_sharded(q.view(B * H, N, D), k.view(B * Hkv, N, D),
+                                    v.view(B * Hkv, N, D), causal=causal, lse=lse_s)
+    grads_s = fa.fp4_attn_bwd_sharded(q.view(B * H, N, D), k.view(B * Hkv, N, D),
+                                      v.view(B * Hkv, N, D), do.view(B * H, N, D), lse_s,
+                                      causal=causal)
+    torch.cuda.synchronize()
+    fa.fp4_status()
+    assert torch.equal(out.view(-1), out_s.view(-1))
+    assert torch.equal(lse.view(-1), lse_s)
+    for a, b in zip(grads, grads_s):
+        assert torch.equal(a.view(-1), b.view(-1))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("case", CASES)
+def test_emulated_training_shards_equal_unsharded(syn, case, world):
+    """The training pass sharded by head, emulated on one GPU: every shard's
+    output, lse and gradients equal its slab of the unsharded pass, bit for
+    bit (the maxima combined by max, as the all-reduce does)."""
+    import torch
+    B, H, Hkv, N, D, causal = case
+    q, k, v, _ = _inputs(syn, B, H, Hkv, N, D, 910 + world)
+    do = to_dev(syn.normal_bf16(B * H * N * D, 911, 4).reshape(B, H, N, D))
+    out, lse = fa.fp4_attn_fwd_lse(q, k, v, causal=causal)
+    gq_, gk_, gv_ = fa.fp4_attn_bwd(q, k, v, do, lse, causal=causal)
+    qf, kf, vf, dof = (t.view(-1, N, D) for t in (q, k, v, do))
+    shards = [fa.shard_rows(B, H, Hkv, world, r) for r in range(world)]
+    shards = [(sq, skv) for sq, skv in shards if skv.stop > skv.start]
+    amax = torch.zeros(3, dtype=torch.float32, device="cuda")
+    for sq, skv in shards:
+        part = torch.stack([fa.fp4_amax(qf[sq]), fa.fp4_amax(kf[skv]), fa.fp4_amax(vf[skv])]).view(3)
+        amax = torch.maximum(amax, part)
+    for sq, skv in shards:
+        g1, g2 = sq.stop - sq.start, skv.stop - skv.start
+        qs = fa.fp4_quantize(qf[sq], fa.FP4_BLOCK_ALONG_D, amax=amax[0:1])
+        ks = fa.fp4_quantize(kf[skv], fa.FP4_BLOCK_ALONG_D, amax=amax[1:2])
+        vs = fa.fp4_quantize(vf[skv], fa.FP4_BLOCK_ALONG_N_T, amax=amax[2:3])
+        lse_s = torch.empty(g1 * N, dtype=torch.float32, device="cuda")
+        out_s = fa.fp4_attn_fwd_quantized(qs, ks, vs, 1, g1, g2, causal=causal, lse=lse_s)
+        as4 = lambda t: t.contiguous().view(1, -1, N, D)
+        d = fa.fp4_attn_bwd(as4(qf[sq]), as4(kf[skv]), as4(vf[skv]), as4(dof[sq]),
+                            lse_s.view(1, g1, N), causal=causal, amax=amax)
+        torch.cuda.synchronize()
+        fa.fp4_status()
+        assert torch.equal(out_s.view(-1), out.view(-1, N, D)[sq].reshape(-1))
+        assert torch.equal(lse_s, lse.view(-1, N)[sq].reshape(-1))
+        assert torch.equal(d[0].view(-1), gq_.view(-1, N, D)[sq].reshape(-1))
+        assert torch.equal(d[1].view(-1), gk_.view(-1, N, D)[skv].reshape(-1))
+        assert torch.equal(d[2].view(-1), gv_.view(-1, N, D)[skv].reshape(-1))
