@@ -1,9 +1,15 @@
-"""NVFP4 (4-bit) FlashAttention forward for B200: Python binding of libfp4attn.
+"""NVFP4 (4-bit) FlashAttention for B200: Python binding of libfp4attn.
 
 A thin ctypes layer over the C ABI in include/fp4attn.h: it marshals torch
 tensors (device memory and streams only) into the library's calls and raises
 on error. Every step of the computation runs in the library's CUDA kernels;
 there is no fallback path. The names are the C ABI's.
+
+Forward: fp4_attn_fwd (P generation: exp-then-quantize, efq=True for
+EFQ-Softmax, fp8pv=True for P and V in FP8; smooth= for Q/K smoothing), the
+steps fp4_quantize / fp4_amax / fp4_quantize_scaled / fp4_attn_fwd_quantized,
+fp4_attn_fwd_host(_many) from host buffers. Training: fp4_attn_fwd_lse and
+fp4_attn_bwd. Several GPUs: fp4_attn_fwd_sharded, fp4_attn_bwd_sharded.
 """
 from __future__ import annotations
 
