@@ -1,5 +1,6 @@
 /*
- * fp4attn: NVFP4 (4-bit) FlashAttention forward on NVIDIA B200 (sm_100a).
+ * fp4attn: NVFP4 (4-bit) FlashAttention on NVIDIA B200 (sm_100a): the forward,
+ * its variants (EFQ-Softmax P, FP8 P and V, Q/K smoothing) and the backward.
  *
  * C ABI. Every pointer argument is a device pointer owned by the caller unless
  * stated otherwise; the library allocates no device memory on any call path,
@@ -63,7 +64,7 @@ typedef enum {
   FP4_OK = 0,
   FP4_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or shape */
   FP4_ERR_UNSUPPORTED = 2, /* head dim not in {64,128}, or the device is not sm_100 */
-  FP4_ERR_WORKSPACE = 3,   /* workspace smaller than fp4_attn_workspace_bytes() */
+  FP4_ERR_WORKSPACE = 3,   /* workspace smaller than the entry's *_workspace_bytes() */
   FP4_ERR_CUDA = 4,        /* a CUDA runtime call failed (message in fp4_last_error) */
   FP4_ERR_TIMEOUT = 5      /* a kernel's bounded wait expired (from fp4_status) */
 } fp4_status_t;
