@@ -72,10 +72,8 @@ def _load():
         lib.ora_channel_mean.restype = None
         lib.ora_smoothed_amax.argtypes = [vp, i64, i32, i32, vp]
         lib.ora_smoothed_amax.restype = f32
-        lib.ora_score_bias.argtypes = [vp, vp, vp, i32, i32, vp]
+        lib.ora_score_bias.argtypes = [vp, vp, vp, i32, i32, vp, vp]
         lib.ora_score_bias.restype = None
-        lib.ora_bias_split.argtypes = [f32, f32, vp, vp]
-        lib.ora_bias_split.restype = None
         lib.ora_quantize_tokens_T.argtypes = [vp, i32, i32, f32, vp, vp, i32]
         lib.ora_quantize_tokens_T.restype = None
         lib.ora_fp8_tensor_scale.argtypes = [f32, vp, vp]
@@ -204,25 +202,21 @@ def smoothed_amax(x_bf16: np.ndarray, means: np.ndarray) -> float:
     return float(_load().ora_smoothed_amax(x.ctypes.data, G, N, D, means.ctypes.data))
 
 
-def bias_split(delta: float, sqsk: float) -> tuple[float, float]:
-    """(hi, lo): the two tf32 parts of beta = fl32(delta sqsk)."""
-    hi, lo = ctypes.c_float(), ctypes.c_float()
-    _load().ora_bias_split(float(delta), float(sqsk), ctypes.byref(hi), ctypes.byref(lo))
-    return hi.value, lo.value
-
-
-def score_bias(qmean, k_bf16: np.ndarray, kmean) -> np.ndarray:
+def score_bias(qmean, k_bf16: np.ndarray, kmean, want_absum: bool = False):
     """Score correction of one query head before its scaling: delta_j = qmean . k'_j
-    (an fp32 fma chain; k' = fl32(k - kmean), or k when kmean is None).
-    k [N, D] bf16 bits; returns N fp32 values."""
+    (k' = fl32(k - kmean), or k when kmean is None), the dot product in double
+    (every product exact). k [N, D] bf16 bits; returns N float64 values, and
+    with want_absum also sum_d |qmean_d k'_jd| per key."""
     k = _c(k_bf16, np.uint16)
     N, D = k.shape
     qmean = _c(qmean, np.float32)
     km = None if kmean is None else _c(kmean, np.float32)
-    out = np.empty(N, dtype=np.float32)
+    out = np.empty(N, dtype=np.float64)
+    mag = np.empty(N, dtype=np.float64)
     _load().ora_score_bias(qmean.ctypes.data, k.ctypes.data,
-                           None if km is None else km.ctypes.data, N, D, out.ctypes.data)
-    return out
+                           None if km is None else km.ctypes.data, N, D, out.ctypes.data,
+                           mag.ctypes.data)
+    return (out, mag) if want_absum else out
 
 
 def quantize_tokens_T(x_bf16: np.ndarray, s_enc: float, npad: int | None = None):

@@ -278,35 +278,17 @@ const float kLog2e = 1.44269504088896340736f;  // fl32(1 / ln 2)
 //   row i, which the softmax cancels: nothing is added back.
 //   Q (flag 64): q_i . k_j = q'_i . k_j + mean_Q . k_j; the second term
 //   depends on the key, so it is added back to the scores:
-//   delta_j = mean_Q . k'_j (k' the smoothed K under flag 32, else K), taken
-//   to the contraction's units, beta_j = fl32(delta_j fl32(s_Q s_K)) (the
-//   encode scales of the quantised Q' and K), and split into two tf32 values
-//   hi_j = tf32_rz(beta_j), lo_j = tf32_rz(fl32(beta_j - hi_j)) (tf32_rz: the
-//   low 13 mantissa bits cleared), beta'_j = hi_j + lo_j; the scores are
-//   x_ij = fl32(fl32(S'_ij + beta'_j) c), the sum exact and rounded once (the
-//   kernel adds beta' to the S accumulator as a rank-1 tensor-core product).
+//   delta_j = mean_Q . k'_j (k' the smoothed K under flag 32, else K), the
+//   dot product itself (each product exact in double, the D terms summed in
+//   double), taken to the contraction's units, beta_j = delta_j s_Q s_K (the
+//   encode scales of the quantised Q' and K, their product exact in double);
+//   the scores are x_ij = fl32(fl32(S'_ij + beta_j) c), S'_ij + beta_j summed
+//   in double and rounded once to fp32.
 // The mean is made independent of summation order so that it is one value on
 // any machine: every element is truncated toward zero to the fixed-point
 // grid 2^-s with s = 44 - E, 2^(E-1) <= amax < 2^E (amax of the raw tensor),
 // the integers are summed exactly (|x| 2^s < 2^44, so N <= 2^19 tokens fit in
 // 64 bits), and mean = fl32(fl64(fl64(T) 2^-s) / N); amax == 0 gives 0.
-// delta_j is a sequential fp32 fma chain over d = 0 .. D-1 from 0.
-const uint32_t kTf32Mask = 0xFFFFE000u;  // tf32: sign, exponent and 10 mantissa bits
-
-float tf32_rz(float x) {
-  uint32_t u;
-  std::memcpy(&u, &x, 4);
-  u &= kTf32Mask;
-  std::memcpy(&x, &u, 4);
-  return x;
-}
-
-// beta' = hi + lo of beta = fl32(delta * sqsk) (see above).
-void bias_split(float delta, float sqsk, float* hi, float* lo) {
-  const float beta = delta * sqsk;
-  *hi = tf32_rz(beta);
-  *lo = tf32_rz(beta - *hi);
-}
 const int kMeanGridBits = 44;
 
 void channel_mean(const uint16_t* x, int N, int D, float amax, float* mean) {
@@ -336,17 +318,20 @@ float smoothed_amax(const uint16_t* x, int64_t G, int N, int D, const float* mea
 }
 
 // delta_j for the N keys of one head: qmean [D]; k [N][D] bf16; kmean [D]
-// (NULL: K not smoothed).
+// (NULL: K not smoothed). absum_j = sum_d |qmean_d k'_jd| (may be NULL).
 void score_bias(const float* qmean, const uint16_t* k, const float* kmean, int N, int D,
-                float* out) {
+                double* delta, double* absum) {
   for (int64_t j = 0; j < N; ++j) {
-    float delta = 0.0f;
+    double acc = 0.0, mag = 0.0;
     for (int d = 0; d < D; ++d) {
       float kv = bf16_to_f32(k[j * D + d]);
       if (kmean) kv = kv - kmean[d];
-      delta = std::fmaf(qmean[d], kv, delta);
+      const double prod = (double)qmean[d] * (double)kv;  // exact: 24 x 24 bits
+      acc += prod;
+      mag += std::fabs(prod);
     }
-    out[j] = delta;
+    delta[j] = acc;
+    if (absum) absum[j] = mag;
   }
 }
 
@@ -357,7 +342,10 @@ struct Tensors {
   bool fp8v;                   // V in FP8 (flag 16): sv, dv are s8, d8
   const float* qmean = nullptr;  // flag 64: [B*H][D]
   const float* kmean = nullptr;  // flag 32: [B*Hkv][D]
-  const double* bias = nullptr;  // flag 64: [B*H][N], beta'_j (contraction units)
+  const double* bias = nullptr;  // flag 64: [B*H][N], beta_j (contraction units)
+  // flag 64: [B*H][N], how far another correct evaluation of beta_j may lie
+  // from it (contraction units; see ora_attn_fwd)
+  const double* bias_unc = nullptr;
 };
 
 // K and V of one (b, kv-head), dequantised to contraction units, [N][D].
@@ -549,7 +537,7 @@ void efq_tile(const std::vector<float>& x, const std::vector<double>& A, double 
 // One query row: the tiled forward over key tiles of Bc keys.
 //   S_ij = fl32(exact dot product of dequantised q_i, k_j)
 //   x_ij = fl32(S_ij * c), c = fl32(fl32(fl32(d_Q d_K) * softmax_scale) * log2 e)
-//          (flag 64: S_ij + beta'_j, exact, before the rounding to fp32)
+//          (flag 64: S_ij + beta_j, exact, before the rounding to fp32)
 //   masked (causal j > i, top-left aligned) -> -inf
 // per tile: m_new = max(m, max_j x_ij); alpha = exp2(m - m_new) (0 while m is -inf)
 //   p_ij = fl32(exp2(x_ij - m_new)) (double exp2, rounded once)
@@ -570,8 +558,9 @@ void efq_tile(const std::vector<float>& x, const std::vector<double>& A, double 
 // like O) to flip[d] (output units), plus eps |out_d| for the continuous
 // change of the denominator. eps is four times the relative
 // uncertainty of p from: S rounding (2^-22 of sum_d |q~_d k~_d|, for the key
-// and for the row maximum), two fp32 roundings of the exponent argument and
-// 2^-21 for the exponential. FLAG_PERTURB_P multiplies each p by
+// and for the row maximum; with flag 64 the sum includes |beta_j|, and the
+// distance of another evaluation of beta_j is added), two fp32 roundings of
+// the exponent argument and 2^-21 for the exponential. FLAG_PERTURB_P multiplies each p by
 // (1 + u eps/4), u uniform in [-1, 1] (seeded by the row), to test the bound.
 void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float c, int Bc,
                  int causal, int flags, double* o_out, double* ml_out, uint16_t* bf_out,
@@ -584,6 +573,7 @@ void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float 
   quantize_rows(qrow, 1, D, T.sq, qc.data(), qs.data(), 1,
                 T.qmean ? T.qmean + ((int64_t)b * T.H + h) * D : nullptr);
   const double* brow = T.bias ? T.bias + ((int64_t)b * T.H + h) * N : nullptr;
+  const double* burow = T.bias_unc ? T.bias_unc + ((int64_t)b * T.H + h) * N : nullptr;
   std::vector<double> qd(D);
   for (int d = 0; d < D; ++d) {
     uint8_t byte = qc[d / 2];
@@ -618,7 +608,9 @@ void row_forward(const Tensors& T, const KVGroup& g, int b, int h, int i, float 
           for (int d = 0; d < D; ++d) aj += std::fabs(qd[d] * kr[d]);
         if (brow) {  // the correction joins the accumulated sum, one rounding
           s += brow[j];
-          aj += std::fabs(brow[j]);
+          // flip bound: the sum's rounding covers |beta_j| too; another
+          // evaluation of beta_j adds its own distance (in units of u)
+          aj += std::fabs(brow[j]) + burow[j] * std::ldexp(1.0, 22);
         }
         float sf = (float)s;
         xv = sf * c;
@@ -929,11 +921,8 @@ float ora_smoothed_amax(const uint16_t* x, int64_t G, int N, int D, const float*
   return smoothed_amax(x, G, N, D, mean);
 }
 void ora_score_bias(const float* qmean, const uint16_t* k, const float* kmean, int N, int D,
-                    float* out) {
-  score_bias(qmean, k, kmean, N, D, out);
-}
-void ora_bias_split(float delta, float sqsk, float* hi, float* lo) {
-  bias_split(delta, sqsk, hi, lo);
+                    double* delta, double* absum) {
+  score_bias(qmean, k, kmean, N, D, delta, absum);
 }
 
 void ora_quantize_tokens_T(const uint16_t* x, int N, int D, float s_enc, uint8_t* codes,
@@ -1124,8 +1113,8 @@ int ora_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B,
   Tensors T{q, k, v, B, H, Hkv, N, D, 0, 0, 0, 0, 0, 0, (flags & FLAG_FP8PV) != 0};
   if (!(softmax_scale > 0.0f)) softmax_scale = 1.0f / std::sqrt((float)D);
   const int64_t Gq = (int64_t)B * H, Gk = (int64_t)B * Hkv;
-  std::vector<float> qmean, kmean, delta;
-  std::vector<double> bias;
+  std::vector<float> qmean, kmean;
+  std::vector<double> delta, absum, bias, bias_unc;
   float amax_q = amax_bf16(q, Gq * N * D), amax_k = amax_bf16(k, Gk * N * D);
   if (flags & FLAG_SMOOTH_K) {
     kmean.resize((size_t)(Gk * D));
@@ -1139,23 +1128,32 @@ int ora_attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B,
     amax_q = smoothed_amax(q, Gq, N, D, qmean.data());
     T.qmean = qmean.data();
     delta.resize((size_t)(Gq * N));
+    absum.resize(delta.size());
     parallel_for(Gq, nthreads, [&](int64_t g) {
       const int64_t gk = (g / H) * Hkv + (g % H) / (H / Hkv);
       score_bias(&qmean[g * D], k + gk * N * D, T.kmean ? T.kmean + gk * D : nullptr, N, D,
-                 &delta[g * N]);
+                 &delta[g * N], &absum[g * N]);
     });
   }
   tensor_scale(amax_q, &T.sq, &T.dq);
   tensor_scale(amax_k, &T.sk, &T.dk);
   if (flags & FLAG_SMOOTH_Q) {
-    const float sqsk = T.sq * T.sk;
+    // beta_j = delta_j s_Q s_K. For the flip bound only: another correct fp32
+    // evaluation of the correction (a D-term fp32 dot product, one fp32
+    // product with fl32(s_Q s_K), and beta carried into the fp32 score sum as
+    // two parts of 11 significant bits each) lies within
+    //   (D + 4) 2^-24 s_Q s_K sum_d |mean_d k'_d| + 2^-20 |beta_j|
+    // of beta_j; bias_unc holds that distance.
+    const double sqsk = (double)T.sq * (double)T.sk;
     bias.resize(delta.size());
+    bias_unc.resize(delta.size());
     for (size_t u = 0; u < delta.size(); ++u) {
-      float hi, lo;
-      bias_split(delta[u], sqsk, &hi, &lo);
-      bias[u] = (double)hi + (double)lo;
+      bias[u] = delta[u] * sqsk;
+      bias_unc[u] = (D + 4) * std::ldexp(1.0, -24) * sqsk * absum[u] +
+                    std::ldexp(1.0, -20) * std::fabs(bias[u]);
     }
     T.bias = bias.data();
+    T.bias_unc = bias_unc.data();
   }
   if (T.fp8v)
     fp8_tensor_scale(amax_bf16(v, (int64_t)B * Hkv * N * D), &T.sv, &T.dv);

@@ -6,19 +6,19 @@ source, at channel_mean): per (batch, head) and channel the mean over the
 head's tokens on a fixed-point grid 2^-(44 - E) (2^(E-1) <= amax < 2^E, each
 element truncated toward zero, the integers summed exactly), x' = fl32(x - mean),
 quantised as usual; K's correction is a per-row constant the softmax cancels;
-Q's is delta_j = mean_Q . k'_j (an fp32 fma chain), taken to the contraction's
-units, beta = fl32(delta fl32(s_Q s_K)), split into two tf32 parts hi + lo
-(mantissas truncated to 10 bits), and added to the scores before their
-rounding: x_ij = fl32(fl32(S'_ij + hi_j + lo_j) c).
+Q's is the dot product delta_j = mean_Q . k'_j, taken to the contraction's
+units, beta_j = delta_j s_Q s_K, and added to the scores before their one
+rounding: x_ij = fl32(fl32(S'_ij + beta_j) c).
 
 Pins: the mean's grid, truncation direction and power-of-two edge by hand; the
 mean within one grid step of the fp64 mean; the smoothed quantiser against the
-pinned block quantiser on numpy fp32 differences; delta against an exact
-rational fma chain; the tf32 split by hand; K-offset invariance of the whole
-forward, bit for bit;
-closed forms where Q's rows are all equal (Q' = 0, the scores are exactly the
-correction), grouped heads included; smoothing lowering the error against
-exact attention when Q and K carry channel offsets.
+pinned block quantiser on numpy fp32 differences; delta against the exact
+rational dot product; smoothing Q leaving the forward unchanged, bit for bit,
+on inputs every step represents exactly (so S' + beta equals the unsmoothed
+score); K-offset invariance of the whole forward, bit for bit; closed forms
+where Q's rows are all equal (Q' = 0, the scores are exactly the correction),
+grouped heads included; smoothing lowering the error against exact attention
+when Q and K carry channel offsets.
 """
 from fractions import Fraction
 
@@ -103,38 +103,86 @@ def test_smoothed_quantiser_and_amax(ora, syn):
 
 
 @pytest.mark.parametrize("smooth_k", [False, True])
-def test_score_bias_is_an_fp32_fma_chain(ora, syn, smooth_k):
+def test_score_bias_is_the_dot_product(ora, syn, smooth_k):
+    """delta_j and sum_d |mean_d k'_jd| against exact rational arithmetic: a
+    double sum of exact products, within D 2^-53 of the magnitude sum."""
     N, D = 9, 32
     k = syn.normal_bf16(N * D, seed=41, scale=3.0).reshape(N, D)
     qmean = bf16_bits_to_f32(syn.normal_bf16(D, seed=42)) * np.float32(1.3)
+    qmean[3] = np.float32(2.0 ** 12 + 1.0)   # a wide exponent spread: the sum needs
+    qmean[5] = np.float32(2.0 ** -14)         # more than fp32's 24 bits
     kmean = (bf16_bits_to_f32(syn.normal_bf16(D, seed=43)) * np.float32(0.7)) if smooth_k else None
-    got = ora.score_bias(qmean, k, kmean)
+    got, mag = ora.score_bias(qmean, k, kmean, want_absum=True)
     kf = bf16_bits_to_f32(k)
     for j in range(N):
         kp = (kf[j] - kmean).astype(np.float32) if smooth_k else kf[j]
-        delta = np.float32(0.0)
-        for d in range(D):
-            delta = fraction_to_f32(Fraction(float(qmean[d])) * Fraction(float(kp[d])) +
-                                    Fraction(float(delta)))
-        assert got[j] == delta, (j, got[j], delta)
+        prods = [Fraction(float(qmean[d])) * Fraction(float(kp[d])) for d in range(D)]
+        exact, absum = sum(prods), sum(abs(t) for t in prods)
+        assert abs(Fraction(got[j]) - exact) <= absum * Fraction(D, 2 ** 53), (j, got[j])
+        assert abs(Fraction(mag[j]) - absum) <= absum * Fraction(D, 2 ** 53), (j, mag[j])
+        # not representable in fp32: the oracle keeps the bits an fp32 sum loses
+        assert Fraction(float(np.float32(got[j]))) != exact
 
 
-def test_bias_split_by_hand(ora):
-    # beta = 1 + 2^-12 + 2^-20: tf32 keeps 10 mantissa bits, hi = 1, lo = 2^-12 (1 + 2^-8)
-    hi, lo = ora.bias_split(1.0 + 2.0 ** -12 + 2.0 ** -20, 1.0)
-    assert (hi, lo) == (1.0, 2.0 ** -12 + 2.0 ** -20)
-    # beta = 3 (1 + 2^-23): the last bits go; hi = 3, lo = tf32(3 2^-23) = 3 2^-23
-    b = float(np.float32(3.0 * (1 + 2.0 ** -23)))
-    hi, lo = ora.bias_split(b, 1.0)
-    assert hi == 3.0 and lo == b - 3.0
-    # negative values truncate toward zero; fl32(delta sqsk) first: -5 * 0.75
-    hi, lo = ora.bias_split(-5.0, 0.75)
-    assert (hi, lo) == (-3.75, 0.0)
-    # a 24-bit mantissa: hi + lo keeps 11 + 11 bits, the rest is dropped (toward zero)
-    m = float(np.float32(1.0 + sum(2.0 ** -i for i in range(1, 24))))  # 2 - 2^-23
-    hi, lo = ora.bias_split(m, 1.0)
-    assert hi == 2.0 - 2.0 ** -10 and lo == float(np.float32(2.0 ** -10 - 2.0 ** -21))
-    assert 0 < m - (hi + lo) < 2.0 ** -20
+def _exact_q_for_smoothing(rng, H, N, D):
+    """Q [1, H, N, D] with channel means m (5.25 on channels 16..31, else 0) such
+    that Q and Q' = Q - m are both exactly representable in NVFP4 with
+    power-of-two tensor scales: every 16-block of a Q' row holds +-5.25 and
+    multiples 0.875 g of E2M1 values g; rows come in pairs q' and -q' (the
+    channel means of Q' are 0), and channels 16..31 of Q' hold only
+    0.875 {0, +-2, +-6} with both +-6 in each row, so Q = Q' + 5.25 there takes
+    0.875 {0, 4, 8, 12}: max |Q| = 10.5 = 2688 / 256, max |Q'| = 5.25 = 2688 / 512."""
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    q = np.zeros((1, H, N, D))
+    for h in range(H):
+        for i in range(0, N, 2):
+            row = np.zeros(D)
+            g0 = rng.choice(grid, size=16) * rng.choice([-1, 1], size=16)
+            g0[rng.integers(16)] = 6 * rng.choice([-1, 1])
+            row[:16] = g0
+            g1 = rng.choice([0, 2, 6], size=16) * rng.choice([-1, 1], size=16)
+            a, b = rng.choice(16, size=2, replace=False)
+            g1[a], g1[b] = 6, -6
+            row[16:32] = g1
+            q[0, h, i], q[0, h, i + 1] = 0.875 * row, -0.875 * row
+    mean = np.zeros(D)
+    mean[16:32] = 5.25
+    return q + mean
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_q_smoothing_is_exact_on_representable_inputs(ora, syn, causal):
+    """When Q, Q' = Q - mean_Q and K are exactly representable in NVFP4 with
+    power-of-two tensor scales, S'_ij + beta_j is the unsmoothed score in the
+    smoothed units (q'_i . k_j + mean_Q . k_j = q_i . k_j), and the two c differ
+    by that same power of two: flag 64 must give the unsmoothed forward bit for
+    bit. A dropped or mis-signed correction, the wrong key, or a missing
+    s_Q s_K factor changes the scores."""
+    H, Hkv, N, D = 2, 1, 64, 32
+    rng = np.random.default_rng(13)
+    q = bf(_exact_q_for_smoothing(rng, H, N, D))
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    k = np.zeros((1, Hkv, N, D))
+    for j in range(N):
+        for b0 in (0, 16):
+            g = rng.choice(grid, size=16) * rng.choice([-1, 1], size=16)
+            g[rng.integers(16)] = 6.0
+            k[0, 0, j, b0:b0 + 16] = 0.875 * g * 2.0 ** -int(rng.integers(0, 3))
+    k[0, 0, 0, :16] = 0.875 * np.where(np.arange(16) == 0, 6.0, 0.0)  # max |K| = 5.25
+    kb = bf(k)
+    v = syn.normal_bf16(Hkv * N * D, seed=17).reshape(1, Hkv, N, D)
+    qf = bf16_bits_to_f32(q).astype(np.float64)
+    assert np.abs(qf).max() == 10.5 and (bf16_bits_to_f32(kb) == k).all()
+    mean = ora.channel_mean(q[0, 0], float(np.abs(qf).max()))
+    assert (mean[16:] == 5.25).all() and (mean[:16] == 0).all()
+    plain = ora.attn_fwd(q, kb, v, causal=causal, want_f64=True)
+    smooth = ora.attn_fwd(q, kb, v, causal=causal, want_f64=True, flags=ora.FLAG_SMOOTH_Q)
+    np.testing.assert_array_equal(smooth["f64"], plain["f64"])
+    np.testing.assert_array_equal(smooth["bf16"], plain["bf16"])
+    # the correction is needed: Q' alone (the same codes, no beta) is different
+    qp = bf(qf - np.concatenate([np.zeros(16), np.full(16, 5.25)]))
+    alone = ora.attn_fwd(qp, kb, v, causal=causal, want_f64=True)
+    assert np.abs(alone["f64"] - plain["f64"]).max() > 1e-3
 
 
 def _unit_cs_scale():

@@ -155,11 +155,10 @@ def _rank_smooth_main(rank, world, port, shapes, arrays, out_dir):
         for x, m in zip(ks, km):
             res["k"].append(oracle.quantize_rows_smoothed(x, s_k, m))
         G = H // Hkv
-        sqsk = np.float32(np.float32(s_q) * np.float32(s_k))
+        sqsk = float(s_q) * float(s_k)
         for i in range(sq.stop - sq.start):
             u = i // G  # the shard's key/value head of this query head
-            delta = oracle.score_bias(qm[i], ks[u], km[u])
-            res["bias"].append(np.array([oracle.bias_split(d, sqsk) for d in delta]))
+            res["bias"].append(oracle.score_bias(qm[i], ks[u], km[u]) * sqsk)
         np.save(os.path.join(out_dir, f"rank{rank}.npy"), np.array(res, dtype=object),
                 allow_pickle=True)
     finally:
@@ -188,7 +187,7 @@ def test_gloo_smoothed_sharding_matches_whole(ora, syn, tmp_path, world, B, H, H
     km = np.stack([ora.channel_mean(x, ak) for x in kf])
     sm = [ora.smoothed_amax(qf, qm), ora.smoothed_amax(kf, km)]
     s_q, s_k = ora.tensor_scale(sm[0])[0], ora.tensor_scale(sm[1])[0]
-    sqsk = np.float32(np.float32(s_q) * np.float32(s_k))
+    sqsk = float(s_q) * float(s_k)
     G = H // Hkv
     for r in range(world):
         res = np.load(tmp_path / f"rank{r}.npy", allow_pickle=True).item()
@@ -198,7 +197,7 @@ def test_gloo_smoothed_sharding_matches_whole(ora, syn, tmp_path, world, B, H, H
             want = ora.quantize_rows_smoothed(qf[i], s_q, qm[i])
             assert np.array_equal(got[0], want[0]) and np.array_equal(got[1], want[1])
             delta = ora.score_bias(qm[i], kf[(i // H) * Hkv + (i % H) // G], km[(i // H) * Hkv + (i % H) // G])
-            wb = np.array([ora.bias_split(d, sqsk) for d in delta])
+            wb = delta * sqsk
             assert np.array_equal(res["bias"][i - sq.start], wb)
         for u, got in zip(range(skv.start, skv.stop), res["k"]):
             want = ora.quantize_rows_smoothed(kf[u], s_k, km[u])
