@@ -34,9 +34,21 @@ def ulp_bf16(x):
     return 2.0 ** (np.floor(np.log2(a)) - 7)
 
 
+FLIP_ROWS_MAX = 1e-3  # at most this fraction of the rows checked may need the flip allowance
+
+
 def compare(gpu_rows, ora, heads, vmax, label):
-    """gpu_rows: uint16 [n, D]; ora: oracle result dict (bf16, f64, flip) of
-    the same rows; heads: [n] head id of each row."""
+    """gpu_rows: uint16 [n, D]; ora: oracle result dict (bf16, f64, flip, ml) of
+    the same rows; heads: [n] head id of each row.
+
+    Every element must lie within 2e-3 max|V| + half a bf16 step + the flip
+    bound of the oracle's unrounded output. The flip bound has a continuous
+    part (eps |out|, the row's p uncertainty moving the denominator; eps is the
+    third column of "ml") and a discrete part (P codes or block scales within
+    their rounding uncertainty of a boundary). Rows that need the discrete part
+    are counted, and their number is capped at FLIP_ROWS_MAX of the rows checked
+    (at least one): a systematic error confined to near-boundary codes would
+    push many rows into the allowance and fail the cap."""
     g = bf16_bits_to_f32(gpu_rows).astype(np.float64)
     o = bf16_bits_to_f32(ora["bf16"]).astype(np.float64)
     f, flip = ora["f64"], ora["flip"]
@@ -45,7 +57,9 @@ def compare(gpu_rows, ora, heads, vmax, label):
     err_bf = np.abs(g - o)
     err = np.abs(g - f)
     plain_bad = (err_bf > tol).any(1)
-    ulp_ok = (err <= tol + 0.5 * ulp_bf16(f)).all(1)
+    cont = ora["ml"][:, 2:3] * np.abs(f) if "ml" in ora else np.zeros_like(f)
+    base = tol + 0.5 * ulp_bf16(f) + np.minimum(cont, flip)
+    ulp_ok = (err <= base).all(1)
     allowed = tol + 0.5 * ulp_bf16(f) + flip
     ok = err <= allowed
     worst_cos = 1.0
@@ -55,13 +69,16 @@ def compare(gpu_rows, ora, heads, vmax, label):
         cos = 1.0 if na == 0 and nb == 0 else float(a @ b / (na * nb))
         worst_cos = min(worst_cos, cos)
     n = len(g)
+    n_flip = int((~ulp_ok).sum())
+    cap = max(1, int(FLIP_ROWS_MAX * n))
     print(f"{label}: max|err| vs oracle bf16 = {err_bf.max():.3g} ({err_bf.max() / vmax:.3g} "
           f"max|V|); rows over 2e-3 max|V|: {int(plain_bad.sum())}/{n} "
           f"(bf16-step ties {int((plain_bad & ulp_ok).sum())}, "
-          f"within flip bound {int((plain_bad & ~ulp_ok).sum())}); "
+          f"within flip bound {n_flip}, cap {cap}); "
           f"worst err/allowance {float((err / allowed).max()):.3f}; "
           f"min head cosine {worst_cos:.7f}")
     assert ok.all(), (label, float((err / allowed).max()))
+    assert n_flip <= cap, (label, n_flip, cap)
     assert worst_cos >= COS_MIN, (label, worst_cos)
 
 
@@ -69,10 +86,10 @@ def run_full(ora, q, k, v, causal, label, softmax_scale=0.0):
     B, H, N, D = q.shape
     got = run_attn(q, k, v, causal, softmax_scale)
     want = ora.attn_fwd(q, k, v, causal=causal, softmax_scale=softmax_scale, want_f64=True,
-                        want_flip=True)
+                        want_flip=True, want_ml=True)
     heads = np.repeat(np.arange(B * H), N)
     vmax = float(np.abs(bf16_bits_to_f32(v)).max())
-    compare(got.reshape(-1, D), {k2: a.reshape(-1, D) for k2, a in want.items()}, heads, vmax,
+    compare(got.reshape(-1, D), {k2: a.reshape(-1, a.shape[-1]) for k2, a in want.items()}, heads, vmax,
             label)
 
 
@@ -140,13 +157,13 @@ def test_attention_workloads(ora, syn, name):
     vmax = float(np.abs(bf16_bits_to_f32(v)).max())
     per_head = _rows_per_head(wl)
     if per_head == 0:
-        want = ora.attn_fwd(q, k, v, causal=wl.causal, want_f64=True, want_flip=True)
+        want = ora.attn_fwd(q, k, v, causal=wl.causal, want_f64=True, want_flip=True, want_ml=True)
         heads = np.repeat(np.arange(wl.B * wl.H), wl.N)
-        compare(got.reshape(-1, wl.D), {k2: a.reshape(-1, wl.D) for k2, a in want.items()},
+        compare(got.reshape(-1, wl.D), {k2: a.reshape(-1, a.shape[-1]) for k2, a in want.items()},
                 heads, vmax, name)
         return
     rows = syn.sample_rows(wl, per_head)
-    want = ora.attn_fwd(q, k, v, causal=wl.causal, rows=rows, want_f64=True, want_flip=True)
+    want = ora.attn_fwd(q, k, v, causal=wl.causal, rows=rows, want_f64=True, want_flip=True, want_ml=True)
     got_rows = got[rows[:, 0], rows[:, 1], rows[:, 2]]
     compare(got_rows, want, rows[:, 0] * wl.H + rows[:, 1], vmax,
             f"{name} ({per_head} rows/head)")

@@ -23,10 +23,10 @@ def run_full(ora, q, k, v, causal, label, softmax_scale=0.0):
     B, H, N, D = q.shape
     got = run_attn(q, k, v, causal, softmax_scale, efq=True)
     want = ora.attn_fwd(q, k, v, causal=causal, softmax_scale=softmax_scale, want_f64=True,
-                        want_flip=True, flags=ora.FLAG_EFQ)
+                        want_flip=True, want_ml=True, flags=ora.FLAG_EFQ)
     heads = np.repeat(np.arange(B * H), N)
     vmax = float(np.abs(bf16_bits_to_f32(v)).max())
-    compare(got.reshape(-1, D), {k2: a.reshape(-1, D) for k2, a in want.items()}, heads, vmax,
+    compare(got.reshape(-1, D), {k2: a.reshape(-1, a.shape[-1]) for k2, a in want.items()}, heads, vmax,
             "EFQ " + label)
 
 
@@ -67,14 +67,14 @@ def test_efq_workloads(ora, syn, name):
     vmax = float(np.abs(bf16_bits_to_f32(v)).max())
     per_head = _rows_per_head(wl)
     if per_head == 0:
-        want = ora.attn_fwd(q, k, v, causal=wl.causal, want_f64=True, want_flip=True,
+        want = ora.attn_fwd(q, k, v, causal=wl.causal, want_f64=True, want_flip=True, want_ml=True,
                             flags=ora.FLAG_EFQ)
         heads = np.repeat(np.arange(wl.B * wl.H), wl.N)
-        compare(got.reshape(-1, wl.D), {k2: a.reshape(-1, wl.D) for k2, a in want.items()},
+        compare(got.reshape(-1, wl.D), {k2: a.reshape(-1, a.shape[-1]) for k2, a in want.items()},
                 heads, vmax, "EFQ " + name)
         return
     rows = syn.sample_rows(wl, per_head)
-    want = ora.attn_fwd(q, k, v, causal=wl.causal, rows=rows, want_f64=True, want_flip=True,
+    want = ora.attn_fwd(q, k, v, causal=wl.causal, rows=rows, want_f64=True, want_flip=True, want_ml=True,
                         flags=ora.FLAG_EFQ)
     got_rows = got[rows[:, 0], rows[:, 1], rows[:, 2]]
     compare(got_rows, want, rows[:, 0] * wl.H + rows[:, 1], vmax,
