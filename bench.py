@@ -12,10 +12,11 @@ is fp4_attn_fwd_sharded: the three tensor maxima of the rank's shard, one NCCL
 all-reduce (MAX) of those three floats, quantisation with the global maxima and
 the fused forward, so codes match a single-GPU run over the whole job.
 Inputs are seeded synthetic tensors; the default workload is the video-DiT
-latent grid (B1 H24 N32760 D128). e2e: the same metric through the host API
-(fp4_attn_fwd_host_many), every step copying its inputs in from pinned host
-memory and its output back, copies overlapped with the neighbouring steps'
-compute.
+latent grid (B1 H24 N32760 D128). e2e: the same metric through the C-ABI call
+on host buffers (fp4_attn_fwd_host), one call per step: the step's q, k, v
+copied in from pinned host memory, the forward, the output copied back, all in
+the timed region. e2e_pipelined: a stream of batches through
+fp4_attn_fwd_host_many, copies overlapped with the neighbouring steps' compute.
 """
 from __future__ import annotations
 
@@ -35,9 +36,9 @@ METRIC = "FP4 attention fwd TFLOPS at 1 B200 and % of dense FP4 tensor peak"
 FP4_DATASHEET_TFLOPS = 9000.0  # NVIDIA B200 dense FP4, no sparsity
 L2_BYTES = 126 * 1024 * 1024
 # DRAM bytes (read + write) of one attention-kernel launch on the full video-DiT
-# workload, from ncu (dram__bytes_read.sum + dram__bytes_write.sum, one pass;
-# profiles/attn_fwd_traffic_video_dit.md). They hold only for the kernel source
-# they were taken on, identified by its hash; otherwise traffic is reported null.
+# workload, from the ncu capture of this kernel (dram__bytes_read.sum +
+# dram__bytes_write.sum, one pass). They hold only for the kernel source they
+# were taken on, identified by its hash; otherwise traffic is reported null.
 ATTN_TRAFFIC = {"workload": "video_dit", "bytes": 170.74e6 + 155.99e6,
                 # sha256 of attn_fwd.cuh's code (comments and whitespace removed)
                 "attn_fwd_code_sha256":
@@ -447,6 +448,7 @@ def main():
 
     houts = [hout, torch.empty(shape_q, dtype=torch.bfloat16, pin_memory=True)]
     n_e2e = max(2, args.steps)
+    e_pipe = None
     if world > 1:
         for _ in range(max(1, args.warmup // 2)):
             e2e()
@@ -454,6 +456,10 @@ def main():
         e_ms = timed(e2e, max(1, args.steps // 2))
         barrier()
     else:
+        # one C-ABI call per step (copies in, forward, copy out), L2 flushed between
+        for _ in range(2):
+            e2e()
+        e_ms = timed(e2e, n_e2e)
         # a stream of batches through the public host API: each step copies its
         # inputs in and its output out, overlapped with the neighbouring steps'
         # compute
@@ -463,7 +469,7 @@ def main():
         _, total = fa.fp4_attn_fwd_host_many(batches, [houts[i % 2] for i in range(n_e2e)],
                                              causal=wl.causal, device=dev, efq=efq,
                                              fp8pv=fp8pv, smooth=smooth, return_ms=True)
-        e_ms = [total / n_e2e] * n_e2e
+        e_pipe = flops / (total / n_e2e * 1e-3) / 1e12
     e_total = sum(e_ms)
     if world > 1:
         t = torch.tensor([e_total], dtype=torch.float64, device=dev)
@@ -512,12 +518,21 @@ def main():
                                     f"{src}); fraction of measured"},
         "e2e": {"value": e2e_value, "unit": "TFLOPS",
                 "h2d_bytes_per_step": (hq.numel() + hk.numel() + hv.numel()) * 2,
-                "d2h_bytes_per_step": hout.numel() * 2},
+                "d2h_bytes_per_step": hout.numel() * 2,
+                "how": ("fp4_attn_fwd_host (C ABI): one host-to-host call per step"
+                        if world == 1 and not (efq or fp8pv or smooth) else
+                        "host copies on the compute stream, then the device entry, one step "
+                        "at a time")},
         # per step: amax (1, or 3 when sharded), 3 quantisations, the fused forward;
         # smoothing adds per smoothed tensor the sums, the means and the smoothed
         # maximum, plus Q's score correction
         "gpu_launches": ((7 if world > 1 else 5) + (7 if smooth else 0)) * args.steps,
     }
+    if e_pipe is not None:
+        line["e2e_pipelined"] = {"value": e_pipe, "unit": "TFLOPS",
+                                 "how": "fp4_attn_fwd_host_many: a stream of batches, step i+1's "
+                                        "copies in and step i-1's copy out overlapped with step "
+                                        "i's compute"}
     c = clk.summary()
     if c:
         line["clocks"] = c

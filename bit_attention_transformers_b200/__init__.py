@@ -47,6 +47,7 @@ EXPORTS = ("fp4_codes_bytes", "fp4_scales_bytes", "fp4_attn_workspace_bytes", "f
            "fp4_score_bias", "fp4_attn_fwd_quantized_bias", "fp4_attn_fwd_lse",
            "fp4_attn_bwd_workspace_bytes", "fp4_attn_bwd", "fp4_attn_bwd_scaled",
            "fp4_attn_fwd_quantized_lse", "fp4_attn_fwd_noalloc",
+           "fp4_attn_host_workspace_bytes", "fp4_attn_fwd_host",
            "fp4_status", "fp4_last_error", "fp4_probe_cvt", "fp4_test_wait_timeout")
 FP4_NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -107,6 +108,10 @@ def lib():
         L.fp4_scales_to_canonical.restype = i32
         L.fp4_attn_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, sz]
         L.fp4_attn_fwd.restype = i32
+        L.fp4_attn_host_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+        L.fp4_attn_host_workspace_bytes.restype = sz
+        L.fp4_attn_fwd_host.argtypes = L.fp4_attn_fwd.argtypes
+        L.fp4_attn_fwd_host.restype = i32
         L.fp4_attn_fwd_quantized.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp]
         L.fp4_attn_fwd_quantized.restype = i32
         L.fp4_attn_fwd_efq.argtypes = L.fp4_attn_fwd.argtypes
@@ -293,17 +298,27 @@ def fp4_amax(x, out=None, stream=None):
 
 
 # -------------------------------------------------------------- attention ----
+# Cached workspaces, one per (device, stream, kind). Calls on one stream run in
+# order, so they can share one; calls on two streams may overlap on the GPU and
+# must not, so each stream gets its own. A caller that passes `ws` itself owns
+# that rule: one workspace must not serve two calls that can overlap.
 _ws_cache: dict = {}
 
 
-def workspace(B, H, Hkv, N, D, device, fp8pv: bool = False, smooth: int = 0):
+def _stream_handle(stream) -> int:
+    return _stream(stream).value or 0
+
+
+def workspace(B, H, Hkv, N, D, device, fp8pv: bool = False, smooth: int = 0, stream=None):
     """A cached device workspace large enough for fp4_attn_fwd (or, with
-    fp8pv, fp4_attn_fwd_fp8pv; with smooth, fp4_attn_fwd_smooth) on this shape."""
+    fp8pv, fp4_attn_fwd_fp8pv; with smooth, fp4_attn_fwd_smooth) on this shape,
+    private to `stream` (default: the current stream) on `device`."""
     import torch
     fn = (fp4_attn_workspace_bytes_smooth if smooth else
           fp4_attn_workspace_bytes_fp8pv if fp8pv else fp4_attn_workspace_bytes)
     need = fn(B, H, Hkv, N, D)
-    key = (str(device),)
+    with torch.cuda.device(device):
+        key = ("fwd", str(device), _stream_handle(stream))
     ws = _ws_cache.get(key)
     if ws is None or ws.numel() < need:
         ws = torch.empty(need, dtype=torch.uint8, device=device)
@@ -340,7 +355,7 @@ def fp4_attn_fwd(q, k, v, causal: bool = False, softmax_scale: float | None = No
         out = torch.empty_like(q)
     fn = _attn_fn(efq, fp8pv, False)
     if ws is None:
-        ws = workspace(B, H, Hkv, N, D, q.device, fp8pv)
+        ws = workspace(B, H, Hkv, N, D, q.device, fp8pv, stream=stream)
     _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, Hkv, N, D, int(bool(causal)),
               float(softmax_scale or 0.0), _stream(stream), _ptr(ws), ws.numel()))
     return out
@@ -361,14 +376,11 @@ def fp4_attn_fwd_lse(q, k, v, causal: bool = False, softmax_scale: float | None 
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     if ws is None:
-        ws = workspace(B, H, Hkv, N, D, q.device)
+        ws = workspace(B, H, Hkv, N, D, q.device, stream=stream)
     _check(lib().fp4_attn_fwd_lse(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, N, D,
                                   int(bool(causal)), float(softmax_scale or 0.0), _stream(stream),
                                   _ptr(ws), ws.numel()))
     return out, lse
-
-
-_ws_bwd: dict = {}
 
 
 def fp4_attn_bwd(q, k, v, dout, lse, causal: bool = False, softmax_scale: float | None = None,
@@ -389,11 +401,12 @@ def fp4_attn_bwd(q, k, v, dout, lse, causal: bool = False, softmax_scale: float 
     dv = torch.empty_like(v) if dv is None else dv
     if ws is None:
         need = lib().fp4_attn_bwd_workspace_bytes(B, H, Hkv, N, D)
-        key = (str(q.device),)
-        ws = _ws_bwd.get(key)
+        with torch.cuda.device(q.device):
+            key = ("bwd", str(q.device), _stream_handle(stream))
+        ws = _ws_cache.get(key)
         if ws is None or ws.numel() < need:
             ws = torch.empty(need, dtype=torch.uint8, device=q.device)
-            _ws_bwd[key] = ws
+            _ws_cache[key] = ws
     if amax is not None:
         assert amax.is_cuda and amax.dtype == torch.float32 and amax.numel() >= 3
         _check(lib().fp4_attn_bwd_scaled(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lse),
@@ -411,9 +424,6 @@ def fp4_attn_workspace_bytes_smooth(B: int, H: int, Hkv: int, N: int, D: int) ->
     return lib().fp4_attn_workspace_bytes_smooth(B, H, Hkv, N, D)
 
 
-_ws_smooth: dict = {}
-
-
 def fp4_attn_fwd_smooth(q, k, v, smooth: int = FP4_SMOOTH_K | FP4_SMOOTH_Q, causal: bool = False,
                         softmax_scale: float | None = None, out=None, stream=None, ws=None):
     """NVFP4 attention forward with Q and/or K smoothed before quantisation
@@ -429,11 +439,12 @@ def fp4_attn_fwd_smooth(q, k, v, smooth: int = FP4_SMOOTH_K | FP4_SMOOTH_Q, caus
         out = torch.empty_like(q)
     if ws is None:
         need = fp4_attn_workspace_bytes_smooth(B, H, Hkv, N, D)
-        key = (str(q.device),)
-        ws = _ws_smooth.get(key)
+        with torch.cuda.device(q.device):
+            key = ("smooth", str(q.device), _stream_handle(stream))
+        ws = _ws_cache.get(key)
         if ws is None or ws.numel() < need:
             ws = torch.empty(need, dtype=torch.uint8, device=q.device)
-            _ws_smooth[key] = ws
+            _ws_cache[key] = ws
     _check(lib().fp4_attn_fwd_smooth(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, Hkv, N, D,
                                      int(bool(causal)), float(softmax_scale or 0.0), int(smooth),
                                      _stream(stream), _ptr(ws), ws.numel()))
@@ -560,19 +571,40 @@ def fp4_attn_fwd_quantized(qq: Fp4Tensor, kq: Fp4Tensor, vq: Fp4Tensor, B: int, 
 def fp4_attn_fwd_host(q, k, v, causal: bool = False, softmax_scale: float | None = None,
                       out=None, device="cuda", stream=None, efq: bool = False,
                       fp8pv: bool = False, smooth: int = 0):
-    """End-to-end call on host buffers: copies q, k, v (pinned CPU bf16
-    tensors) to the device, runs fp4_attn_fwd, copies the output back into
-    `out` (a pinned CPU tensor) and returns it once the stream has finished."""
+    """End-to-end call on host buffers: q, k, v pinned CPU bf16 tensors in,
+    `out` (a pinned CPU tensor, allocated if None) back, returned once it holds
+    the result. The default path is one call of the C entry fp4_attn_fwd_host
+    (copies in, the forward, the copy out, all on `stream`); the variants
+    (efq, fp8pv, smooth) copy with torch on the same stream and call their
+    device entry."""
     import torch
-    dq = q.to(device, non_blocking=True)
-    dk = k.to(device, non_blocking=True)
-    dv = v.to(device, non_blocking=True)
-    o = fp4_attn_fwd(dq, dk, dv, causal, softmax_scale, stream=stream, efq=efq, fp8pv=fp8pv,
-                     smooth=smooth)
+    dev = torch.device(device)
+    for t in (q, k, v):
+        assert not t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()
+    B, H, N, D = q.shape
+    Hkv = k.shape[1]
     if out is None:
-        out = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    out.copy_(o, non_blocking=True)
-    torch.cuda.current_stream().synchronize()
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    assert not out.is_cuda and out.shape == q.shape and out.dtype == q.dtype and out.is_contiguous()
+    with torch.cuda.device(dev):
+        s = torch.cuda.current_stream() if stream is None else stream
+        if not (efq or fp8pv or smooth):
+            need = lib().fp4_attn_host_workspace_bytes(B, H, Hkv, N, D)
+            key = ("host", str(dev), _stream_handle(s))
+            ws = _ws_cache.get(key)
+            if ws is None or ws.numel() < need:
+                ws = torch.empty(need, dtype=torch.uint8, device=dev)
+                _ws_cache[key] = ws
+            _check(lib().fp4_attn_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, Hkv, N, D,
+                                           int(bool(causal)), float(softmax_scale or 0.0),
+                                           _stream(s), _ptr(ws), ws.numel()))
+            return out
+        with torch.cuda.stream(s):
+            dq, dk, dv = (t.to(dev, non_blocking=True) for t in (q, k, v))
+            o = fp4_attn_fwd(dq, dk, dv, causal, softmax_scale, stream=s, efq=efq, fp8pv=fp8pv,
+                             smooth=smooth)
+            out.copy_(o, non_blocking=True)
+        s.synchronize()
     return out
 
 

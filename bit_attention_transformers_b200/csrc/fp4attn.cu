@@ -919,6 +919,44 @@ fp4_status_t fp4_attn_fwd(const void* q, const void* k, const void* v, void* out
                       workspace_bytes, 0);
 }
 
+size_t fp4_attn_host_workspace_bytes(int B, int H, int Hkv, int N, int D) {
+  if (check_shape(B, H, Hkv, N, D) != FP4_OK) return 0;
+  const size_t nq = (size_t)B * H * N * D * 2, nkv = (size_t)B * Hkv * N * D * 2;
+  return 2 * (size_t)round_up((int64_t)nq, 1024) + 2 * (size_t)round_up((int64_t)nkv, 1024) +
+         ws_layout(B, H, Hkv, N, D).total;
+}
+
+fp4_status_t fp4_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
+                               void* out_host, int B, int H, int Hkv, int N, int D, int causal,
+                               float softmax_scale, void* stream, void* dev_workspace,
+                               size_t dev_workspace_bytes) {
+  g_last_error.clear();
+  fp4_status_t s;
+  if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
+  if (!q_host || !k_host || !v_host || !out_host || !dev_workspace)
+    return fail(FP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(dev_workspace))
+    return fail(FP4_ERR_INVALID_ARG, "the device workspace must be 16-byte aligned");
+  const size_t need = fp4_attn_host_workspace_bytes(B, H, Hkv, N, D);
+  if (dev_workspace_bytes < need)
+    return fail(FP4_ERR_WORKSPACE, "device workspace of %zu bytes, %zu needed",
+                dev_workspace_bytes, need);
+  const size_t nq = (size_t)B * H * N * D * 2, nkv = (size_t)B * Hkv * N * D * 2;
+  const size_t aq = (size_t)round_up((int64_t)nq, 1024), akv = (size_t)round_up((int64_t)nkv, 1024);
+  uint8_t* base = static_cast<uint8_t*>(dev_workspace);
+  uint8_t *dq = base, *dk = dq + aq, *dv = dk + akv, *dout = dv + akv, *ws = dout + aq;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  FP4_CUDA(cudaMemcpyAsync(dq, q_host, nq, cudaMemcpyHostToDevice, st));
+  FP4_CUDA(cudaMemcpyAsync(dk, k_host, nkv, cudaMemcpyHostToDevice, st));
+  FP4_CUDA(cudaMemcpyAsync(dv, v_host, nkv, cudaMemcpyHostToDevice, st));
+  if ((s = fp4_attn_fwd(dq, dk, dv, dout, B, H, Hkv, N, D, causal, softmax_scale, stream, ws,
+                        dev_workspace_bytes - (size_t)(ws - base))) != FP4_OK)
+    return s;
+  FP4_CUDA(cudaMemcpyAsync(out_host, dout, nq, cudaMemcpyDeviceToHost, st));
+  FP4_CUDA(cudaStreamSynchronize(st));
+  return FP4_OK;
+}
+
 fp4_status_t fp4_attn_fwd_efq(const void* q, const void* k, const void* v, void* out, int B,
                               int H, int Hkv, int N, int D, int causal, float softmax_scale,
                               void* stream, void* workspace, size_t workspace_bytes) {

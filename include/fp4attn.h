@@ -157,6 +157,27 @@ fp4_status_t fp4_attn_fwd(const void* q, const void* k, const void* v, void* out
                           void* workspace, size_t workspace_bytes);
 
 /*
+ * The attention forward end to end from HOST memory: q_host, k_host, v_host
+ * (bf16, layouts as fp4_attn_fwd) are copied to the device, fp4_attn_fwd runs,
+ * and the output is copied back into out_host; the call returns once
+ * out_host holds the result (it synchronises `stream`). One cudaMemcpyAsync
+ * per tensor in each direction, all on `stream`. Host buffers should be
+ * pinned (cudaHostAlloc / cudaHostRegister) for the copies to run at full
+ * speed; pageable memory works but copies through a staging buffer.
+ * dev_workspace (device, caller-owned, 16-byte aligned) holds the device
+ * copies of q, k, v and out followed by fp4_attn_fwd's workspace:
+ * fp4_attn_host_workspace_bytes() bytes. Errors as fp4_attn_fwd; a failed
+ * copy returns FP4_ERR_CUDA. The pages define no interface (the method is the
+ * forward above); this entry exists so that a whole host-to-host call is one
+ * C function.
+ */
+size_t fp4_attn_host_workspace_bytes(int B, int H, int Hkv, int N, int D);
+fp4_status_t fp4_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
+                               void* out_host, int B, int H, int Hkv, int N, int D, int causal,
+                               float softmax_scale, void* stream, void* dev_workspace,
+                               size_t dev_workspace_bytes);
+
+/*
  * The fused forward alone, on tensors fp4_quantize() produced (q with
  * FP4_BLOCK_ALONG_D and G = B*H; k with FP4_BLOCK_ALONG_D and v with
  * FP4_BLOCK_ALONG_N_T, G = B*Hkv), all for the same N and D.
