@@ -4,18 +4,16 @@ gives them no allocator, or they must avoid cudaMalloc's implicit device
 synchronisation). It uses the library's built-in scratch array instead of a
 workspace. Checked through the C ABI against fp4_attn_fwd on two calls in a
 row, with different shapes, so the second call runs on the first call's
-leftover scratch contents. Collected last on purpose."""
+leftover scratch contents. Both run the same deterministic kernels on the same
+inputs, so the outputs must be identical bit for bit: any difference would be
+leftover scratch (stale padding, a stale maximum) leaking into the result.
+Collected last on purpose."""
 import ctypes
 
-import numpy as np
 import pytest
 
 import bit_attention_transformers_b200 as fa
-from _util import bf16_bits_to_f32
-from gpu_util import from_dev, to_dev
-
-ATOL_REL = 2e-3
-COS_MIN = 0.9999
+from gpu_util import to_dev
 
 
 def _case(syn, B, H, Hkv, N, D, seed):
@@ -43,13 +41,7 @@ def test_noalloc_matches_workspace_entry_point(syn):
                                     vp(stream))
         assert rc == fa.FP4_OK, L.fp4_last_error()
         fa.fp4_status()
-        g = bf16_bits_to_f32(from_dev(out)).astype(np.float64)
-        r = bf16_bits_to_f32(from_dev(ref)).astype(np.float64)
-        vmax = float(np.abs(bf16_bits_to_f32(v)).max())
-        assert np.abs(g - r).max() <= ATOL_REL * vmax
-        for h in range(B * H):
-            a, b = g.reshape(B * H, -1)[h], r.reshape(B * H, -1)[h]
-            assert a @ b / (np.linalg.norm(a) * np.linalg.norm(b)) >= COS_MIN
+        assert torch.equal(out, ref), (B, H, Hkv, N, D, causal)
 
 
 @pytest.mark.gpu
