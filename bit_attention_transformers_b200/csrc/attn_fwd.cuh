@@ -44,8 +44,12 @@
 // the tile's FP4 MMAs; the softmax is unchanged.
 // LSE (the training forward): the epilogue also writes m + log2 l per row.
 //
+// Causal launches order the CTAs longest first across all heads (query tile
+// ntq-1 of every head, then ntq-2, ...), so the short tiles fill the last wave.
+//
 // Every wait is bounded (2 s of %globaltimer); on expiry the kernel sets the
-// device error word, stops issuing, drains its tensor-core work and returns.
+// device error word, stops issuing, drains its tensor-core work and the bulk
+// copies still in flight into shared memory, and returns.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -112,7 +116,7 @@ struct AttnParams {
   const float* amax_v;
   __nv_bfloat16* out;  // [B][H][N][D]
   float* lse;          // [B*H][N]: log2 sum_j 2^(x_ij) per row for the backward, or NULL
-  int H, Hkv, N, Npad, ntq;
+  int B, H, Hkv, N, Npad, ntq;
   float softmax_scale;
 };
 
@@ -200,8 +204,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                            ~uintptr_t(1023));
   const uint32_t sb = smem_u32(sm);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = CAUSAL ? (p.ntq - 1 - (int)blockIdx.x) : (int)blockIdx.x;
-  const int h = blockIdx.y, b = blockIdx.z;
+  // causal: a 1D grid, longest query tiles of every head first
+  int qt, h, b;
+  if (CAUSAL) {
+    const int nbh = p.B * p.H;
+    const int i = (int)blockIdx.x;
+    qt = p.ntq - 1 - i / nbh;
+    h = (i % nbh) % p.H;
+    b = (i % nbh) / p.H;
+  } else {
+    qt = (int)blockIdx.x;
+    h = (int)blockIdx.y;
+    b = (int)blockIdx.z;
+  }
   const int gq = b * p.H + h;
   const int gk = b * p.Hkv + h / (p.H / p.Hkv);
   const int nkv = (p.N + kBN - 1) / kBN;
@@ -270,6 +285,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       bool ok = true;
+      int kissued = 0, vissued = 0;  // tiles whose K / V loads were started
       const int qrow0 = gq * p.Npad + qt * kBM;
       mbar_arrive_expect_tx(bar(kBarQ), L::kQ + L::kSfQK);
       tma_load_2d(sb + L::oQ, &tmQ, 0, qrow0, bar(kBarQ));
@@ -287,6 +303,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         bulk_load(sb + L::oKsf + st * 1024,
                   p.k_sf + ((int64_t)gk * (p.Npad / kBN) + j) * L::kSfQK, L::kSfQK,
                   bar(kBarKFull + st));
+        kissued = j + 1;
         if (j >= kStages && !(ok = wait_bar(bar(kBarVEmpty + st), pe))) break;
         mbar_arrive_expect_tx(bar(kBarVFull + st), L::kV + (FP8 ? 0 : 1024));
         tma_load_2d(sb + L::oV + st * L::kV, &tmV, j * (FP8 ? kBN : kBN / 2), gk * D,
@@ -294,6 +311,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!FP8)
           bulk_load(sb + L::oVsf + st * 1024, p.v_sf + ((int64_t)gk * (p.Npad / 64) + 2 * j) * 512,
                     1024, bar(kBarVFull + st));
+        vissued = j + 1;
+      }
+      if (!ok) {
+        // no bulk copy may outlive the CTA: wait (bounded) for the last load
+        // started on every stage; a stage its consumer already took has
+        // completed that phase, and no later phase was started
+        drain_wait(bar(kBarQ), 0);
+        for (int j = max(0, kissued - kStages); j < kissued; ++j)
+          drain_wait(bar(kBarKFull + j % kStages), (j / kStages) & 1);
+        for (int j = max(0, vissued - kStages); j < vissued; ++j)
+          drain_wait(bar(kBarVFull + j % kStages), (j / kStages) & 1);
       }
     }
   } else if (warp == 1 || warp == 2) {

@@ -419,6 +419,7 @@ fp4_status_t launch_attn(const uint8_t* qc, const uint8_t* qs, const float* qa, 
   p.amax_k = ka;
   p.amax_v = va;
   p.out = static_cast<__nv_bfloat16*>(out);
+  p.B = B;
   p.H = H;
   p.Hkv = Hkv;
   p.N = N;
@@ -426,7 +427,10 @@ fp4_status_t launch_attn(const uint8_t* qc, const uint8_t* qs, const float* qa, 
   p.ntq = (int)(Npad / 128);
   p.lse = lse;
   p.softmax_scale = resolve_scale(softmax_scale, D);
-  dim3 grid(p.ntq, H, B);
+  // causal: one linear grid, the longest query tiles of every head first
+  if (causal && (int64_t)p.ntq * B * H > INT32_MAX)
+    return fail(FP4_ERR_INVALID_ARG, "problem too large");
+  const dim3 grid = causal ? dim3((unsigned)((int64_t)p.ntq * B * H)) : dim3(p.ntq, H, B);
   if ((bias || lse) && pg != fp4::kPgExp)
     return fail(FP4_ERR_UNSUPPORTED, "the score correction and lse need exp-then-quantize P");
   if (bias && lse) return fail(FP4_ERR_UNSUPPORTED, "lse with the score correction");
