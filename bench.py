@@ -229,7 +229,7 @@ def run_bwd(args, wl):
     stream = torch.cuda.current_stream()
 
     def step():
-        fa.fp4_attn_bwd(q, k, v, do, lse, causal=wl.causal, dq=dq, dk=dk, dv=dv)
+        fa.fp4_attn_bwd(q, k, v, out, do, lse, causal=wl.causal, dq=dq, dk=dk, dv=dv)
 
     def timed(fn, n):
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -252,18 +252,22 @@ def run_bwd(args, wl):
     ms_per_step = sum(ms) / len(ms)
     fwd_flops = wl.flops
     value = 2.5 * fwd_flops / (ms_per_step * 1e-3) / 1e12
-    # the kernels' own tensor work: the dq kernel's two sweeps (S, dP twice) and
-    # dQ, the dk/dv kernel's S, dP, dV, dK: 9 contractions of 2 N^2 D per head
-    tensor_flops = 9 * fwd_flops / 2
+    # the kernels' own tensor work: the dq kernel's S, dP and its two dQ sums
+    # (P (dP - c) K^ and P K^), the dk/dv kernel's S, dP, dV, dK: 8 contractions
+    # of 2 N^2 D per head
+    tensor_flops = 8 * fwd_flops / 2
     peaks, src = measured_peaks()
     hlse = torch.empty(lse.shape, dtype=torch.float32, pin_memory=True)
     hlse.copy_(lse)
+    hout = torch.empty(out.shape, dtype=torch.bfloat16, pin_memory=True)
+    hout.copy_(out)
     hdq, hdk, hdv = (torch.empty(t.shape, dtype=torch.bfloat16, pin_memory=True)
                      for t in (dq, dk, dv))
 
     def e2e():
-        gq, gk, gv, gdo, gl = (t.to(dev, non_blocking=True) for t in (hq, hk, hv, hdo, hlse))
-        a, b, c = fa.fp4_attn_bwd(gq, gk, gv, gdo, gl, causal=wl.causal)
+        gq, gk, gv, go, gdo, gl = (t.to(dev, non_blocking=True)
+                                   for t in (hq, hk, hv, hout, hdo, hlse))
+        a, b, c = fa.fp4_attn_bwd(gq, gk, gv, go, gdo, gl, causal=wl.causal)
         hdq.copy_(a, non_blocking=True)
         hdk.copy_(b, non_blocking=True)
         hdv.copy_(c, non_blocking=True)
@@ -284,11 +288,11 @@ def run_bwd(args, wl):
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": tensor_flops / (ms_per_step * 1e-3) / 1e12 / peaks["bf16_tflops"],
                      "traffic": None,
-                     "peak_source": f"measured dense bf16 ({src}); the whole call, 9 bf16 "
+                     "peak_source": f"measured dense bf16 ({src}); the whole call, 8 bf16 "
                                     "contractions of 2 N^2 D per head; fraction of measured"},
         "e2e": {"value": e_val, "unit": "TFLOPS",
-                "h2d_bytes_per_step": (hq.numel() + hk.numel() + hv.numel() + hdo.numel()) * 2
-                                      + hlse.numel() * 4,
+                "h2d_bytes_per_step": (hq.numel() + hk.numel() + hv.numel() + hout.numel()
+                                       + hdo.numel()) * 2 + hlse.numel() * 4,
                 "d2h_bytes_per_step": (hdq.numel() + hdk.numel() + hdv.numel()) * 2},
         # amax, Q^ and K^ decode, V^ decode, dO pad/transpose, lse pad, dq kernel, dk/dv kernel
         "gpu_launches": 8 * args.steps,

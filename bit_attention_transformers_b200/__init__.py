@@ -151,11 +151,11 @@ def lib():
         L.fp4_attn_fwd_lse.restype = i32
         L.fp4_attn_bwd_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
         L.fp4_attn_bwd_workspace_bytes.restype = sz
-        L.fp4_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
-                                   f32, vp, vp, sz]
+        L.fp4_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                   i32, f32, vp, vp, sz]
         L.fp4_attn_bwd.restype = i32
-        L.fp4_attn_bwd_scaled.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
-                                          i32, i32, f32, vp, vp, sz]
+        L.fp4_attn_bwd_scaled.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32,
+                                          i32, i32, i32, f32, vp, vp, sz]
         L.fp4_attn_bwd_scaled.restype = i32
         L.fp4_attn_fwd_quantized_lse.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                                  f32, vp]
@@ -383,18 +383,21 @@ def fp4_attn_fwd_lse(q, k, v, causal: bool = False, softmax_scale: float | None 
     return out, lse
 
 
-def fp4_attn_bwd(q, k, v, dout, lse, causal: bool = False, softmax_scale: float | None = None,
-                 dq=None, dk=None, dv=None, stream=None, ws=None, amax=None):
-    """The FP4 attention backward (reading in include/fp4attn.h): q, dout [B,H,N,D],
-    k, v [B,Hkv,N,D] bf16 CUDA, lse [B,H,N] from fp4_attn_fwd_lse. With `amax`
-    (float32 CUDA [3]: the maxima of Q, K, V, e.g. combined over shards)
-    fp4_attn_bwd_scaled quantises with them. Returns (dq, dk, dv) bf16."""
+def fp4_attn_bwd(q, k, v, out, dout, lse, causal: bool = False,
+                 softmax_scale: float | None = None, dq=None, dk=None, dv=None, stream=None,
+                 ws=None, amax=None):
+    """The FP4 attention backward (reading in include/fp4attn.h): q, out, dout
+    [B,H,N,D], k, v [B,Hkv,N,D] bf16 CUDA; out and lse [B,H,N] from
+    fp4_attn_fwd_lse. With `amax` (float32 CUDA [3]: the maxima of Q, K, V,
+    e.g. combined over shards) fp4_attn_bwd_scaled quantises with them.
+    Returns (dq, dk, dv) bf16."""
     import torch
     B, H, N, D = q.shape
     Hkv = k.shape[1]
-    for t in (q, k, v, dout):
+    for t in (q, k, v, out, dout):
         assert t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()
-    assert k.shape == (B, Hkv, N, D) and v.shape == k.shape and dout.shape == q.shape
+    assert k.shape == (B, Hkv, N, D) and v.shape == k.shape
+    assert dout.shape == q.shape and out.shape == q.shape
     assert lse.dtype == torch.float32 and lse.is_contiguous() and lse.numel() == B * H * N
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
@@ -409,13 +412,14 @@ def fp4_attn_bwd(q, k, v, dout, lse, causal: bool = False, softmax_scale: float 
             _ws_cache[key] = ws
     if amax is not None:
         assert amax.is_cuda and amax.dtype == torch.float32 and amax.numel() >= 3
-        _check(lib().fp4_attn_bwd_scaled(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lse),
-                                         _ptr(amax), _ptr(dq), _ptr(dk), _ptr(dv), B, H, Hkv, N, D,
-                                         int(bool(causal)), float(softmax_scale or 0.0),
-                                         _stream(stream), _ptr(ws), ws.numel()))
+        _check(lib().fp4_attn_bwd_scaled(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout),
+                                         _ptr(lse), _ptr(amax), _ptr(dq), _ptr(dk), _ptr(dv), B, H,
+                                         Hkv, N, D, int(bool(causal)),
+                                         float(softmax_scale or 0.0), _stream(stream), _ptr(ws),
+                                         ws.numel()))
         return dq, dk, dv
-    _check(lib().fp4_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
-                              _ptr(dv), B, H, Hkv, N, D, int(bool(causal)),
+    _check(lib().fp4_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                              _ptr(dq), _ptr(dk), _ptr(dv), B, H, Hkv, N, D, int(bool(causal)),
                               float(softmax_scale or 0.0), _stream(stream), _ptr(ws), ws.numel()))
     return dq, dk, dv
 

@@ -21,8 +21,8 @@
 //       bf16 (Q^, K^ and their transposes; V^), bit-identical codes and scales
 //   pad_transpose_kernel  dO padded to Npad rows, and dO^T
 //   lse_pad_kernel        lse padded with +inf (padded rows get P = 0)
-//   bwd_dq_kernel   one CTA per 128 query rows: sweep 1 over the key tiles
-//       forms D, sweep 2 forms dS and accumulates dQ += dS K^ in TMEM
+//   bwd_dq_kernel   one CTA per 128 query rows, one pass over the key tiles:
+//       D and dQ (dQ from two sums accumulated in TMEM, see the kernel)
 //   bwd_dkdv_kernel one CTA per 128 keys: over the query tiles of every query
 //       head of its key/value head, dV += P^T dO and dK += dS^T Q^ in TMEM
 #pragma once
@@ -241,6 +241,7 @@ struct BwdParams {
   const float* amax;   // [3]: Q, K, V maxima (the forward's tensor scales)
   const float* lse;    // [B*H][Npad], +inf on padded rows
   float* Dvec;         // [B*H][Npad]: D, written by the dq kernel
+  const __nv_bfloat16* out;  // [B][H][N][D]: the forward's output O (centres dP, dq kernel)
   __nv_bfloat16* dq;   // [B][H][N][D]
   __nv_bfloat16* dk;   // [B][Hkv][N][D]
   __nv_bfloat16* dv;
@@ -279,48 +280,64 @@ __device__ __forceinline__ bool bwd_wait(uint32_t bar, uint32_t parity) {
 }
 
 // ------------------------------------------------------------- dq kernel ----
-constexpr int kDqThreads = 384;  // warps 0-3 control (warp 0 loads, warp 1 issues), 4-11 compute
+constexpr int kDqThreads = 384;  // warps 0-3 control, 4-11 compute (two warpgroups)
 constexpr uint32_t kDqRegsCtl = 56, kDqRegsCompute = 224;  // 128 x 56 + 256 x 224 = 384 x 168
 
-// Two rings of key tiles: ring A (K^, V^) feeds S and dP and is released as
-// soon as they complete; ring B (K^T) feeds dQ, needed a tile later, and has
-// its own producer warp, so that neither ring's loads wait on the other's.
-constexpr int kDqRingA = 2, kDqRingB = 3;
+// Key tiles pass once. D_i is not known until every key has been seen, so
+// dQ_i = scale d_K sum_j P_ij (dP_ij - D_i) K^_j is split into two sums that
+// are both accumulated in that one pass (dP in real units, d_V applied):
+//   A_i = sum_j P_ij (dP_ij - c_i) K^_j,   B_i = sum_j P_ij K^_j,
+//   dQ_i = scale d_K (A_i - (D_i - c_i) B_i),
+// an identity for any per-row constant c_i, with D_i = D'_i + c_i sum_j P_ij
+// and D'_i = sum_j P_ij (dP_ij - c_i) formed in the same pass, so D is still
+// this P's and v~'s. c_i = dO_i . O_i with the forward's output O: O_i is
+// sum_j P_ij v~_j up to the FP4 rounding of P, so c_i is close to D_i, the
+// terms of A are as small as those of dS and the subtraction at the end
+// cancels nothing large (with c_i = 0 a row whose P sits on one key loses
+// dQ to the bf16 rounding of P dP). Only the rounding depends on O.
+// Ring A (K^, V^) feeds S and dP and is released when they complete; ring B
+// (K^T) feeds A and B a tile later; each ring has its own producer warp.
+// Warp 1 issues S and dP, warp 3 issues A and B, so that neither kind waits
+// behind the other's barriers.
+constexpr int kDqRingA = 2, kDqRingB = 2;
 
 template <int D>
 struct BwdDqSmem {
   static constexpr int kQ = kBwdQ * D * 2;    // Q^ tile, bf16
   static constexpr int kK = kBwdKt * D * 2;   // K^ tile
   static constexpr int kKT = D * kBwdKt * 2;  // K^T tile (D rows x 64 keys)
-  static constexpr int kDS = kBwdQ * kBwdKt * 2;  // one dS tile: 128 rows x 64 keys, bf16
+  static constexpr int kPT = kBwdQ * kBwdKt * 2;  // one 128 x 64 bf16 operand tile
   static constexpr int oQ = 0;
   static constexpr int oDO = oQ + kQ;
-  static constexpr int oA = oDO + kQ;              // [kDqRingA]: K^ then V^
+  static constexpr int oA = oDO + kQ;                // [kDqRingA]: K^ then V^
   static constexpr int oB = oA + kDqRingA * 2 * kK;  // [kDqRingB]: K^T
-  static constexpr int oDS = oB + kDqRingB * kKT;  // [2]: one dS buffer per compute stream
-  static constexpr int oD = oDS + 2 * kDS;         // float [2][128]: each stream's partial D
-  static constexpr int oBar = oD + 1024;
+  static constexpr int oP = oB + kDqRingB * kKT;     // [2 streams]: P then P (dP - c), bf16
+  static constexpr int oBar = oP + 2 * 2 * kPT;
   static constexpr int oTmem = oBar + 256;
   static constexpr int kBytes = oTmem + 16 + 1024;
+  static_assert(kBytes <= 232448, "shared memory of one CTA");
 };
 
 enum : int {
   kDqBarQ = 0,
-  kDqBarFullA = 1,                     // [kDqRingA]
+  kDqBarFullA = 1,                        // [kDqRingA]
   kDqBarEmptyA = kDqBarFullA + kDqRingA,  // [kDqRingA]
   kDqBarFullB = kDqBarEmptyA + kDqRingA,  // [kDqRingB]
   kDqBarEmptyB = kDqBarFullB + kDqRingB,  // [kDqRingB]
   kDqBarSFull = kDqBarEmptyB + kDqRingB,  // [2] S/dP buffers (= compute streams)
   kDqBarSEmpty = kDqBarSFull + 2,         // [2]
-  kDqBarDsFull = kDqBarSEmpty + 2,        // [2] dS buffers
-  kDqBarDsEmpty = kDqBarDsFull + 2,       // [2]
-  kDqBarDone = kDqBarDsEmpty + 2,
+  kDqBarPFull = kDqBarSEmpty + 2,         // [2] P / P (dP - c) buffers
+  kDqBarPEmpty = kDqBarPFull + 2,         // [2]
+  kDqBarDone = kDqBarPEmpty + 2,          // every A / B contraction complete
+  kDqBarDoneS = kDqBarDone + 1,           // every S / dP contraction complete
+  kDqNumBars = kDqBarDoneS + 1,
 };
+static_assert(kDqNumBars * 8 <= 256, "barrier area");
 
 // One CTA per (128-query tile, head, batch). Two compute streams (warpgroups)
-// take alternate key tiles, so that one forms its P and dS while the tensor
-// core works for the other. TMEM: S[b] at 128 b, dP[b] at 128 b + 64 (64
-// columns each, b = tile parity = stream), dQ at 256 (D columns).
+// take alternate key tiles, so that one forms its P while the tensor core
+// works for the other. TMEM: S[b] at 128 b, dP[b] at 128 b + 64 (64 columns
+// each, b = tile parity = stream), A at 256, B at 256 + D.
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kDqThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
@@ -337,7 +354,6 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   const int gk = b * p.Hkv + h / (p.H / p.Hkv);
   const int nk_all = (p.N + kBwdKt - 1) / kBwdKt;
   const int nkt = CAUSAL ? min(nk_all, (qt * kBwdQ + kBwdQ - 1) / kBwdKt + 1) : nk_all;
-  const int T = 2 * nkt;  // sweep 1 (D), then sweep 2 (dS, dQ)
   auto bar = [&](int i) -> uint32_t { return sb + L::oBar + 8 * i; };
   if (threadIdx.x == 0) {
     mbar_init(bar(kDqBarQ), 1);
@@ -352,10 +368,11 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(kDqBarSFull + s), 1);
       mbar_init(bar(kDqBarSEmpty + s), 4);
-      mbar_init(bar(kDqBarDsFull + s), 4);
-      mbar_init(bar(kDqBarDsEmpty + s), 1);
+      mbar_init(bar(kDqBarPFull + s), 4);
+      mbar_init(bar(kDqBarPEmpty + s), 1);
     }
     mbar_init(bar(kDqBarDone), 1);
+    mbar_init(bar(kDqBarDoneS), 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -379,16 +396,16 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         tma_load_2d(sb + L::oDO + a * kBwdQ * 128, &tmDO, a * 64, gq * p.Npad + qt * kBwdQ,
                     bar(kDqBarQ));
       }
-      for (int t = 0; t < T && ok; ++t) {  // ring A: K^ and V^ of every tile of both sweeps
-        const int st = t % kDqRingA, j = t % nkt;
+      for (int t = 0; t < nkt && ok; ++t) {  // ring A: K^ and V^
+        const int st = t % kDqRingA;
         if (t >= kDqRingA && !(ok = bwd_wait(bar(kDqBarEmptyA + st), ((t / kDqRingA) - 1) & 1)))
           break;
         const uint32_t base = sb + L::oA + st * 2 * L::kK;
         mbar_arrive_expect_tx(bar(kDqBarFullA + st), 2 * L::kK);
         for (int a = 0; a < NA; ++a) {
-          tma_load_2d(base + a * kBwdKt * 128, &tmK, a * 64, gk * p.Npad + j * kBwdKt,
+          tma_load_2d(base + a * kBwdKt * 128, &tmK, a * 64, gk * p.Npad + t * kBwdKt,
                       bar(kDqBarFullA + st));
-          tma_load_2d(base + L::kK + a * kBwdKt * 128, &tmV, a * 64, gk * p.Npad + j * kBwdKt,
+          tma_load_2d(base + L::kK + a * kBwdKt * 128, &tmV, a * 64, gk * p.Npad + t * kBwdKt,
                       bar(kDqBarFullA + st));
         }
         issued = t + 1;
@@ -400,35 +417,20 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     } else if (warp == 2 && lane == 0) {
       bool ok = true;
       int issued = 0;
-      for (int t2 = 0; t2 < nkt && ok; ++t2) {  // ring B: K^T of the sweep-2 tiles
-        const int st = t2 % kDqRingB;
-        if (t2 >= kDqRingB && !(ok = bwd_wait(bar(kDqBarEmptyB + st), ((t2 / kDqRingB) - 1) & 1)))
+      for (int t = 0; t < nkt && ok; ++t) {  // ring B: K^T
+        const int st = t % kDqRingB;
+        if (t >= kDqRingB && !(ok = bwd_wait(bar(kDqBarEmptyB + st), ((t / kDqRingB) - 1) & 1)))
           break;
         mbar_arrive_expect_tx(bar(kDqBarFullB + st), L::kKT);
-        tma_load_2d(sb + L::oB + st * L::kKT, &tmKT, t2 * kBwdKt, gk * D, bar(kDqBarFullB + st));
-        issued = t2 + 1;
+        tma_load_2d(sb + L::oB + st * L::kKT, &tmKT, t * kBwdKt, gk * D, bar(kDqBarFullB + st));
+        issued = t + 1;
       }
-      for (int t2 = max(0, issued - kDqRingB); t2 < issued; ++t2)
-        drain_wait(bar(kDqBarFullB + t2 % kDqRingB), (t2 / kDqRingB) & 1);
-    } else if (warp == 1 && lane == 0) {
+      for (int t = max(0, issued - kDqRingB); t < issued; ++t)
+        drain_wait(bar(kDqBarFullB + t % kDqRingB), (t / kDqRingB) & 1);
+    } else if (warp == 1 && lane == 0) {  // S = Q^ K^T and dP = dO V^T of every key tile
       bool ok = bwd_wait(bar(kDqBarQ), 0);
-      const uint32_t idS = idesc_bf16(kBwdQ, kBwdKt), idQ = idesc_bf16(kBwdQ, D);
-      auto issue_dq = [&](int t) {  // dQ += dS K^ of tile t (sweep 2)
-        const int t2 = t - nkt, sb2 = t2 % kDqRingB;
-        ok = ok && bwd_wait(bar(kDqBarDsFull + (t & 1)), (t2 >> 1) & 1);
-        ok = ok && bwd_wait(bar(kDqBarFullB + sb2), (t2 / kDqRingB) & 1);
-        if (!ok) return;
-        tc_fence_after();
-        const uint32_t kt = sb + L::oB + sb2 * L::kKT;
-        const uint32_t ds = sb + L::oDS + (t & 1) * L::kDS;
-#pragma unroll
-        for (int s = 0; s < kBwdKt / 16; ++s)
-          mma_bf16(tmem + 256, kmaj_desc(ds, kBwdQ, s), kmaj_desc(kt, D, s), idQ,
-                   (t2 > 0 || s > 0) ? 1u : 0u);
-        tc_commit(bar(kDqBarEmptyB + sb2));
-        tc_commit(bar(kDqBarDsEmpty + (t & 1)));
-      };
-      for (int t = 0; t < T && ok; ++t) {
+      const uint32_t idS = idesc_bf16(kBwdQ, kBwdKt);
+      for (int t = 0; t < nkt && ok; ++t) {
         const int st = t % kDqRingA, buf = t & 1;
         if (!(ok = bwd_wait(bar(kDqBarFullA + st), (t / kDqRingA) & 1))) break;
         if (t >= 2 && !(ok = bwd_wait(bar(kDqBarSEmpty + buf), ((t >> 1) - 1) & 1))) break;
@@ -443,11 +445,30 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
         tc_commit(bar(kDqBarSFull + buf));
         tc_commit(bar(kDqBarEmptyA + st));
-        if (t > nkt) issue_dq(t - 1);  // the previous tile's dQ, one step behind
       }
-      if (ok && T > nkt) issue_dq(T - 1);
+      tc_commit(bar(kDqBarDoneS));
+      drain_wait(bar(kDqBarDoneS), 0);  // every MMA complete before TMEM is freed
+    } else if (warp == 3 && lane == 0) {  // A += (P (dP - c)) K^ and B += P K^, a tile behind
+      bool ok = true;
+      const uint32_t idQ = idesc_bf16(kBwdQ, D);
+      for (int t = 0; t < nkt && ok; ++t) {
+        const int buf = t & 1, st = t % kDqRingB;
+        if (!(ok = bwd_wait(bar(kDqBarPFull + buf), (t >> 1) & 1))) break;
+        if (!(ok = bwd_wait(bar(kDqBarFullB + st), (t / kDqRingB) & 1))) break;
+        tc_fence_after();
+        const uint32_t kt = sb + L::oB + st * L::kKT;
+        const uint32_t pp = sb + L::oP + buf * 2 * L::kPT;
+#pragma unroll
+        for (int s = 0; s < kBwdKt / 16; ++s) {
+          const uint32_t acc = (t > 0 || s > 0) ? 1u : 0u;
+          mma_bf16(tmem + 256, kmaj_desc(pp + L::kPT, kBwdQ, s), kmaj_desc(kt, D, s), idQ, acc);
+          mma_bf16(tmem + 256 + D, kmaj_desc(pp, kBwdQ, s), kmaj_desc(kt, D, s), idQ, acc);
+        }
+        tc_commit(bar(kDqBarEmptyB + st));
+        tc_commit(bar(kDqBarPEmpty + buf));
+      }
       tc_commit(bar(kDqBarDone));
-      drain_wait(bar(kDqBarDone), 0);  // every MMA complete before TMEM is freed
+      drain_wait(bar(kDqBarDone), 0);
     }
   } else {
     regs_inc<kDqRegsCompute>();
@@ -456,22 +477,33 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
     const BwdScales sc = bwd_scales(p);
     const float lse = p.lse[(int64_t)gq * p.Npad + qrow];
-    float* Dpart = reinterpret_cast<float*>(sm + L::oD);
-    float Dsum = 0.0f;
-    bool ok = true, combined = false;
-    // both streams' partial D of the row, once every sweep-1 tile is done
-    auto combine = [&]() {
-      Dpart[stream * kBwdQ + row] = Dsum;
-      named_bar_sync(1, 256);
-      Dsum = Dpart[row] + Dpart[kBwdQ + row];
-      if (stream == 0) p.Dvec[(int64_t)gq * p.Npad + qrow] = Dsum;
-      combined = true;
-    };
-    for (int t = stream; t < T; t += 2) {
-      if (!combined && t >= nkt) combine();
-      const int buf = t & 1, j = t % nkt;
+    bool ok = __all_sync(0xFFFFFFFFu, bwd_wait(bar(kDqBarQ), 0));
+    // c_i = dO_i . O_i: dO_i from the row's 128-byte-swizzled chunks, O_i from
+    // the forward's output (0 on padded rows)
+    float cv = 0.0f;
+    if (ok && qrow < p.N) {
+      const __nv_bfloat16* orow = p.out + ((int64_t)gq * p.N + qrow) * D;
+#pragma unroll
+      for (int a = 0; a < NA; ++a) {
+        const uint8_t* src = sm + L::oDO + a * kBwdQ * 128 + row * 128;
+#pragma unroll
+        for (int k2 = 0; k2 < 8; ++k2) {
+          float x[8], o[8];
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(src + ((k2 ^ (row & 7)) * 16)), x);
+          bf16x8_to_f32(ld_nc_v4(orow + a * 64 + k2 * 8), o);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) cv = fmaf(x[e], o[e], cv);
+        }
+      }
+    }
+    // this stream's sums: D' = sum P (dP - c), the same of the bf16-rounded
+    // terms that enter A, and sum P
+    float Dp = 0.0f, Dr = 0.0f, Sp = 0.0f;
+    const int qrow0 = qt * kBwdQ;  // the CTA's first row: tiles below it need no causal mask
+    for (int t = stream; t < nkt && ok; t += 2) {
+      const int buf = stream;
       float s[64], dp[64];
-      ok = ok && __all_sync(0xFFFFFFFFu, bwd_wait(bar(kDqBarSFull + buf), (t >> 1) & 1));
+      ok = __all_sync(0xFFFFFFFFu, bwd_wait(bar(kDqBarSFull + buf), (t >> 1) & 1));
       if (ok) {
         tc_fence_after();
         tmem_ld32(tl + buf * 128, s);
@@ -484,56 +516,94 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kDqBarSEmpty + buf));
       if (!ok) break;
-      const int key0 = j * kBwdKt;
+      const int key0 = t * kBwdKt;
+      if (key0 + kBwdKt <= p.N && (!CAUSAL || key0 + kBwdKt - 1 <= qrow0)) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const int key = key0 + c;
-        const bool live = key < p.N && (!CAUSAL || key <= qrow);
-        s[c] = live ? ex2_approx(fmaf(s[c], sc.c, -lse)) : 0.0f;  // P
+        for (int c = 0; c < 64; ++c) s[c] = ex2_approx(fmaf(s[c], sc.c, -lse));  // P
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const int key = key0 + c;
+          const bool live = key < p.N && (!CAUSAL || key <= qrow);
+          s[c] = live ? ex2_approx(fmaf(s[c], sc.c, -lse)) : 0.0f;
+        }
       }
-      if (t < nkt) {
-        float acc = 0.0f;
+      // x = P (dP - c) and its bf16 rounding r, the operand of A; pairwise
+      // sums (f32x2) of x, r and P, two chains each
+      uint32_t wp[32], wd[32];
+      uint64_t dx[2] = {0, 0}, dr[2] = {0, 0}, dsp[2] = {0, 0};
 #pragma unroll
-        for (int c = 0; c < 64; ++c) acc = fmaf(s[c], dp[c], acc);
-        Dsum = fmaf(acc, sc.dv, Dsum);
-        continue;
+      for (int c = 0; c < 32; ++c) {
+        const float x0 = s[2 * c] * fmaf(dp[2 * c], sc.dv, -cv);
+        const float x1 = s[2 * c + 1] * fmaf(dp[2 * c + 1], sc.dv, -cv);
+        wp[c] = pack_bf16(s[2 * c], s[2 * c + 1]);
+        wd[c] = pack_bf16(x0, x1);
+        dx[c & 1] = add2(dx[c & 1], pk(x0, x1));
+        dr[c & 1] = add2(dr[c & 1], pk(__uint_as_float(wd[c] << 16),
+                                       __uint_as_float(wd[c] & 0xFFFF0000u)));
+        dsp[c & 1] = add2(dsp[c & 1], pk(s[2 * c], s[2 * c + 1]));
       }
-      // dS = P (d_V dP - D) -> bf16, the row's 128 bytes (128-byte swizzle)
-      uint32_t w[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c)
-        w[c] = pack_bf16(s[2 * c] * fmaf(dp[2 * c], sc.dv, -Dsum),
-                         s[2 * c + 1] * fmaf(dp[2 * c + 1], sc.dv, -Dsum));
-      const int t2 = t - nkt;
-      if (t2 >= 2)
-        ok = __all_sync(0xFFFFFFFFu, bwd_wait(bar(kDqBarDsEmpty + buf), ((t2 >> 1) - 1) & 1));
+      {
+        float a0, a1, b0, b1;
+        upk(add2(dx[0], dx[1]), a0, a1);
+        Dp += a0 + a1;
+        upk(add2(dr[0], dr[1]), a0, a1);
+        Dr += a0 + a1;
+        upk(add2(dsp[0], dsp[1]), b0, b1);
+        Sp += b0 + b1;
+      }
+      if (t >= 2)
+        ok = __all_sync(0xFFFFFFFFu, bwd_wait(bar(kDqBarPEmpty + buf), ((t >> 1) - 1) & 1));
       if (!ok) break;
-      uint8_t* dsr = sm + L::oDS + buf * L::kDS + row * 128;
+      uint8_t* pr = sm + L::oP + buf * 2 * L::kPT + row * 128;
 #pragma unroll
-      for (int k2 = 0; k2 < 8; ++k2)
-        *reinterpret_cast<uint4*>(dsr + ((k2 ^ (row & 7)) * 16)) =
-            make_uint4(w[4 * k2], w[4 * k2 + 1], w[4 * k2 + 2], w[4 * k2 + 3]);
+      for (int k2 = 0; k2 < 8; ++k2) {
+        const int off = (k2 ^ (row & 7)) * 16;
+        *reinterpret_cast<uint4*>(pr + off) =
+            make_uint4(wp[4 * k2], wp[4 * k2 + 1], wp[4 * k2 + 2], wp[4 * k2 + 3]);
+        *reinterpret_cast<uint4*>(pr + L::kPT + off) =
+            make_uint4(wd[4 * k2], wd[4 * k2 + 1], wd[4 * k2 + 2], wd[4 * k2 + 3]);
+      }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kDqBarDsFull + buf));
+      if (lane == 0) mbar_arrive(bar(kDqBarPFull + buf));
     }
-    if (!combined) combine();
+    // every A / B contraction has read its P tiles: the P area holds the two
+    // streams' partial sums of the row
     ok = ok && __all_sync(0xFFFFFFFFu, bwd_wait(bar(kDqBarDone), 0));
+    float* part = reinterpret_cast<float*>(sm + L::oP);  // [stream][3][kBwdQ]
+    if (ok) {
+      part[(stream * 3 + 0) * kBwdQ + row] = Dp;
+      part[(stream * 3 + 1) * kBwdQ + row] = Dr;
+      part[(stream * 3 + 2) * kBwdQ + row] = Sp;
+    }
+    named_bar_sync(1, 256);  // both warpgroups, on every path
+    ok = __all_sync(0xFFFFFFFFu, ok && *reinterpret_cast<volatile unsigned*>(&g_fp4_err) == 0u);
     if (ok) {  // warp-uniform: tcgen05.ld is a whole-warp instruction; only the stores are per row
+      const float Dq = part[row] + part[3 * kBwdQ + row];                  // D'_i
+      const float Dqr = part[kBwdQ + row] + part[4 * kBwdQ + row];         // its rounded terms
+      const float Sq = part[2 * kBwdQ + row] + part[5 * kBwdQ + row];      // sum_j P_ij
+      // D_i - c_i for dQ, from the rounded terms that A holds: a row whose P
+      // sits on one key then gets dQ = 0 exactly, as dS = 0 there
+      const float E = fmaf(cv, Sq - 1.0f, Dqr);
+      if (stream == 0) p.Dvec[(int64_t)gq * p.Npad + qrow] = fmaf(cv, Sq, Dq);  // 0 on padded rows
       tc_fence_after();
       constexpr int DH = D / 2;  // each stream writes half the channels
       __nv_bfloat16* dst = p.dq + ((int64_t)gq * p.N + qrow) * D + stream * DH;
 #pragma unroll
       for (int cc = 0; cc < DH; cc += 32) {
-        float o[32];
+        float oa[32], ob[32];
         __syncwarp();
-        tmem_ld32(tl + 256 + stream * DH + cc, o);
+        tmem_ld32(tl + 256 + stream * DH + cc, oa);
+        tmem_ld32(tl + 256 + D + stream * DH + cc, ob);
         tmem_wait_ld();
         if (qrow < p.N) {
           uint32_t w[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) w[i] = pack_bf16(o[2 * i] * sc.sdq, o[2 * i + 1] * sc.sdq);
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack_bf16(fmaf(-E, ob[2 * i], oa[2 * i]) * sc.sdq,
+                             fmaf(-E, ob[2 * i + 1], oa[2 * i + 1]) * sc.sdq);
           uint4* d4 = reinterpret_cast<uint4*>(dst + cc);
 #pragma unroll
           for (int k4 = 0; k4 < 4; ++k4)

@@ -543,17 +543,18 @@ fp4_status_t attn_fwd_smooth_any(const void* q, const void* k, const void* v, vo
 // then the dk/dv kernel.
 // amax_in: the three tensor maxima (Q, K, V) to quantise with, e.g. combined
 // over shards, or NULL to compute them from q, k, v.
-fp4_status_t attn_bwd_any(const void* q, const void* k, const void* v, const void* dout,
-                          const float* lse, void* dq, void* dk, void* dv, int B, int H, int Hkv,
-                          int N, int D, int causal, float softmax_scale, void* stream,
+fp4_status_t attn_bwd_any(const void* q, const void* k, const void* v, const void* out,
+                          const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                          int H, int Hkv, int N, int D, int causal, float softmax_scale, void* stream,
                           void* workspace, size_t workspace_bytes,
                           const float* amax_in = nullptr) {
   g_last_error.clear();
   fp4_status_t s;
   if ((s = check_shape(B, H, Hkv, N, D)) != FP4_OK) return s;
-  if (!q || !k || !v || !dout || !lse || !dq || !dk || !dv || !workspace)
+  if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !workspace)
     return fail(FP4_ERR_INVALID_ARG, "null pointer");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned16(dq) ||
       !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u))
     return fail(FP4_ERR_INVALID_ARG, "pointers must be 16-byte aligned (lse 4-byte)");
@@ -619,6 +620,7 @@ fp4_status_t attn_bwd_any(const void* q, const void* k, const void* v, const voi
   p.amax = amax;
   p.lse = lsep;
   p.Dvec = dvec;
+  p.out = static_cast<const __nv_bfloat16*>(out);
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
@@ -694,25 +696,25 @@ size_t fp4_attn_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D) {
   return bwd_ws_layout(B, H, Hkv, N, D).total;
 }
 
-fp4_status_t fp4_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
-                          const float* lse, void* dq, void* dk, void* dv, int B, int H, int Hkv,
-                          int N, int D, int causal, float softmax_scale, void* stream,
-                          void* workspace, size_t workspace_bytes) {
-  return attn_bwd_any(q, k, v, dout, lse, dq, dk, dv, B, H, Hkv, N, D, causal, softmax_scale,
-                      stream, workspace, workspace_bytes);
+fp4_status_t fp4_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                          const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                          int H, int Hkv, int N, int D, int causal, float softmax_scale,
+                          void* stream, void* workspace, size_t workspace_bytes) {
+  return attn_bwd_any(q, k, v, out, dout, lse, dq, dk, dv, B, H, Hkv, N, D, causal,
+                      softmax_scale, stream, workspace, workspace_bytes);
 }
 
-fp4_status_t fp4_attn_bwd_scaled(const void* q, const void* k, const void* v, const void* dout,
-                                 const float* lse, const float* amax, void* dq, void* dk, void* dv,
-                                 int B, int H, int Hkv, int N, int D, int causal,
-                                 float softmax_scale, void* stream, void* workspace,
+fp4_status_t fp4_attn_bwd_scaled(const void* q, const void* k, const void* v, const void* out,
+                                 const void* dout, const float* lse, const float* amax, void* dq,
+                                 void* dk, void* dv, int B, int H, int Hkv, int N, int D,
+                                 int causal, float softmax_scale, void* stream, void* workspace,
                                  size_t workspace_bytes) {
   if (!amax) {
     g_last_error.clear();
     return fail(FP4_ERR_INVALID_ARG, "null pointer");
   }
-  return attn_bwd_any(q, k, v, dout, lse, dq, dk, dv, B, H, Hkv, N, D, causal, softmax_scale,
-                      stream, workspace, workspace_bytes, amax);
+  return attn_bwd_any(q, k, v, out, dout, lse, dq, dk, dv, B, H, Hkv, N, D, causal,
+                      softmax_scale, stream, workspace, workspace_bytes, amax);
 }
 
 fp4_status_t fp4_attn_fwd_quantized_lse(const fp4_tensor_t* q, const fp4_tensor_t* k,

@@ -133,12 +133,12 @@ def fp4_attn_fwd_sharded(q, k, v, causal: bool = False, softmax_scale: float | N
     return out
 
 
-def fp4_attn_bwd_sharded(q, k, v, dout, lse, causal: bool = False,
+def fp4_attn_bwd_sharded(q, k, v, out, dout, lse, causal: bool = False,
                          softmax_scale: float | None = None, group=None, dq=None, dk=None,
                          dv=None, stream=None):
     """This rank's part of the head-sharded FP4 attention backward: the same
-    units as fp4_attn_fwd_sharded (q, dout, lse: this rank's query heads; k,
-    v: its key/value heads), one all-reduce (MAX) of the three maxima so that
+    units as fp4_attn_fwd_sharded (q, out, dout, lse: this rank's query heads;
+    k, v: its key/value heads; out the forward's output), one all-reduce (MAX) of the three maxima so that
     the operands are quantised as the whole tensors' are, then fp4_attn_bwd
     on the shard. Every rank of `group` calls it, an empty shard included.
     Returns (dq, dk, dv) for the shard."""
@@ -160,6 +160,6 @@ def fp4_attn_bwd_sharded(q, k, v, dout, lse, causal: bool = False,
     if gkv == 0:
         return dq, dk, dv
     as4 = lambda t: t.view(1, -1, N, D)
-    fp4_attn_bwd(as4(q), as4(k), as4(v), as4(dout), lse.reshape(1, gq, N), causal, softmax_scale,
-                 dq=as4(dq), dk=as4(dk), dv=as4(dv), stream=stream, amax=amax)
+    fp4_attn_bwd(as4(q), as4(k), as4(v), as4(out), as4(dout), lse.reshape(1, gq, N), causal,
+                 softmax_scale, dq=as4(dq), dk=as4(dk), dv=as4(dv), stream=stream, amax=amax)
     return dq, dk, dv

@@ -335,11 +335,18 @@ fp4_status_t fp4_attn_fwd_lse(const void* q, const void* k, const void* v, void*
  *               not FlashAttention's dO . O, which assumes O = P V exactly
  *   dS = P (dP - D),  dq = scale dS k~,  dk = scale dS^T q~,  dv = P^T dO
  *   (dk, dv summed over the query heads of each key/value head)
- * with straight-through quantisers. Inputs: q, k, v as fp4_attn_fwd; dout
- * [B][H][N][D] bf16; lse from fp4_attn_fwd_lse. Outputs (bf16): dq
- * [B][H][N][D], dk and dv [B][Hkv][N][D]. The contractions run on the tensor
- * cores in bf16 with fp32 accumulation (P and dS rounded to bf16 for theirs).
- * workspace: fp4_attn_bwd_workspace_bytes(B, H, Hkv, N, D) bytes.
+ * with straight-through quantisers. Inputs: q, k, v as fp4_attn_fwd; out
+ * [B][H][N][D] bf16, the forward's output; dout [B][H][N][D] bf16; lse from
+ * fp4_attn_fwd_lse. Outputs (bf16): dq [B][H][N][D], dk and dv
+ * [B][Hkv][N][D]. The contractions run on the tensor cores in bf16 with fp32
+ * accumulation (P and dS rounded to bf16 for theirs). dq is accumulated in
+ * one pass over the keys as A - (D - c) B with A = sum_j P_ij (dP_ij - c_i)
+ * k~_j, B = sum_j P_ij k~_j and c_i = dO_i . out_i: out enters only through
+ * c, an identity's free constant, so it changes the rounding and not the
+ * definition above (D stays this P's; out close to P v~ keeps the terms of A
+ * small). All device pointers 16-byte aligned (lse 4-byte); none may be NULL
+ * (FP4_ERR_INVALID_ARG). workspace: fp4_attn_bwd_workspace_bytes(B, H, Hkv,
+ * N, D) bytes, else FP4_ERR_WORKSPACE. The library owns no argument.
  */
 size_t fp4_attn_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D);
 /*
@@ -350,19 +357,19 @@ size_t fp4_attn_bwd_workspace_bytes(int B, int H, int Hkv, int N, int D);
  * operands are quantised as the whole tensors' are; and the training forward
  * on quantised tensors (fp4_quantize_scaled with the same maxima) writing lse.
  */
-fp4_status_t fp4_attn_bwd_scaled(const void* q, const void* k, const void* v, const void* dout,
-                                 const float* lse, const float* amax, void* dq, void* dk, void* dv,
-                                 int B, int H, int Hkv, int N, int D, int causal,
-                                 float softmax_scale, void* stream, void* workspace,
+fp4_status_t fp4_attn_bwd_scaled(const void* q, const void* k, const void* v, const void* out,
+                                 const void* dout, const float* lse, const float* amax, void* dq,
+                                 void* dk, void* dv, int B, int H, int Hkv, int N, int D,
+                                 int causal, float softmax_scale, void* stream, void* workspace,
                                  size_t workspace_bytes);
 fp4_status_t fp4_attn_fwd_quantized_lse(const fp4_tensor_t* q, const fp4_tensor_t* k,
                                         const fp4_tensor_t* v, void* out, float* lse, int B,
                                         int H, int Hkv, int N, int D, int causal,
                                         float softmax_scale, void* stream);
-fp4_status_t fp4_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
-                          const float* lse, void* dq, void* dk, void* dv, int B, int H, int Hkv,
-                          int N, int D, int causal, float softmax_scale, void* stream,
-                          void* workspace, size_t workspace_bytes);
+fp4_status_t fp4_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                          const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                          int H, int Hkv, int N, int D, int causal, float softmax_scale,
+                          void* stream, void* workspace, size_t workspace_bytes);
 
 size_t fp4_attn_workspace_bytes_fp8pv(int B, int H, int Hkv, int N, int D);
 fp4_status_t fp4_attn_fwd_fp8pv(const void* q, const void* k, const void* v, void* out, int B,

@@ -130,20 +130,23 @@ def test_argument_errors_launch_nothing(L):
     assert L.fp4_attn_fwd_quantized_bias(ctypes.byref(t), ctypes.byref(t), ctypes.byref(t),
                                          vp(0), vp(16), 1, 1, 1, 8, 128, 0, 0.0, vp(0)) == \
         fa.FP4_ERR_INVALID_ARG
-    # backward: workspace size, null lse, misaligned output, too small a workspace
+    # backward: workspace size, null lse, null out, misaligned output, too small a workspace
     wb = fa.lib().fp4_attn_bwd_workspace_bytes(1, 2, 1, 300, 128)
     assert wb >= 2 * 384 * 128 * 2 * 4  # Q^, Q^T, dO, dO^T at least
     assert fa.lib().fp4_attn_bwd_workspace_bytes(1, 3, 2, 300, 128) == 0
-    bwd = lambda lse=16, dq=16, wsz=1 << 34: L.fp4_attn_bwd(
-        vp(16), vp(16), vp(16), vp(16), vp(lse), vp(dq), vp(16), vp(16), 1, 2, 1, 300, 128, 0,
-        0.0, vp(0), vp(16), wsz)
+    bwd = lambda lse=16, dq=16, o=16, wsz=1 << 34: L.fp4_attn_bwd(
+        vp(16), vp(16), vp(16), vp(o), vp(16), vp(lse), vp(dq), vp(16), vp(16), 1, 2, 1, 300,
+        128, 0, 0.0, vp(0), vp(16), wsz)
     assert bwd(lse=0) == fa.FP4_ERR_INVALID_ARG
+    assert bwd(o=0) == fa.FP4_ERR_INVALID_ARG
+    assert bwd(o=40) == fa.FP4_ERR_INVALID_ARG
     assert bwd(dq=24) == fa.FP4_ERR_INVALID_ARG
     assert bwd(wsz=wb - 1) == fa.FP4_ERR_WORKSPACE
     assert L.fp4_attn_fwd_lse(vp(16), vp(16), vp(16), vp(16), vp(0), 1, 1, 1, 8, 128, 0, 0.0,
                               vp(0), vp(16), 1 << 30) == fa.FP4_ERR_INVALID_ARG
-    assert L.fp4_attn_bwd_scaled(vp(16), vp(16), vp(16), vp(16), vp(16), vp(0), vp(16), vp(16),
-                                 vp(16), 1, 2, 1, 300, 128, 0, 0.0, vp(0), vp(16), 1 << 34) == \
+    assert L.fp4_attn_bwd_scaled(vp(16), vp(16), vp(16), vp(16), vp(16), vp(16), vp(0), vp(16),
+                                 vp(16), vp(16), 1, 2, 1, 300, 128, 0, 0.0, vp(0), vp(16),
+                                 1 << 34) == \
         fa.FP4_ERR_INVALID_ARG  # no maxima
     assert L.fp4_attn_fwd_quantized_lse(ctypes.byref(t), ctypes.byref(t), ctypes.byref(t), vp(16),
                                         vp(0), 1, 1, 1, 8, 128, 0, 0.0, vp(0)) == \

@@ -46,7 +46,7 @@ def run_gpu(q, k, v, do, causal, softmax_scale=0.0):
     import torch
     dq_, dk_, dv_, ddo = (to_dev(t) for t in (q, k, v, do))
     out, lse = fa.fp4_attn_fwd_lse(dq_, dk_, dv_, causal=causal, softmax_scale=softmax_scale or None)
-    gq, gk, gv = fa.fp4_attn_bwd(dq_, dk_, dv_, ddo, lse, causal=causal,
+    gq, gk, gv = fa.fp4_attn_bwd(dq_, dk_, dv_, out, ddo, lse, causal=causal,
                                  softmax_scale=softmax_scale or None)
     torch.cuda.synchronize()
     fa.fp4_status()

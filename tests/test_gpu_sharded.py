@@ -159,13 +159,13 @@ def test_training_pass_one_rank_equals_unsharded(syn, case):
     q, k, v, _ = _inputs(syn, B, H, Hkv, N, D, 900)
     do = to_dev(syn.normal_bf16(B * H * N * D, 901, 4).reshape(B, H, N, D))
     out, lse = fa.fp4_attn_fwd_lse(q, k, v, causal=causal)
-    grads = fa.fp4_attn_bwd(q, k, v, do, lse, causal=causal)
+    grads = fa.fp4_attn_bwd(q, k, v, out, do, lse, causal=causal)
     lse_s = torch.empty(B * H * N, dtype=torch.float32, device="cuda")
     out_s = fa.fp4_attn_fwd_sharded(q.view(B * H, N, D), k.view(B * Hkv, N, D),
                                     v.view(B * Hkv, N, D), causal=causal, lse=lse_s)
     grads_s = fa.fp4_attn_bwd_sharded(q.view(B * H, N, D), k.view(B * Hkv, N, D),
-                                      v.view(B * Hkv, N, D), do.view(B * H, N, D), lse_s,
-                                      causal=causal)
+                                      v.view(B * Hkv, N, D), out_s.view(B * H, N, D),
+                                      do.view(B * H, N, D), lse_s, causal=causal)
     torch.cuda.synchronize()
     fa.fp4_status()
     assert torch.equal(out.view(-1), out_s.view(-1))
@@ -185,7 +185,7 @@ def test_emulated_training_shards_equal_unsharded(syn, case, world):
     q, k, v, _ = _inputs(syn, B, H, Hkv, N, D, 910 + world)
     do = to_dev(syn.normal_bf16(B * H * N * D, 911, 4).reshape(B, H, N, D))
     out, lse = fa.fp4_attn_fwd_lse(q, k, v, causal=causal)
-    gq_, gk_, gv_ = fa.fp4_attn_bwd(q, k, v, do, lse, causal=causal)
+    gq_, gk_, gv_ = fa.fp4_attn_bwd(q, k, v, out, do, lse, causal=causal)
     qf, kf, vf, dof = (t.view(-1, N, D) for t in (q, k, v, do))
     shards = [fa.shard_rows(B, H, Hkv, world, r) for r in range(world)]
     shards = [(sq, skv) for sq, skv in shards if skv.stop > skv.start]
@@ -201,8 +201,8 @@ def test_emulated_training_shards_equal_unsharded(syn, case, world):
         lse_s = torch.empty(g1 * N, dtype=torch.float32, device="cuda")
         out_s = fa.fp4_attn_fwd_quantized(qs, ks, vs, 1, g1, g2, causal=causal, lse=lse_s)
         as4 = lambda t: t.contiguous().view(1, -1, N, D)
-        d = fa.fp4_attn_bwd(as4(qf[sq]), as4(kf[skv]), as4(vf[skv]), as4(dof[sq]),
-                            lse_s.view(1, g1, N), causal=causal, amax=amax)
+        d = fa.fp4_attn_bwd(as4(qf[sq]), as4(kf[skv]), as4(vf[skv]), as4(out_s),
+                            as4(dof[sq]), lse_s.view(1, g1, N), causal=causal, amax=amax)
         torch.cuda.synchronize()
         fa.fp4_status()
         assert torch.equal(out_s.view(-1), out.view(-1, N, D)[sq].reshape(-1))

@@ -81,7 +81,7 @@ def test_sharded_wrappers_check_shapes_first():
     with pytest.raises(ValueError):  # 6 query heads for 4 key/value heads
         fa.fp4_attn_fwd_sharded(q, k, k)
     with pytest.raises(ValueError):
-        fa.fp4_attn_bwd_sharded(q, k, k, q, torch.zeros(6 * 8))
+        fa.fp4_attn_bwd_sharded(q, k, k, q, q, torch.zeros(6 * 8))
     with pytest.raises(ValueError):  # smoothing with another P generation
         fa.fp4_attn_fwd_sharded(q[:4], k, k, smooth=fa.FP4_SMOOTH_Q, efq=True)
     with pytest.raises(ValueError):  # lse with smoothing
