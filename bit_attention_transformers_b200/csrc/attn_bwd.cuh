@@ -13,18 +13,23 @@
 // with straight-through quantisers (the gradients of q~, k~, v~ serve as
 // those of q, k, v).
 //
-// Kernels (all contractions on tcgen05 kind::f16, bf16 operands from shared
-// memory, fp32 accumulators in TMEM; every operand K-major with the 128-byte
-// swizzle, transposed copies prepared by the pre-kernels so that no MN-major
-// operand is needed):
+// Kernels (contractions on tcgen05 with fp32 accumulators in TMEM: the dk/dv
+// kernel's S^T on kind::mxf4nvf4 from the forward's NVFP4 codes, every other
+// one on kind::f16 with bf16 operands, K-major with the 128-byte swizzle,
+// transposed copies prepared by the pre-kernels so that no MN-major operand is
+// needed):
+//   quant_rows_kernel  the forward's own quantiser: Q's and K's NVFP4 codes
+//       and block scales, for S^T
 //   fq_rows_kernel / fq_tokens_kernel  the forward's quantisers, decoded to
 //       bf16 (Q^, K^ and their transposes; V^), bit-identical codes and scales
 //   pad_transpose_kernel  dO padded to Npad rows, and dO^T
 //   lse_pad_kernel        lse padded with +inf (padded rows get P = 0)
 //   bwd_dq_kernel   one CTA per 128 query rows, one pass over the key tiles:
 //       D and dQ (dQ from two sums accumulated in TMEM, see the kernel)
+//   sf64_kernel     Q's block scales regrouped per 64-query tile
 //   bwd_dkdv_kernel one CTA per 128 keys: over the query tiles of every query
-//       head of its key/value head, dV += P^T dO and dK += dS^T Q^ in TMEM
+//       head of its key/value head, S^T from the NVFP4 codes (kind::mxf4nvf4),
+//       dV += P^T dO and dK += dS^T Q^ in TMEM
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -36,7 +41,9 @@
 
 namespace fp4 {
 
-constexpr int kBwdThreads = 256;  // warp 0 loads, warp 1 issues MMAs, warps 4-7 compute
+// dk/dv kernel: warps 0 and 2 load, warp 1 issues MMAs, warps 4-11 compute
+// (two warps per TMEM lane quarter, each on half of a tile's 64 queries)
+constexpr int kBwdThreads = 384;
 constexpr int kBwdQ = 128;        // dq kernel: query rows per CTA
 constexpr int kBwdKt = 64;        // dq kernel: keys per tile
 constexpr int kBwdK = 128;        // dk/dv kernel: keys per CTA
@@ -225,6 +232,22 @@ __global__ void __launch_bounds__(128) pad_transpose_kernel(const __nv_bfloat16*
   }
 }
 
+// Block scales of Q in the forward's layout (atoms of 128 rows: row r of a
+// 64-element chunk at byte (r % 32) 16 + (r / 32) 4 + k) -> one atom per
+// 64-row tile whose 4-byte columns 0 and 1 hold the tile's rows: the lower
+// tile's atom is the same bytes, the upper tile's swaps the two 8-byte halves
+// of every 16-byte lane. One thread per 16 bytes of the input.
+__global__ void sf64_kernel(const uint4* __restrict__ sf, int64_t n16, int atom16,
+                            uint4* __restrict__ sf64) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t tile = i / atom16, j = i % atom16;
+    const uint4 w = sf[i];
+    sf64[(2 * tile) * atom16 + j] = w;
+    sf64[(2 * tile + 1) * atom16 + j] = make_uint4(w.z, w.w, w.x, w.y);
+  }
+}
+
 // lse [G][N] -> [G][Npad], +inf beyond N.
 __global__ void lse_pad_kernel(const float* __restrict__ lse, int64_t G, int N, int Npad,
                                float* __restrict__ out) {
@@ -242,6 +265,8 @@ struct BwdParams {
   const float* lse;    // [B*H][Npad], +inf on padded rows
   float* Dvec;         // [B*H][Npad]: D, written by the dq kernel
   const __nv_bfloat16* out;  // [B][H][N][D]: the forward's output O (centres dP, dq kernel)
+  const uint8_t* k_sf;       // K block scales, the forward's layout (one atom set per 128 keys)
+  const uint8_t* q_sf64;     // Q block scales, one atom set per 64-query tile (sf64_kernel)
   __nv_bfloat16* dq;   // [B][H][N][D]
   __nv_bfloat16* dk;   // [B][Hkv][N][D]
   __nv_bfloat16* dv;
@@ -621,48 +646,72 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 }
 
 // ----------------------------------------------------------- dk/dv kernel ----
+// S^T = K^ Q^T straight from the forward's NVFP4 codes and block scales
+// (tcgen05 kind::mxf4nvf4, M = 128 keys, N = 64 queries, K = 64 per
+// instruction), the other contractions in bf16. The block scales of a
+// 64-query B operand: the forward stores one scale atom per 128 rows (row r
+// of chunk k at byte (r % 32) 16 + (r / 32) 4 + k, copied to TMEM with
+// tcgen05.cp 32x128b.warpx4, where row r's four scales sit in column r / 32);
+// an N = 64 operand reads columns 0 and 1, so sf64_kernel stores for every
+// 64-query tile an atom whose first two columns hold its rows.
 template <int D>
 struct BwdDkvSmem {
-  static constexpr int kK = kBwdK * D * 2;     // K^ or V^ tile, bf16
-  static constexpr int kQ = kBwdQt * D * 2;    // Q^ or dO tile
-  static constexpr int kQT = D * kBwdQt * 2;   // Q^T or dO^T tile
-  static constexpr int oK = 0;
-  static constexpr int oV = oK + kK;
-  static constexpr int oA = oV + kK;          // ring A [2]: Q^ then dO (S^T, dP^T)
-  static constexpr int oB = oA + 2 * 2 * kQ;  // ring B [2]: Q^T then dO^T (dK, dV)
+  static constexpr int kK = kBwdK * D * 2;      // V^ tile (128 keys), bf16
+  static constexpr int kKc = kBwdK * D / 2;     // K codes (128 keys)
+  static constexpr int kSf = (D / 64) * 512;    // scale atoms of one tile, one per 64-element chunk
+  static constexpr int kQ = kBwdQt * D * 2;     // dO tile (64 queries), bf16
+  static constexpr int kQc = kBwdQt * D / 2;    // Q codes (64 queries)
+  static constexpr int kQT = D * kBwdQt * 2;    // Q^T or dO^T tile
+  static constexpr int kSlotA = (kQ + kQc + kSf + 1023) / 1024 * 1024;  // dO, Q codes, Q scales
+  static constexpr int oV = 0;
+  static constexpr int oKc = oV + kK;
+  static constexpr int oKsf = oKc + kKc;
+  static constexpr int oA = oKsf + (kSf + 1023) / 1024 * 1024;  // ring A [2] (S^T, dP^T)
+  static constexpr int oB = oA + 2 * kSlotA;          // ring B [2]: Q^T then dO^T (dK, dV)
   static constexpr int oP = oB + 2 * 2 * kQT;         // P^T: 128 keys x 64 queries, bf16
   static constexpr int oDS = oP + kBwdK * kBwdQt * 2; // dS^T
   static constexpr int oLse = oDS + kBwdK * kBwdQt * 2;  // ring B [2]: lse[64], D[64]
   static constexpr int oBar = oLse + 2 * 512;
   static constexpr int oTmem = oBar + 256;
   static constexpr int kBytes = oTmem + 16 + 1024;
+  static_assert(kBytes <= 232448, "shared memory of one CTA");
 };
 
-// Ring A (Q^, dO) is released when S^T and dP^T complete; ring B (Q^T, dO^T,
-// lse, D) when dV and dK complete; each has its own producer warp.
+// Ring A (dO, Q codes and scales) is released when S^T and dP^T complete;
+// ring B (Q^T, dO^T, lse, D) when dV and dK complete; each has its own
+// producer warp. One S^T/dP^T buffer: the compute warps copy it to registers
+// at once, so the next tile's S^T and dP^T run while they work on this one.
 enum : int {
   kKvBarKV = 0,
   kKvBarFullA = 1,    // [2]
   kKvBarEmptyA = 3,   // [2]
   kKvBarFullB = 5,    // [2]
   kKvBarEmptyB = 7,   // [2]
-  kKvBarSFull = 9,    // [2]
-  kKvBarSEmpty = 11,  // [2]
-  kKvBarPFull = 13,
-  kKvBarPEmpty = 14,
-  kKvBarDone = 15,
+  kKvBarSFull = 9,
+  kKvBarSEmpty = 10,
+  kKvBarPFull = 11,
+  kKvBarPEmpty = 12,
+  kKvBarDone = 13,
+};
+
+// TMEM columns of the dk/dv kernel.
+template <int D>
+struct DkvCols {
+  static constexpr uint32_t kS = 0, kDP = 64, kDV = 128, kDK = 128 + D, kKsf = 128 + 2 * D,
+                            kQsf = kKsf + 8;  // [2] x 8
+  static_assert(kQsf + 16 <= 512, "TMEM columns");
 };
 
 // One CTA per (128-key tile, key/value head, batch); tiles of 64 queries of
-// every query head of the group. TMEM: S^T[b] at 128 b, dP^T[b] at 128 b + 64,
-// dV at 256, dK at 256 + D.
+// every query head of the group.
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kBwdThreads, 1)
-    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                    const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmKc, const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmQc, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmQT,
                     const __grid_constant__ CUtensorMap tmDOT, const BwdParams p) {
   using L = BwdDkvSmem<D>;
+  using TC = DkvCols<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -683,10 +732,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar(kKvBarEmptyA + s), 1);
       mbar_init(bar(kKvBarFullB + s), 1);
       mbar_init(bar(kKvBarEmptyB + s), 1);
-      mbar_init(bar(kKvBarSFull + s), 1);
-      mbar_init(bar(kKvBarSEmpty + s), 4);
     }
-    mbar_init(bar(kKvBarPFull), 4);
+    mbar_init(bar(kKvBarSFull), 1);
+    mbar_init(bar(kKvBarSEmpty), 8);
+    mbar_init(bar(kKvBarPFull), 8);
     mbar_init(bar(kKvBarPEmpty), 1);
     mbar_init(bar(kKvBarDone), 1);
     fence_mbar_init();
@@ -700,30 +749,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + L::oTmem);
   constexpr int NA = D / 64;
+  const int64_t ntq128 = p.Npad / 128;
 
   if (warp == 0) {
     if (lane == 0) {
       bool ok = true;
       int issued = 0;
-      mbar_arrive_expect_tx(bar(kKvBarKV), 2 * L::kK);
-      for (int a = 0; a < NA; ++a) {
-        tma_load_2d(sb + L::oK + a * kBwdK * 128, &tmK, a * 64, gk * p.Npad + kt * kBwdK,
-                    bar(kKvBarKV));
+      mbar_arrive_expect_tx(bar(kKvBarKV), L::kK + L::kKc + L::kSf);
+      for (int a = 0; a < NA; ++a)
         tma_load_2d(sb + L::oV + a * kBwdK * 128, &tmV, a * 64, gk * p.Npad + kt * kBwdK,
                     bar(kKvBarKV));
-      }
-      for (int t = 0; t < T && ok; ++t) {  // ring A: Q^ and dO
+      tma_load_2d(sb + L::oKc, &tmKc, 0, gk * p.Npad + kt * kBwdK, bar(kKvBarKV));
+      bulk_load(sb + L::oKsf, p.k_sf + ((int64_t)gk * ntq128 + kt) * L::kSf, L::kSf,
+                bar(kKvBarKV));
+      for (int t = 0; t < T && ok; ++t) {  // ring A: dO, Q codes and scales
         const int st = t & 1;
         const int gq = b * p.H + hk * G + t / nqt, i = i0 + t % nqt;
         if (t >= 2 && !(ok = bwd_wait(bar(kKvBarEmptyA + st), ((t >> 1) - 1) & 1))) break;
-        const uint32_t base = sb + L::oA + st * 2 * L::kQ;
-        mbar_arrive_expect_tx(bar(kKvBarFullA + st), 2 * L::kQ);
-        for (int a = 0; a < NA; ++a) {
-          tma_load_2d(base + a * kBwdQt * 128, &tmQ, a * 64, gq * p.Npad + i * kBwdQt,
+        const uint32_t base = sb + L::oA + st * L::kSlotA;
+        mbar_arrive_expect_tx(bar(kKvBarFullA + st), L::kQ + L::kQc + L::kSf);
+        for (int a = 0; a < NA; ++a)
+          tma_load_2d(base + a * kBwdQt * 128, &tmDO, a * 64, gq * p.Npad + i * kBwdQt,
                       bar(kKvBarFullA + st));
-          tma_load_2d(base + L::kQ + a * kBwdQt * 128, &tmDO, a * 64, gq * p.Npad + i * kBwdQt,
-                      bar(kKvBarFullA + st));
-        }
+        tma_load_2d(base + L::kQ, &tmQc, 0, gq * p.Npad + i * kBwdQt, bar(kKvBarFullA + st));
+        bulk_load(base + L::kQ + L::kQc, p.q_sf64 + ((int64_t)gq * (2 * ntq128) + i) * L::kSf,
+                  L::kSf, bar(kKvBarFullA + st));
         issued = t + 1;
       }
       drain_wait(bar(kKvBarKV), 0);
@@ -753,8 +803,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
+      constexpr uint32_t kSw = (D == 128) ? 4u : 6u;     // codes: 64- or 32-byte swizzle
+      constexpr uint32_t kSbo = (D == 128) ? 512u : 256u;
+      const uint32_t idS = idesc_mxf4nvf4(kBwdK, kBwdQt), idP = idesc_bf16(kBwdK, kBwdQt);
+      const uint32_t idO = idesc_bf16(kBwdK, D);
       bool ok = bwd_wait(bar(kKvBarKV), 0);
-      const uint32_t idS = idesc_bf16(kBwdK, kBwdQt), idO = idesc_bf16(kBwdK, D);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int kc = 0; kc < NA; ++kc)
+          tc_cp_32x128b_x4(tmem + TC::kKsf + 4 * kc, smem_desc(sb + L::oKsf + 512 * kc, 0, 128, 0));
+      }
       auto issue_kv = [&](int t) {  // dV += P^T dO, dK += dS^T Q^ of tile t
         const int st = t & 1;
         ok = ok && bwd_wait(bar(kKvBarPFull), t & 1);
@@ -765,28 +824,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int s = 0; s < kBwdQt / 16; ++s) {
           const uint32_t acc = (t > 0 || s > 0) ? 1u : 0u;
-          mma_bf16(tmem + 256, kmaj_desc(sb + L::oP, kBwdK, s), kmaj_desc(base + L::kQT, D, s),
+          mma_bf16(tmem + TC::kDV, kmaj_desc(sb + L::oP, kBwdK, s), kmaj_desc(base + L::kQT, D, s),
                    idO, acc);
-          mma_bf16(tmem + 256 + D, kmaj_desc(sb + L::oDS, kBwdK, s), kmaj_desc(base, D, s), idO,
+          mma_bf16(tmem + TC::kDK, kmaj_desc(sb + L::oDS, kBwdK, s), kmaj_desc(base, D, s), idO,
                    acc);
         }
         tc_commit(bar(kKvBarEmptyB + st));
         tc_commit(bar(kKvBarPEmpty));
       };
       for (int t = 0; t < T && ok; ++t) {
-        const int st = t & 1, buf = t & 1;
+        const int st = t & 1;
         if (!(ok = bwd_wait(bar(kKvBarFullA + st), (t >> 1) & 1))) break;
-        if (t >= 2 && !(ok = bwd_wait(bar(kKvBarSEmpty + buf), ((t >> 1) - 1) & 1))) break;
+        if (t >= 1 && !(ok = bwd_wait(bar(kKvBarSEmpty), (t - 1) & 1))) break;
         tc_fence_after();
-        const uint32_t base = sb + L::oA + st * 2 * L::kQ;
+        const uint32_t base = sb + L::oA + st * L::kSlotA;
+        const uint32_t tQsf = tmem + TC::kQsf + 8 * st;
 #pragma unroll
-        for (int s = 0; s < D / 16; ++s) {
-          mma_bf16(tmem + buf * 128, kmaj_desc(sb + L::oK, kBwdK, s), kmaj_desc(base, kBwdQt, s),
-                   idS, s > 0 ? 1u : 0u);
-          mma_bf16(tmem + buf * 128 + 64, kmaj_desc(sb + L::oV, kBwdK, s),
-                   kmaj_desc(base + L::kQ, kBwdQt, s), idS, s > 0 ? 1u : 0u);
-        }
-        tc_commit(bar(kKvBarSFull + buf));
+        for (int kc = 0; kc < NA; ++kc)
+          tc_cp_32x128b_x4(tQsf + 4 * kc, smem_desc(base + L::kQ + L::kQc + 512 * kc, 0, 128, 0));
+#pragma unroll
+        for (int kc = 0; kc < NA; ++kc)
+          mma_mxf4nvf4(tmem + TC::kS, smem_desc(sb + L::oKc + 32 * kc, 16, kSbo, kSw),
+                       smem_desc(base + L::kQ + 32 * kc, 16, kSbo, kSw), idS,
+                       tmem + TC::kKsf + 4 * kc, tQsf + 4 * kc, kc > 0 ? 1u : 0u);
+#pragma unroll
+        for (int s = 0; s < D / 16; ++s)
+          mma_bf16(tmem + TC::kDP, kmaj_desc(sb + L::oV, kBwdK, s), kmaj_desc(base, kBwdQt, s), idP,
+                   s > 0 ? 1u : 0u);
+        tc_commit(bar(kKvBarSFull));
         tc_commit(bar(kKvBarEmptyA + st));
         if (t > 0) issue_kv(t - 1);
       }
@@ -795,39 +860,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       drain_wait(bar(kKvBarDone), 0);
     }
   } else if (warp >= 4) {
-    const int quad = warp & 3, row = quad * 32 + lane, key = kt * kBwdK + row;
+    // this warp: the rows of its lane quarter, queries half * 32 .. + 31 of each tile
+    const int quad = warp & 3, half = (warp - 4) >> 2;
+    const int row = quad * 32 + lane, key = kt * kBwdK + row;
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
     const BwdScales sc = bwd_scales(p);
     bool ok = true;
     for (int t = 0; t < T; ++t) {
-      const int st = t & 1, buf = t & 1, i = i0 + t % nqt;
-      float s[64], dp[64];
-      ok = ok && __all_sync(0xFFFFFFFFu, bwd_wait(bar(kKvBarSFull + buf), (t >> 1) & 1));
+      const int st = t & 1, i = i0 + t % nqt;
+      float s[32], dp[32];
+      ok = ok && __all_sync(0xFFFFFFFFu, bwd_wait(bar(kKvBarSFull), t & 1));
       if (ok) {
         tc_fence_after();
-        tmem_ld32(tl + buf * 128, s);
-        tmem_ld32(tl + buf * 128 + 32, s + 32);
-        tmem_ld32(tl + buf * 128 + 64, dp);
-        tmem_ld32(tl + buf * 128 + 96, dp + 32);
+        tmem_ld32(tl + TC::kS + half * 32, s);
+        tmem_ld32(tl + TC::kDP + half * 32, dp);
         tmem_wait_ld();
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kKvBarSEmpty + buf));
+      if (lane == 0) mbar_arrive(bar(kKvBarSEmpty));
       if (!ok) break;
       // the stage's lse and D: its full barrier has completed (S^T was issued
       // after it); the wait makes the bulk copies' data visible to this thread
       ok = __all_sync(0xFFFFFFFFu, bwd_wait(bar(kKvBarFullB + st), (t >> 1) & 1));
       if (!ok) break;
-      const float* lq = reinterpret_cast<const float*>(sm + L::oLse + st * 512);
+      // this half's lse and D (a predicated select per pair: a separate
+      // unmasked path for full tiles measured slower)
+      const float* lq = reinterpret_cast<const float*>(sm + L::oLse + st * 512) + half * 32;
       const float* dq = lq + 64;
-      uint32_t wp[32], wd[32];
+      const int q0 = i * kBwdQt + half * 32;
+      uint32_t wp[16], wd[16];
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
+      for (int c = 0; c < 32; c += 2) {
         float pv[2], dv2[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-          const int q = i * kBwdQt + c + u;
+          const int q = q0 + c + u;
           const bool live = key < p.N && q < p.N && (!CAUSAL || key <= q);
           pv[u] = live ? ex2_approx(fmaf(s[c + u], sc.c, -lq[c + u])) : 0.0f;
           dv2[u] = pv[u] * fmaf(dp[c + u], sc.dv, -dq[c + u]);
@@ -840,12 +908,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       uint8_t* pr = sm + L::oP + row * 128;
       uint8_t* dr = sm + L::oDS + row * 128;
 #pragma unroll
-      for (int k2 = 0; k2 < 8; ++k2) {
-        const int off = (k2 ^ (row & 7)) * 16;
+      for (int j = 0; j < 4; ++j) {  // 16-byte chunks half * 4 + j of the row (128-byte swizzle)
+        const int off = ((half * 4 + j) ^ (row & 7)) * 16;
         *reinterpret_cast<uint4*>(pr + off) =
-            make_uint4(wp[4 * k2], wp[4 * k2 + 1], wp[4 * k2 + 2], wp[4 * k2 + 3]);
+            make_uint4(wp[4 * j], wp[4 * j + 1], wp[4 * j + 2], wp[4 * j + 3]);
         *reinterpret_cast<uint4*>(dr + off) =
-            make_uint4(wd[4 * k2], wd[4 * k2 + 1], wd[4 * k2 + 2], wd[4 * k2 + 3]);
+            make_uint4(wd[4 * j], wd[4 * j + 1], wd[4 * j + 2], wd[4 * j + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -858,12 +926,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       __nv_bfloat16* dvp = p.dv + ((int64_t)gk * p.N + key) * D;
       __nv_bfloat16* dkp = p.dk + ((int64_t)gk * p.N + key) * D;
 #pragma unroll
-      for (int cc = 0; cc < D; cc += 32) {
+      for (int cc = half * (D / 2); cc < (half + 1) * (D / 2); cc += 32) {  // this warp's channels
         float o[32], o2[32];
         if (T > 0) {
           __syncwarp();
-          tmem_ld32(tl + 256 + cc, o);
-          tmem_ld32(tl + 256 + D + cc, o2);
+          tmem_ld32(tl + TC::kDV + cc, o);
+          tmem_ld32(tl + TC::kDK + cc, o2);
           tmem_wait_ld();
         } else {
 #pragma unroll

@@ -220,7 +220,7 @@ WsLayout ws_layout(int B, int H, int Hkv, int N, int D, bool fp8v = false, bool 
 // Workspace of the backward: the maxima, the decoded operands (Q^, Q^T, K^,
 // K^T, V^), dO padded and transposed, lse padded, D.
 struct BwdWs {
-  size_t amax, qh, qt, kh, kt, vh, dop, dot, lse, dvec, total;
+  size_t amax, qh, qt, kh, kt, vh, dop, dot, lse, dvec, qc, qs, qs64, kc, ks, total;
 };
 
 BwdWs bwd_ws_layout(int B, int H, int Hkv, int N, int D) {
@@ -243,6 +243,11 @@ BwdWs bwd_ws_layout(int B, int H, int Hkv, int N, int D) {
   w.dot = take(q2);
   w.lse = take((size_t)(Gq * Npad * 4));
   w.dvec = take((size_t)(Gq * Npad * 4));
+  w.qc = take(codes_bytes(Gq, N, D));
+  w.qs = take(scales_bytes(Gq, N, D, FP4_BLOCK_ALONG_D));
+  w.qs64 = take(2 * scales_bytes(Gq, N, D, FP4_BLOCK_ALONG_D));
+  w.kc = take(codes_bytes(Gk, N, D));
+  w.ks = take(scales_bytes(Gk, N, D, FP4_BLOCK_ALONG_D));
   w.total = off;
   return w;
 }
@@ -601,18 +606,36 @@ fp4_status_t attn_bwd_any(const void* q, const void* k, const void* v, const voi
     fp4::pad_transpose_kernel<64><<<tq, 128, 0, st>>>(ob, N, (int)Npad, dop, dot);
   }
   FP4_CUDA(cudaGetLastError());
+  // Q's and K's NVFP4 codes and block scales (the forward's quantiser) for S^T,
+  // Q's scales regrouped per 64-query tile
+  if ((s = launch_quant(q, Gq, N, D, FP4_BLOCK_ALONG_D, ws + w.qc, ws + w.qs, amax, sms, st)) !=
+      FP4_OK)
+    return s;
+  if ((s = launch_quant(k, Gk, N, D, FP4_BLOCK_ALONG_D, ws + w.kc, ws + w.ks, amax + 1, sms,
+                        st)) != FP4_OK)
+    return s;
+  {
+    const int64_t n16 = (int64_t)scales_bytes(Gq, N, D, FP4_BLOCK_ALONG_D) / 16;
+    fp4::sf64_kernel<<<(unsigned)std::min<int64_t>((n16 + 255) / 256, (int64_t)sms * 8), 256, 0,
+                       st>>>(reinterpret_cast<const uint4*>(ws + w.qs), n16, D / 64 * 32,
+                             reinterpret_cast<uint4*>(ws + w.qs64));
+    FP4_CUDA(cudaGetLastError());
+  }
   fp4::lse_pad_kernel<<<(unsigned)std::min<int64_t>((Gq * Npad + 255) / 256, (int64_t)sms * 8), 256,
                         0, st>>>(lse, Gq, N, (int)Npad, lsep);
   FP4_CUDA(cudaGetLastError());
-  CUtensorMap mQ, mDO, mK64, mV64, mKT, mK128, mV128, mQ64, mDO64, mQT, mDOT;
+  CUtensorMap mQ, mDO, mK64, mV64, mKT, mKc, mV128, mQc, mDO64, mQT, mDOT;
+  const CUtensorMapSwizzle swQK = D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
   if ((s = tmap_bf16(&mQ, qh, D, Gq * Npad, fp4::kBwdQ)) != FP4_OK) return s;
   if ((s = tmap_bf16(&mDO, dop, D, Gq * Npad, fp4::kBwdQ)) != FP4_OK) return s;
   if ((s = tmap_bf16(&mK64, kh, D, Gk * Npad, fp4::kBwdKt)) != FP4_OK) return s;
   if ((s = tmap_bf16(&mV64, vh, D, Gk * Npad, fp4::kBwdKt)) != FP4_OK) return s;
   if ((s = tmap_bf16(&mKT, kt, Npad, Gk * D, D)) != FP4_OK) return s;
-  if ((s = tmap_bf16(&mK128, kh, D, Gk * Npad, fp4::kBwdK)) != FP4_OK) return s;
+  if ((s = tmap_2d(&mKc, ws + w.kc, D / 2, Gk * Npad, D / 2, fp4::kBwdK, swQK)) != FP4_OK)
+    return s;
   if ((s = tmap_bf16(&mV128, vh, D, Gk * Npad, fp4::kBwdK)) != FP4_OK) return s;
-  if ((s = tmap_bf16(&mQ64, qh, D, Gq * Npad, fp4::kBwdQt)) != FP4_OK) return s;
+  if ((s = tmap_2d(&mQc, ws + w.qc, D / 2, Gq * Npad, D / 2, fp4::kBwdQt, swQK)) != FP4_OK)
+    return s;
   if ((s = tmap_bf16(&mDO64, dop, D, Gq * Npad, fp4::kBwdQt)) != FP4_OK) return s;
   if ((s = tmap_bf16(&mQT, qt, Npad, Gq * D, D)) != FP4_OK) return s;
   if ((s = tmap_bf16(&mDOT, dot, Npad, Gq * D, D)) != FP4_OK) return s;
@@ -621,6 +644,8 @@ fp4_status_t attn_bwd_any(const void* q, const void* k, const void* v, const voi
   p.lse = lsep;
   p.Dvec = dvec;
   p.out = static_cast<const __nv_bfloat16*>(out);
+  p.k_sf = ws + w.ks;
+  p.q_sf64 = ws + w.qs64;
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
@@ -638,7 +663,7 @@ fp4_status_t attn_bwd_any(const void* q, const void* k, const void* v, const voi
   bwd_dkdv_kernel_for(D, causal)<<<g2, fp4::kBwdThreads,
                                    D == 128 ? fp4::BwdDkvSmem<128>::kBytes
                                             : fp4::BwdDkvSmem<64>::kBytes,
-                                   st>>>(mK128, mV128, mQ64, mDO64, mQT, mDOT, p);
+                                   st>>>(mKc, mV128, mQc, mDO64, mQT, mDOT, p);
   FP4_CUDA(cudaGetLastError());
   return FP4_OK;
 }
