@@ -252,10 +252,11 @@ def run_bwd(args, wl):
     ms_per_step = sum(ms) / len(ms)
     fwd_flops = wl.flops
     value = 2.5 * fwd_flops / (ms_per_step * 1e-3) / 1e12
-    # the kernels' own tensor work: the dq kernel's S, dP and its two dQ sums
-    # (P (dP - c) K^ and P K^), the dk/dv kernel's S, dP, dV, dK: 8 contractions
-    # of 2 N^2 D per head
-    tensor_flops = 8 * fwd_flops / 2
+    # the kernels' own tensor work, 8 contractions of 2 N^2 D per head: the dq
+    # kernel's S, dP and its two dQ sums (P (dP - c) K^ and P K^) and the dk/dv
+    # kernel's dP, dV, dK in bf16, and its S^T in NVFP4 (4x the bf16 rate, so
+    # counted as a quarter of a bf16 contraction against the bf16 peak)
+    tensor_flops = 7.25 * fwd_flops / 2
     peaks, src = measured_peaks()
     hlse = torch.empty(lse.shape, dtype=torch.float32, pin_memory=True)
     hlse.copy_(lse)
@@ -288,14 +289,16 @@ def run_bwd(args, wl):
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": tensor_flops / (ms_per_step * 1e-3) / 1e12 / peaks["bf16_tflops"],
                      "traffic": None,
-                     "peak_source": f"measured dense bf16 ({src}); the whole call, 8 bf16 "
-                                    "contractions of 2 N^2 D per head; fraction of measured"},
+                     "peak_source": f"measured dense bf16 ({src}); the whole call, 7 bf16 "
+                                    "contractions of 2 N^2 D per head and one NVFP4 one "
+                                    "counted as 1/4; fraction of measured"},
         "e2e": {"value": e_val, "unit": "TFLOPS",
                 "h2d_bytes_per_step": (hq.numel() + hk.numel() + hv.numel() + hout.numel()
                                        + hdo.numel()) * 2 + hlse.numel() * 4,
                 "d2h_bytes_per_step": (hdq.numel() + hdk.numel() + hdv.numel()) * 2},
-        # amax, Q^ and K^ decode, V^ decode, dO pad/transpose, lse pad, dq kernel, dk/dv kernel
-        "gpu_launches": 8 * args.steps,
+        # amax, Q and K codes (2), Q scale regrouping, Q^ and K^ decode (2), V^ decode,
+        # dO pad/transpose, lse pad, dq kernel, dk/dv kernel
+        "gpu_launches": 11 * args.steps,
     }
     c = clk.summary()
     if c:
