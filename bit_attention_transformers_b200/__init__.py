@@ -21,7 +21,10 @@ from dataclasses import dataclass
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _ROOT = os.path.dirname(_HERE)
 _SRC_DIR = os.path.join(_HERE, "csrc")
-_LIB_PATH = os.path.join(_HERE, "libfp4attn.so")
+_RELEASE_LIB_PATH = os.path.join(_HERE, "libfp4attn.so")
+_DEBUG_LIB_PATH = os.path.join(_HERE, "libfp4attn_debug.so")  # built with -DFP4_DEBUG
+# FP4ATTN_DEBUG=1 in the environment loads the debug build (same entry points)
+_LIB_PATH = _DEBUG_LIB_PATH if os.environ.get("FP4ATTN_DEBUG") == "1" else _RELEASE_LIB_PATH
 _HEADER = os.path.join(_ROOT, "include", "fp4attn.h")
 
 FP4_OK = 0
@@ -30,6 +33,7 @@ FP4_ERR_UNSUPPORTED = 2
 FP4_ERR_WORKSPACE = 3
 FP4_ERR_CUDA = 4
 FP4_ERR_TIMEOUT = 5
+FP4_ERR_BOUNDS = 6
 FP4_BLOCK_ALONG_D = 0
 FP4_BLOCK_ALONG_N_T = 1
 FP8_TOKENS_T = -1  # Fp4Tensor.axis of E4M3 V codes [G][D][Npad] (no block scales)
@@ -48,7 +52,8 @@ EXPORTS = ("fp4_codes_bytes", "fp4_scales_bytes", "fp4_attn_workspace_bytes", "f
            "fp4_attn_bwd_workspace_bytes", "fp4_attn_bwd", "fp4_attn_bwd_scaled",
            "fp4_attn_fwd_quantized_lse", "fp4_attn_fwd_noalloc",
            "fp4_attn_host_workspace_bytes", "fp4_attn_fwd_host",
-           "fp4_status", "fp4_last_error", "fp4_probe_cvt", "fp4_test_wait_timeout")
+           "fp4_status", "fp4_last_error", "fp4_probe_cvt", "fp4_test_wait_timeout",
+           "fp4_debug_build", "fp4_debug_selftest")
 FP4_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
@@ -66,18 +71,33 @@ def _sources():
             if f.endswith((".cu", ".cuh"))] + [_HEADER]
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile libfp4attn.so in-tree for sm_100a (nvcc; no GPU needed)."""
+def build(force: bool = False, verbose: bool = False, debug: bool = True) -> str:
+    """Compile libfp4attn.so in-tree for sm_100a (nvcc; no GPU needed), and
+    with `debug` also libfp4attn_debug.so (-DFP4_DEBUG: the bounds-checking
+    build). Returns the path of the library `lib()` loads."""
     newest = max(os.path.getmtime(s) for s in _sources())
-    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < newest:
-        nvcc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "bin", "nvcc")
-        tmp = _LIB_PATH + f".tmp{os.getpid()}"
-        cmd = [nvcc, *NVCC_FLAGS, "-o", tmp, os.path.join(_SRC_DIR, "fp4attn.cu")]
-        if verbose:
-            cmd.insert(1, "-Xptxas=-v")
-        subprocess.check_call(cmd)
-        os.replace(tmp, _LIB_PATH)
+    nvcc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "bin", "nvcc")
+    for path, extra in ((_RELEASE_LIB_PATH, []), (_DEBUG_LIB_PATH, ["-DFP4_DEBUG"])):
+        if extra and not debug:
+            continue
+        if force or not os.path.exists(path) or os.path.getmtime(path) < newest:
+            tmp = path + f".tmp{os.getpid()}"
+            cmd = [nvcc, *NVCC_FLAGS, *extra, "-o", tmp, os.path.join(_SRC_DIR, "fp4attn.cu")]
+            if verbose:
+                cmd.insert(1, "-Xptxas=-v")
+            subprocess.check_call(cmd)
+            os.replace(tmp, path)
     return _LIB_PATH
+
+
+def load(debug: bool = False) -> ctypes.CDLL:
+    """Select the release (default) or the debug build for `lib()` and load
+    it; the next calls of every entry point go to that library."""
+    global _lib, _LIB_PATH
+    path = _DEBUG_LIB_PATH if debug else _RELEASE_LIB_PATH
+    if path != _LIB_PATH:
+        _LIB_PATH, _lib = path, None
+    return lib()
 
 
 _lib = None
@@ -170,6 +190,10 @@ def lib():
         L.fp4_probe_cvt.restype = i32
         L.fp4_test_wait_timeout.argtypes = [ctypes.c_uint64, vp, vp]
         L.fp4_test_wait_timeout.restype = i32
+        L.fp4_debug_build.argtypes = []
+        L.fp4_debug_build.restype = i32
+        L.fp4_debug_selftest.argtypes = [ctypes.c_uint, vp]
+        L.fp4_debug_selftest.restype = i32
         _lib = L
     return _lib
 
@@ -665,8 +689,20 @@ def fp4_attn_fwd_host_many(batches, outs, causal: bool = False,
 
 
 def fp4_status(stream=None):
-    """Synchronise and raise if a kernel reported an expired wait."""
+    """Synchronise and raise if a kernel reported an expired wait or (debug
+    build) a failed bounds check."""
     _check(lib().fp4_status(_stream(stream)))
+
+
+def fp4_debug_build() -> bool:
+    """Whether the loaded library is the FP4_DEBUG (bounds-checking) build."""
+    return bool(lib().fp4_debug_build())
+
+
+def fp4_debug_selftest(site: int, stream=None):
+    """Debug build only: one check that fails by construction (no memory is
+    addressed); the next fp4_status raises FP4_ERR_BOUNDS naming `site`."""
+    _check(lib().fp4_debug_selftest(int(site), _stream(stream)))
 
 
 def fp4_test_wait_timeout(limit_ns: int, stream=None):

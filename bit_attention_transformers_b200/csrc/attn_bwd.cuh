@@ -143,6 +143,9 @@ __global__ void __launch_bounds__(128) fq_rows_kernel(const __nv_bfloat16* __res
 #pragma unroll
     for (int i = 0; i < 64; ++i)
       w[i] = (uint32_t)tile[(2 * i) * LD + d] | ((uint32_t)tile[(2 * i + 1) * LD + d] << 16);
+    if (!FP4_CHECK(in_range((g * D + d) * (int64_t)Npad + t * 128, 128,
+                            (int64_t)(gridDim.x / ntile) * D * Npad), 321))
+      continue;
     uint4* d4 = reinterpret_cast<uint4*>(xt + (g * D + d) * (int64_t)Npad + t * 128);
 #pragma unroll
     for (int k = 0; k < 16; ++k) d4[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
@@ -226,6 +229,9 @@ __global__ void __launch_bounds__(128) pad_transpose_kernel(const __nv_bfloat16*
 #pragma unroll
     for (int i = 0; i < 64; ++i)
       w[i] = (uint32_t)tile[(2 * i) * LD + d] | ((uint32_t)tile[(2 * i + 1) * LD + d] << 16);
+    if (!FP4_CHECK(in_range((g * D + d) * (int64_t)Npad + t * 128, 128,
+                            (int64_t)(gridDim.x / ntile) * D * Npad), 322))
+      continue;
     uint4* d4 = reinterpret_cast<uint4*>(xt + (g * D + d) * (int64_t)Npad + t * 128);
 #pragma unroll
     for (int k = 0; k < 16; ++k) d4[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
@@ -242,6 +248,7 @@ __global__ void sf64_kernel(const uint4* __restrict__ sf, int64_t n16, int atom1
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16;
        i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t tile = i / atom16, j = i % atom16;
+    if (!FP4_CHECK(in_range((2 * tile + 1) * atom16 + j, 1, 2 * n16), 323)) continue;
     const uint4 w = sf[i];
     sf64[(2 * tile) * atom16 + j] = w;
     sf64[(2 * tile + 1) * atom16 + j] = make_uint4(w.z, w.w, w.x, w.y);
@@ -415,8 +422,11 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     if (warp == 0 && lane == 0) {
       bool ok = true;
       int issued = 0;
+      const int64_t Gq = (int64_t)gridDim.z * p.H, Gk = (int64_t)gridDim.z * p.Hkv;
       mbar_arrive_expect_tx(bar(kDqBarQ), 2 * L::kQ);
       for (int a = 0; a < NA; ++a) {
+        if (!FP4_CHECK(tma_ok(a * 64, 64, D, 2, gq * p.Npad + qt * kBwdQ, kBwdQ, Gq * p.Npad), 301))
+          continue;
         tma_load_2d(sb + L::oQ + a * kBwdQ * 128, &tmQ, a * 64, gq * p.Npad + qt * kBwdQ, bar(kDqBarQ));
         tma_load_2d(sb + L::oDO + a * kBwdQ * 128, &tmDO, a * 64, gq * p.Npad + qt * kBwdQ,
                     bar(kDqBarQ));
@@ -428,6 +438,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         const uint32_t base = sb + L::oA + st * 2 * L::kK;
         mbar_arrive_expect_tx(bar(kDqBarFullA + st), 2 * L::kK);
         for (int a = 0; a < NA; ++a) {
+          if (!FP4_CHECK(tma_ok(a * 64, 64, D, 2, gk * p.Npad + t * kBwdKt, kBwdKt, Gk * p.Npad),
+                         302))
+            continue;
           tma_load_2d(base + a * kBwdKt * 128, &tmK, a * 64, gk * p.Npad + t * kBwdKt,
                       bar(kDqBarFullA + st));
           tma_load_2d(base + L::kK + a * kBwdKt * 128, &tmV, a * 64, gk * p.Npad + t * kBwdKt,
@@ -447,7 +460,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         if (t >= kDqRingB && !(ok = bwd_wait(bar(kDqBarEmptyB + st), ((t / kDqRingB) - 1) & 1)))
           break;
         mbar_arrive_expect_tx(bar(kDqBarFullB + st), L::kKT);
-        tma_load_2d(sb + L::oB + st * L::kKT, &tmKT, t * kBwdKt, gk * D, bar(kDqBarFullB + st));
+        if (FP4_CHECK(tma_ok(t * kBwdKt, kBwdKt, p.Npad, 2, (int64_t)gk * D, D,
+                             (int64_t)gridDim.z * p.Hkv * D), 303))
+          tma_load_2d(sb + L::oB + st * L::kKT, &tmKT, t * kBwdKt, gk * D, bar(kDqBarFullB + st));
         issued = t + 1;
       }
       for (int t = max(0, issued - kDqRingB); t < issued; ++t)
@@ -506,7 +521,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     // c_i = dO_i . O_i: dO_i from the row's 128-byte-swizzled chunks, O_i from
     // the forward's output (0 on padded rows)
     float cv = 0.0f;
-    if (ok && qrow < p.N) {
+    if (ok && qrow < p.N &&
+        FP4_CHECK(in_range(((int64_t)gq * p.N + qrow) * D, D, (int64_t)gridDim.z * p.H * p.N * D),
+                  304)) {
       const __nv_bfloat16* orow = p.out + ((int64_t)gq * p.N + qrow) * D;
 #pragma unroll
       for (int a = 0; a < NA; ++a) {
@@ -612,7 +629,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       // D_i - c_i for dQ, from the rounded terms that A holds: a row whose P
       // sits on one key then gets dQ = 0 exactly, as dS = 0 there
       const float E = fmaf(cv, Sq - 1.0f, Dqr);
-      if (stream == 0) p.Dvec[(int64_t)gq * p.Npad + qrow] = fmaf(cv, Sq, Dq);  // 0 on padded rows
+      if (stream == 0 &&
+          FP4_CHECK(in_range((int64_t)gq * p.Npad + qrow, 1, (int64_t)gridDim.z * p.H * p.Npad), 305))
+        p.Dvec[(int64_t)gq * p.Npad + qrow] = fmaf(cv, Sq, Dq);  // 0 on padded rows
       tc_fence_after();
       constexpr int DH = D / 2;  // each stream writes half the channels
       __nv_bfloat16* dst = p.dq + ((int64_t)gq * p.N + qrow) * D + stream * DH;
@@ -623,7 +642,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         tmem_ld32(tl + 256 + stream * DH + cc, oa);
         tmem_ld32(tl + 256 + D + stream * DH + cc, ob);
         tmem_wait_ld();
-        if (qrow < p.N) {
+        if (qrow < p.N &&
+            FP4_CHECK(in_range(((int64_t)gq * p.N + qrow) * D + stream * DH + cc, 32,
+                               (int64_t)gridDim.z * p.H * p.N * D), 306)) {
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
@@ -755,25 +776,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0) {
       bool ok = true;
       int issued = 0;
+      const int64_t Gq = (int64_t)gridDim.z * p.H, Gk = (int64_t)gridDim.z * p.Hkv;
       mbar_arrive_expect_tx(bar(kKvBarKV), L::kK + L::kKc + L::kSf);
-      for (int a = 0; a < NA; ++a)
-        tma_load_2d(sb + L::oV + a * kBwdK * 128, &tmV, a * 64, gk * p.Npad + kt * kBwdK,
-                    bar(kKvBarKV));
-      tma_load_2d(sb + L::oKc, &tmKc, 0, gk * p.Npad + kt * kBwdK, bar(kKvBarKV));
-      bulk_load(sb + L::oKsf, p.k_sf + ((int64_t)gk * ntq128 + kt) * L::kSf, L::kSf,
-                bar(kKvBarKV));
+      if (FP4_CHECK(tma_ok(0, D / 2, D / 2, 1, gk * p.Npad + kt * kBwdK, kBwdK, Gk * p.Npad), 311)) {
+        for (int a = 0; a < NA; ++a)
+          tma_load_2d(sb + L::oV + a * kBwdK * 128, &tmV, a * 64, gk * p.Npad + kt * kBwdK,
+                      bar(kKvBarKV));
+        tma_load_2d(sb + L::oKc, &tmKc, 0, gk * p.Npad + kt * kBwdK, bar(kKvBarKV));
+      }
+      if (FP4_CHECK(in_range(((int64_t)gk * ntq128 + kt) * L::kSf, L::kSf, Gk * ntq128 * L::kSf),
+                    312))
+        bulk_load(sb + L::oKsf, p.k_sf + ((int64_t)gk * ntq128 + kt) * L::kSf, L::kSf,
+                  bar(kKvBarKV));
       for (int t = 0; t < T && ok; ++t) {  // ring A: dO, Q codes and scales
         const int st = t & 1;
         const int gq = b * p.H + hk * G + t / nqt, i = i0 + t % nqt;
         if (t >= 2 && !(ok = bwd_wait(bar(kKvBarEmptyA + st), ((t >> 1) - 1) & 1))) break;
         const uint32_t base = sb + L::oA + st * L::kSlotA;
         mbar_arrive_expect_tx(bar(kKvBarFullA + st), L::kQ + L::kQc + L::kSf);
-        for (int a = 0; a < NA; ++a)
-          tma_load_2d(base + a * kBwdQt * 128, &tmDO, a * 64, gq * p.Npad + i * kBwdQt,
-                      bar(kKvBarFullA + st));
-        tma_load_2d(base + L::kQ, &tmQc, 0, gq * p.Npad + i * kBwdQt, bar(kKvBarFullA + st));
-        bulk_load(base + L::kQ + L::kQc, p.q_sf64 + ((int64_t)gq * (2 * ntq128) + i) * L::kSf,
-                  L::kSf, bar(kKvBarFullA + st));
+        if (FP4_CHECK(tma_ok(0, D / 2, D / 2, 1, gq * p.Npad + i * kBwdQt, kBwdQt, Gq * p.Npad),
+                      313)) {
+          for (int a = 0; a < NA; ++a)
+            tma_load_2d(base + a * kBwdQt * 128, &tmDO, a * 64, gq * p.Npad + i * kBwdQt,
+                        bar(kKvBarFullA + st));
+          tma_load_2d(base + L::kQ, &tmQc, 0, gq * p.Npad + i * kBwdQt, bar(kKvBarFullA + st));
+        }
+        const int64_t qsf = ((int64_t)gq * (2 * ntq128) + i) * L::kSf;
+        if (FP4_CHECK(in_range(qsf, L::kSf, Gq * 2 * ntq128 * L::kSf), 314))
+          bulk_load(base + L::kQ + L::kQc, p.q_sf64 + qsf, L::kSf, bar(kKvBarFullA + st));
         issued = t + 1;
       }
       drain_wait(bar(kKvBarKV), 0);
@@ -789,13 +819,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int gq = b * p.H + hk * G + t / nqt, i = i0 + t % nqt;
         if (t >= 2 && !(ok = bwd_wait(bar(kKvBarEmptyB + st), ((t >> 1) - 1) & 1))) break;
         const uint32_t base = sb + L::oB + st * 2 * L::kQT;
+        const int64_t Gq = (int64_t)gridDim.z * p.H;
         mbar_arrive_expect_tx(bar(kKvBarFullB + st), 2 * L::kQT + 512);
-        tma_load_2d(base, &tmQT, i * kBwdQt, gq * D, bar(kKvBarFullB + st));
-        tma_load_2d(base + L::kQT, &tmDOT, i * kBwdQt, gq * D, bar(kKvBarFullB + st));
-        bulk_load(sb + L::oLse + st * 512, p.lse + (int64_t)gq * p.Npad + i * kBwdQt, 256,
-                  bar(kKvBarFullB + st));
-        bulk_load(sb + L::oLse + st * 512 + 256, p.Dvec + (int64_t)gq * p.Npad + i * kBwdQt, 256,
-                  bar(kKvBarFullB + st));
+        if (FP4_CHECK(tma_ok(i * kBwdQt, kBwdQt, p.Npad, 2, (int64_t)gq * D, D, Gq * D), 315)) {
+          tma_load_2d(base, &tmQT, i * kBwdQt, gq * D, bar(kKvBarFullB + st));
+          tma_load_2d(base + L::kQT, &tmDOT, i * kBwdQt, gq * D, bar(kKvBarFullB + st));
+        }
+        if (FP4_CHECK(in_range((int64_t)gq * p.Npad + i * kBwdQt, 64, Gq * p.Npad), 316)) {
+          bulk_load(sb + L::oLse + st * 512, p.lse + (int64_t)gq * p.Npad + i * kBwdQt, 256,
+                    bar(kKvBarFullB + st));
+          bulk_load(sb + L::oLse + st * 512 + 256, p.Dvec + (int64_t)gq * p.Npad + i * kBwdQt, 256,
+                    bar(kKvBarFullB + st));
+        }
         issued = t + 1;
       }
       for (int t = max(0, issued - 2); t < issued; ++t)
@@ -937,7 +972,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int u = 0; u < 32; ++u) o[u] = o2[u] = 0.0f;
         }
-        if (key < p.N) {
+        if (key < p.N &&
+            FP4_CHECK(in_range(((int64_t)gk * p.N + key) * D + cc, 32,
+                               (int64_t)gridDim.z * p.Hkv * p.N * D), 317)) {
           uint32_t wv[16], wk[16];
 #pragma unroll
           for (int u = 0; u < 16; ++u) {

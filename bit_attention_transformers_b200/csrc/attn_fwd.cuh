@@ -69,11 +69,6 @@ constexpr int kAttnThreads = 384;  // 12 warps = 3 warpgroups
 constexpr uint32_t kRegsCtl = 56, kRegsSoftmax = 224;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
-enum : unsigned { kDevErrTimeout = 1u };
-
-// Device error word (one per device); read and cleared by fp4_status().
-__device__ unsigned g_fp4_err;
-
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity,
                                          uint64_t limit_ns = kTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -106,6 +101,15 @@ __global__ void wait_timeout_kernel(uint64_t limit_ns, int* ok) {
     *ok = wait_bar(smem_u32(&b), 0, limit_ns) ? 1 : 0;
   }
 }
+
+#ifdef FP4_DEBUG
+// Test support of the debug build: one check that fails by construction and
+// guards no access (the reporting path of FP4_CHECK, nothing else).
+__global__ void dbg_selftest_kernel(unsigned site) {
+  volatile unsigned never = 0u;
+  if (!FP4_CHECK(never != 0u, site)) return;
+}
+#endif
 
 struct AttnParams {
   const uint8_t* q_sf;
@@ -287,30 +291,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       bool ok = true;
       int kissued = 0, vissued = 0;  // tiles whose K / V loads were started
       const int qrow0 = gq * p.Npad + qt * kBM;
+      const int64_t Gq = (int64_t)p.B * p.H, Gk = (int64_t)p.B * p.Hkv;
       mbar_arrive_expect_tx(bar(kBarQ), L::kQ + L::kSfQK);
-      tma_load_2d(sb + L::oQ, &tmQ, 0, qrow0, bar(kBarQ));
-      bulk_load(sb + L::oQsf, p.q_sf + ((int64_t)gq * (p.Npad / kBM) + qt) * L::kSfQK, L::kSfQK,
-                bar(kBarQ));
+      if (FP4_CHECK(tma_ok(0, D / 2, D / 2, 1, qrow0, kBM, Gq * p.Npad), 201))
+        tma_load_2d(sb + L::oQ, &tmQ, 0, qrow0, bar(kBarQ));
+      const int64_t qsf = ((int64_t)gq * (p.Npad / kBM) + qt) * L::kSfQK;
+      if (FP4_CHECK(in_range(qsf, L::kSfQK, Gq * (p.Npad / kBM) * L::kSfQK), 202))
+        bulk_load(sb + L::oQsf, p.q_sf + qsf, L::kSfQK, bar(kBarQ));
       for (int j = 0; j < nt && ok; ++j) {
         const int st = j % kStages;
         const uint32_t pe = ((j / kStages) - 1) & 1;
         if (j >= kStages && !(ok = wait_bar(bar(kBarKEmpty + st), pe))) break;
         mbar_arrive_expect_tx(bar(kBarKFull + st), L::kK + L::kSfQK + (BIAS ? 4096 : 0));
-        tma_load_2d(sb + L::oK + st * L::kK, &tmK, 0, gk * p.Npad + j * kBN, bar(kBarKFull + st));
-        if (BIAS)
+        if (FP4_CHECK(tma_ok(0, D / 2, D / 2, 1, gk * p.Npad + j * kBN, kBN, Gk * p.Npad), 203))
+          tma_load_2d(sb + L::oK + st * L::kK, &tmK, 0, gk * p.Npad + j * kBN, bar(kBarKFull + st));
+        if (BIAS && FP4_CHECK(tma_ok(0, 32, 32, 1, gq * p.Npad + j * kBN, kBN, Gq * p.Npad), 204))
           tma_load_2d(sb + L::oBiasB + st * 4096, &tmB, 0, gq * p.Npad + j * kBN,
                       bar(kBarKFull + st));
-        bulk_load(sb + L::oKsf + st * 1024,
-                  p.k_sf + ((int64_t)gk * (p.Npad / kBN) + j) * L::kSfQK, L::kSfQK,
-                  bar(kBarKFull + st));
+        const int64_t ksf = ((int64_t)gk * (p.Npad / kBN) + j) * L::kSfQK;
+        if (FP4_CHECK(in_range(ksf, L::kSfQK, Gk * (p.Npad / kBN) * L::kSfQK), 205))
+          bulk_load(sb + L::oKsf + st * 1024, p.k_sf + ksf, L::kSfQK, bar(kBarKFull + st));
         kissued = j + 1;
         if (j >= kStages && !(ok = wait_bar(bar(kBarVEmpty + st), pe))) break;
         mbar_arrive_expect_tx(bar(kBarVFull + st), L::kV + (FP8 ? 0 : 1024));
-        tma_load_2d(sb + L::oV + st * L::kV, &tmV, j * (FP8 ? kBN : kBN / 2), gk * D,
-                    bar(kBarVFull + st));
-        if (!FP8)
-          bulk_load(sb + L::oVsf + st * 1024, p.v_sf + ((int64_t)gk * (p.Npad / 64) + 2 * j) * 512,
-                    1024, bar(kBarVFull + st));
+        constexpr int kVx = FP8 ? kBN : kBN / 2;  // bytes of one tile's keys in a V^T row
+        if (FP4_CHECK(tma_ok(j * kVx, kVx, (int64_t)p.Npad * kVx / kBN, 1, gk * D, D, Gk * D), 206))
+          tma_load_2d(sb + L::oV + st * L::kV, &tmV, j * kVx, gk * D, bar(kBarVFull + st));
+        const int64_t vsf = ((int64_t)gk * (p.Npad / 64) + 2 * j) * 512;
+        if (!FP8 && FP4_CHECK(in_range(vsf, 1024, Gk * (p.Npad / 64) * 512), 207))
+          bulk_load(sb + L::oVsf + st * 1024, p.v_sf + vsf, 1024, bar(kBarVFull + st));
         vissued = j + 1;
       }
       if (!ok) {
@@ -650,7 +659,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       } else {
         const float lsum = lval[row] + lval[kBM + row];
         inv = __fdiv_rn(fpv, lsum);
-        if (LSE && stream == 0 && qrow < p.N)
+        if (LSE && stream == 0 && qrow < p.N &&
+            FP4_CHECK(in_range((int64_t)gq * p.N + qrow, 1, (int64_t)p.B * p.H * p.N), 208))
           p.lse[(int64_t)gq * p.N + qrow] = m_fin + log2f(lsum);
       }
       constexpr int DH = D / 2;             // each stream writes half the channels
@@ -660,7 +670,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         float o[32];
         tmem_ld32(tl + kColO + stream * DH + cc, o);
         tmem_wait_ld();
-        if (qrow < p.N) {
+        if (qrow < p.N && FP4_CHECK(in_range(((int64_t)gq * p.N + qrow) * D + stream * DH + cc, 32,
+                                             (int64_t)p.B * p.H * p.N * D), 209)) {
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {

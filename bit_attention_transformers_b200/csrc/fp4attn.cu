@@ -1067,7 +1067,13 @@ fp4_status_t fp4_status(void* stream) {
   FP4_CUDA(cudaMemcpyFromSymbol(&err, fp4::g_fp4_err, sizeof(err)));
   if (err) {
     const unsigned zero = 0;
+    unsigned site = 0;
+    FP4_CUDA(cudaMemcpyFromSymbol(&site, fp4::g_fp4_dbg_site, sizeof(site)));
     FP4_CUDA(cudaMemcpyToSymbol(fp4::g_fp4_err, &zero, sizeof(zero)));
+    FP4_CUDA(cudaMemcpyToSymbol(fp4::g_fp4_dbg_site, &zero, sizeof(zero)));
+    if (err & fp4::kDevErrBounds)
+      return fail(FP4_ERR_BOUNDS, "a bounds or alignment check failed at site %u (error word %u)",
+                  site, err);
     return fail(FP4_ERR_TIMEOUT, "a kernel's bounded wait expired (device error word %u)", err);
   }
   return FP4_OK;
@@ -1105,6 +1111,31 @@ fp4_status_t fp4_scales_to_canonical(const uint8_t* native, int G, int N, int D,
       native, G, N, D, (int)axis, canonical);
   FP4_CUDA(cudaGetLastError());
   return FP4_OK;
+}
+
+int fp4_debug_build(void) {
+#ifdef FP4_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+fp4_status_t fp4_debug_selftest(unsigned site, void* stream) {
+  g_last_error.clear();
+#ifdef FP4_DEBUG
+  if (site < 1 || site > 99) return fail(FP4_ERR_INVALID_ARG, "site must be in 1 .. 99");
+  int dev, sms;
+  fp4_status_t s;
+  if ((s = device_setup(&dev, &sms)) != FP4_OK) return s;
+  fp4::dbg_selftest_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(site);
+  FP4_CUDA(cudaGetLastError());
+  return FP4_OK;
+#else
+  (void)site;
+  (void)stream;
+  return fail(FP4_ERR_UNSUPPORTED, "not a debug build (FP4_DEBUG)");
+#endif
 }
 
 fp4_status_t fp4_test_wait_timeout(uint64_t limit_ns, int* ok, void* stream) {

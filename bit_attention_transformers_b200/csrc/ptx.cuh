@@ -6,6 +6,41 @@
 
 namespace fp4 {
 
+// ---------------------------------------------------- device error word ----
+// One word per device, read and cleared by fp4_status(): bit 0 a bounded wait
+// expired, bit 1 a bounds or alignment check of an FP4_DEBUG build failed.
+enum : unsigned { kDevErrTimeout = 1u, kDevErrBounds = 2u };
+__device__ unsigned g_fp4_err;
+__device__ unsigned g_fp4_dbg_site;  // the first failed check's site number
+
+// FP4_DEBUG builds check the index arithmetic of every guarded global access
+// (bulk copies, TMA coordinates, epilogue stores, quantizer writes) against
+// the extent of the buffer it addresses. A failed check records its site,
+// sets the error word and makes the caller skip the access; nothing traps.
+// Release builds compile FP4_CHECK to `true` without evaluating the condition.
+#ifdef FP4_DEBUG
+__device__ __noinline__ void dbg_fail(unsigned site) {
+  atomicCAS(&g_fp4_dbg_site, 0u, site);
+  atomicOr(&g_fp4_err, kDevErrBounds);
+}
+#define FP4_CHECK(cond, site) ((cond) ? true : (::fp4::dbg_fail(site), false))
+#else
+#define FP4_CHECK(cond, site) true
+#endif
+
+// [off, off + n) inside [0, limit).
+__host__ __device__ __forceinline__ bool in_range(int64_t off, int64_t n, int64_t limit) {
+  return off >= 0 && n >= 0 && off + n <= limit;
+}
+
+// A 2D TMA tile load of an xbox x ybox box at column x (elements of `esize`
+// bytes) and row y of a width x rows tensor map: x on a 16-byte boundary (an
+// unaligned x is an illegal instruction on sm_100a) and the box inside.
+__host__ __device__ __forceinline__ bool tma_ok(int64_t x, int64_t xbox, int64_t width, int esize,
+                                                int64_t y, int64_t ybox, int64_t rows) {
+  return (x * esize) % 16 == 0 && in_range(x, xbox, width) && in_range(y, ybox, rows);
+}
+
 // ------------------------------------------------------------ addresses ----
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -155,7 +155,8 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16* __
     }
     uint32_t lo, hi;
     const uint32_t e = quant_block16(xv, s_enc, lo, hi);
-    if (valid) *reinterpret_cast<uint2*>(codes + r * (D / 2) + kb * 8) = make_uint2(lo, hi);
+    if (valid && FP4_CHECK(in_range(r * (D / 2) + kb * 8, 8, (int64_t)G * Npad * (D / 2)), 101))
+      *reinterpret_cast<uint2*>(codes + r * (D / 2) + kb * 8) = make_uint2(lo, hi);
     // gather the scales of blocks kb..kb+3 (lanes l..l+3) into lane l (kb % 4 == 0)
     const uint32_t e1 = __shfl_down_sync(0xFFFFFFFFu, e, 1);
     const uint32_t e2 = __shfl_down_sync(0xFFFFFFFFu, e, 2);
@@ -163,8 +164,9 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16* __
     if (valid && (kb & 3) == 0) {
       const int tile = n >> 7, rr = n & 127;
       const int64_t atom = (g * (Npad >> 7) + tile) * (D / 64) + (kb >> 2);
-      *reinterpret_cast<uint32_t*>(sf + atom * 512 + (rr & 31) * 16 + (rr >> 5) * 4) =
-          e | (e1 << 8) | (e2 << 16) | (e3 << 24);
+      const int64_t at = atom * 512 + (rr & 31) * 16 + (rr >> 5) * 4;
+      if (FP4_CHECK(in_range(at, 4, (int64_t)G * Npad * (D / 16)), 102))
+        *reinterpret_cast<uint32_t*>(sf + at) = e | (e1 << 8) | (e2 << 16) | (e3 << 24);
     }
   }
 }
@@ -208,16 +210,21 @@ __global__ void __launch_bounds__(128) quant_tokens_T_kernel(const __nv_bfloat16
       out[2 * tb + 1] = hi;
       e4[tb >> 2] |= e << (8 * (tb & 3));
     }
-    uint4* dst = reinterpret_cast<uint4*>(codes + (g * D + d) * (int64_t)(Npad / 2) + t * 64);
+    const int64_t at = (g * D + d) * (int64_t)(Npad / 2) + t * 64;
+    uint4* dst = reinterpret_cast<uint4*>(codes + at);
+    if (FP4_CHECK(in_range(at, 64, (int64_t)G * D * (Npad / 2)), 103)) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      dst[k] = make_uint4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
+      for (int k = 0; k < 4; ++k)
+        dst[k] = make_uint4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
+    }
   }
   // scales: rows are channels (padded to 128 with zeros), two atoms per tile
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
     const int64_t atom = g * (Npad >> 6) + t * 2 + c;
-    *reinterpret_cast<uint32_t*>(sf + atom * 512 + (d & 31) * 16 + (d >> 5) * 4) = e4[c];
+    const int64_t at = atom * 512 + (d & 31) * 16 + (d >> 5) * 4;
+    if (FP4_CHECK(in_range(at, 4, (int64_t)G * (Npad >> 6) * 512), 104))
+      *reinterpret_cast<uint32_t*>(sf + at) = e4[c];
   }
 }
 
@@ -263,10 +270,13 @@ __global__ void __launch_bounds__(128) quant_fp8_tokens_T_kernel(const __nv_bflo
         x[i] = __fmul_rn(__uint_as_float((uint32_t)tile[(w4 * 4 + i) * D + d] << 16), s8);
       out[w4] = cvt_e4m3x2(x[0], x[1]) | (cvt_e4m3x2(x[2], x[3]) << 16);
     }
-    uint4* dst = reinterpret_cast<uint4*>(codes + (g * D + d) * (int64_t)Npad + t * 128);
+    const int64_t at = (g * D + d) * (int64_t)Npad + t * 128;
+    uint4* dst = reinterpret_cast<uint4*>(codes + at);
+    if (FP4_CHECK(in_range(at, 128, (int64_t)G * D * Npad), 105)) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
-      dst[k] = make_uint4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
+      for (int k = 0; k < 8; ++k)
+        dst[k] = make_uint4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
+    }
   }
 }
 

@@ -66,7 +66,9 @@ typedef enum {
   FP4_ERR_UNSUPPORTED = 2, /* head dim not in {64,128}, or the device is not sm_100 */
   FP4_ERR_WORKSPACE = 3,   /* workspace smaller than the entry's *_workspace_bytes() */
   FP4_ERR_CUDA = 4,        /* a CUDA runtime call failed (message in fp4_last_error) */
-  FP4_ERR_TIMEOUT = 5      /* a kernel's bounded wait expired (from fp4_status) */
+  FP4_ERR_TIMEOUT = 5,     /* a kernel's bounded wait expired (from fp4_status) */
+  FP4_ERR_BOUNDS = 6       /* FP4_DEBUG builds: a kernel's bounds or alignment check failed
+                              (from fp4_status; the access was skipped) */
 } fp4_status_t;
 
 typedef enum {
@@ -403,9 +405,11 @@ fp4_status_t fp4_attn_fwd_noalloc(const void* q, const void* k, const void* v, v
                                   void* stream);
 
 /*
- * Synchronises the stream, then returns FP4_ERR_TIMEOUT if a kernel of this
- * library reported an expired wait on the current device since the last call
- * (and clears the report), FP4_ERR_CUDA on a CUDA error, else FP4_OK.
+ * Synchronises the stream, then returns FP4_ERR_BOUNDS if a kernel of an
+ * FP4_DEBUG build failed a bounds or alignment check on the current device
+ * since the last call (the message names the check's site), else
+ * FP4_ERR_TIMEOUT if one reported an expired wait, and clears the report;
+ * FP4_ERR_CUDA on a CUDA error; else FP4_OK.
  */
 fp4_status_t fp4_status(void* stream);
 
@@ -429,6 +433,24 @@ fp4_status_t fp4_probe_cvt(uint32_t start, int64_t count, int kind, uint8_t* out
  * the timeout path can be exercised without breaking a real kernel.
  */
 fp4_status_t fp4_test_wait_timeout(uint64_t limit_ns, int* ok, void* stream);
+
+/*
+ * The debug build. The library built with -DFP4_DEBUG (libfp4attn_debug.so
+ * beside the release library, same entry points) checks the index arithmetic
+ * of its kernels' guarded global accesses (bulk copies, TMA coordinates and
+ * the 16-byte rule for their x, epilogue stores, quantizer writes) against
+ * the extent of the buffer each addresses; a failed check records its site
+ * number, skips the access and sets the device error word, and fp4_status()
+ * returns FP4_ERR_BOUNDS (waits that depended on a skipped copy then expire
+ * within their bound). Nothing traps. This is the bounds checker that stands
+ * in for compute-sanitizer. fp4_debug_build() returns 1 in that build, else
+ * 0. fp4_debug_selftest() launches one thread whose check fails by
+ * construction (it addresses no memory), so that the next fp4_status()
+ * returns FP4_ERR_BOUNDS with site `site` (1 .. 99); in the release build it
+ * launches nothing and returns FP4_ERR_UNSUPPORTED.
+ */
+int fp4_debug_build(void);
+fp4_status_t fp4_debug_selftest(unsigned site, void* stream);
 
 #ifdef __cplusplus
 }

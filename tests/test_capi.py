@@ -33,6 +33,21 @@ def test_every_declared_symbol_is_exported(L):
         assert hasattr(L, name), name
 
 
+def test_debug_build_exports_every_symbol(L):
+    """The FP4_DEBUG build has the release build's entry points and says which
+    it is (host-only calls: no GPU needed)."""
+    import ctypes
+    D = ctypes.CDLL(fa._DEBUG_LIB_PATH)
+    for name in _declared():
+        assert hasattr(D, name), name
+    D.fp4_debug_build.restype = ctypes.c_int
+    L.fp4_debug_build.restype = ctypes.c_int
+    assert D.fp4_debug_build() == 1 and L.fp4_debug_build() == 0
+    # an out-of-range site is rejected before anything is launched
+    D.fp4_debug_selftest.argtypes = [ctypes.c_uint, ctypes.c_void_p]
+    assert D.fp4_debug_selftest(0, None) == fa.FP4_ERR_INVALID_ARG
+
+
 def test_sizes(L):
     # Npad = 384 for N = 300; codes 4 bits per element, scales 1 byte per 16
     assert fa.fp4_codes_bytes(3, 300, 128, fa.FP4_BLOCK_ALONG_D) == 3 * 384 * 64
