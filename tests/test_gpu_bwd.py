@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 
 import bit_attention_transformers_b200 as fa
-from _util import bf16_bits_to_f32
+from _util import bf16_bits_to_f32, f32_to_bf16_bits
 from gpu_util import from_dev, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -140,3 +140,26 @@ def test_backward_workloads(ora, syn, name):
         want = ora.attn_bwd(q, k, v, do, wl.causal, q_rows=np.zeros((0, 3), np.int64), kv_rows=kr)
         check(gk[kr[:, 0], kr[:, 1], kr[:, 2]], want["dk"], np.zeros(16), "dk " + name)
         check(gv[kr[:, 0], kr[:, 1], kr[:, 2]], want["dv"], np.zeros(16), "dv " + name)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_offset_v_and_peaked_rows(ora, syn, causal):
+    """V with a large common offset per channel (dP_ij = dO_i . v_j then shares
+    a large term across the keys of a row) and sharp scores (most rows' P sits
+    on a few keys): the cases where dQ = scale d_K (A - (D - c) B), formed in
+    one pass, could cancel large terms. The bar is the usual one."""
+    B, H, Hkv, N, D = 1, 2, 1, 300, 128
+    q, k, v, do = _inputs(syn, B, H, Hkv, N, D, 321)
+    qf = bf16_bits_to_f32(q) * 3.0
+    kf = bf16_bits_to_f32(k) * 3.0
+    offs = (np.arange(D, dtype=np.float32) % 7 - 3.0) * 4.0  # per-channel offsets up to 12
+    vf = bf16_bits_to_f32(v) + offs
+    q, k, v = (f32_to_bf16_bits(x) for x in (qf, kf, vf))
+    _, _, gq, gk, gv = run_gpu(q, k, v, do, causal)
+    want = ora.attn_bwd(q, k, v, do, causal)
+    label = f"offset V, peaked, causal={causal}"
+    check(gq.reshape(-1, D), want["dq"].reshape(-1, D), np.repeat(np.arange(B * H), N), "dq " + label)
+    check(gk.reshape(-1, D), want["dk"].reshape(-1, D), np.repeat(np.arange(B * Hkv), N),
+          "dk " + label)
+    check(gv.reshape(-1, D), want["dv"].reshape(-1, D), np.repeat(np.arange(B * Hkv), N),
+          "dv " + label)
