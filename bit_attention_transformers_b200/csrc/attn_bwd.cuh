@@ -29,7 +29,7 @@
 //   sf64_kernel     Q's block scales regrouped per 64-query tile
 //   bwd_dkdv_kernel one CTA per 128 keys: over the query tiles of every query
 //       head of its key/value head, S^T from the NVFP4 codes (kind::mxf4nvf4),
-//       dV += P^T dO and dK += dS^T Q^ in TMEM
+//       dV += P^T dO and dK += dS^T Q^ in TMEM (P^T and dS^T from TMEM)
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -62,6 +62,19 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, bf16 operands, K = 16 per instruction; A
+// (M = 128 rows, one per TMEM lane) holds two consecutive K elements per
+// 32-bit column, the even one in the low half.
+__device__ __forceinline__ void mma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -689,9 +702,7 @@ struct BwdDkvSmem {
   static constexpr int oKsf = oKc + kKc;
   static constexpr int oA = oKsf + (kSf + 1023) / 1024 * 1024;  // ring A [2] (S^T, dP^T)
   static constexpr int oB = oA + 2 * kSlotA;          // ring B [2]: Q^T then dO^T (dK, dV)
-  static constexpr int oP = oB + 2 * 2 * kQT;         // P^T: 128 keys x 64 queries, bf16
-  static constexpr int oDS = oP + kBwdK * kBwdQt * 2; // dS^T
-  static constexpr int oLse = oDS + kBwdK * kBwdQt * 2;  // ring B [2]: lse[64], D[64]
+  static constexpr int oLse = oB + 2 * 2 * kQT;       // ring B [2]: lse[64], D[64]
   static constexpr int oBar = oLse + 2 * 512;
   static constexpr int oTmem = oBar + 256;
   static constexpr int kBytes = oTmem + 16 + 1024;
@@ -702,6 +713,8 @@ struct BwdDkvSmem {
 // ring B (Q^T, dO^T, lse, D) when dV and dK complete; each has its own
 // producer warp. One S^T/dP^T buffer: the compute warps copy it to registers
 // at once, so the next tile's S^T and dP^T run while they work on this one.
+// P^T and dS^T go back to TMEM (tcgen05.st) as the A operands of dV and dK:
+// no shared-memory store and no proxy fence on the compute warps' path.
 enum : int {
   kKvBarKV = 0,
   kKvBarFullA = 1,    // [2]
@@ -719,8 +732,10 @@ enum : int {
 template <int D>
 struct DkvCols {
   static constexpr uint32_t kS = 0, kDP = 64, kDV = 128, kDK = 128 + D, kKsf = 128 + 2 * D,
-                            kQsf = kKsf + 8;  // [2] x 8
-  static_assert(kQsf + 16 <= 512, "TMEM columns");
+                            kQsf = kKsf + 8,                 // [2] x 8
+                            kPT = (kQsf + 16 + 31) / 32 * 32,  // P^T: 64 bf16 per key = 32 columns
+                            kDST = kPT + 32;                   // dS^T
+  static_assert(kDST + 32 <= 512, "TMEM columns");
 };
 
 // One CTA per (128-key tile, key/value head, batch); tiles of 64 queries of
@@ -857,12 +872,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         const uint32_t base = sb + L::oB + st * 2 * L::kQT;
 #pragma unroll
-        for (int s = 0; s < kBwdQt / 16; ++s) {
+        for (int s = 0; s < kBwdQt / 16; ++s) {  // A (P^T, dS^T) from TMEM, 8 columns per K step
           const uint32_t acc = (t > 0 || s > 0) ? 1u : 0u;
-          mma_bf16(tmem + TC::kDV, kmaj_desc(sb + L::oP, kBwdK, s), kmaj_desc(base + L::kQT, D, s),
-                   idO, acc);
-          mma_bf16(tmem + TC::kDK, kmaj_desc(sb + L::oDS, kBwdK, s), kmaj_desc(base, D, s), idO,
-                   acc);
+          mma_bf16_ta(tmem + TC::kDV, tmem + TC::kPT + 8 * s, kmaj_desc(base + L::kQT, D, s), idO,
+                      acc);
+          mma_bf16_ta(tmem + TC::kDK, tmem + TC::kDST + 8 * s, kmaj_desc(base, D, s), idO, acc);
         }
         tc_commit(bar(kKvBarEmptyB + st));
         tc_commit(bar(kKvBarPEmpty));
@@ -940,17 +954,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       if (t > 0) ok = __all_sync(0xFFFFFFFFu, bwd_wait(bar(kKvBarPEmpty), (t - 1) & 1));
       if (!ok) break;
-      uint8_t* pr = sm + L::oP + row * 128;
-      uint8_t* dr = sm + L::oDS + row * 128;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {  // 16-byte chunks half * 4 + j of the row (128-byte swizzle)
-        const int off = ((half * 4 + j) ^ (row & 7)) * 16;
-        *reinterpret_cast<uint4*>(pr + off) =
-            make_uint4(wp[4 * j], wp[4 * j + 1], wp[4 * j + 2], wp[4 * j + 3]);
-        *reinterpret_cast<uint4*>(dr + off) =
-            make_uint4(wd[4 * j], wd[4 * j + 1], wd[4 * j + 2], wd[4 * j + 3]);
-      }
-      fence_proxy_async_smem();
+      // P^T and dS^T of this warp's 32 queries: TMEM columns half * 16 .. + 15
+      tc_fence_after();
+      tmem_st16(tl + TC::kPT + half * 16, reinterpret_cast<const float*>(wp));
+      tmem_st16(tl + TC::kDST + half * 16, reinterpret_cast<const float*>(wd));
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kKvBarPFull));
