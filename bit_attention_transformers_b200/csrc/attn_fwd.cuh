@@ -20,8 +20,11 @@
 //               (S buffer s, P buffer s), so two tiles are in flight on every
 //               SM sub-partition; the running maximum, the only value a tile
 //               needs from the one before, passes between the two streams
-//               through shared memory
-// TMEM columns: S0 [0,128) S1 [128,256) O [256,256+D) scales from 384.
+//               through shared memory; NVFP4 P (codes and block scales) goes
+//               to TMEM with tcgen05.st, where PV reads it as its A operand
+//               (FP8 P goes through shared memory)
+// TMEM columns: S0 [0,128) S1 [128,256) O [256,256+D) scales from 384, then
+// P's codes (two buffers of 16 columns).
 //
 // EFQ variant (template flag EFQ) [EFQ-Softmax abstract]: P is generated
 // without exponentials. Per 16-key block, E = floor(max z) - 2 with z = x - m
@@ -180,7 +183,8 @@ template <bool EFQ>
 struct TmemCols {
   static constexpr uint32_t kSf = EFQ ? 400 : 384;
   static constexpr uint32_t kQsf = kSf, kKsf = kSf + 8, kPsf = kSf + 24, kVsf = kSf + 40,
-                            kOnesSf = kSf + 56;
+                            kOnesSf = kSf + 56,
+                            kPc = kSf + 64;  // [2] x 16: P codes (NVFP4 paths), 8 per column
 };
 constexpr float kInv7 = 1.0f / 7.0f;
 constexpr float kRound = 8388608.0f;  // 2^23: x + 2^23 rounds x (0 <= x < 2^22) to an integer
@@ -395,23 +399,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                          idesc_f8e4m3(kBM, D), (t > 0 || c > 0) ? 1u : 0u);
           } else {
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              tc_cp_32x128b_x4(tPsf + 4 * c,
-                               smem_desc(sb + L::oPsf + (t & 1) * 1024 + 512 * c, 0, 128, 0));
+            for (int c = 0; c < 2; ++c)
               tc_cp_32x128b_x4(tVsf + 4 * c, smem_desc(sb + L::oVsf + st * 1024 + 512 * c, 0, 128, 0));
-            }
+            // P's codes and block scales were written to TMEM by the softmax warps
 #pragma unroll
             for (int c = 0; c < 2; ++c)
-              mma_mxf4nvf4(tO, smem_desc(sb + L::oP + (t & 1) * L::kP + 32 * c, 16, 512, 4),
-                           smem_desc(sb + L::oV + st * L::kV + 32 * c, 16, 512, 4), kIdO,
-                           tPsf + 4 * c, tVsf + 4 * c, (t > 0 || c > 0) ? 1u : 0u);
+              mma_mxf4nvf4_ta(tO, tmem + TC::kPc + 16 * (t & 1) + 8 * c,
+                              smem_desc(sb + L::oV + st * L::kV + 32 * c, 16, 512, 4), kIdO,
+                              tPsf + 4 * c, tVsf + 4 * c, (t > 0 || c > 0) ? 1u : 0u);
           }
           if (EFQ) {
 #pragma unroll
             for (int c = 0; c < 2; ++c)
-              mma_mxf4nvf4(tmem + kColL, smem_desc(sb + L::oP + (t & 1) * L::kP + 32 * c, 16, 512, 4),
-                           smem_desc(sb + L::oOnes + 32 * c, 16, 512, 4), idesc_mxf4nvf4(kBM, 16),
-                           tPsf + 4 * c, tmem + TC::kOnesSf, (t > 0 || c > 0) ? 1u : 0u);
+              mma_mxf4nvf4_ta(tmem + kColL, tmem + TC::kPc + 16 * (t & 1) + 8 * c,
+                              smem_desc(sb + L::oOnes + 32 * c, 16, 512, 4), idesc_mxf4nvf4(kBM, 16),
+                              tPsf + 4 * c, tmem + TC::kOnesSf, (t > 0 || c > 0) ? 1u : 0u);
           }
           tc_commit(bar(kBarO + (t & 1)));
           tc_commit(bar(kBarVEmpty + st));
@@ -622,17 +624,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           *reinterpret_cast<uint4*>(pbuf + ((k2 ^ (row & 7)) * 16)) =
               make_uint4(pc[4 * k2], pc[4 * k2 + 1], pc[4 * k2 + 2], pc[4 * k2 + 3]);
       } else {
-        // codes: the row's 64 bytes (64-byte swizzle); scales: two 4-block atoms
-        uint8_t* pbuf = sm + L::oP + stream * L::kP + row * 64;
-#pragma unroll
-        for (int k2 = 0; k2 < 4; ++k2)
-          *reinterpret_cast<uint4*>(pbuf + ((k2 ^ ((row >> 1) & 3)) * 16)) =
-              make_uint4(pc[4 * k2], pc[4 * k2 + 1], pc[4 * k2 + 2], pc[4 * k2 + 3]);
-        uint8_t* psf = sm + L::oPsf + stream * 1024 + (row & 31) * 16 + (row >> 5) * 4;
-        *reinterpret_cast<uint32_t*>(psf) = sfw[0];
-        *reinterpret_cast<uint32_t*>(psf + 512) = sfw[1];
+        // codes to TMEM, where PV takes them as its A operand (eight codes per
+        // column), and the row's scale word of each 64-key chunk into all four
+        // columns of the chunk's scale group in its own lane: no shared-memory
+        // store and no proxy fence on the softmax's path
+        tc_fence_after();
+        tmem_st16(tl + TC::kPc + 16 * stream, reinterpret_cast<const float*>(pc));
+        const uint32_t sw8[8] = {sfw[0], sfw[0], sfw[0], sfw[0], sfw[1], sfw[1], sfw[1], sfw[1]};
+        tmem_st8u(tl + kColPsf + 8 * stream, sw8);
+        tmem_wait_st();
       }
-      fence_proxy_async_smem();
+      if constexpr (FP8) fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kBarPFull + stream));

@@ -257,6 +257,28 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
       : "memory");
 }
 
+// Eight 32-bit TMEM columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, E2M1 operands with UE4M3 block scales
+// (scale_vec::4X); A: M = 128 rows, one per TMEM lane, eight codes per column.
+__device__ __forceinline__ void mma_mxf4nvf4_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X"
+      " [%0], [%1], %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
 // ---------------------------------------------------------- conversions ----
 // E4M3 (round to nearest even, saturating to +-448) of x, in the low byte.
 __device__ __forceinline__ uint32_t cvt_e4m3(float x) {
