@@ -20,11 +20,11 @@
 //               (S buffer s, P buffer s), so two tiles are in flight on every
 //               SM sub-partition; the running maximum, the only value a tile
 //               needs from the one before, passes between the two streams
-//               through shared memory; NVFP4 P (codes and block scales) goes
-//               to TMEM with tcgen05.st, where PV reads it as its A operand
-//               (FP8 P goes through shared memory)
+//               through shared memory; P (NVFP4 codes and block scales, or
+//               FP8 codes) goes to TMEM with tcgen05.st, where PV reads it as
+//               its A operand
 // TMEM columns: S0 [0,128) S1 [128,256) O [256,256+D) scales from 384, then
-// P's codes (two buffers of 16 columns).
+// P's codes (two buffers: 16 columns NVFP4, 32 columns FP8).
 //
 // EFQ variant (template flag EFQ) [EFQ-Softmax abstract]: P is generated
 // without exponentials. Per 16-key block, E = floor(max z) - 2 with z = x - m
@@ -184,7 +184,8 @@ struct TmemCols {
   static constexpr uint32_t kSf = EFQ ? 400 : 384;
   static constexpr uint32_t kQsf = kSf, kKsf = kSf + 8, kPsf = kSf + 24, kVsf = kSf + 40,
                             kOnesSf = kSf + 56,
-                            kPc = kSf + 64;  // [2] x 16: P codes (NVFP4 paths), 8 per column
+                            kPc = kSf + 64,  // [2] x 16: P codes (NVFP4 paths), 8 per column
+                            kP8 = kSf + 32;  // [2] x 32: P codes (FP8 path), 4 per column
 };
 constexpr float kInv7 = 1.0f / 7.0f;
 constexpr float kRound = 8388608.0f;  // 2^23: x + 2^23 rounds x (0 <= x < 2^22) to an integer
@@ -394,9 +395,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             // E4M3 P (128 bytes per row) times E4M3 V^T, 128-byte swizzle, K = 32 per MMA
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-              mma_f8e4m3(tO, smem_desc(sb + L::oP + (t & 1) * L::kP + 32 * c, 16, 1024, 2),
-                         smem_desc(sb + L::oV + st * L::kV + 32 * c, 16, 1024, 2),
-                         idesc_f8e4m3(kBM, D), (t > 0 || c > 0) ? 1u : 0u);
+              mma_f8e4m3_ta(tO, tmem + TC::kP8 + 32 * (t & 1) + 8 * c,
+                            smem_desc(sb + L::oV + st * L::kV + 32 * c, 16, 1024, 2),
+                            idesc_f8e4m3(kBM, D), (t > 0 || c > 0) ? 1u : 0u);
           } else {
 #pragma unroll
             for (int c = 0; c < 2; ++c)
@@ -617,12 +618,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_wait_st();
       }
       if constexpr (FP8) {
-        // codes: the row's 128 bytes (128-byte swizzle)
-        uint8_t* pbuf = sm + L::oP + stream * L::kP + row * 128;
-#pragma unroll
-        for (int k2 = 0; k2 < 8; ++k2)
-          *reinterpret_cast<uint4*>(pbuf + ((k2 ^ (row & 7)) * 16)) =
-              make_uint4(pc[4 * k2], pc[4 * k2 + 1], pc[4 * k2 + 2], pc[4 * k2 + 3]);
+        // codes to TMEM, where PV takes them as its A operand (four per column)
+        tc_fence_after();
+        tmem_st32u(tl + TC::kP8 + 32 * stream, pc);
+        tmem_wait_st();
       } else {
         // codes to TMEM, where PV takes them as its A operand (eight codes per
         // column), and the row's scale word of each 64-key chunk into all four
@@ -634,7 +633,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_st8u(tl + kColPsf + 8 * stream, sw8);
         tmem_wait_st();
       }
-      if constexpr (FP8) fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kBarPFull + stream));
