@@ -136,7 +136,7 @@ struct AttnSmem {
   static constexpr int kQ = kBM * D / 2;   // Q codes tile
   static constexpr int kK = kBN * D / 2;   // K codes tile
   static constexpr int kV = FP8 ? D * kBN : D * kBN / 2;    // V^T codes tile
-  static constexpr int kP = FP8 ? kBM * kBN : kBM * kBN / 2;  // P codes tile
+  static constexpr int kP = FP8 ? kBM * kBN : kBM * kBN / 2;  // P codes tile (reserved; P lives in TMEM)
   static constexpr int kSfQK = (D / 64) * 512;
   static constexpr int oQ = 0;
   static constexpr int oK = oQ + kQ;
@@ -147,7 +147,7 @@ struct AttnSmem {
   static constexpr int oQsf = oOnesSf + 512;
   static constexpr int oKsf = oQsf + 1024;
   static constexpr int oVsf = oKsf + kStages * 1024;
-  static constexpr int oPsf = oVsf + kStages * 1024;
+  static constexpr int oPsf = oVsf + kStages * 1024;  // reserved (P scales live in TMEM)
   static constexpr int oRed = oPsf + 2 * 1024;  // float [2][128] running max per stream, [2][128] l
   static constexpr int oPtab = oRed + 2048;     // float [128]
   static constexpr int oBar = oPtab + 512;      // mbarriers
